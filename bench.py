@@ -1,0 +1,391 @@
+#!/usr/bin/env python
+"""Benchmark of the CSA2 decode step on B200.
+
+One step = one csa2_decode_stack call: the append of this step's keys and Main
+KV rows (FP4 quantiser), the Full layer's indexer scan over the whole visible
+context with its block top-P pool and own top-K, the Reindex layers' pool
+rescoring and top-K, and attention for every layer (sparse FP4 Main KV, plus
+the FP8 sliding window where the workload has one).
+
+Default workload: the million-token configuration (4 sequences x 1,048,576
+cached positions, 1 query token each, 1 Full + 3 Reindex + 16 Reuse layers).
+Metric: decode query tokens per second through the layer stack; the indexer
+scan's HBM GB/s is reported as the roofline of the dominant kernel.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU: one process per GPU (torchrun); sequences are independent, so each
+rank decodes its own batch of the workload (weak scaling, no collective on the
+data path); the time is the max over ranks.  The reference arm times the CPU
+oracle (there is no reference implementation to run).
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import math
+import os
+import signal
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA2 decode query-tokens/s per layer stack at 1M ctx; indexer-scan HBM GB/s"
+UNIT = "qtok/s"
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", type=int, default=4, help="workload number (1..5)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle sample")
+    return ap.parse_args()
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def _workload_desc(cfg, w):
+    return {
+        "workload": f"{cfg.name}: B={cfg.B}, L={'x'.join(str(int(x)) for x in sorted(set(w.lens.tolist())))[:60]}"
+                    f", T={w.T}, H_I={cfg.H_I}, d_I={cfg.d_I}, P={cfg.P}, K={cfg.K}, Hq={cfg.Hq}, D={cfg.D}, "
+                    f"layers={''.join(w.modes)}{', paged' if cfg.paged else ''}{', swa' if cfg.swa else ''}",
+        "sum_context": int(w.lens.sum()),
+        "query_tokens_per_step": int(w.T),
+        "layers": len(w.modes),
+        "q_dtype": cfg.q_dtype,
+        "out_dtype": cfg.out_dtype,
+        "l2": "flushed (256 MiB write) before every timed step; caches 1.36 GB > L2",
+    }
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.3)
+        self.proc.send_signal(signal.SIGTERM)
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    sm.append(float(f[1]))
+                    mx.append(float(f[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, f[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+            os.remove(self.path)
+        except Exception:
+            pass
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- oracle sample
+def oracle_sample(cfg_id: int, seconds: float, seed_offset: int = 0):
+    """Times the CPU oracle on a bounded sample of the workload: whole query
+    tokens (all layers of the stack), as many as fit in `seconds` (>= 1).
+    Input preparation (regenerating and quantising the cached keys) is not
+    timed, as the GPU timing excludes the cache fill."""
+    import numpy as np
+
+    import oracle
+    from synth.workloads import BLOCK, CONFIGS, make_workload
+    cfg = CONFIGS[cfg_id]
+    w = make_workload(cfg.with_(seed=cfg.seed + seed_offset))
+    c = cfg
+    timed, toks = 0.0, 0
+    tok = 0
+    while toks == 0 or (timed < seconds and toks < w.T):
+        b, p = int(w.tok_seq[tok]), int(w.tok_pos[tok])
+        kx = w.kidx.rows_f32(b, 0, p + 1)
+        kc, ks, _ = oracle.quantize_fp4(kx)
+        del kx
+        qs = {l: w.iq_f32(l, tok) for l, m in enumerate(w.modes) if m in "FR"}
+        ws = {l: w.iw_f32(l, tok).astype(np.float64) for l in qs}
+        qm = {l: w.qmain_f64(l, tok) for l in range(len(w.modes))}
+        sw = {}
+        if c.swa:
+            for l in range(len(w.modes)):
+                codes, sc = w.swa_rows_e4m3(l, tok)
+                sw[l] = (codes, sc)
+        t0 = time.perf_counter()
+        idx = None
+        pool = None
+        for l, m in enumerate(w.modes):
+            if m in "FR":
+                qc, qsc, _ = oracle.quantize_fp4(qs[l])
+                q = oracle.dequant_fp4(qc, qsc)
+                if m == "F":
+                    r = oracle.full_select(q, ws[l], kc, ks, p, c.P, c.K, BLOCK)
+                    pool, idx = r.pool, r.idx
+                else:
+                    idx, _, _ = oracle.reindex_select(q, ws[l], kc, ks, p, pool, c.K, BLOCK)
+                rows_x = w.kv.select_rows_f32(b, idx)
+                vc, vs, _ = oracle.quantize_fp4(rows_x)
+                kv_rows = oracle.dequant_fp4(vc, vs)
+            swr = None
+            if c.swa:
+                codes, sc = sw[l]
+                swr = oracle.e4m3_decode_array(codes) * sc.astype(np.float64)[:, None]
+            oracle.attend_rows(qm[l], kv_rows, swr, 1.0 / math.sqrt(c.D))
+        timed += time.perf_counter() - t0
+        toks += 1
+        tok = (tok + 1) % w.T
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return toks / timed, toks, timed, cores
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from synth.workloads import CONFIGS, make_workload
+    cfg = CONFIGS[args.config]
+    w = make_workload(cfg)
+    per_step = max(1.0, min(args.cpu_seconds, 15.0))
+    for _ in range(args.warmup):
+        oracle_sample(args.config, 0.0)
+    vals, times = [], []
+    for _ in range(args.steps):
+        v, toks, t, cores = oracle_sample(args.config, per_step)
+        vals.append(v)
+        times.append(t / toks)
+    value = sum(1.0 / t for t in times) / len(times)
+    sample = f"whole query tokens of {cfg.name} through all {len(w.modes)} layers, >= 1 per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * sum(times) / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": _workload_desc(cfg, w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    import csa2_fp4_sparse_b200 as C
+    from synth.gpu import DeviceWorkload
+    from synth.workloads import CONFIGS, algorithmic_bytes, make_workload
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def allmax(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    cfg = CONFIGS[args.config]
+    cfg = cfg.with_(seed=cfg.seed + 1000 * rank)
+    w = make_workload(cfg)
+    dw = DeviceWorkload(w)
+    dw.fill_caches(include_new=False)
+    desc = dw.stack_desc(append=True, copies=False)
+    ws = dw.stack_workspace(desc)
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def step():
+        rc = C.csa2_decode_stack(ctypes.byref(desc), ws.data_ptr(), ws.numel(), sp)
+        if rc != 0:
+            raise RuntimeError(f"csa2_decode_stack: {rc} {C.csa2_last_error()}")
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    st = C.csa2_get_status(sp)
+    assert st == 0, f"device status {st}"
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.4)
+    barrier()
+    torch.cuda.synchronize()
+    n0 = C.csa2_launch_count()
+    for k in range(args.steps):
+        flush.zero_()
+        ev[k][0].record(stream)
+        step()
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    n_launch = C.csa2_launch_count() - n0
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = allmax(sum(step_ms))
+    st = C.csa2_get_status(sp)
+    assert st == 0, f"device status {st}"
+    value = world * w.T * args.steps / (total_ms / 1000.0)
+
+    # per-kernel times (second pass, profiler on; same steps)
+    C.csa2_profiler_read()
+    C.csa2_profiler_enable(1)
+    for _ in range(args.steps):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    kstats = C.csa2_profiler_read()
+    C.csa2_profiler_enable(0)
+    ab = algorithmic_bytes(w)
+    peak_hbm, peak_bf16, peak_kind = _peaks()
+    scan_name = next((n for n in kstats if n.startswith("scan")), None)
+    roof = None
+    kernels = {}
+    tot_prof = sum(v[1] for v in kstats.values())
+    for n, (cnt, ms) in sorted(kstats.items(), key=lambda kv: -kv[1][1]):
+        kernels[n] = {"launches_per_step": cnt / args.steps, "us_per_step": 1000.0 * ms / args.steps,
+                      "share": ms / tot_prof if tot_prof else None}
+    if scan_name:
+        cnt, ms = kstats[scan_name]
+        avg_s = ms / cnt / 1000.0
+        achieved = ab["scan"] / avg_s / 1e9
+        roof = {"kernel": scan_name, "bound": "hbm", "achieved": achieved, "peak": peak_hbm, "unit": "GB/s",
+                "frac": achieved / peak_hbm, "peak_source": peak_kind, "traffic": None,
+                "algorithmic_bytes_per_launch": ab["scan"], "avg_launch_us": avg_s * 1e6}
+
+    # end to end through the public call with host buffers (pinned)
+    e2e = None
+    try:
+        e2e = _e2e(args, C, dw, desc, ws, stream, flush, w)
+        e2e["value"] = world * e2e["value"] if e2e else None
+    except Exception as ex:  # reported, not hidden
+        e2e = {"value": None, "unit": UNIT, "error": str(ex)[:200]}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, toks, t, cores = oracle_sample(args.config, args.cpu_seconds)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{toks} whole query token(s) of {cfg.name} through all {len(w.modes)} layers "
+                         f"({t:.1f} s of CPU time; cache fill excluded)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "fp4", "data": "synthetic",
+            "config": dict(_workload_desc(cfg, w), parallelism=f"replicas x{world}"),
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(n_launch),
+            "clocks": clk, "kernels": kernels,
+            "scan_gbs": roof["achieved"] if roof else None,
+            "algorithmic_bytes_per_step": ab,
+            "step_ms_min_max": [min(step_ms), max(step_ms)],
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _e2e(args, C, dw, desc, ws, stream, flush, w):
+    """Same step through the public call, with every per-step input copied in
+    from pinned host memory and every output read back, inside the timing."""
+    import torch
+    ins, outs = [], []
+    for l in range(len(w.modes)):
+        if l in dw.iq:
+            ins += [dw.iq[l], dw.iw[l]]
+        ins.append(dw.q[l])
+        outs.append(dw.out[l])
+    ins += [dw.new_kidx, dw.new_kv]
+    h_in = [t.cpu().pin_memory() for t in ins]
+    h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
+    bi = sum(t.numel() * t.element_size() for t in h_in)
+    bo = sum(t.numel() * t.element_size() for t in h_out)
+    sp = stream.cuda_stream
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        flush.zero_()
+        ev[k][0].record(stream)
+        for d, h in zip(ins, h_in):
+            d.copy_(h, non_blocking=True)
+        rc = C.csa2_decode_stack(ctypes.byref(desc), ws.data_ptr(), ws.numel(), sp)
+        if rc != 0:
+            raise RuntimeError(C.csa2_last_error())
+        for h, d in zip(h_out, outs):
+            h.copy_(d, non_blocking=True)
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in ev)
+    return {"value": w.T * args.steps / (ms / 1000.0), "unit": UNIT, "h2d_bytes_per_step": bi,
+            "d2h_bytes_per_step": bo, "ms_per_step": ms / args.steps}
+
+
+def main():
+    args = _args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

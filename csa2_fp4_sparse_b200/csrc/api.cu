@@ -1,0 +1,546 @@
+// api.cu -- the C ABI of libcsa2.so: argument validation, workspace carving
+// and kernel launches on the caller's stream.  No device allocation here.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <algorithm>
+#include <atomic>
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "internal.h"
+#include "kernels_simt.cuh"
+
+namespace csa2 {
+
+__device__ int g_status;  // per-device status word (first device-side error)
+
+static thread_local char t_err[512];
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_err, sizeof(t_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_check(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return CSA2_OK;
+  return fail(CSA2_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int* status_ptr() {
+  static int* cache[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+    cache[dev] = static_cast<int*>(p);
+  }
+  return cache[dev];
+}
+
+// ---------------------------------------------------------------- profiler
+namespace {
+std::atomic<int64_t> g_launches{0};
+std::atomic<bool> g_prof_on{false};
+std::mutex g_prof_mu;
+struct ProfRec {
+  const char* name;
+  cudaEvent_t a, b;
+};
+std::vector<ProfRec> g_prof_recs;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t pool_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+}  // namespace
+
+Launch::Launch(const char* n, cudaStream_t s) : name(n), st(s), slot(-1) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (!g_prof_on.load(std::memory_order_relaxed)) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  ProfRec r{n, pool_event(), pool_event()};
+  cudaEventRecord(r.a, s);
+  g_prof_recs.push_back(r);
+  slot = (int)g_prof_recs.size() - 1;
+}
+
+Launch::~Launch() {
+  if (slot < 0) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (slot < (int)g_prof_recs.size()) cudaEventRecord(g_prof_recs[slot].b, st);
+}
+
+// ---------------------------------------------------------------- validation
+static int check_batch(const csa2_query_batch* qb) {
+  if (!qb) return fail(CSA2_ERR_INVALID_ARG, "query batch is NULL");
+  if (qb->n_seq < 1 || qb->n_tok < 1) return fail(CSA2_ERR_INVALID_ARG, "n_seq and n_tok must be >= 1");
+  if (qb->max_seq_len < 1 || qb->max_q_per_seq < 1 || qb->max_q_per_seq > qb->max_seq_len)
+    return fail(CSA2_ERR_INVALID_ARG, "bad max_seq_len/max_q_per_seq");
+  if (!qb->seq_len || !qb->tok_start || !qb->tok_seq || !qb->tok_pos)
+    return fail(CSA2_ERR_INVALID_ARG, "query batch arrays must be non-NULL");
+  return CSA2_OK;
+}
+
+static int check_cache(const csa2_fp4_cache* c, const char* name) {
+  if (!c) return fail(CSA2_ERR_INVALID_ARG, "%s cache is NULL", name);
+  if (!c->codes || !c->scales || c->n_rows < 1) return fail(CSA2_ERR_INVALID_ARG, "%s cache buffers missing", name);
+  if (c->dim < 32 || c->dim % 32) return fail(CSA2_ERR_UNSUPPORTED, "%s dim %d not a multiple of 32", name, c->dim);
+  if (c->page_table) {
+    if (c->page_size < 64 || c->page_size % 64 || c->max_pages < 1)
+      return fail(CSA2_ERR_UNSUPPORTED, "%s page_size must be a positive multiple of 64", name);
+  } else if (!c->seq_base) {
+    return fail(CSA2_ERR_INVALID_ARG, "%s: unpaged cache needs seq_base", name);
+  }
+  return CSA2_OK;
+}
+
+struct Carve {
+  uint8_t* base;
+  size_t cap, used = 0;
+  void* take(size_t bytes) {
+    size_t off = (used + 255) & ~size_t(255);
+    used = off + bytes;
+    return base ? base + off : nullptr;
+  }
+  bool ok() const { return used <= cap; }
+};
+
+static int n_blocks_max(const csa2_query_batch* qb) { return (qb->max_seq_len + kBlock - 1) / kBlock; }
+
+static size_t index_ws(const csa2_query_batch* qb, int P) {
+  Carve c{nullptr, 0};
+  c.take((size_t)qb->n_tok * n_blocks_max(qb) * 4);  // block scores
+  c.take((size_t)qb->n_tok * P * kBlock * 4);        // pool position scores
+  return c.used + 256;
+}
+
+static int n_att_splits(int K, const csa2_swa_desc* swa, int* n_sp) {
+  *n_sp = (K + kAttRows - 1) / kAttRows;
+  return *n_sp + (swa ? (swa->window + kAttRows - 1) / kAttRows : 0);
+}
+
+static size_t attend_ws(const csa2_query_batch* qb, int Hq, int D, int K, const csa2_swa_desc* swa) {
+  int n_sp;
+  int ns = n_att_splits(K, swa, &n_sp);
+  Carve c{nullptr, 0};
+  c.take((size_t)qb->n_tok * ns * Hq * D * 4);
+  c.take((size_t)qb->n_tok * ns * Hq * 2 * 4);
+  return c.used + 256;
+}
+
+// ---------------------------------------------------------------- launches
+int launch_quantize(const float* x, int64_t n_rows, int dim, const int64_t* slot, uint8_t* codes, uint8_t* scales,
+                    cudaStream_t st) {
+  if (n_rows == 0) return CSA2_OK;
+  int64_t work = n_rows * (dim / 8);
+  int64_t grid = (work + 255) / 256;
+  if (grid > 148 * 32) grid = 148 * 32;
+  Launch L_("quantize_fp4", st);
+  k_quantize_fp4<<<(int)grid, 256, 0, st>>>(x, n_rows, dim, slot, codes, scales, status_ptr());
+  return cuda_check(cudaGetLastError(), "k_quantize_fp4");
+}
+
+template <int DI>
+static int launch_scan_simt(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
+                            const csa2_fp4_cache* kc, float* bs, int64_t ld, cudaStream_t st) {
+  size_t smem = (size_t)H * DI * 4 + H * 4;
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(k_scan_simt<DI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    attr = true;
+  }
+  dim3 grid((qb->max_seq_len + 127) / 128, qb->n_tok);
+  Launch L_("scan_simt", st);
+  k_scan_simt<DI><<<grid, 128, smem, st>>>(*qb, qc, qs, w, H, *kc, bs, ld, status_ptr());
+  return cuda_check(cudaGetLastError(), "k_scan_simt");
+}
+
+template <int DI>
+static int launch_rescore_simt(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
+                               const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n, int P,
+                               float* scores, cudaStream_t st) {
+  size_t smem = (size_t)H * DI * 4 + H * 4;
+  dim3 grid((P * kBlock + 127) / 128, qb->n_tok);
+  Launch L_("rescore_simt", st);
+  k_rescore_simt<DI><<<grid, 128, smem, st>>>(*qb, qc, qs, w, H, *kc, pool, pool_n, P, scores, status_ptr());
+  return cuda_check(cudaGetLastError(), "k_rescore_simt");
+}
+
+int launch_scan(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
+                const csa2_fp4_cache* kc, float* bs, int64_t ld, cudaStream_t st) {
+  if (kc->dim == 128) return launch_scan_simt<128>(qb, qc, qs, w, H, kc, bs, ld, st);
+  return launch_scan_simt<64>(qb, qc, qs, w, H, kc, bs, ld, st);
+}
+
+int launch_rescore(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
+                   const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n, int P, float* scores,
+                   cudaStream_t st) {
+  if (kc->dim == 128) return launch_rescore_simt<128>(qb, qc, qs, w, H, kc, pool, pool_n, P, scores, st);
+  return launch_rescore_simt<64>(qb, qc, qs, w, H, kc, pool, pool_n, P, scores, st);
+}
+
+int launch_select(const csa2_query_batch* qb, const float* score, int64_t ld, int mode, const int32_t* pool,
+                  const int32_t* pool_n, int P, int k_out, int32_t* out, int32_t* out_n, cudaStream_t st) {
+  Launch L_(mode == 0 ? "select_blocks" : "select_positions", st);
+  k_select_topk<<<qb->n_tok, kSelThreads, 0, st>>>(*qb, score, ld, mode, pool, pool_n, P, k_out, out, out_n);
+  return cuda_check(cudaGetLastError(), "k_select_topk");
+}
+
+int launch_attend(const csa2_query_batch* qb, const void* q, int q_dtype, int Hq, const csa2_fp4_cache* kv,
+                  const int32_t* idx, const int32_t* idx_n, int K, const csa2_swa_desc* swa, float scale, void* out,
+                  int out_dtype, float* lse, void* ws, cudaStream_t st) {
+  const int D = kv->dim;
+  int n_sp;
+  const int ns = n_att_splits(K, swa, &n_sp);
+  Carve c{static_cast<uint8_t*>(ws), ~size_t(0)};
+  float* part_o = static_cast<float*>(c.take((size_t)qb->n_tok * ns * Hq * D * 4));
+  float* part_ml = static_cast<float*>(c.take((size_t)qb->n_tok * ns * Hq * 2 * 4));
+  csa2_swa_desc sw{};
+  if (swa) sw = *swa;
+  size_t smem = (size_t)kAttRows * D * 4 + kAttRows * 4;
+  dim3 grid(ns, qb->n_tok);
+  {
+  Launch L_("attend_simt", st);
+  if (D == 512) {
+    static bool attr = false;
+    if (!attr) {
+      cudaFuncSetAttribute(k_attend_simt<512>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      attr = true;
+    }
+    k_attend_simt<512><<<grid, 256, smem, st>>>(*qb, q, q_dtype, Hq, *kv, idx, idx_n, K, sw, n_sp, scale, part_o,
+                                                part_ml, ns, status_ptr());
+  } else {
+    k_attend_simt<128><<<grid, 256, smem, st>>>(*qb, q, q_dtype, Hq, *kv, idx, idx_n, K, sw, n_sp, scale, part_o,
+                                                part_ml, ns, status_ptr());
+  }
+  }
+  int rc = cuda_check(cudaGetLastError(), "k_attend_simt");
+  if (rc) return rc;
+  Launch L_("merge", st);
+  k_merge<<<dim3(Hq, qb->n_tok), 128, 0, st>>>(part_o, part_ml, ns, Hq, D, out, out_dtype, lse);
+  return cuda_check(cudaGetLastError(), "k_merge");
+}
+
+}  // namespace csa2
+
+using namespace csa2;
+
+// ============================================================================
+// C ABI
+// ============================================================================
+extern "C" {
+
+const char* csa2_last_error(void) { return t_err; }
+
+int csa2_version(void) { return 100; }
+
+int csa2_get_status(void* stream) {
+  int rc = cuda_check(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)), "cudaStreamSynchronize");
+  if (rc) return rc;
+  int v = 0, zero = 0;
+  rc = cuda_check(cudaMemcpyFromSymbol(&v, g_status, sizeof(int)), "read status");
+  if (rc) return rc;
+  rc = cuda_check(cudaMemcpyToSymbol(g_status, &zero, sizeof(int)), "clear status");
+  if (rc) return rc;
+  return v;
+}
+
+int csa2_quantize_fp4(const float* x, int64_t n_rows, int32_t dim, const int64_t* slot, uint8_t* codes,
+                      uint8_t* scales, void* stream) {
+  t_err[0] = 0;
+  if (n_rows < 0) return fail(CSA2_ERR_INVALID_ARG, "n_rows < 0");
+  if (dim < 32 || dim > 8192 || dim % 32) return fail(CSA2_ERR_UNSUPPORTED, "dim %d unsupported", dim);
+  if (n_rows > 0 && (!x || !codes || !scales)) return fail(CSA2_ERR_INVALID_ARG, "NULL buffer");
+  if (reinterpret_cast<uintptr_t>(x) % 16 || reinterpret_cast<uintptr_t>(codes) % 4)
+    return fail(CSA2_ERR_INVALID_ARG, "x must be 16-byte aligned and codes 4-byte aligned");
+  return launch_quantize(x, n_rows, dim, slot, codes, scales, static_cast<cudaStream_t>(stream));
+}
+
+int csa2_index_workspace_size(const csa2_query_batch* qb, int32_t H_I, int32_t d_I, int32_t P, int32_t K,
+                              size_t* bytes) {
+  t_err[0] = 0;
+  if (int rc = check_batch(qb)) return rc;
+  if (!bytes || P < 1 || K < 1 || H_I < 1) return fail(CSA2_ERR_INVALID_ARG, "bad arguments");
+  (void)d_I;
+  *bytes = index_ws(qb, P);
+  return CSA2_OK;
+}
+
+int csa2_attend_workspace_size(const csa2_query_batch* qb, int32_t Hq, int32_t D, int32_t K, int32_t has_swa,
+                               size_t* bytes) {
+  t_err[0] = 0;
+  if (int rc = check_batch(qb)) return rc;
+  if (!bytes || Hq < 1 || D < 32 || K < 1) return fail(CSA2_ERR_INVALID_ARG, "bad arguments");
+  csa2_swa_desc sw{};
+  sw.window = 256;
+  *bytes = attend_ws(qb, Hq, D, K, has_swa ? &sw : nullptr);
+  return CSA2_OK;
+}
+
+static int check_index_common(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w,
+                              int H_I, const csa2_fp4_cache* kc, int P, int K) {
+  if (int rc = check_batch(qb)) return rc;
+  if (int rc = check_cache(kc, "k_idx")) return rc;
+  if (!qc || !qs || !w) return fail(CSA2_ERR_INVALID_ARG, "indexer query buffers must be non-NULL");
+  if (kc->dim != 64 && kc->dim != 128) return fail(CSA2_ERR_UNSUPPORTED, "d_I must be 64 or 128");
+  if (H_I < 1 || H_I > 64) return fail(CSA2_ERR_UNSUPPORTED, "H_I must be in [1, 64]");
+  if (P < 1 || P > 4096) return fail(CSA2_ERR_UNSUPPORTED, "P must be in [1, 4096]");
+  if (K < 1 || K > 2048 || K > P * kBlock) return fail(CSA2_ERR_UNSUPPORTED, "K must be in [1, min(2048, 8P)]");
+  return CSA2_OK;
+}
+
+int csa2_index_full(const csa2_query_batch* qb, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
+                    int32_t H_I, const csa2_fp4_cache* k_idx, int32_t P, int32_t K, int32_t* pool, int32_t* pool_n,
+                    int32_t* idx, int32_t* idx_n, float* blockscore, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  t_err[0] = 0;
+  if (int rc = check_index_common(qb, q_codes, q_scales, w, H_I, k_idx, P, K)) return rc;
+  if (!pool || !pool_n || !idx || !idx_n) return fail(CSA2_ERR_INVALID_ARG, "output buffers must be non-NULL");
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256 || workspace_bytes < index_ws(qb, P))
+    return fail(CSA2_ERR_WORKSPACE, "workspace too small or misaligned (need %zu)", index_ws(qb, P));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Carve c{static_cast<uint8_t*>(workspace), workspace_bytes};
+  const int64_t ld = n_blocks_max(qb);
+  float* bs = static_cast<float*>(c.take((size_t)qb->n_tok * ld * 4));
+  float* sc = static_cast<float*>(c.take((size_t)qb->n_tok * P * kBlock * 4));
+  if (blockscore) bs = blockscore;
+  if (int rc = launch_scan(qb, q_codes, q_scales, w, H_I, k_idx, bs, ld, st)) return rc;
+  if (int rc = launch_select(qb, bs, ld, 0, nullptr, nullptr, P, P, pool, pool_n, st)) return rc;
+  if (int rc = launch_rescore(qb, q_codes, q_scales, w, H_I, k_idx, pool, pool_n, P, sc, st)) return rc;
+  return launch_select(qb, sc, (int64_t)P * kBlock, 1, pool, pool_n, P, K, idx, idx_n, st);
+}
+
+int csa2_index_reindex(const csa2_query_batch* qb, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
+                       int32_t H_I, const csa2_fp4_cache* k_idx, const int32_t* pool, const int32_t* pool_n,
+                       int32_t P, int32_t K, int32_t* idx, int32_t* idx_n, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  t_err[0] = 0;
+  if (int rc = check_index_common(qb, q_codes, q_scales, w, H_I, k_idx, P, K)) return rc;
+  if (!pool || !pool_n || !idx || !idx_n) return fail(CSA2_ERR_INVALID_ARG, "pool/idx buffers must be non-NULL");
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256 || workspace_bytes < index_ws(qb, P))
+    return fail(CSA2_ERR_WORKSPACE, "workspace too small or misaligned (need %zu)", index_ws(qb, P));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Carve c{static_cast<uint8_t*>(workspace), workspace_bytes};
+  c.take((size_t)qb->n_tok * n_blocks_max(qb) * 4);
+  float* sc = static_cast<float*>(c.take((size_t)qb->n_tok * P * kBlock * 4));
+  if (int rc = launch_rescore(qb, q_codes, q_scales, w, H_I, k_idx, pool, pool_n, P, sc, st)) return rc;
+  return launch_select(qb, sc, (int64_t)P * kBlock, 1, pool, pool_n, P, K, idx, idx_n, st);
+}
+
+static int check_attend(const csa2_query_batch* qb, const void* q, int q_dtype, int Hq, const csa2_fp4_cache* kv,
+                        bool have_idx, int K, const csa2_swa_desc* swa, void* out, int out_dtype) {
+  if (int rc = check_batch(qb)) return rc;
+  if (int rc = check_cache(kv, "kv")) return rc;
+  if (kv->dim != 128 && kv->dim != 512) return fail(CSA2_ERR_UNSUPPORTED, "D must be 128 or 512");
+  if (Hq != 16 && Hq != 32 && Hq != 64) return fail(CSA2_ERR_UNSUPPORTED, "Hq must be 16, 32 or 64");
+  if (K < 1 || K > 2048) return fail(CSA2_ERR_UNSUPPORTED, "K must be in [1, 2048]");
+  if (!q || !have_idx || !out) return fail(CSA2_ERR_INVALID_ARG, "NULL buffer");
+  if ((q_dtype != CSA2_F32 && q_dtype != CSA2_BF16) || (out_dtype != CSA2_F32 && out_dtype != CSA2_BF16))
+    return fail(CSA2_ERR_INVALID_ARG, "bad dtype");
+  if (swa) {
+    if (!swa->codes || !swa->scale) return fail(CSA2_ERR_INVALID_ARG, "swa buffers missing");
+    if (swa->dim != kv->dim) return fail(CSA2_ERR_INVALID_ARG, "swa dim must equal the Main KV dim");
+    if (swa->window < 1 || swa->window > 256) return fail(CSA2_ERR_UNSUPPORTED, "swa window must be in [1,256]");
+    if (swa->cap < swa->window + qb->max_q_per_seq - 1)
+      return fail(CSA2_ERR_INVALID_ARG, "swa cap must be >= window + max_q_per_seq - 1");
+  }
+  return CSA2_OK;
+}
+
+int csa2_attend_reuse(const csa2_query_batch* qb, const void* q, int32_t q_dtype, int32_t Hq, const csa2_fp4_cache* kv,
+                      const int32_t* idx, const int32_t* idx_n, int32_t K, const csa2_swa_desc* swa,
+                      float softmax_scale, void* out, int32_t out_dtype, float* lse, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  t_err[0] = 0;
+  if (int rc = check_attend(qb, q, q_dtype, Hq, kv, idx && idx_n, K, swa, out, out_dtype)) return rc;
+  size_t need = attend_ws(qb, Hq, kv->dim, K, swa);
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256 || workspace_bytes < need)
+    return fail(CSA2_ERR_WORKSPACE, "workspace too small or misaligned (need %zu)", need);
+  float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / std::sqrt((float)kv->dim);
+  return launch_attend(qb, q, q_dtype, Hq, kv, idx, idx_n, K, swa, scale, out, out_dtype, lse, workspace,
+                       static_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------- stack
+static size_t stack_ws(const csa2_stack_desc* d, size_t* sub_off) {
+  const csa2_query_batch* qb = &d->qb;
+  const int dI = d->k_idx.dim;
+  Carve c{nullptr, 0};
+  c.take((size_t)qb->n_tok * d->H_I * (dI / 2));   // quantised indexer query codes
+  c.take((size_t)qb->n_tok * d->H_I * (dI / 32));  // and scales
+  c.take((size_t)qb->n_tok * d->P * 4);            // pool
+  c.take((size_t)qb->n_tok * 4);                   // pool_n
+  c.take((size_t)qb->n_tok * d->K * 4);            // idx
+  c.take((size_t)qb->n_tok * 4);                   // idx_n
+  size_t sub = std::max(index_ws(qb, d->P), (size_t)0);
+  bool any_swa = false;
+  int win = 0;
+  for (int l = 0; l < d->n_layers; ++l)
+    if (d->layers[l].swa) {
+      any_swa = true;
+      win = std::max(win, d->layers[l].swa->window);
+    }
+  csa2_swa_desc sw{};
+  sw.window = win;
+  sub = std::max(sub, attend_ws(qb, d->Hq, d->kv.dim, d->K, any_swa ? &sw : nullptr));
+  c.take(0);
+  *sub_off = c.used;
+  c.take(sub);
+  return c.used + 256;
+}
+
+int csa2_stack_workspace_size(const csa2_stack_desc* d, size_t* bytes) {
+  t_err[0] = 0;
+  if (!d || !bytes) return fail(CSA2_ERR_INVALID_ARG, "NULL argument");
+  if (int rc = check_batch(&d->qb)) return rc;
+  if (d->n_layers < 1 || !d->layers) return fail(CSA2_ERR_INVALID_ARG, "no layers");
+  size_t off;
+  *bytes = stack_ws(d, &off);
+  return CSA2_OK;
+}
+
+int csa2_decode_stack(const csa2_stack_desc* d, void* workspace, size_t workspace_bytes, void* stream) {
+  t_err[0] = 0;
+  if (!d) return fail(CSA2_ERR_INVALID_ARG, "desc is NULL");
+  const csa2_query_batch* qb = &d->qb;
+  if (int rc = check_batch(qb)) return rc;
+  if (d->n_layers < 1 || !d->layers) return fail(CSA2_ERR_INVALID_ARG, "no layers");
+  if (d->layers[0].mode != CSA2_MODE_FULL) return fail(CSA2_ERR_INVALID_ARG, "layer 0 must be FULL");
+  for (int l = 0; l < d->n_layers; ++l) {
+    const csa2_layer_desc& L = d->layers[l];
+    if (L.mode < CSA2_MODE_FULL || L.mode > CSA2_MODE_REUSE) return fail(CSA2_ERR_INVALID_ARG, "layer %d: bad mode", l);
+    if (L.mode != CSA2_MODE_REUSE && (!L.iq || !L.iw))
+      return fail(CSA2_ERR_INVALID_ARG, "layer %d: selector layer needs iq and iw", l);
+    if (int rc = check_attend(qb, L.q, d->q_dtype, d->Hq, &d->kv, true, d->K, L.swa, L.out, d->out_dtype))
+      return rc;
+  }
+  if (int rc = check_cache(&d->k_idx, "k_idx")) return rc;
+  if (d->k_idx.dim != 64 && d->k_idx.dim != 128) return fail(CSA2_ERR_UNSUPPORTED, "d_I must be 64 or 128");
+  if (d->H_I < 1 || d->H_I > 64 || d->P < 1 || d->P > 4096 || d->K < 1 || d->K > 2048 || d->K > d->P * kBlock)
+    return fail(CSA2_ERR_UNSUPPORTED, "H_I/P/K out of the supported range");
+  size_t sub_off;
+  size_t need = stack_ws(d, &sub_off);
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256 || workspace_bytes < need)
+    return fail(CSA2_ERR_WORKSPACE, "workspace too small or misaligned (need %zu)", need);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int T = qb->n_tok, dI = d->k_idx.dim;
+  Carve c{static_cast<uint8_t*>(workspace), workspace_bytes};
+  uint8_t* qc = static_cast<uint8_t*>(c.take((size_t)T * d->H_I * (dI / 2)));
+  uint8_t* qsc = static_cast<uint8_t*>(c.take((size_t)T * d->H_I * (dI / 32)));
+  int32_t* pool = static_cast<int32_t*>(c.take((size_t)T * d->P * 4));
+  int32_t* pool_n = static_cast<int32_t*>(c.take((size_t)T * 4));
+  int32_t* idx = static_cast<int32_t*>(c.take((size_t)T * d->K * 4));
+  int32_t* idx_n = static_cast<int32_t*>(c.take((size_t)T * 4));
+  uint8_t* sub = static_cast<uint8_t*>(workspace) + sub_off;
+  size_t sub_bytes = workspace_bytes - sub_off;
+  const float scale = d->softmax_scale > 0.0f ? d->softmax_scale : 1.0f / std::sqrt((float)d->kv.dim);
+
+  // append this step's keys and Main KV rows
+  if (d->new_k_idx) {
+    if (!d->new_slot_k_idx) return fail(CSA2_ERR_INVALID_ARG, "new_k_idx needs new_slot_k_idx");
+    if (int rc = launch_quantize(d->new_k_idx, T, dI, d->new_slot_k_idx, d->k_idx.codes, d->k_idx.scales, st))
+      return rc;
+  }
+  if (d->new_kv) {
+    if (!d->new_slot_kv) return fail(CSA2_ERR_INVALID_ARG, "new_kv needs new_slot_kv");
+    if (int rc = launch_quantize(d->new_kv, T, d->kv.dim, d->new_slot_kv, d->kv.codes, d->kv.scales, st)) return rc;
+  }
+  const int32_t* cur_idx = idx;
+  const int32_t* cur_idx_n = idx_n;
+  for (int l = 0; l < d->n_layers; ++l) {
+    const csa2_layer_desc& L = d->layers[l];
+    if (L.mode != CSA2_MODE_REUSE) {
+      if (int rc = launch_quantize(L.iq, (int64_t)T * d->H_I, dI, nullptr, qc, qsc, st)) return rc;
+      Carve s{sub, sub_bytes};
+      const int64_t ld = n_blocks_max(qb);
+      float* bs = static_cast<float*>(s.take((size_t)T * ld * 4));
+      float* sc = static_cast<float*>(s.take((size_t)T * d->P * kBlock * 4));
+      if (L.mode == CSA2_MODE_FULL) {
+        if (int rc = launch_scan(qb, qc, qsc, L.iw, d->H_I, &d->k_idx, bs, ld, st)) return rc;
+        if (int rc = launch_select(qb, bs, ld, 0, nullptr, nullptr, d->P, d->P, pool, pool_n, st)) return rc;
+        if (L.pool_out) {
+          Launch L_("copy", st);
+          k_copy_i32<<<64, 256, 0, st>>>(pool, L.pool_out, (int64_t)T * d->P);
+          if (int rc = cuda_check(cudaGetLastError(), "copy pool")) return rc;
+        }
+      }
+      if (int rc = launch_rescore(qb, qc, qsc, L.iw, d->H_I, &d->k_idx, pool, pool_n, d->P, sc, st)) return rc;
+      if (int rc = launch_select(qb, sc, (int64_t)d->P * kBlock, 1, pool, pool_n, d->P, d->K, idx, idx_n, st))
+        return rc;
+      if (L.idx_out) {
+        Launch L_("copy", st);
+        k_copy_i32<<<64, 256, 0, st>>>(idx, L.idx_out, (int64_t)T * d->K);
+        if (int rc = cuda_check(cudaGetLastError(), "copy idx")) return rc;
+      }
+    }
+    if (int rc = launch_attend(qb, L.q, d->q_dtype, d->Hq, &d->kv, cur_idx, cur_idx_n, d->K, L.swa, scale, L.out,
+                               d->out_dtype, L.lse, sub, st))
+      return rc;
+  }
+  return CSA2_OK;
+}
+
+int csa2_profiler_enable(int on) {
+  t_err[0] = 0;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on.store(on != 0);
+  return CSA2_OK;
+}
+
+int csa2_profiler_read(csa2_kernel_stat* out, int32_t cap, int32_t* n_out) {
+  t_err[0] = 0;
+  if (!n_out || (cap > 0 && !out)) return fail(CSA2_ERR_INVALID_ARG, "NULL output");
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  std::map<std::string, std::pair<int64_t, double>> agg;
+  int rc = CSA2_OK;
+  for (auto& r : g_prof_recs) {
+    float ms = 0.0f;
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.a, r.b);
+    if (e != cudaSuccess && rc == CSA2_OK) rc = cuda_check(e, "profiler event");
+    auto& a = agg[r.name];
+    a.first += 1;
+    a.second += ms;
+    g_event_pool.push_back(r.a);
+    g_event_pool.push_back(r.b);
+  }
+  g_prof_recs.clear();
+  int n = 0;
+  for (auto& kv : agg) {
+    if (n < cap) {
+      snprintf(out[n].name, sizeof(out[n].name), "%s", kv.first.c_str());
+      out[n].launches = kv.second.first;
+      out[n].total_ms = kv.second.second;
+    }
+    ++n;
+  }
+  *n_out = n < cap ? n : cap;
+  return rc;
+}
+
+int64_t csa2_launch_count(void) { return g_launches.load(); }
+
+int csa2_selftest_wait_timeout(int64_t limit_ns, void* stream) {
+  t_err[0] = 0;
+  if (limit_ns < 1000 || limit_ns > 10000000000LL) return fail(CSA2_ERR_INVALID_ARG, "limit_ns out of range");
+  Launch L_("selftest_wait", static_cast<cudaStream_t>(stream));
+  k_selftest_wait<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, status_ptr());
+  return cuda_check(cudaGetLastError(), "k_selftest_wait");
+}
+
+}  // extern "C"

@@ -1,0 +1,103 @@
+"""The C ABI: the library loads, exports every entry point declared in
+include/csa2.h, and rejects bad arguments on the host (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import csa2_fp4_sparse_b200 as C
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "csa2.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(csa2_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported_and_bound():
+    lib = ctypes.CDLL(C._lib.LIB_PATH)
+    names = _declared()
+    assert "csa2_decode_stack" in names and len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in C.EXPORTED, n
+
+
+def test_version_and_error_string():
+    assert C.csa2_version() >= 100
+    assert isinstance(C.csa2_last_error(), str)
+
+
+def _batch(**kw):
+    b = C.csa2_query_batch(1, 1, 100, 1, 8, 8, 8, 8)
+    for k, v in kw.items():
+        setattr(b, k, v)
+    return b
+
+
+def test_quantize_rejects_bad_shapes():
+    assert C.csa2_quantize_fp4(16, 10, 48, None, 16, 16, None) == C.CSA2_ERR_UNSUPPORTED
+    assert "dim" in C.csa2_last_error()
+    assert C.csa2_quantize_fp4(16, -1, 64, None, 16, 16, None) == C.CSA2_ERR_INVALID_ARG
+    assert C.csa2_quantize_fp4(None, 10, 64, None, 16, 16, None) == C.CSA2_ERR_INVALID_ARG
+    assert C.csa2_quantize_fp4(8, 10, 64, None, 16, 16, None) == C.CSA2_ERR_INVALID_ARG  # misaligned x
+
+
+def test_index_rejects_bad_arguments():
+    kc = C.csa2_fp4_cache(16, 16, 100, 128, 0, None, 0, 16)
+    b = _batch()
+    args = lambda qb, H, kc_, P, K, ws_bytes=1 << 30: C.csa2_index_full(  # noqa: E731
+        ctypes.byref(qb) if qb is not None else None, 256, 256, 256, H, ctypes.byref(kc_), P, K, 256, 256, 256,
+        256, None, 256, ws_bytes, None)
+    assert args(None, 64, kc, 2048, 512) == C.CSA2_ERR_INVALID_ARG
+    assert args(_batch(n_tok=0), 64, kc, 2048, 512) == C.CSA2_ERR_INVALID_ARG
+    assert args(b, 65, kc, 2048, 512) == C.CSA2_ERR_UNSUPPORTED
+    assert args(b, 64, kc, 16, 512) == C.CSA2_ERR_UNSUPPORTED  # K > 8P
+    assert args(b, 64, C.csa2_fp4_cache(16, 16, 100, 96, 0, None, 0, 16), 2048, 512) == C.CSA2_ERR_UNSUPPORTED
+    assert args(b, 64, C.csa2_fp4_cache(16, 16, 100, 128, 32, 16, 4, None), 2048, 512) == C.CSA2_ERR_UNSUPPORTED
+    assert args(b, 64, C.csa2_fp4_cache(16, 16, 100, 128, 0, None, 0, None), 2048, 512) == C.CSA2_ERR_INVALID_ARG
+    assert args(b, 64, kc, 2048, 512, ws_bytes=10) == C.CSA2_ERR_WORKSPACE
+
+
+def test_workspace_size_queries():
+    b = _batch(n_tok=4, max_seq_len=1 << 20)
+    n = ctypes.c_size_t(0)
+    assert C.csa2_index_workspace_size(ctypes.byref(b), 64, 128, 2048, 512, ctypes.byref(n)) == 0
+    assert n.value >= 4 * (1 << 17) * 4 + 4 * 16384 * 4
+    assert C.csa2_attend_workspace_size(ctypes.byref(b), 64, 512, 512, 1, ctypes.byref(n)) == 0
+    assert n.value > 0
+
+
+def test_attend_rejects_bad_swa():
+    kv = C.csa2_fp4_cache(16, 16, 100, 512, 0, None, 0, 16)
+    b = _batch(max_q_per_seq=4)
+    sw = C.csa2_swa_desc(16, 16, 128, 128, 512)  # cap < window + W - 1
+    rc = C.csa2_attend_reuse(ctypes.byref(b), 256, C.CSA2_BF16, 64, ctypes.byref(kv), 256, 256, 512,
+                             ctypes.byref(sw), 0.0, 256, C.CSA2_BF16, None, 256, 1 << 30, None)
+    assert rc == C.CSA2_ERR_INVALID_ARG
+    rc = C.csa2_attend_reuse(ctypes.byref(b), 256, C.CSA2_BF16, 48, ctypes.byref(kv), 256, 256, 512, None, 0.0,
+                             256, C.CSA2_BF16, None, 256, 1 << 30, None)
+    assert rc == C.CSA2_ERR_UNSUPPORTED
+
+
+def test_stack_rejects_non_full_first_layer():
+    layers = (C.csa2_layer_desc * 1)()
+    layers[0].mode = C.CSA2_MODE_REUSE
+    d = C.csa2_stack_desc()
+    d.qb = _batch()
+    d.n_layers = 1
+    d.layers = layers
+    assert C.csa2_decode_stack(ctypes.byref(d), 256, 1 << 30, None) == C.CSA2_ERR_INVALID_ARG
+    assert "FULL" in C.csa2_last_error()
+
+
+def test_product_package_does_not_import_oracle():
+    pkg = os.path.join(ROOT, "csa2_fp4_sparse_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".c")):
+                txt = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert "oracle" not in txt.replace("Oracle", "").lower() or f == "__init__.py", f
