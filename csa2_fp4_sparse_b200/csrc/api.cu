@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <cstdlib>
 #include <algorithm>
 #include <atomic>
 #include <map>
@@ -181,8 +182,20 @@ static int launch_rescore_simt(const csa2_query_batch* qb, const uint8_t* qc, co
   return cuda_check(cudaGetLastError(), "k_rescore_simt");
 }
 
+// CSA2_SCAN_IMPL=simt selects the CUDA-core scan (comparison runs); the
+// tensor-core scan is the default wherever its shape limits hold.
+static bool use_scan_tc(const csa2_query_batch* qb, int H) {
+  static int env = -1;
+  if (env < 0) {
+    const char* e = getenv("CSA2_SCAN_IMPL");
+    env = (e && strcmp(e, "simt") == 0) ? 0 : 1;
+  }
+  return env == 1 && qb->max_q_per_seq <= 8 && H <= 64;
+}
+
 int launch_scan(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
                 const csa2_fp4_cache* kc, float* bs, int64_t ld, cudaStream_t st) {
+  if (use_scan_tc(qb, H)) return launch_scan_tc(qb, qc, qs, w, H, kc, bs, ld, st);
   if (kc->dim == 128) return launch_scan_simt<128>(qb, qc, qs, w, H, kc, bs, ld, st);
   return launch_scan_simt<64>(qb, qc, qs, w, H, kc, bs, ld, st);
 }

@@ -1,0 +1,504 @@
+// scan_tc.cu -- the Full layer's indexer scan on the 5th-generation tensor
+// cores (sm_100a).
+//
+// For every query token i of sequence b and visible position t <= p_i:
+//   s_t = sum_h w[i][h] * max(0, q~_{i,h} . k~_t),   B_j = max_{t in block j} s_t
+// (hierarchical indexer of the DeepSeek-V4.1-Flash pages, dbyun.net article
+// 10794, section "KV Cache 成为这一代架构改造的核心": the first Full layer scans
+// the whole visible context and keeps blocks of 8 positions).
+//
+// Design (one persistent CTA per SM, warp-specialised):
+//   warp 0      TMA producer: tiles of 128 positions of the FP4 indexer K cache
+//               (codes with the 64B/32B swizzle the MMA expects, plus the raw
+//               E4M3 scales) into an 8-stage shared-memory ring;
+//   warp 1      MMA issuer: rearranges the tile's scales into the tensor-core
+//               scale-factor layout (each per-32 E4M3 scale written twice, as
+//               the block-scaled MMA takes one UE4M3 scale per 16 elements),
+//               copies them to TMEM (tcgen05.cp), and issues
+//               tcgen05.mma kind::mxf4nvf4 (M = 128 positions, N = heads,
+//               K = 64 per instruction) per query token into a ring of TMEM
+//               accumulators; commits release the smem stage and hand the
+//               accumulator to the epilogue;
+//   warps 2..5  epilogue: TMEM -> registers (one position per thread),
+//               ReLU, weighted head sum, block max over 8 lanes, block-score
+//               store.
+// The key cache is streamed from HBM exactly once per sequence for all of its
+// query tokens.  All waits are bounded; on timeout the kernel records
+// CSA2_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace csa2 {
+namespace scan_tc {
+
+constexpr int kStages = 8;
+constexpr int kTile = 128;      // positions per tile = MMA M
+constexpr int kChunk = 64;      // rows per TMA box
+constexpr int kAccUnits = 4;    // TMEM accumulator ring, 64 columns each
+constexpr int kMaxW = 8;        // query tokens of one sequence per tile
+constexpr int kThreads = 192;   // 6 warps
+constexpr uint32_t kColAcc = 0;
+constexpr uint32_t kColSfa = kAccUnits * 64;              // 256
+constexpr uint32_t kColSfb = kColSfa + kStages * 8;      // 320
+constexpr uint32_t kTmemCols = 512;
+
+// shared-memory map (offsets from a 1024-aligned base)
+constexpr uint32_t kOffA = 0;                             // [kStages][8192]
+constexpr uint32_t kOffRaw = kOffA + kStages * 8192;      // [kStages][512]
+constexpr uint32_t kOffSfa = kOffRaw + kStages * 512;     // [kStages][2][512]
+constexpr uint32_t kOffB = kOffSfa + kStages * 1024;      // [kMaxW][64 rows][64 B]
+constexpr uint32_t kOffSfb = kOffB + kMaxW * 4096;        // [kMaxW][2][512]
+constexpr uint32_t kOffW = kOffSfb + kMaxW * 1024;        // [kMaxW][64] f32
+constexpr uint32_t kOffBar = kOffW + kMaxW * 64 * 4;      // mbarriers
+constexpr uint32_t kNumBars = 2 * kStages + 2 * kAccUnits + 1;
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;     // tmem base, abort flag
+constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;     // + alignment slack
+static_assert(kOffB % 1024 == 0, "B tiles must be 1024-aligned");
+
+struct Params {
+  csa2_query_batch qb;
+  const uint8_t* q_codes;
+  const uint8_t* q_scales;
+  const float* w;
+  int H, N, DI;
+  int64_t n_rows;
+  int page_size, max_pages;
+  const int32_t* page_table;
+  const int64_t* seq_base;
+  float* bscore;
+  int64_t ld_bs;
+  int* status;
+  uint64_t wait_ns;
+};
+
+__device__ __forceinline__ int ntiles_of(const Params& P, int b) {
+  return (__ldg(P.qb.seq_len + b) + kTile - 1) / kTile;
+}
+
+// this CTA's contiguous range of (sequence, tile) work in sequence-major order
+__device__ __forceinline__ void work_range(const Params& P, int64_t* begin, int64_t* end) {
+  int64_t total = 0;
+  for (int b = 0; b < P.qb.n_seq; ++b) total += ntiles_of(P, b);
+  *begin = total * blockIdx.x / gridDim.x;
+  *end = total * (blockIdx.x + 1) / gridDim.x;
+}
+
+// iterator over the tiles of [begin, end)
+struct TileIter {
+  int b, tile, ntile;
+  int64_t left;
+  __device__ void init(const Params& P, int64_t begin, int64_t end) {
+    b = 0;
+    int64_t acc = 0;
+    ntile = ntiles_of(P, 0);
+    while (b < P.qb.n_seq - 1 && acc + ntile <= begin) {
+      acc += ntile;
+      ++b;
+      ntile = ntiles_of(P, b);
+    }
+    tile = (int)(begin - acc);
+    left = end - begin;
+  }
+  __device__ bool valid() const { return left > 0; }
+  __device__ void next(const Params& P) {
+    --left;
+    if (++tile >= ntile && left > 0) {
+      do {
+        ++b;
+        ntile = ntiles_of(P, b);
+      } while (ntile == 0 && b < P.qb.n_seq - 1);
+      tile = 0;
+    }
+  }
+};
+
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, const Params& P, volatile int* abort) {
+  if (*abort) return false;
+  if (mbar_wait_bounded(bar, parity, P.wait_ns)) return true;
+  set_status(P.status, CSA2_ERR_TIMEOUT);
+  *abort = 1;
+  return false;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_scan_tc(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales,
+              const Params P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar_full = sbase + kOffBar;
+  const uint32_t bar_empty = bar_full + kStages * 8;
+  const uint32_t bar_accf = bar_empty + kStages * 8;
+  const uint32_t bar_acce = bar_accf + kAccUnits * 8;
+  const uint32_t bar_drain = bar_acce + kAccUnits * 8;
+  volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(smem + kOffMisc);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+  float* w_s = reinterpret_cast<float*>(smem + kOffW);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row_bytes = P.DI / 2, spr = P.DI / 32, ksteps = P.DI / 64;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(bar_full + 8 * i, 1);
+      mbar_init(bar_empty + 8 * i, 1);
+    }
+    for (int i = 0; i < kAccUnits; ++i) {
+      mbar_init(bar_accf + 8 * i, 1);
+      mbar_init(bar_acce + 8 * i, 4);
+    }
+    mbar_init(bar_drain, 1);
+    *abort = 0;
+    tc::fence_barrier_init();
+    tc::tma_prefetch_desc(&tm_codes);
+    tc::tma_prefetch_desc(&tm_scales);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(sbase + kOffMisc, kTmemCols);
+    tc::tmem_relinquish();
+    tc::fence_before_sync();
+  }
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_holder;
+
+  int64_t wb, we;
+  work_range(P, &wb, &we);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint32_t tx = 2u * kChunk * row_bytes + 2u * kChunk * spr;
+      const int32_t oob_row = (int32_t)P.n_rows;
+      const int32_t oob_x = (int32_t)(((P.n_rows * spr) + 15) / 16 * 16);
+      TileIter ti;
+      ti.init(P, wb, we);
+      int64_t it = 0;
+      for (; ti.valid(); ti.next(P), ++it) {
+        const int s = (int)(it % kStages);
+        const uint32_t n = (uint32_t)(it / kStages);
+        if (!wait_or_abort(bar_empty + 8 * s, (n & 1) ^ 1, P, abort)) break;
+        tc::mbar_arrive_expect_tx(bar_full + 8 * s, tx);
+        const int L = __ldg(P.qb.seq_len + ti.b);
+        for (int c = 0; c < 2; ++c) {
+          const int64_t pos0 = (int64_t)ti.tile * kTile + c * kChunk;
+          int64_t row0 = -1;
+          if (pos0 < L) {
+            if (P.page_table) {
+              int32_t pg = __ldg(P.page_table + (int64_t)ti.b * P.max_pages + pos0 / P.page_size);
+              row0 = (int64_t)pg * P.page_size + pos0 % P.page_size;
+            } else {
+              row0 = __ldg(P.seq_base + ti.b) + pos0;
+            }
+          }
+          int32_t ry = oob_row, sx = oob_x;
+          if (row0 >= 0 && row0 < P.n_rows && ((row0 * spr) & 15) == 0) {
+            ry = (int32_t)row0;
+            sx = (int32_t)(row0 * spr);
+          } else if (row0 >= 0) {
+            set_status(P.status, CSA2_ERR_RANGE);  // misplaced row: read as zeros
+          }
+          tc::tma_load_2d(sbase + kOffA + s * 8192 + c * kChunk * row_bytes, &tm_codes, bar_full + 8 * s, 0, ry);
+          tc::tma_load_1d(sbase + kOffRaw + s * 512 + c * kChunk * spr, &tm_scales, bar_full + 8 * s, sx);
+        }
+      }
+      // no copy of ours may be in flight when the CTA leaves
+      for (int s = 0; s < kStages && it > 0; ++s) {
+        int64_t uses = it / kStages + (s < it % kStages ? 1 : 0);
+        if (uses == 0) continue;
+        uint32_t last = (uint32_t)(uses - 1);
+        if (!mbar_wait_bounded(bar_full + 8 * s, last & 1, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t idesc = tc::idesc_mxf4nvf4(128, P.N);
+    const tc::SmemLayout sw = (P.DI == 128) ? tc::kSwizzle64B : tc::kSwizzle32B;
+    const uint32_t sbo = 8u * row_bytes;  // 8 rows per swizzle atom
+    TileIter ti;
+    ti.init(P, wb, we);
+    int64_t it = 0, acc_it = 0;
+    uint32_t drain_n = 0;
+    int cur_b = -1, W = 0, tok0 = 0;
+    for (; ti.valid(); ti.next(P), ++it) {
+      if (ti.b != cur_b) {
+        if (cur_b >= 0) {  // every MMA reading the old queries must finish first
+          if (lane == 0) tc::commit(bar_drain);
+          __syncwarp();
+          bool ok = wait_or_abort(bar_drain, drain_n & 1, P, abort);
+          ++drain_n;
+          if (!__all_sync(0xffffffffu, ok)) break;
+          tc::fence_after_sync();
+        }
+        cur_b = ti.b;
+        tok0 = __ldg(P.qb.tok_start + cur_b);
+        W = __ldg(P.qb.tok_start + cur_b + 1) - tok0;
+        if (W > kMaxW) {
+          if (lane == 0) set_status(P.status, CSA2_ERR_RANGE);
+          W = kMaxW;
+        }
+        // B operand: query codes, swizzled like the TMA-written A tiles
+        const int chunks_per_row = row_bytes / 16;
+        for (int e = lane; e < W * 64 * chunks_per_row; e += 32) {
+          const int j = e / (64 * chunks_per_row);
+          const int n = (e / chunks_per_row) % 64;
+          const int ch = e % chunks_per_row;
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (n < P.H)
+            v = __ldg(reinterpret_cast<const uint4*>(P.q_codes + ((int64_t)(tok0 + j) * P.H + n) * row_bytes) + ch);
+          const int sch = (P.DI == 128) ? (ch ^ ((n >> 1) & 3)) : (ch ^ ((n >> 2) & 1));
+          *reinterpret_cast<uint4*>(smem + kOffB + j * 4096 + n * row_bytes + sch * 16) = v;
+        }
+        // B scale factors: [m0 (32)][m1 (4)][k (4)] per 64-element K step
+        for (int e = lane; e < W * ksteps * 32; e += 32) {
+          const int j = e / (ksteps * 32), ks = (e / 32) % ksteps, m0 = e % 32;
+          uint32_t v[4];
+#pragma unroll
+          for (int m1 = 0; m1 < 4; ++m1) {
+            const int n = m1 * 32 + m0;
+            uint32_t a = 0, b2 = 0;
+            if (n < P.H) {
+              const uint8_t* sp = P.q_scales + ((int64_t)(tok0 + j) * P.H + n) * spr + 2 * ks;
+              a = __ldg(sp);
+              b2 = __ldg(sp + 1);
+            }
+            v[m1] = a | (a << 8) | (b2 << 16) | (b2 << 24);
+          }
+          *reinterpret_cast<uint4*>(smem + kOffSfb + (j * 2 + ks) * 512 + m0 * 16) = make_uint4(v[0], v[1], v[2], v[3]);
+        }
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          for (int j = 0; j < W; ++j)
+            for (int ks = 0; ks < ksteps; ++ks)
+              tc::cp_32x128b_warpx4(tmem + kColSfb + j * 8 + ks * 4,
+                                    tc::smem_desc(sbase + kOffSfb + (j * 2 + ks) * 512, 16, 128, tc::kSwizzleNone));
+        }
+        __syncwarp();
+      }
+      const int s = (int)(it % kStages);
+      const uint32_t n = (uint32_t)(it / kStages);
+      bool ok = wait_or_abort(bar_full + 8 * s, n & 1, P, abort);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      // A scale factors: raw [row][spr] -> [m0][m1][k] per K step (each scale twice)
+      {
+        const uint8_t* raw = smem + kOffRaw + s * 512;
+        uint32_t wv[4];
+#pragma unroll
+        for (int m1 = 0; m1 < 4; ++m1) {
+          const int r = m1 * 32 + lane;
+          wv[m1] = (spr == 4) ? *reinterpret_cast<const uint32_t*>(raw + r * 4)
+                              : (uint32_t)*reinterpret_cast<const uint16_t*>(raw + r * 2);
+        }
+        for (int ks = 0; ks < ksteps; ++ks) {
+          const uint32_t sel = ks == 0 ? 0x1100u : 0x3322u;
+          *reinterpret_cast<uint4*>(smem + kOffSfa + (s * 2 + ks) * 512 + lane * 16) =
+              make_uint4(__byte_perm(wv[0], 0, sel), __byte_perm(wv[1], 0, sel), __byte_perm(wv[2], 0, sel),
+                         __byte_perm(wv[3], 0, sel));
+        }
+      }
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      bool okw = true;
+      if (lane == 0) {
+        tc::fence_after_sync();
+        for (int ks = 0; ks < ksteps; ++ks)
+          tc::cp_32x128b_warpx4(tmem + kColSfa + s * 8 + ks * 4,
+                                tc::smem_desc(sbase + kOffSfa + (s * 2 + ks) * 512, 16, 128, tc::kSwizzleNone));
+        const int64_t t0 = (int64_t)ti.tile * kTile;
+        for (int j = 0; j < W && okw; ++j) {
+          if (t0 > __ldg(P.qb.tok_pos + tok0 + j)) continue;
+          const int u = (int)(acc_it % kAccUnits);
+          const uint32_t m = (uint32_t)(acc_it / kAccUnits);
+          if (!wait_or_abort(bar_acce + 8 * u, (m & 1) ^ 1, P, abort)) {
+            okw = false;
+            break;
+          }
+          tc::fence_after_sync();
+          for (int ks = 0; ks < ksteps; ++ks) {
+            const uint64_t ad = tc::smem_desc(sbase + kOffA + s * 8192 + ks * 32, 16, sbo, sw);
+            const uint64_t bd = tc::smem_desc(sbase + kOffB + j * 4096 + ks * 32, 16, sbo, sw);
+            tc::mma_mxf4nvf4(tmem + kColAcc + u * 64, ad, bd, idesc, tmem + kColSfa + s * 8 + ks * 4,
+                             tmem + kColSfb + j * 8 + ks * 4, ks > 0 ? 1u : 0u);
+          }
+          tc::commit(bar_accf + 8 * u);
+          ++acc_it;
+        }
+        tc::commit(bar_empty + 8 * s);
+      }
+      acc_it = __shfl_sync(0xffffffffu, acc_it, 0);
+      if (!__shfl_sync(0xffffffffu, (int)okw, 0)) break;
+    }
+    // drain: no MMA or copy of ours in flight at teardown
+    if (lane == 0) {
+      tc::commit(bar_drain);
+      if (!mbar_wait_bounded(bar_drain, drain_n & 1, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int ept = threadIdx.x - 64;  // 0..127
+    TileIter ti;
+    ti.init(P, wb, we);
+    int64_t acc_it = 0;
+    int cur_b = -1, W = 0, tok0 = 0;
+    bool alive = true;
+    for (; ti.valid() && alive; ti.next(P)) {
+      if (ti.b != cur_b) {
+        tc::named_sync(1, 128);
+        cur_b = ti.b;
+        tok0 = __ldg(P.qb.tok_start + cur_b);
+        W = min(__ldg(P.qb.tok_start + cur_b + 1) - tok0, kMaxW);
+        for (int e = ept; e < W * 64; e += 128) {
+          const int j = e / 64, h = e % 64;
+          w_s[e] = h < P.H ? __ldg(P.w + (int64_t)(tok0 + j) * P.H + h) : 0.0f;
+        }
+        tc::named_sync(1, 128);
+      }
+      const int64_t t0 = (int64_t)ti.tile * kTile;
+      for (int j = 0; j < W; ++j) {
+        const int tok = tok0 + j;
+        const int64_t p = __ldg(P.qb.tok_pos + tok);
+        if (t0 > p) continue;
+        const int u = (int)(acc_it % kAccUnits);
+        const uint32_t m = (uint32_t)(acc_it / kAccUnits);
+        bool ok = wait_or_abort(bar_accf + 8 * u, m & 1, P, abort);
+        if (!__all_sync(0xffffffffu, ok)) {
+          alive = false;
+          break;
+        }
+        tc::fence_after_sync();
+        const float* wj = w_s + j * 64;
+        float acc = 0.0f;
+        const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + kColAcc + u * 64;
+        for (int g = 0; g < P.N / 16; ++g) {
+          uint32_t r[16];
+          tc::ld_32x32b_x16(taddr + g * 16, r);
+          tc::ld_wait();
+#pragma unroll
+          for (int k = 0; k < 16; ++k) acc = fmaf(wj[g * 16 + k], fmaxf(__uint_as_float(r[k]), 0.0f), acc);
+        }
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(bar_acce + 8 * u);
+        ++acc_it;
+        const int64_t t = t0 + row;
+        float sc = (t <= p) ? acc : -INFINITY;
+        sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 1));
+        sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 2));
+        sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 4));
+        if ((lane & 7) == 0 && t <= p) P.bscore[(int64_t)tok * P.ld_bs + t / kBlock] = sc;
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace scan_tc
+
+// ---------------------------------------------------------------- host side
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// codes: [n_rows][row_bytes] u8, box {row_bytes, 64}, swizzle = row_bytes
+int make_codes_map(CUtensorMap* m, const uint8_t* codes, int64_t n_rows, int row_bytes) {
+  auto fn = encode_fn();
+  if (!fn) return fail(CSA2_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)n_rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)row_bytes, (cuuint32_t)scan_tc::kChunk};
+  cuuint32_t es[2] = {1, 1};
+  CUtensorMapSwizzle sw = row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CSA2_ERR_CUDA, "cuTensorMapEncodeTiled(codes) failed: %d", (int)r);
+  return CSA2_OK;
+}
+
+// scales: 1-D byte array [n_rows * spr], box of 64 rows
+int make_scales_map(CUtensorMap* m, const uint8_t* scales, int64_t n_rows, int spr) {
+  auto fn = encode_fn();
+  if (!fn) return fail(CSA2_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[1] = {(cuuint64_t)(n_rows * spr)};
+  cuuint64_t strides[1] = {0};
+  cuuint32_t box[1] = {(cuuint32_t)(scan_tc::kChunk * spr)};
+  cuuint32_t es[1] = {1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, const_cast<uint8_t*>(scales), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CSA2_ERR_CUDA, "cuTensorMapEncodeTiled(scales) failed: %d", (int)r);
+  return CSA2_OK;
+}
+
+static int num_sms() {
+  static int n[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (!n[dev]) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    n[dev] = v > 0 ? v : 148;
+  }
+  return n[dev];
+}
+
+int launch_scan_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
+                   const csa2_fp4_cache* kc, float* bs, int64_t ld, cudaStream_t st) {
+  using namespace scan_tc;
+  if (qb->max_q_per_seq > kMaxW) return fail(CSA2_ERR_UNSUPPORTED, "scan: more than %d query tokens per sequence", kMaxW);
+  if (kc->n_rows * (kc->dim / 32) >= (int64_t(1) << 31)) return fail(CSA2_ERR_UNSUPPORTED, "cache too large for TMA");
+  CUtensorMap tmc, tms;
+  if (int rc = make_codes_map(&tmc, kc->codes, kc->n_rows, kc->dim / 2)) return rc;
+  if (int rc = make_scales_map(&tms, kc->scales, kc->n_rows, kc->dim / 32)) return rc;
+  Params p{};
+  p.qb = *qb;
+  p.q_codes = qc;
+  p.q_scales = qs;
+  p.w = w;
+  p.H = H;
+  p.N = (H + 15) / 16 * 16;
+  p.DI = kc->dim;
+  p.n_rows = kc->n_rows;
+  p.page_size = kc->page_size;
+  p.max_pages = kc->max_pages;
+  p.page_table = kc->page_table;
+  p.seq_base = kc->seq_base;
+  p.bscore = bs;
+  p.ld_bs = ld;
+  p.status = status_ptr();
+  p.wait_ns = 1000000000ull;  // 1 s
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    if (int rc = cuda_check(cudaFuncSetAttribute(k_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes),
+                            "scan smem attribute"))
+      return rc;
+    attr_done[dev] = true;
+  }
+  Launch L_("scan_tc", st);
+  k_scan_tc<<<num_sms(), kThreads, kSmemBytes, st>>>(tmc, tms, p);
+  return cuda_check(cudaGetLastError(), "k_scan_tc");
+}
+
+}  // namespace csa2

@@ -108,7 +108,11 @@ def grade_attention(gpu, ref, out_dtype, what=""):
     ulp = 2.0 ** (e - 7)
     d = np.abs(gpu - r16)
     bad = d > ulp * (1 + 1e-9)
-    assert not bad.any(), f"{what}: {int(bad.sum())} outputs beyond 1 bf16 ulp (max {float(d.max())})"
+    if bad.any():
+        i = np.flatnonzero(bad.reshape(-1))[:4]
+        raise AssertionError(f"{what}: {int(bad.sum())} outputs beyond 1 bf16 ulp: gpu {gpu.reshape(-1)[i]} "
+                             f"ref {ref.reshape(-1)[i]} ref_bf16 {r16.reshape(-1)[i]} (out rms "
+                             f"{float(np.sqrt((ref ** 2).mean()))}, max |gpu-ref| {float(np.abs(gpu - ref).max())})")
     return float(d.max()), float(np.abs(gpu - ref).sum() / max(np.abs(ref).sum(), 1e-30))
 
 

@@ -72,8 +72,9 @@ def test_quantize_slot_mapping_and_nonfinite():
     slot = rng.permutation(200)[:100].astype(np.int64)
     codes = torch.full((200, 64), 0xAB, dtype=torch.uint8, device="cuda")
     scales = torch.full((200, 4), 0xAB, dtype=torch.uint8, device="cuda")
-    C.check(C.csa2_quantize_fp4(torch.from_numpy(x).cuda().data_ptr(), 100, 128,
-                                torch.from_numpy(slot).cuda().data_ptr(), codes.data_ptr(), scales.data_ptr(),
+    xd = torch.from_numpy(x).cuda()  # kept alive until the kernel has run
+    sd = torch.from_numpy(slot).cuda()
+    C.check(C.csa2_quantize_fp4(xd.data_ptr(), 100, 128, sd.data_ptr(), codes.data_ptr(), scales.data_ptr(),
                                 _stream()))
     assert _status() == C.CSA2_ERR_NONFINITE
     assert _status() == 0  # cleared
@@ -149,6 +150,7 @@ def test_stack_config1_full_size():
     dict(i=3, B=4, lengths=("uniform8", 2000, 20000)),                     # paged, permuted pages
     dict(i=4, B=2, lengths=("fixed", 20000)),                              # outliers, needles
     dict(i=5, B=6, lengths=("loguniform", 60, 30000)),                     # SWA + W in 1..6, window truncated
+    dict(i=5, B=3, lengths=("list", [7, 200, 5000]), out_dtype="f32"),     # SWA, fp32 output graded strictly
 ])
 def test_stack_small_variants(case):
     case = dict(case)
