@@ -8,7 +8,9 @@ Grading (the workload's stated tolerances):
     k-th best score -- i.e. exact except for swaps across a gap below 1e-5
     relative.
   * attention (fp32 out): max |d| <= 2e-3 and sum|d| / sum|ref| <= 1e-3;
-    (bf16 out): within one bf16 ulp of the oracle rounded to bf16.
+    (bf16 out): within one bf16 ulp of the oracle rounded to bf16, plus an
+    absolute floor of 1e-5 * max|ref| for outputs near zero, where the fp32
+    accumulation's absolute error (not the bf16 rounding) is what remains.
 Downstream steps are graded on the GPU's upstream choice (Reindex on the GPU's
 pool, attention on the GPU's index list), so one near-tie never cascades.
 """
@@ -107,7 +109,7 @@ def grade_attention(gpu, ref, out_dtype, what=""):
     e = np.floor(np.log2(np.maximum(np.abs(r16), 2.0 ** -126)))
     ulp = 2.0 ** (e - 7)
     d = np.abs(gpu - r16)
-    bad = d > ulp * (1 + 1e-9)
+    bad = d > ulp * (1 + 1e-9) + 1e-5 * float(np.abs(ref).max())
     if bad.any():
         i = np.flatnonzero(bad.reshape(-1))[:4]
         raise AssertionError(f"{what}: {int(bad.sum())} outputs beyond 1 bf16 ulp: gpu {gpu.reshape(-1)[i]} "

@@ -92,4 +92,6 @@ def test_host_device_identity():
     sw.dev_rows_e4m3(2, 1000, 130, 136, codes.data_ptr(), scale.data_ptr(), s)
     torch.cuda.synchronize()
     hc, hs = sw.rows_e4m3(2, 1000, 130, ring=136)
-    assert np.array_equal(codes.cpu().numpy(), hc) and np.array_equal(scale.cpu().numpy(), hs)
+    slots = np.arange(1000, 1130) % 136  # slots the 130 positions land in
+    assert np.array_equal(codes.cpu().numpy()[slots], hc[slots])
+    assert np.array_equal(scale.cpu().numpy()[slots], hs[slots])
