@@ -64,6 +64,8 @@ _SIGS = {
     "csa2_attend_reuse": [_P(csa2_query_batch), _vp, _i32, _i32, _P(csa2_fp4_cache), _vp, _vp, _i32,
                           _P(csa2_swa_desc), ctypes.c_float, _vp, _i32, _vp, _vp, ctypes.c_size_t, _vp],
     "csa2_decode_stack": [_P(csa2_stack_desc), _vp, ctypes.c_size_t, _vp],
+    "csa2_index_reindex_noalloc": [_P(csa2_query_batch), _vp, _vp, _vp, _i32, _P(csa2_fp4_cache), _vp, _vp, _i32,
+                                   _i32, _vp, _vp, _vp],
     "csa2_index_workspace_size": [_P(csa2_query_batch), _i32, _i32, _i32, _i32, _P(ctypes.c_size_t)],
     "csa2_attend_workspace_size": [_P(csa2_query_batch), _i32, _i32, _i32, _i32, _P(ctypes.c_size_t)],
     "csa2_stack_workspace_size": [_P(csa2_stack_desc), _P(ctypes.c_size_t)],
@@ -118,6 +120,7 @@ csa2_index_full = _wrap("csa2_index_full")
 csa2_index_reindex = _wrap("csa2_index_reindex")
 csa2_attend_reuse = _wrap("csa2_attend_reuse")
 csa2_decode_stack = _wrap("csa2_decode_stack")
+csa2_index_reindex_noalloc = _wrap("csa2_index_reindex_noalloc")
 csa2_index_workspace_size = _wrap("csa2_index_workspace_size")
 csa2_attend_workspace_size = _wrap("csa2_attend_workspace_size")
 csa2_stack_workspace_size = _wrap("csa2_stack_workspace_size")

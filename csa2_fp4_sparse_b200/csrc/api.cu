@@ -317,6 +317,18 @@ static int check_index_common(const csa2_query_batch* qb, const uint8_t* qc, con
   return CSA2_OK;
 }
 
+}  // extern "C"
+
+namespace csa2 {
+int check_index_args(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H_I,
+                     const csa2_fp4_cache* kc, int P, int K) {
+  return check_index_common(qb, qc, qs, w, H_I, kc, P, K);
+}
+void clear_last_error() { t_err[0] = 0; }
+}  // namespace csa2
+
+extern "C" {
+
 int csa2_index_full(const csa2_query_batch* qb, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
                     int32_t H_I, const csa2_fp4_cache* k_idx, int32_t P, int32_t K, int32_t* pool, int32_t* pool_n,
                     int32_t* idx, int32_t* idx_n, float* blockscore, void* workspace, size_t workspace_bytes,

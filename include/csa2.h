@@ -210,6 +210,27 @@ const char* csa2_last_error(void);
 /* Library version, major*10000 + minor*100 + patch. */
 int csa2_version(void);
 
+/* csa2_index_reindex without a workspace, for callers that cannot allocate
+ * device memory or pass one (for example a serving engine that reserves all
+ * device memory for its KV pool at start-up and forbids later allocations,
+ * or a plug-in interface with no workspace argument).  The method described
+ * on the pages has no counterpart to this call; it computes exactly what
+ * csa2_index_reindex computes, with the same kernels.
+ * Scratch: a fixed file-scope device array of 2^20 fp32 candidate scores
+ * (4 MiB) that every GPU loading the library holds until the process exits;
+ * requires n_tok * P * 8 <= 2^20, else returns CSA2_ERR_WORKSPACE and
+ * launches nothing.  The call allocates nothing (no cudaMalloc, cudaFree or
+ * allocating library routine).  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture.  Every call shares the one
+ * array and leaves its contents behind; each call overwrites every slot it
+ * reads, so nothing needs clearing, but calls that overlap on the GPU (other
+ * streams, other threads) race on the array and must be serialised. */
+int csa2_index_reindex_noalloc(const csa2_query_batch* qb, const uint8_t* q_codes, const uint8_t* q_scales,
+                               const float* w, int32_t H_I, const csa2_fp4_cache* k_idx, const int32_t* pool,
+                               const int32_t* pool_n, int32_t P, int32_t K, int32_t* idx, int32_t* idx_n,
+                               void* stream);
+
 /* Kernel timing (the tracing hook).  While enabled, every kernel the library
  * launches is bracketed by a pair of CUDA events on its stream, aggregated per
  * kernel name.  Off by default; costs two event records per launch when on. */
