@@ -214,6 +214,16 @@ int launch_select(const csa2_query_batch* qb, const float* score, int64_t ld, in
   return cuda_check(cudaGetLastError(), "k_select_topk");
 }
 
+// CSA2_ATTEND_IMPL=simt selects the CUDA-core attention (comparison runs).
+static bool use_attend_tc(int D, int Hq, int q_dtype) {
+  static int env = -1;
+  if (env < 0) {
+    const char* e = getenv("CSA2_ATTEND_IMPL");
+    env = (e && strcmp(e, "simt") == 0) ? 0 : 1;
+  }
+  return env == 1 && attend_tc_supported(D, Hq, q_dtype);
+}
+
 int launch_attend(const csa2_query_batch* qb, const void* q, int q_dtype, int Hq, const csa2_fp4_cache* kv,
                   const int32_t* idx, const int32_t* idx_n, int K, const csa2_swa_desc* swa, float scale, void* out,
                   int out_dtype, float* lse, void* ws, cudaStream_t st) {
@@ -223,6 +233,19 @@ int launch_attend(const csa2_query_batch* qb, const void* q, int q_dtype, int Hq
   Carve c{static_cast<uint8_t*>(ws), ~size_t(0)};
   float* part_o = static_cast<float*>(c.take((size_t)qb->n_tok * ns * Hq * D * 4));
   float* part_ml = static_cast<float*>(c.take((size_t)qb->n_tok * ns * Hq * 2 * 4));
+  if (use_attend_tc(D, Hq, q_dtype)) {
+    // 128-row chunks; small batches spread one token's chunks over several CTAs
+    const int chunks = (K + 127) / 128 + (swa ? (swa->window + 127) / 128 : 0);
+    int nsplit = 1;
+    if (qb->n_tok < 148) nsplit = std::min(chunks, (148 + qb->n_tok - 1) / qb->n_tok);
+    if (int rc = launch_attend_tc(qb, q, q_dtype, Hq, kv, idx, idx_n, K, swa, scale, out, out_dtype, lse, part_o,
+                                  part_ml, nsplit, st))
+      return rc;
+    if (nsplit == 1) return CSA2_OK;
+    Launch L_("merge", st);
+    k_merge<<<dim3(Hq, qb->n_tok), 128, 0, st>>>(part_o, part_ml, nsplit, Hq, D, out, out_dtype, lse);
+    return cuda_check(cudaGetLastError(), "k_merge");
+  }
   csa2_swa_desc sw{};
   if (swa) sw = *swa;
   size_t smem = (size_t)kAttRows * D * 4 + kAttRows * 4;
