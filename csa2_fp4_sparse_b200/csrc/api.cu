@@ -14,6 +14,7 @@
 
 #include "internal.h"
 #include "kernels_simt.cuh"
+#include "select.cuh"
 
 namespace csa2 {
 
@@ -210,7 +211,7 @@ int launch_rescore(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t*
 int launch_select(const csa2_query_batch* qb, const float* score, int64_t ld, int mode, const int32_t* pool,
                   const int32_t* pool_n, int P, int k_out, int32_t* out, int32_t* out_n, cudaStream_t st) {
   Launch L_(mode == 0 ? "select_blocks" : "select_positions", st);
-  k_select_topk<<<qb->n_tok, kSelThreads, 0, st>>>(*qb, score, ld, mode, pool, pool_n, P, k_out, out, out_n);
+  k_select_topk2<<<qb->n_tok, kSel2Threads, 0, st>>>(*qb, score, ld, mode, pool, pool_n, P, k_out, out, out_n);
   return cuda_check(cudaGetLastError(), "k_select_topk");
 }
 

@@ -71,7 +71,8 @@ struct Layout {
   static constexpr uint32_t kOffL = kOffM + HQ * 4;              // running sum [HQ]
   static constexpr uint32_t kOffRs = kOffL + HQ * 4;             // row scale [128] f32
   static constexpr uint32_t kOffValid = kOffRs + kRows * 4;      // row valid [128] i32
-  static constexpr uint32_t kOffMu = kOffValid + kRows * 4;      // max used for this chunk [HQ]
+  static constexpr uint32_t kOffRows = kOffValid + kRows * 4;    // gathered row index [128] i64
+  static constexpr uint32_t kOffMu = kOffRows + kRows * 8;       // max used for this chunk [HQ]
   static constexpr uint32_t kOffCorr = kOffMu + HQ * 4;          // rescale factor [HQ]
   static constexpr uint32_t kOffBar = kOffCorr + HQ * 4;         // 3 mbarriers (S, PV, drain)
   static constexpr uint32_t kOffMisc = kOffBar + 24;             // tmem base, abort, rescale flag
@@ -146,6 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
   float* l_s = reinterpret_cast<float*>(smem + Ly::kOffL);
   float* rs = reinterpret_cast<float*>(smem + Ly::kOffRs);
   int* valid = reinterpret_cast<int*>(smem + Ly::kOffValid);
+  int64_t* rows_s = reinterpret_cast<int64_t*>(smem + Ly::kOffRows);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tok = blockIdx.y, split = blockIdx.x, nsplit = gridDim.x;
@@ -235,82 +237,104 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
     }
     // ---- 1. gather + dequantise the chunk into the K/V tile
     const bool swa_chunk = chunk >= n_sp;
-    if (!swa_chunk) {
-      constexpr int kUnits = D / 32;  // 16-byte code units (32 values, one scale) per row
-      for (int u = threadIdx.x; u < kRows * kUnits; u += kThreads) {
-        const int r = u / kUnits, g = u % kUnits;
+    // row addresses first (one index load per row), so the code loads below
+    // are independent of each other and all in flight together
+    if (threadIdx.x < kRows) {
+      const int r = threadIdx.x;
+      int64_t row = -1;
+      float scale_r = 1.0f;
+      if (!swa_chunk) {
         const int j = chunk * kRows + r;
-        bool ok = false;
-        int64_t row = 0;
         if (j < n_sel) {
           const int32_t t = __ldg(P.idx + (int64_t)tok * P.K + j);
           if (t >= 0 && t <= p) {
             row = cache_row(P.kv, b, t);
-            ok = row >= 0 && row < P.kv.n_rows;
-            if (!ok && g == 0) set_status(P.status, CSA2_ERR_RANGE);
-          } else if (g == 0) {
-            set_status(P.status, CSA2_ERR_RANGE);
+            if (row < 0 || row >= P.kv.n_rows) row = -1;
           }
+          if (row < 0) set_status(P.status, CSA2_ERR_RANGE);
         }
-        uint32_t outw[16];
-        if (ok) {
-          const uint4 cw = __ldg(reinterpret_cast<const uint4*>(P.kv.codes + row * (D / 2)) + g);
-          const uint32_t sb = __ldg(P.kv.scales + row * (D / 32) + g);
-          const __half sh = __float2half_rn(e4m3_to_f32(sb));
-          const __half2 s2 = __halves2half2(sh, sh);
-          const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-#pragma unroll
-            for (int bb = 0; bb < 4; ++bb) {
-              uint32_t h2 = tc::e2m1x2_to_f16x2((words[k] >> (8 * bb)) & 0xFFu);
-              __half2 v = __hmul2(*reinterpret_cast<__half2*>(&h2), s2);
-              outw[k * 4 + bb] = *reinterpret_cast<uint32_t*>(&v);
-            }
+      } else {
+        const int64_t t = w_lo + (int64_t)(chunk - n_sp) * kRows + r;
+        if (t <= p) {
+          row = (int64_t)b * P.swa.cap + t % P.swa.cap;
+          scale_r = __ldg(P.swa.scale + row);
         } else {
-#pragma unroll
-          for (int k = 0; k < 16; ++k) outw[k] = 0;
+          scale_r = 0.0f;
         }
+      }
+      rows_s[r] = row;
+      valid[r] = row >= 0;
+      rs[r] = scale_r;
+    }
+    __syncthreads();
+    if (!swa_chunk) {
+      constexpr int kUnits = D / 32;  // 16-byte code units (32 values, one scale) per row
+      constexpr int kPer = kRows * kUnits / kThreads;
+      uint4 cw[kPer];
+      uint32_t sb[kPer];
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int u = threadIdx.x + i * kThreads;
+        const int r = u / kUnits, g = u % kUnits;
+        const int64_t row = rows_s[r];
+        if (row >= 0) {
+          cw[i] = __ldg(reinterpret_cast<const uint4*>(P.kv.codes + row * (D / 2)) + g);
+          sb[i] = __ldg(P.kv.scales + row * (D / 32) + g);
+        } else {
+          cw[i] = make_uint4(0, 0, 0, 0);
+          sb[i] = 0;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int u = threadIdx.x + i * kThreads;
+        const int r = u / kUnits, g = u % kUnits;
+        const __half sh = __float2half_rn(e4m3_to_f32(sb[i]));
+        const __half2 s2 = __halves2half2(sh, sh);
+        const uint32_t words[4] = {cw[i].x, cw[i].y, cw[i].z, cw[i].w};
+        uint32_t outw[16];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+          for (int bb = 0; bb < 4; ++bb) {
+            uint32_t h2 = tc::e2m1x2_to_f16x2((words[k] >> (8 * bb)) & 0xFFu);
+            __half2 v = __hmul2(*reinterpret_cast<__half2*>(&h2), s2);
+            outw[k * 4 + bb] = *reinterpret_cast<uint32_t*>(&v);
+          }
         // 32 values = d in [32g, 32g+32): d-block g/2, 16-byte chunks (g%2)*4 .. +4
         const int kb = g / 2, c0 = (g % 2) * 4;
 #pragma unroll
         for (int k = 0; k < 4; ++k)
           *reinterpret_cast<uint4*>(smem + Ly::kOffK + kb * (kRows * 128) + swz(r, c0 + k, 128)) =
               make_uint4(outw[4 * k], outw[4 * k + 1], outw[4 * k + 2], outw[4 * k + 3]);
-        if (g == 0) {
-          valid[r] = ok;
-          rs[r] = 1.0f;
-        }
       }
     } else {
       constexpr int kUnits = D / 16;  // 16 FP8 codes per unit
-      const int c_w = chunk - n_sp;
-      for (int u = threadIdx.x; u < kRows * kUnits; u += kThreads) {
+      constexpr int kPer = kRows * kUnits / kThreads;
+      uint4 cw[kPer];
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int u = threadIdx.x + i * kThreads;
         const int r = u / kUnits, g = u % kUnits;
-        const int64_t t = w_lo + (int64_t)c_w * kRows + r;
-        const bool ok = t <= p;
+        const int64_t row = rows_s[r];
+        cw[i] = row >= 0 ? __ldg(reinterpret_cast<const uint4*>(P.swa.codes + row * D) + g) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int u = threadIdx.x + i * kThreads;
+        const int r = u / kUnits, g = u % kUnits;
+        const uint32_t words[4] = {cw[i].x, cw[i].y, cw[i].z, cw[i].w};
         uint32_t outw[8];
-        if (ok) {
-          const int64_t row = (int64_t)b * P.swa.cap + t % P.swa.cap;
-          const uint4 cw = __ldg(reinterpret_cast<const uint4*>(P.swa.codes + row * D) + g);
-          const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            outw[2 * k] = tc::e4m3x2_to_f16x2(words[k] & 0xFFFFu);
-            outw[2 * k + 1] = tc::e4m3x2_to_f16x2(words[k] >> 16);
-          }
-          if (g == 0) rs[r] = __ldg(P.swa.scale + row);
-        } else {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) outw[k] = 0;
-          if (g == 0) rs[r] = 0.0f;
+        for (int k = 0; k < 4; ++k) {
+          outw[2 * k] = tc::e4m3x2_to_f16x2(words[k] & 0xFFFFu);
+          outw[2 * k + 1] = tc::e4m3x2_to_f16x2(words[k] >> 16);
         }
         const int kb = g / 4, c0 = (g % 4) * 2;
 #pragma unroll
         for (int k = 0; k < 2; ++k)
           *reinterpret_cast<uint4*>(smem + Ly::kOffK + kb * (kRows * 128) + swz(r, c0 + k, 128)) =
               make_uint4(outw[4 * k], outw[4 * k + 1], outw[4 * k + 2], outw[4 * k + 3]);
-        if (g == 0) valid[r] = ok;
       }
     }
     tc::fence_proxy_async_smem();
@@ -347,20 +371,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
       const bool rv = valid[r] != 0;
       const float zscale = P.scale * kLog2e * rs[r];  // log2-domain score scale (window rows: * s_t)
       constexpr int kPer = HQ >= 32 ? HQ / 32 : 1;
-      float z[HQ];
+      const uint32_t s_addr = tmem + ((uint32_t)(warp * 32) << 16) + Ly::kColS;
+      // the chunk's scores, scaled to the log2 domain (window rows: * s_t); invalid rows -inf
+      auto load_scores = [&](float (&z)[HQ]) {
 #pragma unroll
-      for (int g = 0; g < HQ / 16; ++g) {
-        uint32_t v[16];
-        tc::ld_32x32b_x16(tmem + ((uint32_t)(warp * 32) << 16) + Ly::kColS + g * 16, v);
-        tc::ld_wait();
+        for (int g = 0; g < HQ / 16; ++g) {
+          uint32_t v[16];
+          tc::ld_32x32b_x16(s_addr + g * 16, v);
+          tc::ld_wait();
 #pragma unroll
-        for (int k = 0; k < 16; ++k) z[g * 16 + k] = rv ? __uint_as_float(v[k]) * zscale : -INFINITY;
-      }
+          for (int k = 0; k < 16; ++k) z[g * 16 + k] = rv ? __uint_as_float(v[k]) * zscale : -INFINITY;
+        }
+      };
       // per-head maximum of this chunk
       {
         float mx[HQ];
-#pragma unroll
-        for (int h = 0; h < HQ; ++h) mx[h] = z[h];
+        load_scores(mx);
         warp_transpose_reduce<HQ, true>(mx, lane);
 #pragma unroll
         for (int i = 0; i < kPer; ++i) red[warp * HQ + reduced_head<HQ>(lane, i)] = mx[i];
@@ -398,6 +424,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
       // z[] is reused for the weights entering the row sum.
       uint8_t* prow = smem + Ly::kOffP;
       const float rsr = rs[r];
+      float z[HQ];
+      load_scores(z);
 #pragma unroll
       for (int c = 0; c < HQ / 8; ++c) {
         uint32_t pk[4];

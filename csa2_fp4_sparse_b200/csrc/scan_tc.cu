@@ -19,9 +19,9 @@
 //               K = 64 per instruction) per query token into a ring of TMEM
 //               accumulators; commits release the smem stage and hand the
 //               accumulator to the epilogue;
-//   warps 2..5  epilogue: TMEM -> registers (one position per thread),
-//               ReLU, weighted head sum, block max over 8 lanes, block-score
-//               store.
+//   warps 2..9  epilogue, two warpgroups taking alternate accumulators:
+//               TMEM -> registers (one position per thread), ReLU, weighted
+//               head sum, block max over 8 lanes, block-score store.
 // The key cache is streamed from HBM exactly once per sequence for all of its
 // query tokens.  All waits are bounded; on timeout the kernel records
 // CSA2_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
@@ -39,7 +39,7 @@ constexpr int kTile = 128;      // positions per tile = MMA M
 constexpr int kChunk = 64;      // rows per TMA box
 constexpr int kAccUnits = 4;    // TMEM accumulator ring, 64 columns each
 constexpr int kMaxW = 8;        // query tokens of one sequence per tile
-constexpr int kThreads = 192;   // 6 warps
+constexpr int kThreads = 320;   // 10 warps: producer, MMA, two epilogue warpgroups
 constexpr uint32_t kColAcc = 0;
 constexpr uint32_t kColSfa = kAccUnits * 64;              // 256
 constexpr uint32_t kColSfb = kColSfa + kStages * 8;      // 320
@@ -51,8 +51,8 @@ constexpr uint32_t kOffRaw = kOffA + kStages * 8192;      // [kStages][512]
 constexpr uint32_t kOffSfa = kOffRaw + kStages * 512;     // [kStages][2][512]
 constexpr uint32_t kOffB = kOffSfa + kStages * 1024;      // [kMaxW][64 rows][64 B]
 constexpr uint32_t kOffSfb = kOffB + kMaxW * 4096;        // [kMaxW][2][512]
-constexpr uint32_t kOffW = kOffSfb + kMaxW * 1024;        // [kMaxW][64] f32
-constexpr uint32_t kOffBar = kOffW + kMaxW * 64 * 4;      // mbarriers
+constexpr uint32_t kOffW = kOffSfb + kMaxW * 1024;        // [2 warpgroups][kMaxW][64] f32
+constexpr uint32_t kOffBar = kOffW + 2 * kMaxW * 64 * 4;  // mbarriers
 constexpr uint32_t kNumBars = 2 * kStages + 2 * kAccUnits + 1;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;     // tmem base, abort flag
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;     // + alignment slack
@@ -340,9 +340,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;
+    const int wg = (warp - 2) / 4;        // warpgroup 0: warps 2..5, 1: warps 6..9
+    const int quarter = warp & 3;         // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
-    const int ept = threadIdx.x - 64;  // 0..127
+    const int ept = threadIdx.x - 64 - wg * 128;  // 0..127 within the warpgroup
+    float* w_g = w_s + wg * kMaxW * 64;
     TileIter ti;
     ti.init(P, wb, we);
     int64_t acc_it = 0;
@@ -350,43 +352,49 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool alive = true;
     for (; ti.valid() && alive; ti.next(P)) {
       if (ti.b != cur_b) {
-        tc::named_sync(1, 128);
+        tc::named_sync(1 + wg, 128);
         cur_b = ti.b;
         tok0 = __ldg(P.qb.tok_start + cur_b);
         W = min(__ldg(P.qb.tok_start + cur_b + 1) - tok0, kMaxW);
         for (int e = ept; e < W * 64; e += 128) {
           const int j = e / 64, h = e % 64;
-          w_s[e] = h < P.H ? __ldg(P.w + (int64_t)(tok0 + j) * P.H + h) : 0.0f;
+          w_g[e] = h < P.H ? __ldg(P.w + (int64_t)(tok0 + j) * P.H + h) : 0.0f;
         }
-        tc::named_sync(1, 128);
+        tc::named_sync(1 + wg, 128);
       }
       const int64_t t0 = (int64_t)ti.tile * kTile;
       for (int j = 0; j < W; ++j) {
         const int tok = tok0 + j;
         const int64_t p = __ldg(P.qb.tok_pos + tok);
         if (t0 > p) continue;
-        const int u = (int)(acc_it % kAccUnits);
-        const uint32_t m = (uint32_t)(acc_it / kAccUnits);
+        const int64_t my = acc_it++;
+        if ((my & 1) != wg) continue;  // the other warpgroup takes this accumulator
+        const int u = (int)(my % kAccUnits);
+        const uint32_t m = (uint32_t)(my / kAccUnits);
         bool ok = wait_or_abort(bar_accf + 8 * u, m & 1, P, abort);
         if (!__all_sync(0xffffffffu, ok)) {
           alive = false;
           break;
         }
         tc::fence_after_sync();
-        const float* wj = w_s + j * 64;
-        float acc = 0.0f;
+        const float* wj = w_g + j * 64;
         const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + kColAcc + u * 64;
-        for (int g = 0; g < P.N / 16; ++g) {
-          uint32_t r[16];
-          tc::ld_32x32b_x16(taddr + g * 16, r);
-          tc::ld_wait();
+        uint32_t r[4][16];
+        const int ng = P.N / 16;
 #pragma unroll
-          for (int k = 0; k < 16; ++k) acc = fmaf(wj[g * 16 + k], fmaxf(__uint_as_float(r[k]), 0.0f), acc);
-        }
+        for (int g = 0; g < 4; ++g)
+          if (g < ng) tc::ld_32x32b_x16(taddr + g * 16, r[g]);
+        tc::ld_wait();
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(bar_acce + 8 * u);
-        ++acc_it;
+        float acc = 0.0f;
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+          if (g < ng) {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) acc = fmaf(wj[g * 16 + k], fmaxf(__uint_as_float(r[g][k]), 0.0f), acc);
+          }
         const int64_t t = t0 + row;
         float sc = (t <= p) ? acc : -INFINITY;
         sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 1));

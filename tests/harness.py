@@ -8,9 +8,11 @@ Grading (the workload's stated tolerances):
     k-th best score -- i.e. exact except for swaps across a gap below 1e-5
     relative.
   * attention (fp32 out): max |d| <= 2e-3 and sum|d| / sum|ref| <= 1e-3;
-    (bf16 out): within one bf16 ulp of the oracle rounded to bf16, plus an
-    absolute floor of 1e-5 * max|ref| for outputs near zero, where the fp32
-    accumulation's absolute error (not the bf16 rounding) is what remains.
+    (bf16 out): the same tolerances with the output's own rounding taken out:
+    max |d| <= 2e-3 + half a bf16 ulp of the value, and
+    sum|gpu - bf16(ref)| / sum|ref| <= 1e-3 (bf16 rounding alone is ~1e-3
+    relative on average, so comparing with the unrounded oracle would grade
+    the format, not the kernel).
 Downstream steps are graded on the GPU's upstream choice (Reindex on the GPU's
 pool, attention on the GPU's index list), so one near-tie never cascades.
 """
@@ -105,17 +107,17 @@ def grade_attention(gpu, ref, out_dtype, what=""):
         assert mrel <= ATT_MEAN_REL, f"{what}: mean rel {mrel}"
         return mx, mrel
     r16 = bf16_round(ref).astype(np.float64)
-    # one bf16 ulp at the rounded reference's magnitude
-    e = np.floor(np.log2(np.maximum(np.abs(r16), 2.0 ** -126)))
-    ulp = 2.0 ** (e - 7)
-    d = np.abs(gpu - r16)
-    bad = d > ulp * (1 + 1e-9) + 1e-5 * float(np.abs(ref).max())
+    e = np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** -126)))
+    half_ulp = 2.0 ** (e - 8)
+    d = np.abs(gpu - ref)
+    bad = d > ATT_MAX_ABS + half_ulp
     if bad.any():
         i = np.flatnonzero(bad.reshape(-1))[:4]
-        raise AssertionError(f"{what}: {int(bad.sum())} outputs beyond 1 bf16 ulp: gpu {gpu.reshape(-1)[i]} "
-                             f"ref {ref.reshape(-1)[i]} ref_bf16 {r16.reshape(-1)[i]} (out rms "
-                             f"{float(np.sqrt((ref ** 2).mean()))}, max |gpu-ref| {float(np.abs(gpu - ref).max())})")
-    return float(d.max()), float(np.abs(gpu - ref).sum() / max(np.abs(ref).sum(), 1e-30))
+        raise AssertionError(f"{what}: {int(bad.sum())} outputs beyond 2e-3 + half ulp: gpu {gpu.reshape(-1)[i]} "
+                             f"ref {ref.reshape(-1)[i]}")
+    mrel = float(np.abs(gpu - r16).sum() / max(np.abs(ref).sum(), 1e-30))
+    assert mrel <= ATT_MEAN_REL, f"{what}: mean rel vs bf16(ref) {mrel}"
+    return float(d.max()), mrel
 
 
 def selector_of(modes, layer):
