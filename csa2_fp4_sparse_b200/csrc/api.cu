@@ -204,6 +204,7 @@ int launch_scan(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs
 int launch_rescore(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
                    const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n, int P, float* scores,
                    cudaStream_t st) {
+  if (use_scan_tc(qb, H)) return launch_rescore_tc(qb, qc, qs, w, H, kc, pool, pool_n, P, scores, st);
   if (kc->dim == 128) return launch_rescore_simt<128>(qb, qc, qs, w, H, kc, pool, pool_n, P, scores, st);
   return launch_rescore_simt<64>(qb, qc, qs, w, H, kc, pool, pool_n, P, scores, st);
 }

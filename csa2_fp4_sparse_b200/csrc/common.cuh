@@ -72,14 +72,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete; gives up after
-// limit_ns and returns false (the caller records CSA2_ERR_TIMEOUT).
+// limit_ns and returns false (the caller records CSA2_ERR_TIMEOUT).  The
+// clock is only read once a long run of probes has failed, so the common,
+// short waits cost nothing but the probes.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = globaltimer_ns();
+  uint64_t t0 = 0;
   while (true) {
-    for (int i = 0; i < 32; ++i)
+    for (int i = 0; i < 1024; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > limit_ns) return false;
+    const uint64_t now = globaltimer_ns();
+    if (t0 == 0)
+      t0 = now;
+    else if (now - t0 > limit_ns)
+      return false;
   }
 }
 

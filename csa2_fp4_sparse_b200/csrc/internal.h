@@ -15,6 +15,9 @@ int* status_ptr();
 int launch_scan_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
                    const csa2_fp4_cache* kc, float* bs, int64_t ld, cudaStream_t st);
 
+int launch_rescore_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
+                      const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n, int P, float* scores,
+                      cudaStream_t st);
 bool attend_tc_supported(int D, int Hq, int q_dtype);
 int launch_attend_tc(const csa2_query_batch* qb, const void* q, int q_dtype, int Hq, const csa2_fp4_cache* kv,
                      const int32_t* idx, const int32_t* idx_n, int K, const csa2_swa_desc* swa, float scale, void* out,

@@ -1,5 +1,7 @@
-// scan_tc.cu -- the Full layer's indexer scan on the 5th-generation tensor
-// cores (sm_100a).
+// scan_tc.cu -- the indexer scoring on the 5th-generation tensor cores
+// (sm_100a): the Full layer's scan of the whole visible context (block scores)
+// and the pool rescoring of the Full layer's own top-K and of every Reindex
+// layer (position scores), one templated kernel.
 //
 // For every query token i of sequence b and visible position t <= p_i:
 //   s_t = sum_h w[i][h] * max(0, q~_{i,h} . k~_t),   B_j = max_{t in block j} s_t
@@ -23,7 +25,9 @@
 //               TMEM -> registers (one position per thread), ReLU, weighted
 //               head sum, block max over 8 lanes, block-score store.
 // The key cache is streamed from HBM exactly once per sequence for all of its
-// query tokens.  All waits are bounded; on timeout the kernel records
+// query tokens.  In rescoring mode the producer instead gathers the 16 pool
+// blocks of a tile (8 rows each, one swizzle atom per block) for one query
+// token, and the epilogue writes one score per pool position.  All waits are bounded; on timeout the kernel records
 // CSA2_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -37,12 +41,12 @@ namespace scan_tc {
 constexpr int kStages = 8;
 constexpr int kTile = 128;      // positions per tile = MMA M
 constexpr int kChunk = 64;      // rows per TMA box
-constexpr int kAccUnits = 4;    // TMEM accumulator ring, 64 columns each
+constexpr int kAccUnits = 6;    // TMEM accumulator ring, 64 columns each
 constexpr int kMaxW = 8;        // query tokens of one sequence per tile
 constexpr int kThreads = 320;   // 10 warps: producer, MMA, two epilogue warpgroups
 constexpr uint32_t kColAcc = 0;
-constexpr uint32_t kColSfa = kAccUnits * 64;              // 256
-constexpr uint32_t kColSfb = kColSfa + kStages * 8;      // 320
+constexpr uint32_t kColSfa = kAccUnits * 64;              // 384
+constexpr uint32_t kColSfb = kColSfa + kStages * 8;      // 448
 constexpr uint32_t kTmemCols = 512;
 
 // shared-memory map (offsets from a 1024-aligned base)
@@ -68,36 +72,65 @@ struct Params {
   int page_size, max_pages;
   const int32_t* page_table;
   const int64_t* seq_base;
-  float* bscore;
-  int64_t ld_bs;
+  float* out;        // scan: block scores [T][ld]; rescore: pool-position scores [T][ld]
+  int64_t ld;
+  const int32_t* pool;   // rescore: [T][pool_cap] block ids
+  const int32_t* pool_n; // rescore: [T]
+  int pool_cap;
   int* status;
   uint64_t wait_ns;
 };
 
-__device__ __forceinline__ int ntiles_of(const Params& P, int b) {
-  return (__ldg(P.qb.seq_len + b) + kTile - 1) / kTile;
+// Work groups: a sequence (scan: all of its query tokens share every tile) or
+// a query token (rescore: its own pool).  Tiles are 128 positions.
+template <bool kRescore>
+__device__ __forceinline__ int n_groups(const Params& P) {
+  return kRescore ? P.qb.n_tok : P.qb.n_seq;
 }
 
-// this CTA's contiguous range of (sequence, tile) work in sequence-major order
+template <bool kRescore>
+__device__ __forceinline__ int group_tiles(const Params& P, int g) {
+  if (kRescore) return (min(__ldg(P.pool_n + g), P.pool_cap) + 15) / 16;
+  return (__ldg(P.qb.seq_len + g) + kTile - 1) / kTile;
+}
+
+// first query token, number of query tokens, sequence of group g
+template <bool kRescore>
+__device__ __forceinline__ void group_info(const Params& P, int g, int* tok0, int* W, int* b) {
+  if (kRescore) {
+    *tok0 = g;
+    *W = 1;
+    *b = __ldg(P.qb.tok_seq + g);
+  } else {
+    *tok0 = __ldg(P.qb.tok_start + g);
+    *W = __ldg(P.qb.tok_start + g + 1) - *tok0;
+    *b = g;
+  }
+}
+
+// this CTA's contiguous range of (group, tile) work in group-major order
+template <bool kRescore>
 __device__ __forceinline__ void work_range(const Params& P, int64_t* begin, int64_t* end) {
   int64_t total = 0;
-  for (int b = 0; b < P.qb.n_seq; ++b) total += ntiles_of(P, b);
+  for (int g = 0; g < n_groups<kRescore>(P); ++g) total += group_tiles<kRescore>(P, g);
   *begin = total * blockIdx.x / gridDim.x;
   *end = total * (blockIdx.x + 1) / gridDim.x;
 }
 
 // iterator over the tiles of [begin, end)
+template <bool kRescore>
 struct TileIter {
-  int b, tile, ntile;
+  int b, tile, ntile;  // b: group
   int64_t left;
   __device__ void init(const Params& P, int64_t begin, int64_t end) {
     b = 0;
     int64_t acc = 0;
-    ntile = ntiles_of(P, 0);
-    while (b < P.qb.n_seq - 1 && acc + ntile <= begin) {
+    const int ng = n_groups<kRescore>(P);
+    ntile = group_tiles<kRescore>(P, 0);
+    while (b < ng - 1 && acc + ntile <= begin) {
       acc += ntile;
       ++b;
-      ntile = ntiles_of(P, b);
+      ntile = group_tiles<kRescore>(P, b);
     }
     tile = (int)(begin - acc);
     left = end - begin;
@@ -106,10 +139,11 @@ struct TileIter {
   __device__ void next(const Params& P) {
     --left;
     if (++tile >= ntile && left > 0) {
+      const int ng = n_groups<kRescore>(P);
       do {
         ++b;
-        ntile = ntiles_of(P, b);
-      } while (ntile == 0 && b < P.qb.n_seq - 1);
+        ntile = group_tiles<kRescore>(P, b);
+      } while (ntile == 0 && b < ng - 1);
       tile = 0;
     }
   }
@@ -123,9 +157,10 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, con
   return false;
 }
 
+template <bool kRescore>
 __global__ void __launch_bounds__(kThreads, 1)
-    k_scan_tc(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales,
-              const Params P) {
+    k_index_tc(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales,
+               const Params P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -166,46 +201,65 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_holder;
 
   int64_t wb, we;
-  work_range(P, &wb, &we);
+  work_range<kRescore>(P, &wb, &we);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      const uint32_t tx = 2u * kChunk * row_bytes + 2u * kChunk * spr;
-      const int32_t oob_row = (int32_t)P.n_rows;
-      const int32_t oob_x = (int32_t)(((P.n_rows * spr) + 15) / 16 * 16);
-      TileIter ti;
-      ti.init(P, wb, we);
-      int64_t it = 0;
-      for (; ti.valid(); ti.next(P), ++it) {
-        const int s = (int)(it % kStages);
-        const uint32_t n = (uint32_t)(it / kStages);
-        if (!wait_or_abort(bar_empty + 8 * s, (n & 1) ^ 1, P, abort)) break;
-        tc::mbar_arrive_expect_tx(bar_full + 8 * s, tx);
-        const int L = __ldg(P.qb.seq_len + ti.b);
-        for (int c = 0; c < 2; ++c) {
-          const int64_t pos0 = (int64_t)ti.tile * kTile + c * kChunk;
-          int64_t row0 = -1;
-          if (pos0 < L) {
-            if (P.page_table) {
-              int32_t pg = __ldg(P.page_table + (int64_t)ti.b * P.max_pages + pos0 / P.page_size);
-              row0 = (int64_t)pg * P.page_size + pos0 % P.page_size;
-            } else {
-              row0 = __ldg(P.seq_base + ti.b) + pos0;
-            }
-          }
-          int32_t ry = oob_row, sx = oob_x;
-          if (row0 >= 0 && row0 < P.n_rows && ((row0 * spr) & 15) == 0) {
-            ry = (int32_t)row0;
-            sx = (int32_t)(row0 * spr);
-          } else if (row0 >= 0) {
-            set_status(P.status, CSA2_ERR_RANGE);  // misplaced row: read as zeros
-          }
-          tc::tma_load_2d(sbase + kOffA + s * 8192 + c * kChunk * row_bytes, &tm_codes, bar_full + 8 * s, 0, ry);
-          tc::tma_load_1d(sbase + kOffRaw + s * 512 + c * kChunk * spr, &tm_scales, bar_full + 8 * s, sx);
-        }
+    const uint32_t tx = (uint32_t)kTile * row_bytes + (uint32_t)kTile * spr;
+    const int32_t oob_row = (int32_t)P.n_rows;
+    const int32_t oob_x = (int32_t)(((P.n_rows * spr) + 15) / 16 * 16);
+    TileIter<kRescore> ti;
+    ti.init(P, wb, we);
+    int64_t it = 0;
+    for (; ti.valid(); ti.next(P), ++it) {
+      const int s = (int)(it % kStages);
+      const uint32_t n = (uint32_t)(it / kStages);
+      bool ok = true;
+      if (lane == 0) {
+        ok = wait_or_abort(bar_empty + 8 * s, (n & 1) ^ 1, P, abort);
+        if (ok) tc::mbar_arrive_expect_tx(bar_full + 8 * s, tx);
       }
-      // no copy of ours may be in flight when the CTA leaves
+      if (!__shfl_sync(0xffffffffu, (int)ok, 0)) break;
+      // each issuing lane loads one box: scan 2 boxes of 64 rows, rescore 16 blocks of 8 rows
+      const int boxes = kRescore ? 16 : 2;
+      const int rows_per_box = kTile / boxes;
+      if (lane < boxes) {
+        int tok0, W, b;
+        group_info<kRescore>(P, ti.b, &tok0, &W, &b);
+        int64_t pos0 = -1;
+        if (kRescore) {
+          const int e = ti.tile * 16 + lane;
+          const int np = min(__ldg(P.pool_n + tok0), P.pool_cap);
+          const int32_t blk = e < np ? __ldg(P.pool + (int64_t)tok0 * P.pool_cap + e) : -1;
+          if (blk >= 0) pos0 = (int64_t)blk * kBlock;
+        } else {
+          pos0 = (int64_t)ti.tile * kTile + lane * kChunk;
+          if (pos0 >= __ldg(P.qb.seq_len + b)) pos0 = -1;
+        }
+        int64_t row0 = -1;
+        if (pos0 >= 0) {
+          if (P.page_table) {
+            const int32_t pg = __ldg(P.page_table + (int64_t)b * P.max_pages + pos0 / P.page_size);
+            row0 = (int64_t)pg * P.page_size + pos0 % P.page_size;
+          } else {
+            row0 = __ldg(P.seq_base + b) + pos0;
+          }
+        }
+        int32_t ry = oob_row, sx = oob_x;
+        if (row0 >= 0 && row0 < P.n_rows && ((row0 * spr) & 15) == 0) {
+          ry = (int32_t)row0;
+          sx = (int32_t)(row0 * spr);
+        } else if (row0 >= 0) {
+          set_status(P.status, CSA2_ERR_RANGE);  // misplaced row: read as zeros
+        }
+        tc::tma_load_2d(sbase + kOffA + s * 8192 + lane * rows_per_box * row_bytes, &tm_codes, bar_full + 8 * s, 0,
+                        ry);
+        tc::tma_load_1d(sbase + kOffRaw + s * 512 + lane * rows_per_box * spr, &tm_scales, bar_full + 8 * s, sx);
+      }
+      __syncwarp();
+    }
+    // no copy of ours may be in flight when the CTA leaves
+    if (lane == 0) {
       for (int s = 0; s < kStages && it > 0; ++s) {
         int64_t uses = it / kStages + (s < it % kStages ? 1 : 0);
         if (uses == 0) continue;
@@ -218,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t idesc = tc::idesc_mxf4nvf4(128, P.N);
     const tc::SmemLayout sw = (P.DI == 128) ? tc::kSwizzle64B : tc::kSwizzle32B;
     const uint32_t sbo = 8u * row_bytes;  // 8 rows per swizzle atom
-    TileIter ti;
+    TileIter<kRescore> ti;
     ti.init(P, wb, we);
     int64_t it = 0, acc_it = 0;
     uint32_t drain_n = 0;
@@ -234,8 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::fence_after_sync();
         }
         cur_b = ti.b;
-        tok0 = __ldg(P.qb.tok_start + cur_b);
-        W = __ldg(P.qb.tok_start + cur_b + 1) - tok0;
+        int bseq;
+        group_info<kRescore>(P, cur_b, &tok0, &W, &bseq);
         if (W > kMaxW) {
           if (lane == 0) set_status(P.status, CSA2_ERR_RANGE);
           W = kMaxW;
@@ -310,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 tc::smem_desc(sbase + kOffSfa + (s * 2 + ks) * 512, 16, 128, tc::kSwizzleNone));
         const int64_t t0 = (int64_t)ti.tile * kTile;
         for (int j = 0; j < W && okw; ++j) {
-          if (t0 > __ldg(P.qb.tok_pos + tok0 + j)) continue;
+          if (!kRescore && t0 > __ldg(P.qb.tok_pos + tok0 + j)) continue;
           const int u = (int)(acc_it % kAccUnits);
           const uint32_t m = (uint32_t)(acc_it / kAccUnits);
           if (!wait_or_abort(bar_acce + 8 * u, (m & 1) ^ 1, P, abort)) {
@@ -345,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = quarter * 32 + lane;
     const int ept = threadIdx.x - 64 - wg * 128;  // 0..127 within the warpgroup
     float* w_g = w_s + wg * kMaxW * 64;
-    TileIter ti;
+    TileIter<kRescore> ti;
     ti.init(P, wb, we);
     int64_t acc_it = 0;
     int cur_b = -1, W = 0, tok0 = 0;
@@ -354,8 +408,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ti.b != cur_b) {
         tc::named_sync(1 + wg, 128);
         cur_b = ti.b;
-        tok0 = __ldg(P.qb.tok_start + cur_b);
-        W = min(__ldg(P.qb.tok_start + cur_b + 1) - tok0, kMaxW);
+        int bseq;
+        group_info<kRescore>(P, cur_b, &tok0, &W, &bseq);
+        W = min(W, kMaxW);
         for (int e = ept; e < W * 64; e += 128) {
           const int j = e / 64, h = e % 64;
           w_g[e] = h < P.H ? __ldg(P.w + (int64_t)(tok0 + j) * P.H + h) : 0.0f;
@@ -366,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < W; ++j) {
         const int tok = tok0 + j;
         const int64_t p = __ldg(P.qb.tok_pos + tok);
-        if (t0 > p) continue;
+        if (!kRescore && t0 > p) continue;
         const int64_t my = acc_it++;
         if ((my & 1) != wg) continue;  // the other warpgroup takes this accumulator
         const int u = (int)(my % kAccUnits);
@@ -395,12 +450,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k = 0; k < 16; ++k) acc = fmaf(wj[g * 16 + k], fmaxf(__uint_as_float(r[g][k]), 0.0f), acc);
           }
-        const int64_t t = t0 + row;
-        float sc = (t <= p) ? acc : -INFINITY;
-        sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 1));
-        sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 2));
-        sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 4));
-        if ((lane & 7) == 0 && t <= p) P.bscore[(int64_t)tok * P.ld_bs + t / kBlock] = sc;
+        if (kRescore) {
+          // pool entry i = tile*128 + row: position pool[i/8]*8 + i%8
+          const int i = ti.tile * kTile + row;
+          const int np = min(__ldg(P.pool_n + tok), P.pool_cap);
+          const int32_t blk = (i / kBlock) < np ? __ldg(P.pool + (int64_t)tok * P.pool_cap + i / kBlock) : -1;
+          const int64_t pos = (int64_t)blk * kBlock + (i % kBlock);
+          if (i < P.pool_cap * kBlock) P.out[(int64_t)tok * P.ld + i] = (blk >= 0 && pos <= p) ? acc : -INFINITY;
+        } else {
+          const int64_t t = t0 + row;
+          float sc = (t <= p) ? acc : -INFINITY;
+          sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 1));
+          sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 2));
+          sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 4));
+          if ((lane & 7) == 0 && t <= p) P.out[(int64_t)tok * P.ld + t / kBlock] = sc;
+        }
       }
     }
   }
@@ -426,13 +490,13 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// codes: [n_rows][row_bytes] u8, box {row_bytes, 64}, swizzle = row_bytes
-int make_codes_map(CUtensorMap* m, const uint8_t* codes, int64_t n_rows, int row_bytes) {
+// codes: [n_rows][row_bytes] u8, box {row_bytes, box_rows}, swizzle = row_bytes
+int make_codes_map(CUtensorMap* m, const uint8_t* codes, int64_t n_rows, int row_bytes, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return fail(CSA2_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)n_rows};
   cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-  cuuint32_t box[2] = {(cuuint32_t)row_bytes, (cuuint32_t)scan_tc::kChunk};
+  cuuint32_t box[2] = {(cuuint32_t)row_bytes, (cuuint32_t)box_rows};
   cuuint32_t es[2] = {1, 1};
   CUtensorMapSwizzle sw = row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, es,
@@ -442,13 +506,13 @@ int make_codes_map(CUtensorMap* m, const uint8_t* codes, int64_t n_rows, int row
   return CSA2_OK;
 }
 
-// scales: 1-D byte array [n_rows * spr], box of 64 rows
-int make_scales_map(CUtensorMap* m, const uint8_t* scales, int64_t n_rows, int spr) {
+// scales: 1-D byte array [n_rows * spr], box of box_rows rows
+int make_scales_map(CUtensorMap* m, const uint8_t* scales, int64_t n_rows, int spr, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return fail(CSA2_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[1] = {(cuuint64_t)(n_rows * spr)};
   cuuint64_t strides[1] = {0};
-  cuuint32_t box[1] = {(cuuint32_t)(scan_tc::kChunk * spr)};
+  cuuint32_t box[1] = {(cuuint32_t)(box_rows * spr)};
   cuuint32_t es[1] = {1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, const_cast<uint8_t*>(scales), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -470,14 +534,18 @@ static int num_sms() {
   return n[dev];
 }
 
-int launch_scan_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
-                   const csa2_fp4_cache* kc, float* bs, int64_t ld, cudaStream_t st) {
+template <bool kRescore>
+static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
+                           const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n, int pool_cap,
+                           float* out, int64_t ld, cudaStream_t st) {
   using namespace scan_tc;
-  if (qb->max_q_per_seq > kMaxW) return fail(CSA2_ERR_UNSUPPORTED, "scan: more than %d query tokens per sequence", kMaxW);
+  if (!kRescore && qb->max_q_per_seq > kMaxW)
+    return fail(CSA2_ERR_UNSUPPORTED, "scan: more than %d query tokens per sequence", kMaxW);
   if (kc->n_rows * (kc->dim / 32) >= (int64_t(1) << 31)) return fail(CSA2_ERR_UNSUPPORTED, "cache too large for TMA");
+  const int box_rows = kRescore ? kBlock : kChunk;
   CUtensorMap tmc, tms;
-  if (int rc = make_codes_map(&tmc, kc->codes, kc->n_rows, kc->dim / 2)) return rc;
-  if (int rc = make_scales_map(&tms, kc->scales, kc->n_rows, kc->dim / 32)) return rc;
+  if (int rc = make_codes_map(&tmc, kc->codes, kc->n_rows, kc->dim / 2, box_rows)) return rc;
+  if (int rc = make_scales_map(&tms, kc->scales, kc->n_rows, kc->dim / 32, box_rows)) return rc;
   Params p{};
   p.qb = *qb;
   p.q_codes = qc;
@@ -491,22 +559,37 @@ int launch_scan_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t*
   p.max_pages = kc->max_pages;
   p.page_table = kc->page_table;
   p.seq_base = kc->seq_base;
-  p.bscore = bs;
-  p.ld_bs = ld;
+  p.out = out;
+  p.ld = ld;
+  p.pool = pool;
+  p.pool_n = pool_n;
+  p.pool_cap = pool_cap;
   p.status = status_ptr();
   p.wait_ns = 1000000000ull;  // 1 s
   static bool attr_done[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-    if (int rc = cuda_check(cudaFuncSetAttribute(k_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes),
-                            "scan smem attribute"))
+    if (int rc = cuda_check(
+            cudaFuncSetAttribute(k_index_tc<kRescore>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes),
+            "index smem attribute"))
       return rc;
     attr_done[dev] = true;
   }
-  Launch L_("scan_tc", st);
-  k_scan_tc<<<num_sms(), kThreads, kSmemBytes, st>>>(tmc, tms, p);
-  return cuda_check(cudaGetLastError(), "k_scan_tc");
+  Launch L_(kRescore ? "rescore_tc" : "scan_tc", st);
+  k_index_tc<kRescore><<<num_sms(), kThreads, kSmemBytes, st>>>(tmc, tms, p);
+  return cuda_check(cudaGetLastError(), "k_index_tc");
+}
+
+int launch_scan_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
+                   const csa2_fp4_cache* kc, float* bs, int64_t ld, cudaStream_t st) {
+  return launch_index_tc<false>(qb, qc, qs, w, H, kc, nullptr, nullptr, 0, bs, ld, st);
+}
+
+int launch_rescore_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
+                      const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n, int P, float* scores,
+                      cudaStream_t st) {
+  return launch_index_tc<true>(qb, qc, qs, w, H, kc, pool, pool_n, P, scores, (int64_t)P * kBlock, st);
 }
 
 }  // namespace csa2

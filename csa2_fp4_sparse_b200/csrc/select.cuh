@@ -86,6 +86,22 @@ __device__ __forceinline__ int32_t sel_id(int mode, int i, const int32_t* pool_r
   return mode == 0 ? i : __ldg(pool_row + i / kBlock) * kBlock + (i % kBlock);
 }
 
+// key of candidate i (0 past the end)
+__device__ __forceinline__ uint32_t key_at(const float* sc, int i, int n) { return i < n ? score_key(sc[i]) : 0u; }
+
+// visit every candidate: f(i, key) for i in [0, n), several loads in flight per thread
+template <typename F>
+__device__ __forceinline__ void for_keys(const float* sc, int n, F&& f) {
+  constexpr int kU = 8;
+  for (int base = 0; base < n; base += kSel2Threads * kU) {
+    uint32_t k[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) k[u] = key_at(sc, base + u * kSel2Threads + threadIdx.x, n);
+#pragma unroll
+    for (int u = 0; u < kU; ++u) f(base + u * kSel2Threads + threadIdx.x, k[u]);
+  }
+}
+
 __global__ void __launch_bounds__(kSel2Threads) k_select_topk2(csa2_query_batch qb, const float* __restrict__ score,
                                                                int64_t ld, int mode, const int32_t* __restrict__ pool,
                                                                const int32_t* __restrict__ pool_n, int P, int k_out,
@@ -107,12 +123,10 @@ __global__ void __launch_bounds__(kSel2Threads) k_select_topk2(csa2_query_batch 
   __syncthreads();
   // pass 1: top byte, and the number of valid candidates
   int nv = 0;
-  for (int base = 0; base < n; base += kSel2Threads) {
-    const int i = base + threadIdx.x;
-    const uint32_t key = i < n ? score_key(sc[i]) : 0u;
+  for_keys(sc, n, [&](int, uint32_t key) {
     nv += key != 0u;
     hist_add(S.hist, key >> 24, key != 0u);
-  }
+  });
   nv = __reduce_add_sync(0xffffffffu, nv);
   if (lane == 0) atomicAdd(&S.n_valid, nv);
   __syncthreads();
@@ -128,22 +142,18 @@ __global__ void __launch_bounds__(kSel2Threads) k_select_topk2(csa2_query_batch 
     for (int i = threadIdx.x; i < 256; i += kSel2Threads) S.hist[i] = 0;
     __syncthreads();
     const uint32_t p1 = S.prefix;
-    for (int base = 0; base < n; base += kSel2Threads) {
-      const int i = base + threadIdx.x;
-      const uint32_t key = i < n ? score_key(sc[i]) : 0u;
+    for_keys(sc, n, [&](int, uint32_t key) {
       hist_add(S.hist, (key >> 16) & 255u, key != 0u && (key >> 24) == (p1 >> 24));
-    }
+    });
     pick_digit(S, 16);
     const uint32_t p2 = S.prefix;
     // pass 3: gather the keys sharing the 16-bit prefix
-    for (int base = 0; base < n; base += kSel2Threads) {
-      const int i = base + threadIdx.x;
-      const uint32_t key = i < n ? score_key(sc[i]) : 0u;
+    for_keys(sc, n, [&](int, uint32_t key) {
       if (key != 0u && (key >> 16) == (p2 >> 16)) {
         const int slot = atomicAdd(&S.cand_n, 1);
         if (slot < kSelCand) S.cand_key[slot] = key;
       }
-    }
+    });
     __syncthreads();
     const int nc = S.cand_n;
     for (int shift = 8; shift >= 0; shift -= 8) {
@@ -158,11 +168,9 @@ __global__ void __launch_bounds__(kSel2Threads) k_select_topk2(csa2_query_batch 
           hist_add(S.hist, (key >> shift) & 255u, i < nc && (key & hi_mask) == (pre & hi_mask));
         }
       } else {
-        for (int base = 0; base < n; base += kSel2Threads) {
-          const int i = base + threadIdx.x;
-          const uint32_t key = i < n ? score_key(sc[i]) : 0u;
+        for_keys(sc, n, [&](int, uint32_t key) {
           hist_add(S.hist, (key >> shift) & 255u, key != 0u && (key & hi_mask) == (pre & hi_mask));
-        }
+        });
       }
       pick_digit(S, shift);
     }
@@ -173,13 +181,18 @@ __global__ void __launch_bounds__(kSel2Threads) k_select_topk2(csa2_query_batch 
   const int span = (n + 31) / 32;
   const int lo = min(n, wid * span), hi = min(n, lo + span);
   int gt = 0, eq = 0;
-  for (int b0 = lo; b0 < hi; b0 += 32) {
-    const int i = b0 + lane;
-    const uint32_t key = i < hi ? score_key(sc[i]) : 0u;
-    const bool g = key != 0u && (take_all || key > T);
-    const bool e = !take_all && key != 0u && key == T;
-    gt += __popc(__ballot_sync(0xffffffffu, g));
-    eq += __popc(__ballot_sync(0xffffffffu, e));
+  for (int b0 = lo; b0 < hi; b0 += 32 * 8) {
+    uint32_t k8[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) k8[u] = key_at(sc, b0 + u * 32 + lane, hi);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint32_t key = k8[u];
+      const bool g = key != 0u && (take_all || key > T);
+      const bool e = !take_all && key != 0u && key == T;
+      gt += __popc(__ballot_sync(0xffffffffu, g));
+      eq += __popc(__ballot_sync(0xffffffffu, e));
+    }
   }
   if (lane == 0) {
     S.wsum[wid] = gt;
@@ -195,18 +208,24 @@ __global__ void __launch_bounds__(kSel2Threads) k_select_topk2(csa2_query_batch 
   for (int w = 0; w < wid; ++w) out_before += S.wsum[w] + S.wsum2[w];
   int32_t* o = out + (int64_t)tok * k_out;
   int written = out_before, eq_taken = 0;
-  for (int b0 = lo; b0 < hi; b0 += 32) {
-    const int i = b0 + lane;
-    const uint32_t key = i < hi ? score_key(sc[i]) : 0u;
-    const bool g = key != 0u && (take_all || key > T);
-    const bool e = !take_all && key != 0u && key == T;
-    const uint32_t em = __ballot_sync(0xffffffffu, e);
-    const int e_rank = __popc(em & ((1u << lane) - 1u));
-    const bool sel = g || (e && eq_taken + e_rank < take_eq);
-    const uint32_t sm = __ballot_sync(0xffffffffu, sel);
-    if (sel) o[written + __popc(sm & ((1u << lane) - 1u))] = sel_id(mode, i, pool_row);
-    written += __popc(sm);
-    eq_taken = min(take_eq, eq_taken + __popc(em));
+  for (int b0 = lo; b0 < hi; b0 += 32 * 8) {
+    uint32_t k8[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) k8[u] = key_at(sc, b0 + u * 32 + lane, hi);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = b0 + u * 32 + lane;
+      const uint32_t key = k8[u];
+      const bool g = key != 0u && (take_all || key > T);
+      const bool e = !take_all && key != 0u && key == T;
+      const uint32_t em = __ballot_sync(0xffffffffu, e);
+      const int e_rank = __popc(em & ((1u << lane) - 1u));
+      const bool sel = g || (e && eq_taken + e_rank < take_eq);
+      const uint32_t sm = __ballot_sync(0xffffffffu, sel);
+      if (sel) o[written + __popc(sm & ((1u << lane) - 1u))] = sel_id(mode, i, pool_row);
+      written += __popc(sm);
+      eq_taken = min(take_eq, eq_taken + __popc(em));
+    }
   }
   __syncthreads();
   for (int j = k_eff + threadIdx.x; j < k_out; j += kSel2Threads) o[j] = -1;
