@@ -51,8 +51,12 @@ constexpr uint32_t kTmemCols = 512;
 
 // shared-memory map (offsets from a 1024-aligned base)
 constexpr uint32_t kOffA = 0;                             // [kStages][8192]
-constexpr uint32_t kOffRaw = kOffA + kStages * 8192;      // [kStages][512]
-constexpr uint32_t kOffSfa = kOffRaw + kStages * 512;     // [kStages][2][512]
+// raw scales: every TMA box gets its own 128-byte-aligned slot (TMA writes
+// shared memory at 128-byte-aligned addresses): scan 2 boxes at 1024-byte
+// slots, rescoring 16 boxes at 128-byte slots
+constexpr uint32_t kRawStage = 2048;
+constexpr uint32_t kOffRaw = kOffA + kStages * 8192;      // [kStages][2048]
+constexpr uint32_t kOffSfa = kOffRaw + kStages * kRawStage;  // [kStages][2][512]
 constexpr uint32_t kOffB = kOffSfa + kStages * 1024;      // [kMaxW][64 rows][64 B]
 constexpr uint32_t kOffSfb = kOffB + kMaxW * 4096;        // [kMaxW][2][512]
 constexpr uint32_t kOffW = kOffSfb + kMaxW * 1024;        // [2 warpgroups][kMaxW][64] f32
@@ -254,7 +258,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc::tma_load_2d(sbase + kOffA + s * 8192 + lane * rows_per_box * row_bytes, &tm_codes, bar_full + 8 * s, 0,
                         ry);
-        tc::tma_load_1d(sbase + kOffRaw + s * 512 + lane * rows_per_box * spr, &tm_scales, bar_full + 8 * s, sx);
+        tc::tma_load_1d(sbase + kOffRaw + s * kRawStage + lane * (kRawStage / boxes), &tm_scales, bar_full + 8 * s,
+                        sx);
       }
       __syncwarp();
     }
@@ -339,13 +344,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, ok)) break;
       // A scale factors: raw [row][spr] -> [m0][m1][k] per K step (each scale twice)
       {
-        const uint8_t* raw = smem + kOffRaw + s * 512;
+        const uint8_t* raw = smem + kOffRaw + s * kRawStage;
+        constexpr int kBoxRows = kRescore ? kBlock : kChunk;
+        constexpr uint32_t kSlot = kRescore ? kRawStage / 16 : kRawStage / 2;
         uint32_t wv[4];
 #pragma unroll
         for (int m1 = 0; m1 < 4; ++m1) {
           const int r = m1 * 32 + lane;
-          wv[m1] = (spr == 4) ? *reinterpret_cast<const uint32_t*>(raw + r * 4)
-                              : (uint32_t)*reinterpret_cast<const uint16_t*>(raw + r * 2);
+          const uint8_t* src = raw + (r / kBoxRows) * kSlot + (r % kBoxRows) * spr;
+          wv[m1] = (spr == 4) ? *reinterpret_cast<const uint32_t*>(src) : (uint32_t)*reinterpret_cast<const uint16_t*>(src);
         }
         for (int ks = 0; ks < ksteps; ++ks) {
           const uint32_t sel = ks == 0 ? 0x1100u : 0x3322u;
