@@ -142,6 +142,7 @@ static size_t attend_ws(const csa2_query_batch* qb, int Hq, int D, int K, const 
   Carve c{nullptr, 0};
   c.take((size_t)qb->n_tok * ns * Hq * D * 4);
   c.take((size_t)qb->n_tok * ns * Hq * 2 * 4);
+  c.take((size_t)qb->n_tok * 4);  // split arrival counters
   return c.used + 256;
 }
 
@@ -235,18 +236,18 @@ int launch_attend(const csa2_query_batch* qb, const void* q, int q_dtype, int Hq
   Carve c{static_cast<uint8_t*>(ws), ~size_t(0)};
   float* part_o = static_cast<float*>(c.take((size_t)qb->n_tok * ns * Hq * D * 4));
   float* part_ml = static_cast<float*>(c.take((size_t)qb->n_tok * ns * Hq * 2 * 4));
+  int* done = static_cast<int*>(c.take((size_t)qb->n_tok * 4));
   if (use_attend_tc(D, Hq, q_dtype)) {
-    // 128-row chunks; small batches spread one token's chunks over several CTAs
+    // 128-row chunks; small batches spread one token's chunks over up to 4 CTAs,
+    // whose partials the last one to finish merges
     const int chunks = (K + 127) / 128 + (swa ? (swa->window + 127) / 128 : 0);
     int nsplit = 1;
-    if (qb->n_tok < 148) nsplit = std::min(chunks, (148 + qb->n_tok - 1) / qb->n_tok);
-    if (int rc = launch_attend_tc(qb, q, q_dtype, Hq, kv, idx, idx_n, K, swa, scale, out, out_dtype, lse, part_o,
-                                  part_ml, nsplit, st))
-      return rc;
-    if (nsplit == 1) return CSA2_OK;
-    Launch L_("merge", st);
-    k_merge<<<dim3(Hq, qb->n_tok), 128, 0, st>>>(part_o, part_ml, nsplit, Hq, D, out, out_dtype, lse);
-    return cuda_check(cudaGetLastError(), "k_merge");
+    if (qb->n_tok < 148) nsplit = std::min(std::min(chunks, 4), (148 + qb->n_tok - 1) / qb->n_tok);
+    if (nsplit > 1) {
+      if (int rc = cuda_check(cudaMemsetAsync(done, 0, (size_t)qb->n_tok * 4, st), "clear split counters")) return rc;
+    }
+    return launch_attend_tc(qb, q, q_dtype, Hq, kv, idx, idx_n, K, swa, scale, out, out_dtype, lse, part_o, part_ml,
+                            done, nsplit, st);
   }
   csa2_swa_desc sw{};
   if (swa) sw = *swa;

@@ -53,6 +53,7 @@ struct Params {
   float* lse;
   float* part_o;   // split mode: [T][S][Hq][D]
   float* part_ml;  // split mode: [T][S][Hq][2] (natural-log max, sum)
+  int* done;       // split mode: [T] arrival counters, zero on entry, left zero on exit
   int* status;
   uint64_t wait_ns;
 };
@@ -171,38 +172,55 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
     m_s[h] = -INFINITY;
     l_s[h] = 0.0f;
   }
-  // query -> fp16 (K-major, 128B swizzle); f32 queries also keep the residual
-  for (int e = threadIdx.x; e < HQ * D / 8; e += kThreads) {
-    const int h = e / (D / 8), c8 = e % (D / 8);  // 8 consecutive d per unit
-    const int kb = c8 / 8, c = c8 % 8;
-    const int64_t off = ((int64_t)tok * HQ + h) * D + c8 * 8;
-    float f[8];
-    if (P.q_f32) {
-      const float4* s4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(P.q) + off);
-      float4 a = __ldg(s4), bb = __ldg(s4 + 1);
-      f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = bb.x; f[5] = bb.y; f[6] = bb.z; f[7] = bb.w;
-    } else {
-      uint4 u = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(P.q) + off));
-      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+  // query -> fp16 (K-major, 128B swizzle); f32 queries also keep the residual.
+  // Loads are issued in batches of 8 independent 16-byte reads per thread.
+  {
+    constexpr int kUnitsQ = HQ * D / 8;  // 8 consecutive d per unit
+    constexpr int kBatch = 8;
+    for (int e0 = 0; e0 < kUnitsQ; e0 += kThreads * kBatch) {
+      float f[kBatch][8];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        f[2 * k] = __uint_as_float(w4[k] << 16);
-        f[2 * k + 1] = __uint_as_float(w4[k] & 0xFFFF0000u);
+      for (int u = 0; u < kBatch; ++u) {
+        const int e = e0 + u * kThreads + threadIdx.x;
+        if (e >= kUnitsQ) continue;
+        const int h = e / (D / 8), c8 = e % (D / 8);
+        const int64_t off = ((int64_t)tok * HQ + h) * D + c8 * 8;
+        if (P.q_f32) {
+          const float4* s4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(P.q) + off);
+          float4 a = __ldg(s4), bb = __ldg(s4 + 1);
+          f[u][0] = a.x; f[u][1] = a.y; f[u][2] = a.z; f[u][3] = a.w;
+          f[u][4] = bb.x; f[u][5] = bb.y; f[u][6] = bb.z; f[u][7] = bb.w;
+        } else {
+          uint4 w4 = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(P.q) + off));
+          const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            f[u][2 * k] = __uint_as_float(ww[k] << 16);
+            f[u][2 * k + 1] = __uint_as_float(ww[k] & 0xFFFF0000u);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int e = e0 + u * kThreads + threadIdx.x;
+        if (e >= kUnitsQ) continue;
+        const int h = e / (D / 8), c8 = e % (D / 8);
+        const int kb = c8 / 8, c = c8 % 8;
+        uint4 hi, lo;
+        uint32_t* hp = &hi.x;
+        uint32_t* lp = &lo.x;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          __half2 h2 = __floats2half2_rn(f[u][2 * k], f[u][2 * k + 1]);
+          hp[k] = *reinterpret_cast<uint32_t*>(&h2);
+          float2 back = __half22float2(h2);
+          lp[k] = pack_half2(f[u][2 * k] - back.x, f[u][2 * k + 1] - back.y);
+        }
+        const uint32_t o = kb * (HQ * 128) + swz(h, c, 128);
+        *reinterpret_cast<uint4*>(smem + Ly::kOffQ + o) = hi;
+        if (QLO) *reinterpret_cast<uint4*>(smem + Ly::kOffQlo + o) = lo;
       }
     }
-    uint4 hi, lo;
-    uint32_t* hp = &hi.x;
-    uint32_t* lp = &lo.x;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      __half2 h2 = __floats2half2_rn(f[2 * k], f[2 * k + 1]);
-      hp[k] = *reinterpret_cast<uint32_t*>(&h2);
-      float2 back = __half22float2(h2);
-      lp[k] = pack_half2(f[2 * k] - back.x, f[2 * k + 1] - back.y);
-    }
-    const uint32_t o = kb * (HQ * 128) + swz(h, c, 128);
-    *reinterpret_cast<uint4*>(smem + Ly::kOffQ + o) = hi;
-    if (QLO) *reinterpret_cast<uint4*>(smem + Ly::kOffQlo + o) = lo;
   }
   tc::fence_proxy_async_smem();
   __syncthreads();
@@ -535,6 +553,51 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
       }
     }
   }
+  // split mode: the last CTA of this token to finish merges the partials
+  // (log-sum-exp weights) and restores the arrival counter to zero
+  if (nsplit > 1) {
+    __shared__ int s_last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(P.done + tok, 1) == nsplit - 1;
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      float* wgt = red;  // [nsplit][HQ] weights, reusing the reduction scratch (nsplit <= 4 here)
+      for (int h = threadIdx.x; h < HQ; h += kThreads) {
+        float M = -INFINITY;
+        for (int sp = 0; sp < nsplit; ++sp) {
+          const float* ml = P.part_ml + (((int64_t)tok * nsplit + sp) * HQ + h) * 2;
+          if (__ldcg(ml + 1) > 0.0f) M = fmaxf(M, __ldcg(ml));
+        }
+        float L = 0.0f;
+        for (int sp = 0; sp < nsplit; ++sp) {
+          const float* ml = P.part_ml + (((int64_t)tok * nsplit + sp) * HQ + h) * 2;
+          const float l = __ldcg(ml + 1);
+          const float a = l > 0.0f ? __expf(__ldcg(ml) - M) : 0.0f;
+          wgt[sp * HQ + h] = a;
+          L += a * l;
+        }
+        const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+        for (int sp = 0; sp < nsplit; ++sp) wgt[sp * HQ + h] *= inv;
+        if (P.lse) P.lse[(int64_t)tok * HQ + h] = L > 0.0f ? M + logf(L) : -INFINITY;
+      }
+      __syncthreads();
+      for (int e = threadIdx.x; e < HQ * D; e += kThreads) {
+        const int h = e / D;
+        float acc = 0.0f;
+#pragma unroll 4
+        for (int sp = 0; sp < nsplit; ++sp)
+          acc += wgt[sp * HQ + h] * __ldcg(P.part_o + ((int64_t)tok * nsplit + sp) * HQ * D + e);
+        const int64_t oi = (int64_t)tok * HQ * D + e;
+        if (P.out_f32)
+          reinterpret_cast<float*>(P.out)[oi] = acc;
+        else
+          reinterpret_cast<__nv_bfloat16*>(P.out)[oi] = __float2bfloat16_rn(acc);
+      }
+      if (threadIdx.x == 0) P.done[tok] = 0;
+    }
+  }
   // no MMA of ours may be in flight when TMEM is released
   if (threadIdx.x == 0) {
     tc::commit(bar_drain);
@@ -577,7 +640,8 @@ bool attend_tc_supported(int D, int Hq, int q_dtype) {
 
 int launch_attend_tc(const csa2_query_batch* qb, const void* q, int q_dtype, int Hq, const csa2_fp4_cache* kv,
                      const int32_t* idx, const int32_t* idx_n, int K, const csa2_swa_desc* swa, float scale, void* out,
-                     int out_dtype, float* lse, float* part_o, float* part_ml, int nsplit, cudaStream_t st) {
+                     int out_dtype, float* lse, float* part_o, float* part_ml, int* done, int nsplit,
+                     cudaStream_t st) {
   using namespace attend_tc;
   Params p{};
   p.qb = *qb;
@@ -597,6 +661,7 @@ int launch_attend_tc(const csa2_query_batch* qb, const void* q, int q_dtype, int
   p.lse = lse;
   p.part_o = part_o;
   p.part_ml = part_ml;
+  p.done = done;
   p.status = status_ptr();
   p.wait_ns = 1000000000ull;
   const int D = kv->dim;

@@ -3,12 +3,13 @@
 //
 //   keys      order-preserving unsigned images of the fp32 scores (score_key);
 //             invalid candidates map to 0 and are never selected
-//   passes 1-2  256-bin histograms of the top two key bytes (shared-memory
-//             atomics aggregated per warp with __match_any_sync), each fixing
-//             one byte of the k-th largest key;
-//   pass 3    candidates that share those 16 bits are gathered into shared
-//             memory (few in practice) and the last two bytes are resolved
-//             there; if they do not fit, two more global passes resolve them;
+//   pass A    range [min, max] and count of the valid scores;
+//   pass B    4096-bin linear histogram over that range (monotone in the
+//             score, so bins are ordered); the bin where the count from the
+//             top reaches k holds the k-th largest score;
+//   pass C    that bin's keys are gathered into shared memory (few in
+//             practice) and its exact k-th key is found by byte-wise radix
+//             steps there (or on global memory if they do not fit);
 //   output    every warp owns a contiguous id range: it counts its selections,
 //             a scan over the 32 warps gives each its output offset, and ties
 //             at the k-th key go to the lowest ids (warp ranges are in id
@@ -102,11 +103,86 @@ __device__ __forceinline__ void for_keys(const float* sc, int n, F&& f) {
   }
 }
 
-__global__ void __launch_bounds__(kSel2Threads) k_select_topk2(csa2_query_batch qb, const float* __restrict__ score,
+// block-wide float min/max and int sum (all threads get the result)
+struct MinMaxCount {
+  float mn, mx;
+  int cnt;
+};
+
+__device__ __forceinline__ MinMaxCount block_minmax_count(MinMaxCount v, float* smf, int* smi) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    v.mn = fminf(v.mn, __shfl_xor_sync(0xffffffffu, v.mn, o));
+    v.mx = fmaxf(v.mx, __shfl_xor_sync(0xffffffffu, v.mx, o));
+    v.cnt += __shfl_xor_sync(0xffffffffu, v.cnt, o);
+  }
+  __syncthreads();
+  if (lane == 0) {
+    smf[wid] = v.mn;
+    smf[32 + wid] = v.mx;
+    smi[wid] = v.cnt;
+  }
+  __syncthreads();
+  MinMaxCount r{smf[0], smf[32], smi[0]};
+  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) {
+    r.mn = fminf(r.mn, smf[w]);
+    r.mx = fmaxf(r.mx, smf[32 + w]);
+    r.cnt += smi[w];
+  }
+  return r;
+}
+
+constexpr int kLinBins = 4096;
+
+struct SelShared2 {
+  int hist[kLinBins];
+  float redf[64];
+  int redi[32];
+  int wsum[32];
+  int wsum2[32];
+  uint32_t cand_key[kSelCand];
+  int cand_n;
+  int bstar, above;
+  uint32_t prefix;
+  int remaining;
+};
+
+// linear bin of a valid score within [mn, mx] (monotone non-decreasing in s)
+__device__ __forceinline__ int lin_bin(float s, float mn, float scale) {
+  int b = (int)__fmul_rn(__fsub_rn(s, mn), scale);
+  return b < 0 ? 0 : (b >= kLinBins ? kLinBins - 1 : b);
+}
+
+// radix step over the shared candidates: fixes the byte at `shift` of the
+// remaining-th largest key among candidates matching S.prefix above it
+__device__ __forceinline__ void cand_radix_step(SelShared2& S, int nc, int shift) {
+  for (int i = threadIdx.x; i < 256; i += kSel2Threads) S.hist[i] = 0;
+  __syncthreads();
+  const uint32_t hi_mask = shift >= 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
+  const uint32_t pre = S.prefix;
+  for (int i = threadIdx.x; i < nc; i += kSel2Threads) {
+    const uint32_t key = S.cand_key[i];
+    if ((key & hi_mask) == (pre & hi_mask)) atomicAdd(&S.hist[(key >> shift) & 255u], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int rem = S.remaining, cum = 0, d = 255;
+    for (; d > 0; --d) {
+      if (cum + S.hist[d] >= rem) break;
+      cum += S.hist[d];
+    }
+    S.prefix = pre | ((uint32_t)d << shift);
+    S.remaining = rem - cum;
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kSel2Threads, 1) k_select_topk2(csa2_query_batch qb, const float* __restrict__ score,
                                                                int64_t ld, int mode, const int32_t* __restrict__ pool,
                                                                const int32_t* __restrict__ pool_n, int P, int k_out,
                                                                int32_t* __restrict__ out, int32_t* __restrict__ out_n) {
-  __shared__ SelShared S;
+  __shared__ SelShared2 S;
   const int tok = blockIdx.x;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int64_t p = __ldg(qb.tok_pos + tok);
@@ -114,65 +190,99 @@ __global__ void __launch_bounds__(kSel2Threads) k_select_topk2(csa2_query_batch 
   const float* sc = score + (int64_t)tok * ld;
   const int32_t* pool_row = pool + (int64_t)tok * P;
 
-  for (int i = threadIdx.x; i < 256; i += kSel2Threads) S.hist[i] = 0;
-  if (threadIdx.x == 0) {
-    S.prefix = 0;
-    S.cand_n = 0;
-    S.n_valid = 0;
-  }
-  __syncthreads();
-  // pass 1: top byte, and the number of valid candidates
-  int nv = 0;
-  for_keys(sc, n, [&](int, uint32_t key) {
-    nv += key != 0u;
-    hist_add(S.hist, key >> 24, key != 0u);
+  // pass A: range and count of the valid scores
+  MinMaxCount v{INFINITY, -INFINITY, 0};
+  for_keys(sc, n, [&](int i, uint32_t key) {
+    if (key != 0u) {
+      const float f = sc[i];
+      v.mn = fminf(v.mn, f);
+      v.mx = fmaxf(v.mx, f);
+      v.cnt += 1;
+    }
   });
-  nv = __reduce_add_sync(0xffffffffu, nv);
-  if (lane == 0) atomicAdd(&S.n_valid, nv);
-  __syncthreads();
-  const int n_valid = S.n_valid;
+  const MinMaxCount r = block_minmax_count(v, S.redf, S.redi);
+  const int n_valid = r.cnt;
   const int k_eff = min(k_out, n_valid);
   const bool take_all = k_eff == n_valid;
   uint32_t T = 0;
   int need_eq = 0;
-  if (!take_all) {
-    if (threadIdx.x == 0) S.remaining = k_eff;
-    pick_digit(S, 24);
-    // pass 2: second byte among keys with the chosen top byte
-    for (int i = threadIdx.x; i < 256; i += kSel2Threads) S.hist[i] = 0;
+  if (!take_all && r.mx == r.mn) {
+    T = score_key(r.mx);  // every valid score ties: the lowest ids win
+    need_eq = k_eff;
+  } else if (!take_all) {
+    // pass B: linear histogram over [mn, mx]
+    const float mn = r.mn, scale = (float)kLinBins / (r.mx - r.mn);
+    for (int i = threadIdx.x; i < kLinBins; i += kSel2Threads) S.hist[i] = 0;
     __syncthreads();
-    const uint32_t p1 = S.prefix;
-    for_keys(sc, n, [&](int, uint32_t key) {
-      hist_add(S.hist, (key >> 16) & 255u, key != 0u && (key >> 24) == (p1 >> 24));
+    for_keys(sc, n, [&](int i, uint32_t key) {
+      if (key != 0u) atomicAdd(&S.hist[lin_bin(sc[i], mn, scale)], 1);
     });
-    pick_digit(S, 16);
-    const uint32_t p2 = S.prefix;
-    // pass 3: gather the keys sharing the 16-bit prefix
-    for_keys(sc, n, [&](int, uint32_t key) {
-      if (key != 0u && (key >> 16) == (p2 >> 16)) {
+    __syncthreads();
+    // threshold bin: suffix sums from the top, 4 bins per thread
+    {
+      constexpr int kPerT = kLinBins / kSel2Threads;
+      const int hb = kLinBins - 1 - threadIdx.x * kPerT;  // this thread's highest bin
+      int c[kPerT], tot = 0;
+#pragma unroll
+      for (int j = 0; j < kPerT; ++j) {
+        c[j] = S.hist[hb - j];
+        tot += c[j];
+      }
+      int total;
+      const int before = block_exclusive_scan(tot, S.wsum, &total);
+      int cum = before;
+#pragma unroll
+      for (int j = 0; j < kPerT; ++j) {
+        if (cum < k_eff && cum + c[j] >= k_eff) {
+          S.bstar = hb - j;
+          S.above = cum;
+        }
+        cum += c[j];
+      }
+    }
+    __syncthreads();
+    const int bstar = S.bstar;
+    // pass C: gather the keys of the threshold bin
+    if (threadIdx.x == 0) S.cand_n = 0;
+    __syncthreads();
+    for_keys(sc, n, [&](int i, uint32_t key) {
+      if (key != 0u && lin_bin(sc[i], mn, scale) == bstar) {
         const int slot = atomicAdd(&S.cand_n, 1);
         if (slot < kSelCand) S.cand_key[slot] = key;
       }
     });
     __syncthreads();
     const int nc = S.cand_n;
-    for (int shift = 8; shift >= 0; shift -= 8) {
-      for (int i = threadIdx.x; i < 256; i += kSel2Threads) S.hist[i] = 0;
-      __syncthreads();
-      const uint32_t pre = S.prefix;
-      const uint32_t hi_mask = 0xFFFFFFFFu << (shift + 8);
-      if (nc <= kSelCand) {
-        for (int base = 0; base < nc; base += kSel2Threads) {
-          const int i = base + threadIdx.x;
-          const uint32_t key = i < nc ? S.cand_key[i] : 0u;
-          hist_add(S.hist, (key >> shift) & 255u, i < nc && (key & hi_mask) == (pre & hi_mask));
-        }
-      } else {
-        for_keys(sc, n, [&](int, uint32_t key) {
-          hist_add(S.hist, (key >> shift) & 255u, key != 0u && (key & hi_mask) == (pre & hi_mask));
+    if (threadIdx.x == 0) {
+      S.prefix = 0;
+      S.remaining = k_eff - S.above;
+    }
+    __syncthreads();
+    if (nc <= kSelCand) {
+      for (int shift = 24; shift >= 0; shift -= 8) cand_radix_step(S, nc, shift);
+    } else {
+      // more threshold-bin members than fit: resolve the bytes on global memory
+      for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int i = threadIdx.x; i < 256; i += kSel2Threads) S.hist[i] = 0;
+        __syncthreads();
+        const uint32_t hi_mask = shift >= 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
+        const uint32_t pre = S.prefix;
+        for_keys(sc, n, [&](int i, uint32_t key) {
+          if (key != 0u && lin_bin(sc[i], mn, scale) == bstar && (key & hi_mask) == (pre & hi_mask))
+            atomicAdd(&S.hist[(key >> shift) & 255u], 1);
         });
+        __syncthreads();
+        if (threadIdx.x == 0) {
+          int rem = S.remaining, cum = 0, d = 255;
+          for (; d > 0; --d) {
+            if (cum + S.hist[d] >= rem) break;
+            cum += S.hist[d];
+          }
+          S.prefix = pre | ((uint32_t)d << shift);
+          S.remaining = rem - cum;
+        }
+        __syncthreads();
       }
-      pick_digit(S, shift);
     }
     T = S.prefix;
     need_eq = S.remaining;
