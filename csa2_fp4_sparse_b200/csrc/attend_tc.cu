@@ -583,17 +583,44 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
         if (P.lse) P.lse[(int64_t)tok * HQ + h] = L > 0.0f ? M + logf(L) : -INFINITY;
       }
       __syncthreads();
-      for (int e = threadIdx.x; e < HQ * D; e += kThreads) {
-        const int h = e / D;
-        float acc = 0.0f;
-#pragma unroll 4
-        for (int sp = 0; sp < nsplit; ++sp)
-          acc += wgt[sp * HQ + h] * __ldcg(P.part_o + ((int64_t)tok * nsplit + sp) * HQ * D + e);
-        const int64_t oi = (int64_t)tok * HQ * D + e;
-        if (P.out_f32)
-          reinterpret_cast<float*>(P.out)[oi] = acc;
-        else
-          reinterpret_cast<__nv_bfloat16*>(P.out)[oi] = __float2bfloat16_rn(acc);
+      // 16-byte loads, all splits of 4 groups in flight per thread (nsplit <= 4)
+      constexpr int kTot4 = HQ * D / 4;
+      const float4* po = reinterpret_cast<const float4*>(P.part_o) + (int64_t)tok * nsplit * kTot4;
+      for (int e0 = threadIdx.x; e0 < kTot4; e0 += kThreads * 4) {
+        float4 v[4][4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int sp = 0; sp < 4; ++sp) {
+            const int e = e0 + u * kThreads;
+            v[u][sp] = (sp < nsplit && e < kTot4) ? __ldcg(po + (int64_t)sp * kTot4 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = e0 + u * kThreads;
+          if (e >= kTot4) continue;
+          const int h = (e * 4) / D;
+          float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int sp = 0; sp < 4; ++sp) {
+            if (sp >= nsplit) continue;
+            const float wv = wgt[sp * HQ + h];
+            a.x += wv * v[u][sp].x;
+            a.y += wv * v[u][sp].y;
+            a.z += wv * v[u][sp].z;
+            a.w += wv * v[u][sp].w;
+          }
+          const int64_t oi = (int64_t)tok * HQ * D + (int64_t)e * 4;
+          if (P.out_f32) {
+            *reinterpret_cast<float4*>(reinterpret_cast<float*>(P.out) + oi) = a;
+          } else {
+            __nv_bfloat162 lo2 = __floats2bfloat162_rn(a.x, a.y), hi2 = __floats2bfloat162_rn(a.z, a.w);
+            uint2 pk;
+            pk.x = *reinterpret_cast<uint32_t*>(&lo2);
+            pk.y = *reinterpret_cast<uint32_t*>(&hi2);
+            *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(P.out) + oi) = pk;
+          }
+        }
       }
       if (threadIdx.x == 0) P.done[tok] = 0;
     }

@@ -13,10 +13,12 @@
 //   warp 0      TMA producer: tiles of 128 positions of the FP4 indexer K cache
 //               (codes with the 64B/32B swizzle the MMA expects, plus the raw
 //               E4M3 scales) into an 8-stage shared-memory ring;
-//   warp 1      MMA issuer: rearranges the tile's scales into the tensor-core
-//               scale-factor layout (each per-32 E4M3 scale written twice, as
-//               the block-scaled MMA takes one UE4M3 scale per 16 elements),
-//               copies them to TMEM (tcgen05.cp), and issues
+//   warp 10     scale-factor warp: rearranges each landed tile's scales into
+//               the tensor-core scale-factor layout (each per-32 E4M3 scale
+//               written twice, as the block-scaled MMA takes one UE4M3 scale
+//               per 16 elements) and hands the stage to the MMA warp;
+//   warp 1      MMA issuer: copies the scale factors to TMEM (tcgen05.cp) and
+//               issues
 //               tcgen05.mma kind::mxf4nvf4 (M = 128 positions, N = heads,
 //               K = 64 per instruction) per query token into a ring of TMEM
 //               accumulators; commits release the smem stage and hand the
@@ -43,7 +45,8 @@ constexpr int kTile = 128;      // positions per tile = MMA M
 constexpr int kChunk = 64;      // rows per TMA box
 constexpr int kAccUnits = 6;    // TMEM accumulator ring, 64 columns each
 constexpr int kMaxW = 8;        // query tokens of one sequence per tile
-constexpr int kThreads = 320;   // 10 warps: producer, MMA, two epilogue warpgroups
+constexpr int kThreads = 352;   // 11 warps: producer, MMA, two epilogue warpgroups, scale-factor warp
+constexpr int kSfWarp = 10;
 constexpr uint32_t kColAcc = 0;
 constexpr uint32_t kColSfa = kAccUnits * 64;              // 384
 constexpr uint32_t kColSfb = kColSfa + kStages * 8;      // 448
@@ -60,8 +63,9 @@ constexpr uint32_t kOffSfa = kOffRaw + kStages * kRawStage;  // [kStages][2][512
 constexpr uint32_t kOffB = kOffSfa + kStages * 1024;      // [kMaxW][64 rows][64 B]
 constexpr uint32_t kOffSfb = kOffB + kMaxW * 4096;        // [kMaxW][2][512]
 constexpr uint32_t kOffW = kOffSfb + kMaxW * 1024;        // [2 warpgroups][kMaxW][64] f32
-constexpr uint32_t kOffBar = kOffW + 2 * kMaxW * 64 * 4;  // mbarriers
-constexpr uint32_t kNumBars = 2 * kStages + 2 * kAccUnits + 1;
+constexpr uint32_t kOffPos = kOffW + 2 * kMaxW * 64 * 4;  // [3][kMaxW] i64 query positions (MMA warp, 2 epilogue warpgroups)
+constexpr uint32_t kOffBar = kOffPos + 3 * kMaxW * 8;     // mbarriers
+constexpr uint32_t kNumBars = 3 * kStages + 2 * kAccUnits + 1;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;     // tmem base, abort flag
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;     // + alignment slack
 static_assert(kOffB % 1024 == 0, "B tiles must be 1024-aligned");
@@ -173,6 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_accf = bar_empty + kStages * 8;
   const uint32_t bar_acce = bar_accf + kAccUnits * 8;
   const uint32_t bar_drain = bar_acce + kAccUnits * 8;
+  const uint32_t bar_sfr = bar_drain + 8;
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(smem + kOffMisc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   float* w_s = reinterpret_cast<float*>(smem + kOffW);
@@ -190,6 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_acce + 8 * i, 4);
     }
     mbar_init(bar_drain, 1);
+    for (int i = 0; i < kStages; ++i) mbar_init(bar_sfr + 8 * i, 1);
     *abort = 0;
     tc::fence_barrier_init();
     tc::tma_prefetch_desc(&tm_codes);
@@ -299,6 +305,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) set_status(P.status, CSA2_ERR_RANGE);
           W = kMaxW;
         }
+        int64_t* pos_s = reinterpret_cast<int64_t*>(smem + kOffPos);
+        if (lane < W) pos_s[lane] = __ldg(P.qb.tok_pos + tok0 + lane);
         // B operand: query codes, swizzled like the TMA-written A tiles
         const int chunks_per_row = row_bytes / 16;
         for (int e = lane; e < W * 64 * chunks_per_row; e += 32) {
@@ -340,38 +348,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int s = (int)(it % kStages);
       const uint32_t n = (uint32_t)(it / kStages);
-      bool ok = wait_or_abort(bar_full + 8 * s, n & 1, P, abort);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      // A scale factors: raw [row][spr] -> [m0][m1][k] per K step (each scale twice)
-      {
-        const uint8_t* raw = smem + kOffRaw + s * kRawStage;
-        constexpr int kBoxRows = kRescore ? kBlock : kChunk;
-        constexpr uint32_t kSlot = kRescore ? kRawStage / 16 : kRawStage / 2;
-        uint32_t wv[4];
-#pragma unroll
-        for (int m1 = 0; m1 < 4; ++m1) {
-          const int r = m1 * 32 + lane;
-          const uint8_t* src = raw + (r / kBoxRows) * kSlot + (r % kBoxRows) * spr;
-          wv[m1] = (spr == 4) ? *reinterpret_cast<const uint32_t*>(src) : (uint32_t)*reinterpret_cast<const uint16_t*>(src);
-        }
-        for (int ks = 0; ks < ksteps; ++ks) {
-          const uint32_t sel = ks == 0 ? 0x1100u : 0x3322u;
-          *reinterpret_cast<uint4*>(smem + kOffSfa + (s * 2 + ks) * 512 + lane * 16) =
-              make_uint4(__byte_perm(wv[0], 0, sel), __byte_perm(wv[1], 0, sel), __byte_perm(wv[2], 0, sel),
-                         __byte_perm(wv[3], 0, sel));
-        }
-      }
-      tc::fence_proxy_async_smem();
-      __syncwarp();
       bool okw = true;
       if (lane == 0) {
+        okw = wait_or_abort(bar_sfr + 8 * s, n & 1, P, abort);  // tile landed, scale factors laid out
         tc::fence_after_sync();
-        for (int ks = 0; ks < ksteps; ++ks)
+        const int64_t* pos_s = reinterpret_cast<const int64_t*>(smem + kOffPos);
+        for (int ks = 0; ks < ksteps && okw; ++ks)
           tc::cp_32x128b_warpx4(tmem + kColSfa + s * 8 + ks * 4,
                                 tc::smem_desc(sbase + kOffSfa + (s * 2 + ks) * 512, 16, 128, tc::kSwizzleNone));
         const int64_t t0 = (int64_t)ti.tile * kTile;
         for (int j = 0; j < W && okw; ++j) {
-          if (!kRescore && t0 > __ldg(P.qb.tok_pos + tok0 + j)) continue;
+          if (!kRescore && t0 > pos_s[j]) continue;
           const int u = (int)(acc_it % kAccUnits);
           const uint32_t m = (uint32_t)(acc_it / kAccUnits);
           if (!wait_or_abort(bar_acce + 8 * u, (m & 1) ^ 1, P, abort)) {
@@ -388,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::commit(bar_accf + 8 * u);
           ++acc_it;
         }
-        tc::commit(bar_empty + 8 * s);
+        if (okw) tc::commit(bar_empty + 8 * s);
       }
       acc_it = __shfl_sync(0xffffffffu, acc_it, 0);
       if (!__shfl_sync(0xffffffffu, (int)okw, 0)) break;
@@ -399,6 +386,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait_bounded(bar_drain, drain_n & 1, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
     }
     __syncwarp();
+  } else if (warp == kSfWarp) {
+    // ------------------------------------------------------------ scale factors
+    // raw [row][spr] -> [m0 (32)][m1 (4)][k (4)] per 64-element K step, each
+    // per-32 scale written twice (the MMA takes one scale per 16 elements)
+    TileIter<kRescore> ti;
+    ti.init(P, wb, we);
+    int64_t it = 0;
+    constexpr int kBoxRows = kRescore ? kBlock : kChunk;
+    constexpr uint32_t kSlot = kRescore ? kRawStage / 16 : kRawStage / 2;
+    for (; ti.valid(); ti.next(P), ++it) {
+      const int s = (int)(it % kStages);
+      const uint32_t n = (uint32_t)(it / kStages);
+      bool ok = wait_or_abort(bar_full + 8 * s, n & 1, P, abort);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const uint8_t* raw = smem + kOffRaw + s * kRawStage;
+      uint32_t wv[4];
+#pragma unroll
+      for (int m1 = 0; m1 < 4; ++m1) {
+        const int r = m1 * 32 + lane;
+        const uint8_t* src = raw + (r / kBoxRows) * kSlot + (r % kBoxRows) * spr;
+        wv[m1] = (spr == 4) ? *reinterpret_cast<const uint32_t*>(src) : (uint32_t)*reinterpret_cast<const uint16_t*>(src);
+      }
+      for (int ks = 0; ks < ksteps; ++ks) {
+        const uint32_t sel = ks == 0 ? 0x1100u : 0x3322u;
+        *reinterpret_cast<uint4*>(smem + kOffSfa + (s * 2 + ks) * 512 + lane * 16) =
+            make_uint4(__byte_perm(wv[0], 0, sel), __byte_perm(wv[1], 0, sel), __byte_perm(wv[2], 0, sel),
+                       __byte_perm(wv[3], 0, sel));
+      }
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar_sfr + 8 * s);
+    }
   } else {
     // ------------------------------------------------------------ epilogue
     const int wg = (warp - 2) / 4;        // warpgroup 0: warps 2..5, 1: warps 6..9
@@ -406,6 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = quarter * 32 + lane;
     const int ept = threadIdx.x - 64 - wg * 128;  // 0..127 within the warpgroup
     float* w_g = w_s + wg * kMaxW * 64;
+    int64_t* pos_g = reinterpret_cast<int64_t*>(smem + kOffPos) + (1 + wg) * kMaxW;
     TileIter<kRescore> ti;
     ti.init(P, wb, we);
     int64_t acc_it = 0;
@@ -422,12 +442,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int j = e / 64, h = e % 64;
           w_g[e] = h < P.H ? __ldg(P.w + (int64_t)(tok0 + j) * P.H + h) : 0.0f;
         }
+        if (ept < W) pos_g[ept] = __ldg(P.qb.tok_pos + tok0 + ept);
         tc::named_sync(1 + wg, 128);
       }
       const int64_t t0 = (int64_t)ti.tile * kTile;
       for (int j = 0; j < W; ++j) {
         const int tok = tok0 + j;
-        const int64_t p = __ldg(P.qb.tok_pos + tok);
+        const int64_t p = pos_g[j];
         if (!kRescore && t0 > p) continue;
         const int64_t my = acc_it++;
         if ((my & 1) != wg) continue;  // the other warpgroup takes this accumulator

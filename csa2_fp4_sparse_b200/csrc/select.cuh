@@ -154,6 +154,44 @@ __device__ __forceinline__ int lin_bin(float s, float mn, float scale) {
   return b < 0 ? 0 : (b >= kLinBins ? kLinBins - 1 : b);
 }
 
+// warp 0: the byte where the count from the top of hist[256] reaches *remaining;
+// updates *prefix and *remaining (callers synchronise around it)
+__device__ __forceinline__ void warp_pick_byte(const int* hist, uint32_t* prefix, int* remaining, int shift) {
+  const int lane = threadIdx.x & 31;
+  int c[8], tot = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    c[i] = hist[255 - (lane * 8 + i)];
+    tot += c[i];
+  }
+  int incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  int before = incl - tot;
+  const int rem = *remaining;
+  int found = -1, above = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (found < 0 && before + c[i] >= rem) {
+      found = 255 - (lane * 8 + i);
+      above = before;
+    }
+    before += c[i];
+  }
+  const uint32_t mask = __ballot_sync(0xffffffffu, found >= 0);
+  const int src = mask ? __ffs(mask) - 1 : 31;
+  found = __shfl_sync(0xffffffffu, found, src);
+  above = __shfl_sync(0xffffffffu, above, src);
+  if (found < 0) found = 0;
+  if (lane == 0) {
+    *prefix |= (uint32_t)found << shift;
+    *remaining = rem - above;
+  }
+}
+
 // radix step over the shared candidates: fixes the byte at `shift` of the
 // remaining-th largest key among candidates matching S.prefix above it
 __device__ __forceinline__ void cand_radix_step(SelShared2& S, int nc, int shift) {
@@ -166,15 +204,7 @@ __device__ __forceinline__ void cand_radix_step(SelShared2& S, int nc, int shift
     if ((key & hi_mask) == (pre & hi_mask)) atomicAdd(&S.hist[(key >> shift) & 255u], 1);
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int rem = S.remaining, cum = 0, d = 255;
-    for (; d > 0; --d) {
-      if (cum + S.hist[d] >= rem) break;
-      cum += S.hist[d];
-    }
-    S.prefix = pre | ((uint32_t)d << shift);
-    S.remaining = rem - cum;
-  }
+  if (threadIdx.x < 32) warp_pick_byte(S.hist, &S.prefix, &S.remaining, shift);
   __syncthreads();
 }
 
@@ -272,15 +302,7 @@ __global__ void __launch_bounds__(kSel2Threads, 1) k_select_topk2(csa2_query_bat
             atomicAdd(&S.hist[(key >> shift) & 255u], 1);
         });
         __syncthreads();
-        if (threadIdx.x == 0) {
-          int rem = S.remaining, cum = 0, d = 255;
-          for (; d > 0; --d) {
-            if (cum + S.hist[d] >= rem) break;
-            cum += S.hist[d];
-          }
-          S.prefix = pre | ((uint32_t)d << shift);
-          S.remaining = rem - cum;
-        }
+        if (threadIdx.x < 32) warp_pick_byte(S.hist, &S.prefix, &S.remaining, shift);
         __syncthreads();
       }
     }
@@ -309,13 +331,21 @@ __global__ void __launch_bounds__(kSel2Threads, 1) k_select_topk2(csa2_query_bat
     S.wsum2[wid] = eq;
   }
   __syncthreads();
-  int eq_before = 0, out_before = 0;
-  for (int w = 0; w < wid; ++w) eq_before += S.wsum2[w];
+  // exclusive prefix over the 32 warps (each lane of a warp reads one warp's sum)
+  int eq_before = __shfl_sync(0xffffffffu, 0, 0);
+  {
+    const int v = lane < wid ? S.wsum2[lane] : 0;
+    eq_before = __reduce_add_sync(0xffffffffu, v);
+  }
   const int take_eq = max(0, min(eq, need_eq - eq_before));
   __syncthreads();
   if (lane == 0) S.wsum2[wid] = take_eq;
   __syncthreads();
-  for (int w = 0; w < wid; ++w) out_before += S.wsum[w] + S.wsum2[w];
+  int out_before;
+  {
+    const int v = lane < wid ? S.wsum[lane] + S.wsum2[lane] : 0;
+    out_before = __reduce_add_sync(0xffffffffu, v);
+  }
   int32_t* o = out + (int64_t)tok * k_out;
   int written = out_before, eq_taken = 0;
   for (int b0 = lo; b0 < hi; b0 += 32 * 8) {
