@@ -16,10 +16,10 @@
 //   warp 10     scale-factor warp: rearranges each landed tile's scales into
 //               the tensor-core scale-factor layout (each per-32 E4M3 scale
 //               written twice, as the block-scaled MMA takes one UE4M3 scale
-//               per 16 elements) and hands the stage to the MMA warp;
-//   warp 1      MMA issuer: copies the scale factors to TMEM (tcgen05.cp) and
-//               issues
-//               tcgen05.mma kind::mxf4nvf4 (M = 128 positions, N = heads,
+//               per 16 elements) and copies them to TMEM (tcgen05.cp); a
+//               commit hands the stage to the MMA warp, so the copy never
+//               queues behind that warp's earlier MMAs;
+//   warp 1      MMA issuer: issues tcgen05.mma kind::mxf4nvf4 (M = 128 positions, N = heads,
 //               K = 64 per instruction) per query token into a ring of TMEM
 //               accumulators; commits release the smem stage and hand the
 //               accumulator to the epilogue;
@@ -65,7 +65,7 @@ constexpr uint32_t kOffSfb = kOffB + kMaxW * 4096;        // [kMaxW][2][512]
 constexpr uint32_t kOffW = kOffSfb + kMaxW * 1024;        // [2 warpgroups][kMaxW][64] f32
 constexpr uint32_t kOffPos = kOffW + 2 * kMaxW * 64 * 4;  // [3][kMaxW] i64 query positions (MMA warp, 2 epilogue warpgroups)
 constexpr uint32_t kOffBar = kOffPos + 3 * kMaxW * 8;     // mbarriers
-constexpr uint32_t kNumBars = 3 * kStages + 2 * kAccUnits + 1;
+constexpr uint32_t kNumBars = 3 * kStages + 2 * kAccUnits + 2;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;     // tmem base, abort flag
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;     // + alignment slack
 static_assert(kOffB % 1024 == 0, "B tiles must be 1024-aligned");
@@ -178,6 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_acce = bar_accf + kAccUnits * 8;
   const uint32_t bar_drain = bar_acce + kAccUnits * 8;
   const uint32_t bar_sfr = bar_drain + 8;
+  const uint32_t bar_drain2 = bar_sfr + 8 * kStages;
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(smem + kOffMisc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   float* w_s = reinterpret_cast<float*>(smem + kOffW);
@@ -196,6 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar_drain, 1);
     for (int i = 0; i < kStages; ++i) mbar_init(bar_sfr + 8 * i, 1);
+    mbar_init(bar_drain2, 1);
     *abort = 0;
     tc::fence_barrier_init();
     tc::tma_prefetch_desc(&tm_codes);
@@ -350,12 +352,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t n = (uint32_t)(it / kStages);
       bool okw = true;
       if (lane == 0) {
-        okw = wait_or_abort(bar_sfr + 8 * s, n & 1, P, abort);  // tile landed, scale factors laid out
+        okw = wait_or_abort(bar_sfr + 8 * s, n & 1, P, abort);  // tile landed, scale factors in TMEM
         tc::fence_after_sync();
         const int64_t* pos_s = reinterpret_cast<const int64_t*>(smem + kOffPos);
-        for (int ks = 0; ks < ksteps && okw; ++ks)
-          tc::cp_32x128b_warpx4(tmem + kColSfa + s * 8 + ks * 4,
-                                tc::smem_desc(sbase + kOffSfa + (s * 2 + ks) * 512, 16, 128, tc::kSwizzleNone));
         const int64_t t0 = (int64_t)ti.tile * kTile;
         for (int j = 0; j < W && okw; ++j) {
           if (!kRescore && t0 > pos_s[j]) continue;
@@ -416,8 +415,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc::fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(bar_sfr + 8 * s);
+      // copy to TMEM from this warp, so the copy is not queued behind the MMA
+      // warp's earlier MMAs; the commit hands the stage over once it landed
+      if (lane == 0) {
+        tc::fence_after_sync();
+        for (int ks = 0; ks < ksteps; ++ks)
+          tc::cp_32x128b_warpx4(tmem + kColSfa + s * 8 + ks * 4,
+                                tc::smem_desc(sbase + kOffSfa + (s * 2 + ks) * 512, 16, 128, tc::kSwizzleNone));
+        tc::commit(bar_sfr + 8 * s);
+      }
+      __syncwarp();
     }
+    // drain: our copies must have landed before teardown
+    if (lane == 0) {
+      tc::commit(bar_drain2);
+      if (!mbar_wait_bounded(bar_drain2, 0, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
+    }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
     const int wg = (warp - 2) / 4;        // warpgroup 0: warps 2..5, 1: warps 6..9
