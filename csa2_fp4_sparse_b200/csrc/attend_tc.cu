@@ -243,9 +243,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
 
   int it = 0;
   for (int chunk = split; chunk < n_chunks; chunk += nsplit, ++it) {
-    if (it > 0) {  // the previous chunk's PV still reads the tile
-      bool ok = mbar_wait_bounded(bar_pv, (it - 1) & 1, P.wait_ns);
-      if (!ok) {
+    if (it > 0) {  // the previous chunk's PV still reads the tile (thread 0 probes, the rest park)
+      if (threadIdx.x == 0 && !mbar_wait_bounded(bar_pv, (it - 1) & 1, P.wait_ns)) {
         set_status(P.status, CSA2_ERR_TIMEOUT);
         *abort = 1;
       }
@@ -379,8 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
 
     // ---- 3. softmax over the rows (warps 0..3: one row per thread)
     if (warp < 4) {
-      bool ok = mbar_wait_bounded(bar_s, it & 1, P.wait_ns);
-      if (!ok) {
+      if (!mbar_wait_warp(bar_s, it & 1, P.wait_ns)) {
         set_status(P.status, CSA2_ERR_TIMEOUT);
         *abort = 1;
       }
@@ -502,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
     }
   }
   // ---- epilogue
-  if (it > 0 && !*abort) {
+  if (it > 0 && !*abort && threadIdx.x == 0) {
     if (!mbar_wait_bounded(bar_pv, (it - 1) & 1, P.wait_ns)) {
       set_status(P.status, CSA2_ERR_TIMEOUT);
       *abort = 1;

@@ -88,6 +88,14 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
+// Warp-wide wait: only lane 0 probes the barrier (the other lanes are parked
+// at the shuffle and take no issue slots); every lane gets the result.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait_bounded(bar, parity, limit_ns);
+  return __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
+}
+
 // ---------------------------------------------------------------- reductions
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll

@@ -165,6 +165,14 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, con
   return false;
 }
 
+// the same for a whole warp, probed by lane 0 only
+__device__ __forceinline__ bool warp_wait_or_abort(uint32_t bar, uint32_t parity, const Params& P,
+                                                   volatile int* abort) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = wait_or_abort(bar, parity, P, abort);
+  return __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
+}
+
 template <bool kRescore>
 __global__ void __launch_bounds__(kThreads, 1)
     k_index_tc(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales,
@@ -295,9 +303,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (cur_b >= 0) {  // every MMA reading the old queries must finish first
           if (lane == 0) tc::commit(bar_drain);
           __syncwarp();
-          bool ok = wait_or_abort(bar_drain, drain_n & 1, P, abort);
+          bool ok = warp_wait_or_abort(bar_drain, drain_n & 1, P, abort);
           ++drain_n;
-          if (!__all_sync(0xffffffffu, ok)) break;
+          if (!ok) break;
           tc::fence_after_sync();
         }
         cur_b = ti.b;
@@ -397,8 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (; ti.valid(); ti.next(P), ++it) {
       const int s = (int)(it % kStages);
       const uint32_t n = (uint32_t)(it / kStages);
-      bool ok = wait_or_abort(bar_full + 8 * s, n & 1, P, abort);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      if (!warp_wait_or_abort(bar_full + 8 * s, n & 1, P, abort)) break;
       const uint8_t* raw = smem + kOffRaw + s * kRawStage;
       uint32_t wv[4];
 #pragma unroll
@@ -468,8 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if ((my & 1) != wg) continue;  // the other warpgroup takes this accumulator
         const int u = (int)(my % kAccUnits);
         const uint32_t m = (uint32_t)(my / kAccUnits);
-        bool ok = wait_or_abort(bar_accf + 8 * u, m & 1, P, abort);
-        if (!__all_sync(0xffffffffu, ok)) {
+        if (!warp_wait_or_abort(bar_accf + 8 * u, m & 1, P, abort)) {
           alive = false;
           break;
         }
