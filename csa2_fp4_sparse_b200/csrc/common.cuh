@@ -71,20 +71,30 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread is parked (issuing nothing)
+// until the phase completes or about `hint_ns` have passed
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete; gives up after
-// limit_ns and returns false (the caller records CSA2_ERR_TIMEOUT).  The
-// clock is only read once a long run of probes has failed, so the common,
-// short waits cost nothing but the probes.
+// limit_ns and returns false (the caller records CSA2_ERR_TIMEOUT).  Waiting
+// threads are suspended by the hardware between probes (they take no issue
+// slots from the warps doing work); the clock is read once per probe.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
-  uint64_t t0 = 0;
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
   while (true) {
-    for (int i = 0; i < 1024; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t now = globaltimer_ns();
-    if (t0 == 0)
-      t0 = now;
-    else if (now - t0 > limit_ns)
-      return false;
+    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
 
