@@ -19,11 +19,13 @@
 //               per 16 elements) and copies them to TMEM (tcgen05.cp); a
 //               commit hands the stage to the MMA warp, so the copy never
 //               queues behind that warp's earlier MMAs;
-//   warp 1      MMA issuer: issues tcgen05.mma kind::mxf4nvf4 (M = 128 positions, N = heads,
+//   warps 1, 11 MMA issuers (alternate tiles, one epilogue warpgroup each):
+//               issue tcgen05.mma kind::mxf4nvf4 (M = 128 positions, N = heads,
 //               K = 64 per instruction) per query token into a ring of TMEM
 //               accumulators; commits release the smem stage and hand the
 //               accumulator to the epilogue;
-//   warps 2..9  epilogue, two warpgroups taking alternate accumulators:
+//   warps 2..9  epilogue, two warpgroups (warps 2..5 for MMA warp 1's tiles,
+//               6..9 for warp 11's):
 //               TMEM -> registers (one position per thread), ReLU, weighted
 //               head sum, block max over 8 lanes, block-score store.
 // The key cache is streamed from HBM exactly once per sequence for all of its
@@ -45,8 +47,10 @@ constexpr int kTile = 128;      // positions per tile = MMA M
 constexpr int kChunk = 64;      // rows per TMA box
 constexpr int kAccUnits = 6;    // TMEM accumulator ring, 64 columns each
 constexpr int kMaxW = 8;        // query tokens of one sequence per tile
-constexpr int kThreads = 352;   // 11 warps: producer, MMA, two epilogue warpgroups, scale-factor warp
+constexpr int kThreads = 384;   // 12 warps: producer, 2 MMA issuers, 2 epilogue warpgroups, scale-factor warp
 constexpr int kSfWarp = 10;
+constexpr int kMmaWarpB = 11;   // second MMA issuer (the first is warp 1); they take alternate tiles
+constexpr int kUnitsPer = kAccUnits / 2;  // accumulator units of each MMA issuer
 constexpr uint32_t kColAcc = 0;
 constexpr uint32_t kColSfa = kAccUnits * 64;              // 384
 constexpr uint32_t kColSfb = kColSfa + kStages * 8;      // 448
@@ -65,7 +69,7 @@ constexpr uint32_t kOffSfb = kOffB + kMaxW * 4096;        // [kMaxW][2][512]
 constexpr uint32_t kOffW = kOffSfb + kMaxW * 1024;        // [2 warpgroups][kMaxW][64] f32
 constexpr uint32_t kOffPos = kOffW + 2 * kMaxW * 64 * 4;  // [3][kMaxW] i64 query positions (MMA warp, 2 epilogue warpgroups)
 constexpr uint32_t kOffBar = kOffPos + 3 * kMaxW * 8;     // mbarriers
-constexpr uint32_t kNumBars = 3 * kStages + 2 * kAccUnits + 2;
+constexpr uint32_t kNumBars = 3 * kStages + 2 * kAccUnits + 4;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;     // tmem base, abort flag
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;     // + alignment slack
 static_assert(kOffB % 1024 == 0, "B tiles must be 1024-aligned");
@@ -187,6 +191,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_drain = bar_acce + kAccUnits * 8;
   const uint32_t bar_sfr = bar_drain + 8;
   const uint32_t bar_drain2 = bar_sfr + 8 * kStages;
+  const uint32_t bar_drain_b = bar_drain2 + 8;
+  const uint32_t bar_sfb = bar_drain_b + 8;
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(smem + kOffMisc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   float* w_s = reinterpret_cast<float*>(smem + kOffW);
@@ -206,6 +212,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_drain, 1);
     for (int i = 0; i < kStages; ++i) mbar_init(bar_sfr + 8 * i, 1);
     mbar_init(bar_drain2, 1);
+    mbar_init(bar_drain_b, 1);
+    mbar_init(bar_sfb, 1);
     *abort = 0;
     tc::fence_barrier_init();
     tc::tma_prefetch_desc(&tm_codes);
@@ -288,74 +296,93 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait_bounded(bar_full + 8 * s, last & 1, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == kMmaWarpB) {
+    // ------------------------------------------------------------ MMA issuers
+    // Both issuers walk every tile (so both see every change of group) and
+    // issue the MMAs of the tiles of their parity; a single issuing thread is
+    // limited by the latency of its barrier tests and MMA issues, two overlap.
+    const int mw = warp == 1 ? 0 : 1;
+    const uint32_t my_drain = mw == 0 ? bar_drain : bar_drain_b;
     const uint32_t idesc = tc::idesc_mxf4nvf4(128, P.N);
     const tc::SmemLayout sw = (P.DI == 128) ? tc::kSwizzle64B : tc::kSwizzle32B;
     const uint32_t sbo = 8u * row_bytes;  // 8 rows per swizzle atom
     TileIter<kRescore> ti;
     ti.init(P, wb, we);
-    int64_t it = 0, acc_it = 0;
-    uint32_t drain_n = 0;
+    int64_t it = 0;
+    int cnt = 0;  // jobs issued by this warp
+    uint32_t drain_n = 0, sfb_n = 0;
     int cur_b = -1, W = 0, tok0 = 0;
+    // No early exit from this loop: both issuers must meet at the same named
+    // barriers, so after a failed wait a warp keeps walking the tiles without
+    // issuing anything (every later wait returns at once once *abort is set).
     for (; ti.valid(); ti.next(P), ++it) {
       if (ti.b != cur_b) {
         if (cur_b >= 0) {  // every MMA reading the old queries must finish first
-          if (lane == 0) tc::commit(bar_drain);
+          if (lane == 0) tc::commit(my_drain);
           __syncwarp();
-          bool ok = warp_wait_or_abort(bar_drain, drain_n & 1, P, abort);
+          warp_wait_or_abort(my_drain, drain_n & 1, P, abort);
           ++drain_n;
-          if (!ok) break;
-          tc::fence_after_sync();
         }
+        tc::named_sync(3, 64);  // both issuers drained
         cur_b = ti.b;
         int bseq;
         group_info<kRescore>(P, cur_b, &tok0, &W, &bseq);
         if (W > kMaxW) {
-          if (lane == 0) set_status(P.status, CSA2_ERR_RANGE);
+          if (lane == 0 && mw == 0) set_status(P.status, CSA2_ERR_RANGE);
           W = kMaxW;
         }
-        int64_t* pos_s = reinterpret_cast<int64_t*>(smem + kOffPos);
-        if (lane < W) pos_s[lane] = __ldg(P.qb.tok_pos + tok0 + lane);
-        // B operand: query codes, swizzled like the TMA-written A tiles
-        const int chunks_per_row = row_bytes / 16;
-        for (int e = lane; e < W * 64 * chunks_per_row; e += 32) {
-          const int j = e / (64 * chunks_per_row);
-          const int n = (e / chunks_per_row) % 64;
-          const int ch = e % chunks_per_row;
-          uint4 v = make_uint4(0, 0, 0, 0);
-          if (n < P.H)
-            v = __ldg(reinterpret_cast<const uint4*>(P.q_codes + ((int64_t)(tok0 + j) * P.H + n) * row_bytes) + ch);
-          const int sch = (P.DI == 128) ? (ch ^ ((n >> 1) & 3)) : (ch ^ ((n >> 2) & 1));
-          *reinterpret_cast<uint4*>(smem + kOffB + j * 4096 + n * row_bytes + sch * 16) = v;
-        }
-        // B scale factors: [m0 (32)][m1 (4)][k (4)] per 64-element K step
-        for (int e = lane; e < W * ksteps * 32; e += 32) {
-          const int j = e / (ksteps * 32), ks = (e / 32) % ksteps, m0 = e % 32;
-          uint32_t v[4];
-#pragma unroll
-          for (int m1 = 0; m1 < 4; ++m1) {
-            const int n = m1 * 32 + m0;
-            uint32_t a = 0, b2 = 0;
-            if (n < P.H) {
-              const uint8_t* sp = P.q_scales + ((int64_t)(tok0 + j) * P.H + n) * spr + 2 * ks;
-              a = __ldg(sp);
-              b2 = __ldg(sp + 1);
-            }
-            v[m1] = a | (a << 8) | (b2 << 16) | (b2 << 24);
+        if (mw == 0 && !*abort) {
+          int64_t* pos_s = reinterpret_cast<int64_t*>(smem + kOffPos);
+          if (lane < W) pos_s[lane] = __ldg(P.qb.tok_pos + tok0 + lane);
+          // B operand: query codes, swizzled like the TMA-written A tiles
+          const int chunks_per_row = row_bytes / 16;
+          for (int e = lane; e < W * 64 * chunks_per_row; e += 32) {
+            const int j = e / (64 * chunks_per_row);
+            const int n = (e / chunks_per_row) % 64;
+            const int ch = e % chunks_per_row;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (n < P.H)
+              v = __ldg(reinterpret_cast<const uint4*>(P.q_codes + ((int64_t)(tok0 + j) * P.H + n) * row_bytes) + ch);
+            const int sch = (P.DI == 128) ? (ch ^ ((n >> 1) & 3)) : (ch ^ ((n >> 2) & 1));
+            *reinterpret_cast<uint4*>(smem + kOffB + j * 4096 + n * row_bytes + sch * 16) = v;
           }
-          *reinterpret_cast<uint4*>(smem + kOffSfb + (j * 2 + ks) * 512 + m0 * 16) = make_uint4(v[0], v[1], v[2], v[3]);
+          // B scale factors: [m0 (32)][m1 (4)][k (4)] per 64-element K step
+          for (int e = lane; e < W * ksteps * 32; e += 32) {
+            const int j = e / (ksteps * 32), ks = (e / 32) % ksteps, m0 = e % 32;
+            uint32_t v[4];
+#pragma unroll
+            for (int m1 = 0; m1 < 4; ++m1) {
+              const int n = m1 * 32 + m0;
+              uint32_t a = 0, b2 = 0;
+              if (n < P.H) {
+                const uint8_t* sp = P.q_scales + ((int64_t)(tok0 + j) * P.H + n) * spr + 2 * ks;
+                a = __ldg(sp);
+                b2 = __ldg(sp + 1);
+              }
+              v[m1] = a | (a << 8) | (b2 << 16) | (b2 << 24);
+            }
+            *reinterpret_cast<uint4*>(smem + kOffSfb + (j * 2 + ks) * 512 + m0 * 16) =
+                make_uint4(v[0], v[1], v[2], v[3]);
+          }
+          tc::fence_proxy_async_smem();
+          __syncwarp();
+          bool ok = true;
+          if (lane == 0) {
+            tc::fence_after_sync();
+            for (int j = 0; j < W; ++j)
+              for (int ks = 0; ks < ksteps; ++ks)
+                tc::cp_32x128b_warpx4(tmem + kColSfb + j * 8 + ks * 4,
+                                      tc::smem_desc(sbase + kOffSfb + (j * 2 + ks) * 512, 16, 128, tc::kSwizzleNone));
+            tc::commit(bar_sfb);
+            ok = wait_or_abort(bar_sfb, sfb_n & 1, P, abort);  // the copies landed before anyone issues
+          }
+          ++sfb_n;
+          (void)ok;
         }
-        tc::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          for (int j = 0; j < W; ++j)
-            for (int ks = 0; ks < ksteps; ++ks)
-              tc::cp_32x128b_warpx4(tmem + kColSfb + j * 8 + ks * 4,
-                                    tc::smem_desc(sbase + kOffSfb + (j * 2 + ks) * 512, 16, 128, tc::kSwizzleNone));
-        }
-        __syncwarp();
+        tc::named_sync(4, 64);  // new queries and positions in place
+        tc::fence_after_sync();
       }
+      if ((int)(it & 1) != mw || *abort) continue;  // the other issuer's tile (or nothing left to do)
       const int s = (int)(it % kStages);
       const uint32_t n = (uint32_t)(it / kStages);
       bool okw = true;
@@ -366,8 +393,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t t0 = (int64_t)ti.tile * kTile;
         for (int j = 0; j < W && okw; ++j) {
           if (!kRescore && t0 > pos_s[j]) continue;
-          const int u = (int)(acc_it % kAccUnits);
-          const uint32_t m = (uint32_t)(acc_it / kAccUnits);
+          const int u = mw + 2 * (cnt % kUnitsPer);
+          const uint32_t m = (uint32_t)(cnt / kUnitsPer);
           if (!wait_or_abort(bar_acce + 8 * u, (m & 1) ^ 1, P, abort)) {
             okw = false;
             break;
@@ -380,17 +407,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                              tmem + kColSfb + j * 8 + ks * 4, ks > 0 ? 1u : 0u);
           }
           tc::commit(bar_accf + 8 * u);
-          ++acc_it;
+          ++cnt;
         }
         if (okw) tc::commit(bar_empty + 8 * s);
       }
-      acc_it = __shfl_sync(0xffffffffu, acc_it, 0);
-      if (!__shfl_sync(0xffffffffu, (int)okw, 0)) break;
+      cnt = __shfl_sync(0xffffffffu, cnt, 0);
+      (void)okw;
     }
     // drain: no MMA or copy of ours in flight at teardown
     if (lane == 0) {
-      tc::commit(bar_drain);
-      if (!mbar_wait_bounded(bar_drain, drain_n & 1, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
+      tc::commit(my_drain);
+      if (!mbar_wait_bounded(my_drain, drain_n & 1, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
     }
     __syncwarp();
   } else if (warp == kSfWarp) {
@@ -449,10 +476,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     int64_t* pos_g = reinterpret_cast<int64_t*>(smem + kOffPos) + (1 + wg) * kMaxW;
     TileIter<kRescore> ti;
     ti.init(P, wb, we);
-    int64_t acc_it = 0;
+    int64_t it = 0;
+    int cnt = 0;  // jobs of this warpgroup's issuer
     int cur_b = -1, W = 0, tok0 = 0;
-    bool alive = true;
-    for (; ti.valid() && alive; ti.next(P)) {
+    // no early exit: the four warps of the warpgroup meet at named barriers
+    for (; ti.valid(); ti.next(P), ++it) {
       if (ti.b != cur_b) {
         tc::named_sync(1 + wg, 128);
         cur_b = ti.b;
@@ -466,19 +494,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ept < W) pos_g[ept] = __ldg(P.qb.tok_pos + tok0 + ept);
         tc::named_sync(1 + wg, 128);
       }
+      if ((int)(it & 1) != wg || *abort) continue;  // the other issuer's tile (or nothing left to do)
       const int64_t t0 = (int64_t)ti.tile * kTile;
       for (int j = 0; j < W; ++j) {
         const int tok = tok0 + j;
         const int64_t p = pos_g[j];
         if (!kRescore && t0 > p) continue;
-        const int64_t my = acc_it++;
-        if ((my & 1) != wg) continue;  // the other warpgroup takes this accumulator
-        const int u = (int)(my % kAccUnits);
-        const uint32_t m = (uint32_t)(my / kAccUnits);
-        if (!warp_wait_or_abort(bar_accf + 8 * u, m & 1, P, abort)) {
-          alive = false;
-          break;
-        }
+        const int u = wg + 2 * (cnt % kUnitsPer);
+        const uint32_t m = (uint32_t)(cnt / kUnitsPer);
+        ++cnt;
+        if (!warp_wait_or_abort(bar_accf + 8 * u, m & 1, P, abort)) break;
         tc::fence_after_sync();
         const float* wj = w_g + j * 64;
         const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + kColAcc + u * 64;
