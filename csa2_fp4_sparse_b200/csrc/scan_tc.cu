@@ -12,7 +12,7 @@
 // Design (one persistent CTA per SM, warp-specialised):
 //   warp 0      TMA producer: tiles of 128 positions of the FP4 indexer K cache
 //               (codes with the 64B/32B swizzle the MMA expects, plus the raw
-//               E4M3 scales) into an 8-stage shared-memory ring;
+//               E4M3 scales) into a 12-stage shared-memory ring;
 //   warp 10     scale-factor warp: rearranges each landed tile's scales into
 //               the tensor-core scale-factor layout (each per-32 E4M3 scale
 //               written twice, as the block-scaled MMA takes one UE4M3 scale
@@ -42,18 +42,19 @@
 namespace csa2 {
 namespace scan_tc {
 
-constexpr int kStages = 8;
+constexpr int kStages = 12;
 constexpr int kTile = 128;      // positions per tile = MMA M
 constexpr int kChunk = 64;      // rows per TMA box
-constexpr int kAccUnits = 6;    // TMEM accumulator ring, 64 columns each
+constexpr int kAccUnits = 4;    // TMEM accumulator ring, 64 columns each
 constexpr int kMaxW = 8;        // query tokens of one sequence per tile
 constexpr int kThreads = 384;   // 12 warps: producer, 2 MMA issuers, 2 epilogue warpgroups, scale-factor warp
 constexpr int kSfWarp = 10;
 constexpr int kMmaWarpB = 11;   // second MMA issuer (the first is warp 1); they take alternate tiles
 constexpr int kUnitsPer = kAccUnits / 2;  // accumulator units of each MMA issuer
 constexpr uint32_t kColAcc = 0;
-constexpr uint32_t kColSfa = kAccUnits * 64;              // 384
-constexpr uint32_t kColSfb = kColSfa + kStages * 8;      // 448
+constexpr uint32_t kColSfa = kAccUnits * 64;              // 256
+constexpr uint32_t kColSfb = kColSfa + kStages * 8;      // 352
+static_assert(kColSfb + kMaxW * 8 <= 512, "TMEM budget");
 constexpr uint32_t kTmemCols = 512;
 
 // shared-memory map (offsets from a 1024-aligned base)
