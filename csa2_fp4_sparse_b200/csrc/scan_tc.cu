@@ -13,7 +13,7 @@
 //   warp 0      TMA producer: tiles of 128 positions of the FP4 indexer K cache
 //               (codes with the 64B/32B swizzle the MMA expects, plus the raw
 //               E4M3 scales) into a 12-stage shared-memory ring;
-//   warp 10     scale-factor warp: rearranges each landed tile's scales into
+//   warps 10,12 scale-factor warps (alternate tiles): rearrange each landed tile's scales into
 //               the tensor-core scale-factor layout (each per-32 E4M3 scale
 //               written twice, as the block-scaled MMA takes one UE4M3 scale
 //               per 16 elements) and copies them to TMEM (tcgen05.cp); a
@@ -47,8 +47,9 @@ constexpr int kTile = 128;      // positions per tile = MMA M
 constexpr int kChunk = 64;      // rows per TMA box
 constexpr int kAccUnits = 4;    // TMEM accumulator ring, 64 columns each
 constexpr int kMaxW = 8;        // query tokens of one sequence per tile
-constexpr int kThreads = 384;   // 12 warps: producer, 2 MMA issuers, 2 epilogue warpgroups, scale-factor warp
-constexpr int kSfWarp = 10;
+constexpr int kThreads = 416;   // 13 warps: producer, 2 MMA issuers, 2 epilogue warpgroups, 2 scale-factor warps
+constexpr int kSfWarp = 10;     // scale-factor warps 10 and 12 take alternate tiles
+constexpr int kSfWarpB = 12;
 constexpr int kMmaWarpB = 11;   // second MMA issuer (the first is warp 1); they take alternate tiles
 constexpr int kUnitsPer = kAccUnits / 2;  // accumulator units of each MMA issuer
 constexpr uint32_t kColAcc = 0;
@@ -70,7 +71,7 @@ constexpr uint32_t kOffSfb = kOffB + kMaxW * 4096;        // [kMaxW][2][512]
 constexpr uint32_t kOffW = kOffSfb + kMaxW * 1024;        // [2 warpgroups][kMaxW][64] f32
 constexpr uint32_t kOffPos = kOffW + 2 * kMaxW * 64 * 4;  // [3][kMaxW] i64 query positions (MMA warp, 2 epilogue warpgroups)
 constexpr uint32_t kOffBar = kOffPos + 3 * kMaxW * 8;     // mbarriers
-constexpr uint32_t kNumBars = 3 * kStages + 2 * kAccUnits + 4;
+constexpr uint32_t kNumBars = 3 * kStages + 2 * kAccUnits + 5;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;     // tmem base, abort flag
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;     // + alignment slack
 static_assert(kOffB % 1024 == 0, "B tiles must be 1024-aligned");
@@ -194,6 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_drain2 = bar_sfr + 8 * kStages;
   const uint32_t bar_drain_b = bar_drain2 + 8;
   const uint32_t bar_sfb = bar_drain_b + 8;
+  const uint32_t bar_drain_c = bar_sfb + 8;
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(smem + kOffMisc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   float* w_s = reinterpret_cast<float*>(smem + kOffW);
@@ -215,6 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_drain2, 1);
     mbar_init(bar_drain_b, 1);
     mbar_init(bar_sfb, 1);
+    mbar_init(bar_drain_c, 1);
     *abort = 0;
     tc::fence_barrier_init();
     tc::tma_prefetch_desc(&tm_codes);
@@ -421,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait_bounded(my_drain, drain_n & 1, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
     }
     __syncwarp();
-  } else if (warp == kSfWarp) {
+  } else if (warp == kSfWarp || warp == kSfWarpB) {
     // ------------------------------------------------------------ scale factors
     // raw [row][spr] -> [m0 (32)][m1 (4)][k (4)] per 64-element K step, each
     // per-32 scale written twice (the MMA takes one scale per 16 elements)
@@ -430,7 +433,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int64_t it = 0;
     constexpr int kBoxRows = kRescore ? kBlock : kChunk;
     constexpr uint32_t kSlot = kRescore ? kRawStage / 16 : kRawStage / 2;
+    const int sfw = warp == kSfWarp ? 0 : 1;
     for (; ti.valid(); ti.next(P), ++it) {
+      if ((int)(it & 1) != sfw) continue;  // the other scale-factor warp's tile
       const int s = (int)(it % kStages);
       const uint32_t n = (uint32_t)(it / kStages);
       if (!warp_wait_or_abort(bar_full + 8 * s, n & 1, P, abort)) break;
@@ -463,8 +468,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // drain: our copies must have landed before teardown
     if (lane == 0) {
-      tc::commit(bar_drain2);
-      if (!mbar_wait_bounded(bar_drain2, 0, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
+      const uint32_t dr = sfw == 0 ? bar_drain2 : bar_drain_c;
+      tc::commit(dr);
+      if (!mbar_wait_bounded(dr, 0, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
     }
     __syncwarp();
   } else {
