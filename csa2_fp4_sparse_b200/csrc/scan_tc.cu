@@ -237,36 +237,50 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // G tiles per iteration, `boxes` lanes per tile (scan: 2 boxes of 64 rows,
+    // rescore: 16 blocks of 8 rows): the lanes of different tiles wait for
+    // their stages and issue their copies concurrently.
     const uint32_t tx = (uint32_t)kTile * row_bytes + (uint32_t)kTile * spr;
     const int32_t oob_row = (int32_t)P.n_rows;
     const int32_t oob_x = (int32_t)(((P.n_rows * spr) + 15) / 16 * 16);
+    constexpr int boxes = kRescore ? 16 : 2;
+    constexpr int rows_per_box = kTile / boxes;
+    constexpr int G = (32 / boxes) < 8 ? (32 / boxes) : 8;  // <= kStages: no lane waits on a tile of its own group
+    const int lt = lane / boxes, bx = lane % boxes;
+    const bool has_slot = lane < G * boxes;
     TileIter<kRescore> ti;
     ti.init(P, wb, we);
-    int64_t it = 0;
-    for (; ti.valid(); ti.next(P), ++it) {
+    for (int k = 0; k < lt; ++k) ti.next(P);
+    int64_t it = lt;  // this lane's tile
+    const int64_t total = we - wb;
+    int64_t issued = 0;
+    int cur_g = -1, tok0 = 0, b = 0;
+    int64_t base = 0, len = 0;
+    for (int64_t g0 = 0; g0 < total; g0 += G) {
+      const bool act = has_slot && ti.valid();
       const int s = (int)(it % kStages);
       const uint32_t n = (uint32_t)(it / kStages);
-      bool ok = true;
-      if (lane == 0) {
-        ok = wait_or_abort(bar_empty + 8 * s, (n & 1) ^ 1, P, abort);
-        if (ok) tc::mbar_arrive_expect_tx(bar_full + 8 * s, tx);
+      if (act && bx == 0) {
+        if (wait_or_abort(bar_empty + 8 * s, (n & 1) ^ 1, P, abort)) tc::mbar_arrive_expect_tx(bar_full + 8 * s, tx);
       }
-      if (!__shfl_sync(0xffffffffu, (int)ok, 0)) break;
-      // each issuing lane loads one box: scan 2 boxes of 64 rows, rescore 16 blocks of 8 rows
-      const int boxes = kRescore ? 16 : 2;
-      const int rows_per_box = kTile / boxes;
-      if (lane < boxes) {
-        int tok0, W, b;
-        group_info<kRescore>(P, ti.b, &tok0, &W, &b);
+      __syncwarp();  // every stage of this group armed before any copy lands
+      if (act && !*abort) {
+        if (ti.b != cur_g) {
+          cur_g = ti.b;
+          int W;
+          group_info<kRescore>(P, cur_g, &tok0, &W, &b);
+          len = __ldg(P.qb.seq_len + b);
+          base = P.page_table ? 0 : __ldg(P.seq_base + b);
+        }
         int64_t pos0 = -1;
         if (kRescore) {
-          const int e = ti.tile * 16 + lane;
+          const int e = ti.tile * 16 + bx;
           const int np = min(__ldg(P.pool_n + tok0), P.pool_cap);
           const int32_t blk = e < np ? __ldg(P.pool + (int64_t)tok0 * P.pool_cap + e) : -1;
           if (blk >= 0) pos0 = (int64_t)blk * kBlock;
         } else {
-          pos0 = (int64_t)ti.tile * kTile + lane * kChunk;
-          if (pos0 >= __ldg(P.qb.seq_len + b)) pos0 = -1;
+          pos0 = (int64_t)ti.tile * kTile + bx * kChunk;
+          if (pos0 >= len) pos0 = -1;
         }
         int64_t row0 = -1;
         if (pos0 >= 0) {
@@ -274,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int32_t pg = __ldg(P.page_table + (int64_t)b * P.max_pages + pos0 / P.page_size);
             row0 = (int64_t)pg * P.page_size + pos0 % P.page_size;
           } else {
-            row0 = __ldg(P.seq_base + b) + pos0;
+            row0 = base + pos0;
           }
         }
         int32_t ry = oob_row, sx = oob_x;
@@ -284,20 +298,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (row0 >= 0) {
           set_status(P.status, CSA2_ERR_RANGE);  // misplaced row: read as zeros
         }
-        tc::tma_load_2d(sbase + kOffA + s * 8192 + lane * rows_per_box * row_bytes, &tm_codes, bar_full + 8 * s, 0,
+        tc::tma_load_2d(sbase + kOffA + s * 8192 + bx * rows_per_box * row_bytes, &tm_codes, bar_full + 8 * s, 0,
                         ry);
-        tc::tma_load_1d(sbase + kOffRaw + s * kRawStage + lane * (kRawStage / boxes), &tm_scales, bar_full + 8 * s,
+        tc::tma_load_1d(sbase + kOffRaw + s * kRawStage + bx * (kRawStage / boxes), &tm_scales, bar_full + 8 * s,
                         sx);
       }
       __syncwarp();
+      if (*abort) break;
+      issued = min(total, g0 + G);
+      for (int k = 0; k < G; ++k) ti.next(P);
+      it += G;
     }
     // no copy of ours may be in flight when the CTA leaves
     if (lane == 0) {
-      for (int s = 0; s < kStages && it > 0; ++s) {
-        int64_t uses = it / kStages + (s < it % kStages ? 1 : 0);
+      const uint64_t lim = *abort ? 1000000ull : P.wait_ns;
+      for (int s = 0; s < kStages && issued > 0; ++s) {
+        int64_t uses = issued / kStages + (s < issued % kStages ? 1 : 0);
         if (uses == 0) continue;
         uint32_t last = (uint32_t)(uses - 1);
-        if (!mbar_wait_bounded(bar_full + 8 * s, last & 1, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
+        if (!mbar_wait_bounded(bar_full + 8 * s, last & 1, lim)) set_status(P.status, CSA2_ERR_TIMEOUT);
       }
     }
   } else if (warp == 1 || warp == kMmaWarpB) {
