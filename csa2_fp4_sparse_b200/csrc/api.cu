@@ -136,13 +136,19 @@ static int n_att_splits(int K, const csa2_swa_desc* swa, int* n_sp) {
   return *n_sp + (swa ? (swa->window + kAttRows - 1) / kAttRows : 0);
 }
 
+// tensor-core attention: split partials exist only while the launch has fewer
+// than 148 (token, layer) pairs, so at most 296 partial slots are ever used
+constexpr int64_t kMaxPartialSlots = 296;
+constexpr int kMaxAttLayers = 8;
+
 static size_t attend_ws(const csa2_query_batch* qb, int Hq, int D, int K, const csa2_swa_desc* swa) {
   int n_sp;
   int ns = n_att_splits(K, swa, &n_sp);
+  const int64_t slots = std::max<int64_t>((int64_t)qb->n_tok * ns, kMaxPartialSlots);
   Carve c{nullptr, 0};
-  c.take((size_t)qb->n_tok * ns * Hq * D * 4);
-  c.take((size_t)qb->n_tok * ns * Hq * 2 * 4);
-  c.take((size_t)qb->n_tok * 4);  // split arrival counters
+  c.take((size_t)slots * Hq * D * 4);
+  c.take((size_t)slots * Hq * 2 * 4);
+  c.take((size_t)qb->n_tok * kMaxAttLayers * 4);  // split arrival counters
   return c.used + 256;
 }
 
@@ -227,52 +233,67 @@ static bool use_attend_tc(int D, int Hq, int q_dtype) {
   return env == 1 && attend_tc_supported(D, Hq, q_dtype);
 }
 
+// Attention of n_layers layers that share one index list (one launch on the
+// tensor-core path).  ws: attend_ws() bytes.
+int launch_attend_layers(const csa2_query_batch* qb, int q_dtype, int Hq, const csa2_fp4_cache* kv,
+                         const int32_t* idx, const int32_t* idx_n, int K, const AttendLayer* layers, int n_layers,
+                         float scale, int out_dtype, void* ws, cudaStream_t st) {
+  const int D = kv->dim;
+  const csa2_swa_desc* swa = layers[0].swa;
+  int n_sp;
+  const int ns = n_att_splits(K, swa, &n_sp);
+  const int64_t slots = std::max<int64_t>((int64_t)qb->n_tok * ns, kMaxPartialSlots);
+  Carve c{static_cast<uint8_t*>(ws), ~size_t(0)};
+  float* part_o = static_cast<float*>(c.take((size_t)slots * Hq * D * 4));
+  float* part_ml = static_cast<float*>(c.take((size_t)slots * Hq * 2 * 4));
+  int* done = static_cast<int*>(c.take((size_t)qb->n_tok * kMaxAttLayers * 4));
+  if (use_attend_tc(D, Hq, q_dtype)) {
+    // 128-row chunks; with fewer than 148 (token, layer) pairs one token's
+    // chunks are spread over up to 4 CTAs, whose partials the last one merges
+    const int chunks = (K + 127) / 128 + (swa ? (swa->window + 127) / 128 : 0);
+    const int64_t pairs = (int64_t)qb->n_tok * n_layers;
+    int nsplit = 1;
+    if (pairs < 148) nsplit = (int)std::min<int64_t>(std::min(chunks, 4), (148 + pairs - 1) / pairs);
+    if (nsplit > 1) {
+      if (int rc = cuda_check(cudaMemsetAsync(done, 0, (size_t)pairs * 4, st), "clear split counters")) return rc;
+    }
+    return launch_attend_tc(qb, q_dtype, Hq, kv, idx, idx_n, K, layers, n_layers, scale, out_dtype, part_o, part_ml,
+                            done, nsplit, st);
+  }
+  // CUDA-core path, one layer at a time
+  for (int l = 0; l < n_layers; ++l) {
+    csa2_swa_desc sw{};
+    if (layers[l].swa) sw = *layers[l].swa;
+    size_t smem = (size_t)kAttRows * D * 4 + kAttRows * 4;
+    dim3 grid(ns, qb->n_tok);
+    {
+      Launch L_("attend_simt", st);
+      if (D == 512) {
+        static bool attr = false;
+        if (!attr) {
+          cudaFuncSetAttribute(k_attend_simt<512>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+          attr = true;
+        }
+        k_attend_simt<512><<<grid, 256, smem, st>>>(*qb, layers[l].q, q_dtype, Hq, *kv, idx, idx_n, K, sw, n_sp,
+                                                    scale, part_o, part_ml, ns, status_ptr());
+      } else {
+        k_attend_simt<128><<<grid, 256, smem, st>>>(*qb, layers[l].q, q_dtype, Hq, *kv, idx, idx_n, K, sw, n_sp,
+                                                    scale, part_o, part_ml, ns, status_ptr());
+      }
+    }
+    if (int rc = cuda_check(cudaGetLastError(), "k_attend_simt")) return rc;
+    Launch L_("merge", st);
+    k_merge<<<dim3(Hq, qb->n_tok), 128, 0, st>>>(part_o, part_ml, ns, Hq, D, layers[l].out, out_dtype, layers[l].lse);
+    if (int rc = cuda_check(cudaGetLastError(), "k_merge")) return rc;
+  }
+  return CSA2_OK;
+}
+
 int launch_attend(const csa2_query_batch* qb, const void* q, int q_dtype, int Hq, const csa2_fp4_cache* kv,
                   const int32_t* idx, const int32_t* idx_n, int K, const csa2_swa_desc* swa, float scale, void* out,
                   int out_dtype, float* lse, void* ws, cudaStream_t st) {
-  const int D = kv->dim;
-  int n_sp;
-  const int ns = n_att_splits(K, swa, &n_sp);
-  Carve c{static_cast<uint8_t*>(ws), ~size_t(0)};
-  float* part_o = static_cast<float*>(c.take((size_t)qb->n_tok * ns * Hq * D * 4));
-  float* part_ml = static_cast<float*>(c.take((size_t)qb->n_tok * ns * Hq * 2 * 4));
-  int* done = static_cast<int*>(c.take((size_t)qb->n_tok * 4));
-  if (use_attend_tc(D, Hq, q_dtype)) {
-    // 128-row chunks; small batches spread one token's chunks over up to 4 CTAs,
-    // whose partials the last one to finish merges
-    const int chunks = (K + 127) / 128 + (swa ? (swa->window + 127) / 128 : 0);
-    int nsplit = 1;
-    if (qb->n_tok < 148) nsplit = std::min(std::min(chunks, 4), (148 + qb->n_tok - 1) / qb->n_tok);
-    if (nsplit > 1) {
-      if (int rc = cuda_check(cudaMemsetAsync(done, 0, (size_t)qb->n_tok * 4, st), "clear split counters")) return rc;
-    }
-    return launch_attend_tc(qb, q, q_dtype, Hq, kv, idx, idx_n, K, swa, scale, out, out_dtype, lse, part_o, part_ml,
-                            done, nsplit, st);
-  }
-  csa2_swa_desc sw{};
-  if (swa) sw = *swa;
-  size_t smem = (size_t)kAttRows * D * 4 + kAttRows * 4;
-  dim3 grid(ns, qb->n_tok);
-  {
-  Launch L_("attend_simt", st);
-  if (D == 512) {
-    static bool attr = false;
-    if (!attr) {
-      cudaFuncSetAttribute(k_attend_simt<512>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      attr = true;
-    }
-    k_attend_simt<512><<<grid, 256, smem, st>>>(*qb, q, q_dtype, Hq, *kv, idx, idx_n, K, sw, n_sp, scale, part_o,
-                                                part_ml, ns, status_ptr());
-  } else {
-    k_attend_simt<128><<<grid, 256, smem, st>>>(*qb, q, q_dtype, Hq, *kv, idx, idx_n, K, sw, n_sp, scale, part_o,
-                                                part_ml, ns, status_ptr());
-  }
-  }
-  int rc = cuda_check(cudaGetLastError(), "k_attend_simt");
-  if (rc) return rc;
-  Launch L_("merge", st);
-  k_merge<<<dim3(Hq, qb->n_tok), 128, 0, st>>>(part_o, part_ml, ns, Hq, D, out, out_dtype, lse);
-  return cuda_check(cudaGetLastError(), "k_merge");
+  AttendLayer one{q, out, lse, swa};
+  return launch_attend_layers(qb, q_dtype, Hq, kv, idx, idx_n, K, &one, 1, scale, out_dtype, ws, st);
 }
 
 }  // namespace csa2
@@ -513,7 +534,8 @@ int csa2_decode_stack(const csa2_stack_desc* d, void* workspace, size_t workspac
   }
   const int32_t* cur_idx = idx;
   const int32_t* cur_idx_n = idx_n;
-  for (int l = 0; l < d->n_layers; ++l) {
+  int l = 0;
+  while (l < d->n_layers) {
     const csa2_layer_desc& L = d->layers[l];
     if (L.mode != CSA2_MODE_REUSE) {
       if (int rc = launch_quantize(L.iq, (int64_t)T * d->H_I, dI, nullptr, qc, qsc, st)) return rc;
@@ -539,8 +561,16 @@ int csa2_decode_stack(const csa2_stack_desc* d, void* workspace, size_t workspac
         if (int rc = cuda_check(cudaGetLastError(), "copy idx")) return rc;
       }
     }
-    if (int rc = launch_attend(qb, L.q, d->q_dtype, d->Hq, &d->kv, cur_idx, cur_idx_n, d->K, L.swa, scale, L.out,
-                               d->out_dtype, L.lse, sub, st))
+    // this layer and the Reuse layers after it share the index list: one launch
+    AttendLayer group[kMaxAttLayers];
+    int ng = 0;
+    do {
+      const csa2_layer_desc& G = d->layers[l];
+      group[ng++] = AttendLayer{G.q, G.out, G.lse, G.swa};
+      ++l;
+    } while (l < d->n_layers && d->layers[l].mode == CSA2_MODE_REUSE && ng < kMaxAttLayers);
+    if (int rc = launch_attend_layers(qb, d->q_dtype, d->Hq, &d->kv, cur_idx, cur_idx_n, d->K, group, ng, scale,
+                                      d->out_dtype, sub, st))
       return rc;
   }
   return CSA2_OK;

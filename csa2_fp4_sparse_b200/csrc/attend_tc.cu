@@ -37,23 +37,30 @@ constexpr int kThreads = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;  // P stays <= 2^8 between rescales (fp16-safe)
 
+constexpr int kMaxLayers = 8;  // layers sharing one index list, attended in one launch (grid.z)
+
+struct LayerIO {
+  const void* q;
+  void* out;
+  float* lse;
+  const uint8_t* swa_codes;
+  const float* swa_scale;
+};
+
 struct Params {
   csa2_query_batch qb;
-  const void* q;
   int q_f32;
   csa2_fp4_cache kv;
   const int32_t* idx;
   const int32_t* idx_n;
   int K;
-  csa2_swa_desc swa;
-  int has_swa;
+  int has_swa, swa_cap, swa_window;
   float scale;
-  void* out;
   int out_f32;
-  float* lse;
-  float* part_o;   // split mode: [T][S][Hq][D]
-  float* part_ml;  // split mode: [T][S][Hq][2] (natural-log max, sum)
-  int* done;       // split mode: [T] arrival counters, zero on entry, left zero on exit
+  LayerIO io[kMaxLayers];
+  float* part_o;   // split mode: [layers][T][S][Hq][D]
+  float* part_ml;  // split mode: [layers][T][S][Hq][2] (natural-log max, sum)
+  int* done;       // split mode: [layers][T] arrival counters, zero on entry, left zero on exit
   int* status;
   uint64_t wait_ns;
 };
@@ -78,8 +85,10 @@ struct Layout {
   static constexpr uint32_t kOffBar = kOffCorr + HQ * 4;         // 3 mbarriers (S, PV, drain)
   static constexpr uint32_t kOffMisc = kOffBar + 24;             // tmem base, abort, rescale flag
   static constexpr uint32_t kBytes = kOffMisc + 16 + 1024;
-  static constexpr uint32_t kColS = 0;
-  static constexpr uint32_t kColO = 64;
+  static constexpr int kChains = kKB < 4 ? kKB : 4;  // S = K q^T split over this many issuing threads
+  static constexpr uint32_t kColS = 0;                // chain c accumulates at kColS + c * HQ
+  static constexpr uint32_t kColO = 256;              // O^T tile mt at kColO + mt * HQ
+  static_assert(kChains * HQ <= 256 && kMT * HQ <= 256, "TMEM budget");
 };
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
@@ -151,14 +160,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
   int64_t* rows_s = reinterpret_cast<int64_t*>(smem + Ly::kOffRows);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tok = blockIdx.y, split = blockIdx.x, nsplit = gridDim.x;
+  const int tok = blockIdx.y, split = blockIdx.x, nsplit = gridDim.x, layer = blockIdx.z;
+  const LayerIO io = P.io[layer];
+  const int64_t slot0 = ((int64_t)layer * P.qb.n_tok + tok) * nsplit;  // this token's partial slots
   const int b = __ldg(P.qb.tok_seq + tok);
   const int64_t p = __ldg(P.qb.tok_pos + tok);
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_s, 1);
-    mbar_init(bar_pv, 1);
-    mbar_init(bar_drain, 1);
+    mbar_init(bar_s, Ly::kChains);
+    mbar_init(bar_pv, Ly::kMT);
+    mbar_init(bar_drain, 4);
     *abort = 0;
     *any_rescale = 0;
     tc::fence_barrier_init();
@@ -186,12 +197,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
         const int h = e / (D / 8), c8 = e % (D / 8);
         const int64_t off = ((int64_t)tok * HQ + h) * D + c8 * 8;
         if (P.q_f32) {
-          const float4* s4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(P.q) + off);
+          const float4* s4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(io.q) + off);
           float4 a = __ldg(s4), bb = __ldg(s4 + 1);
           f[u][0] = a.x; f[u][1] = a.y; f[u][2] = a.z; f[u][3] = a.w;
           f[u][4] = bb.x; f[u][5] = bb.y; f[u][6] = bb.z; f[u][7] = bb.w;
         } else {
-          uint4 w4 = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(P.q) + off));
+          uint4 w4 = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(io.q) + off));
           const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
@@ -232,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
   int64_t w_lo = 0;
   int n_w = 0;
   if (P.has_swa) {
-    w_lo = p - P.swa.window + 1;
+    w_lo = p - P.swa_window + 1;
     if (w_lo < 0) w_lo = 0;
     n_w = (int)(p - w_lo + 1);
   }
@@ -273,8 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
       } else {
         const int64_t t = w_lo + (int64_t)(chunk - n_sp) * kRows + r;
         if (t <= p) {
-          row = (int64_t)b * P.swa.cap + t % P.swa.cap;
-          scale_r = __ldg(P.swa.scale + row);
+          row = (int64_t)b * P.swa_cap + t % P.swa_cap;
+          scale_r = __ldg(io.swa_scale + row);
         } else {
           scale_r = 0.0f;
         }
@@ -334,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
         const int u = threadIdx.x + i * kThreads;
         const int r = u / kUnits, g = u % kUnits;
         const int64_t row = rows_s[r];
-        cw[i] = row >= 0 ? __ldg(reinterpret_cast<const uint4*>(P.swa.codes + row * D) + g) : make_uint4(0, 0, 0, 0);
+        cw[i] = row >= 0 ? __ldg(reinterpret_cast<const uint4*>(io.swa_codes + row * D) + g) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
       for (int i = 0; i < kPer; ++i) {
@@ -357,24 +368,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
     tc::fence_proxy_async_smem();
     __syncthreads();
 
-    // ---- 2. S^T = K q^T
-    if (threadIdx.x == 0) {
+    // ---- 2. S^T = K q^T, the K chain split over kChains issuing threads
+    //         (chain c: d-blocks c, c + kChains, ...; its own accumulator)
+    if (warp == 0 && lane < Ly::kChains) {
       tc::fence_after_sync();
+      const int c = lane;
 #pragma unroll 1
-      for (int kb = 0; kb < Ly::kKB; ++kb)
+      for (int kb = c; kb < Ly::kKB; kb += Ly::kChains)
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
           const uint64_t ad = tc::smem_desc(sbase + Ly::kOffK + kb * (kRows * 128) + ks * 32, 16, 1024, tc::kSwizzle128B);
           const uint64_t bd = tc::smem_desc(sbase + Ly::kOffQ + kb * (HQ * 128) + ks * 32, 16, 1024, tc::kSwizzle128B);
-          tc::mma_f16(tmem + Ly::kColS, ad, bd, idesc_s, (kb | ks) ? 1u : 0u);
+          tc::mma_f16(tmem + Ly::kColS + c * HQ, ad, bd, idesc_s, (kb != c || ks) ? 1u : 0u);
           if (QLO) {
             const uint64_t bl =
                 tc::smem_desc(sbase + Ly::kOffQlo + kb * (HQ * 128) + ks * 32, 16, 1024, tc::kSwizzle128B);
-            tc::mma_f16(tmem + Ly::kColS, ad, bl, idesc_s, 1u);
+            tc::mma_f16(tmem + Ly::kColS + c * HQ, ad, bl, idesc_s, 1u);
           }
         }
       tc::commit(bar_s);
     }
+    __syncwarp();
 
     // ---- 3. softmax over the rows (warps 0..3: one row per thread)
     if (warp < 4) {
@@ -388,15 +402,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
       const float zscale = P.scale * kLog2e * rs[r];  // log2-domain score scale (window rows: * s_t)
       constexpr int kPer = HQ >= 32 ? HQ / 32 : 1;
       const uint32_t s_addr = tmem + ((uint32_t)(warp * 32) << 16) + Ly::kColS;
-      // the chunk's scores, scaled to the log2 domain (window rows: * s_t); invalid rows -inf
+      // the chunk's scores (sum of the chains), scaled to the log2 domain
+      // (window rows: * s_t); invalid rows -inf
       auto load_scores = [&](float (&z)[HQ]) {
 #pragma unroll
         for (int g = 0; g < HQ / 16; ++g) {
-          uint32_t v[16];
-          tc::ld_32x32b_x16(s_addr + g * 16, v);
+          uint32_t v[Ly::kChains][16];
+#pragma unroll
+          for (int c = 0; c < Ly::kChains; ++c) tc::ld_32x32b_x16(s_addr + c * HQ + g * 16, v[c]);
           tc::ld_wait();
 #pragma unroll
-          for (int k = 0; k < 16; ++k) z[g * 16 + k] = rv ? __uint_as_float(v[k]) * zscale : -INFINITY;
+          for (int k = 0; k < 16; ++k) {
+            float acc = __uint_as_float(v[0][k]);
+#pragma unroll
+            for (int c = 1; c < Ly::kChains; ++c) acc += __uint_as_float(v[c][k]);
+            z[g * 16 + k] = rv ? acc * zscale : -INFINITY;
+          }
         }
       };
       // per-head maximum of this chunk
@@ -484,20 +505,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
     __syncthreads();
     if (*abort) break;
 
-    // ---- 4. O^T += V^T P^T
-    if (threadIdx.x == 0) {
+    // ---- 4. O^T += V^T P^T, one M tile (128 latent dims) per issuing thread
+    if (warp == 0 && lane < Ly::kMT) {
       tc::fence_after_sync();
-#pragma unroll 1
-      for (int mt = 0; mt < Ly::kMT; ++mt)
+      const int mt = lane;
 #pragma unroll
-        for (int ks = 0; ks < kRows / 16; ++ks) {
-          const uint64_t ad =
-              tc::smem_desc(sbase + Ly::kOffK + (2 * mt) * (kRows * 128) + ks * 2048, kRows * 128, 1024, tc::kSwizzle128B);
-          const uint64_t bd = tc::smem_desc(sbase + Ly::kOffP + ks * 16 * Ly::kPRow, 8 * Ly::kPRow, 8 * Ly::kPRow, p_sw);
-          tc::mma_f16(tmem + Ly::kColO + mt * HQ, ad, bd, idesc_pv, (it > 0 || ks > 0) ? 1u : 0u);
-        }
+      for (int ks = 0; ks < kRows / 16; ++ks) {
+        const uint64_t ad =
+            tc::smem_desc(sbase + Ly::kOffK + (2 * mt) * (kRows * 128) + ks * 2048, kRows * 128, 1024, tc::kSwizzle128B);
+        const uint64_t bd = tc::smem_desc(sbase + Ly::kOffP + ks * 16 * Ly::kPRow, 8 * Ly::kPRow, 8 * Ly::kPRow, p_sw);
+        tc::mma_f16(tmem + Ly::kColO + mt * HQ, ad, bd, idesc_pv, (it > 0 || ks > 0) ? 1u : 0u);
+      }
       tc::commit(bar_pv);
     }
+    __syncwarp();
   }
   // ---- epilogue
   if (it > 0 && !*abort && threadIdx.x == 0) {
@@ -529,11 +550,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
             const float val = l > 0.0f ? o / l : 0.0f;
             const int64_t oi = ((int64_t)tok * HQ + h) * D + d;
             if (P.out_f32)
-              reinterpret_cast<float*>(P.out)[oi] = val;
+              reinterpret_cast<float*>(io.out)[oi] = val;
             else
-              reinterpret_cast<__nv_bfloat16*>(P.out)[oi] = __float2bfloat16_rn(val);
+              reinterpret_cast<__nv_bfloat16*>(io.out)[oi] = __float2bfloat16_rn(val);
           } else {
-            P.part_o[(((int64_t)tok * nsplit + split) * HQ + h) * D + d] = o;
+            P.part_o[((slot0 + split) * HQ + h) * D + d] = o;
           }
         }
       }
@@ -543,9 +564,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
       const float l = have ? l_s[h] : 0.0f;
       const float m2 = have ? m_s[h] : -INFINITY;
       if (nsplit == 1) {
-        if (P.lse) P.lse[(int64_t)tok * HQ + h] = l > 0.0f ? (m2 + log2f(l)) * 0.6931471805599453f : -INFINITY;
+        if (io.lse) io.lse[(int64_t)tok * HQ + h] = l > 0.0f ? (m2 + log2f(l)) * 0.6931471805599453f : -INFINITY;
       } else {
-        float* ml = P.part_ml + (((int64_t)tok * nsplit + split) * HQ + h) * 2;
+        float* ml = P.part_ml + ((slot0 + split) * HQ + h) * 2;
         ml[0] = l > 0.0f ? m2 * 0.6931471805599453f : -INFINITY;
         ml[1] = l;
       }
@@ -557,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
     __shared__ int s_last;
     __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) s_last = atomicAdd(P.done + tok, 1) == nsplit - 1;
+    if (threadIdx.x == 0) s_last = atomicAdd(P.done + (int64_t)layer * P.qb.n_tok + tok, 1) == nsplit - 1;
     __syncthreads();
     if (s_last) {
       __threadfence();
@@ -565,12 +586,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
       for (int h = threadIdx.x; h < HQ; h += kThreads) {
         float M = -INFINITY;
         for (int sp = 0; sp < nsplit; ++sp) {
-          const float* ml = P.part_ml + (((int64_t)tok * nsplit + sp) * HQ + h) * 2;
+          const float* ml = P.part_ml + ((slot0 + sp) * HQ + h) * 2;
           if (__ldcg(ml + 1) > 0.0f) M = fmaxf(M, __ldcg(ml));
         }
         float L = 0.0f;
         for (int sp = 0; sp < nsplit; ++sp) {
-          const float* ml = P.part_ml + (((int64_t)tok * nsplit + sp) * HQ + h) * 2;
+          const float* ml = P.part_ml + ((slot0 + sp) * HQ + h) * 2;
           const float l = __ldcg(ml + 1);
           const float a = l > 0.0f ? __expf(__ldcg(ml) - M) : 0.0f;
           wgt[sp * HQ + h] = a;
@@ -578,12 +599,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
         }
         const float inv = L > 0.0f ? 1.0f / L : 0.0f;
         for (int sp = 0; sp < nsplit; ++sp) wgt[sp * HQ + h] *= inv;
-        if (P.lse) P.lse[(int64_t)tok * HQ + h] = L > 0.0f ? M + logf(L) : -INFINITY;
+        if (io.lse) io.lse[(int64_t)tok * HQ + h] = L > 0.0f ? M + logf(L) : -INFINITY;
       }
       __syncthreads();
       // 16-byte loads, all splits of 4 groups in flight per thread (nsplit <= 4)
       constexpr int kTot4 = HQ * D / 4;
-      const float4* po = reinterpret_cast<const float4*>(P.part_o) + (int64_t)tok * nsplit * kTot4;
+      const float4* po = reinterpret_cast<const float4*>(P.part_o) + slot0 * kTot4;
       for (int e0 = threadIdx.x; e0 < kTot4; e0 += kThreads * 4) {
         float4 v[4][4];
 #pragma unroll
@@ -610,22 +631,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
           }
           const int64_t oi = (int64_t)tok * HQ * D + (int64_t)e * 4;
           if (P.out_f32) {
-            *reinterpret_cast<float4*>(reinterpret_cast<float*>(P.out) + oi) = a;
+            *reinterpret_cast<float4*>(reinterpret_cast<float*>(io.out) + oi) = a;
           } else {
             __nv_bfloat162 lo2 = __floats2bfloat162_rn(a.x, a.y), hi2 = __floats2bfloat162_rn(a.z, a.w);
             uint2 pk;
             pk.x = *reinterpret_cast<uint32_t*>(&lo2);
             pk.y = *reinterpret_cast<uint32_t*>(&hi2);
-            *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(P.out) + oi) = pk;
+            *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(io.out) + oi) = pk;
           }
         }
       }
-      if (threadIdx.x == 0) P.done[tok] = 0;
+      if (threadIdx.x == 0) P.done[(int64_t)layer * P.qb.n_tok + tok] = 0;
     }
   }
   // no MMA of ours may be in flight when TMEM is released
+  if (warp == 0 && lane < 4) tc::commit(bar_drain);  // every issuing thread
+  __syncwarp();
   if (threadIdx.x == 0) {
-    tc::commit(bar_drain);
     if (!mbar_wait_bounded(bar_drain, 0, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
   }
   __syncthreads();
@@ -636,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
 }
 
 template <int D, int HQ, bool QLO>
-int launch_t(const Params& p, int nsplit, cudaStream_t st) {
+int launch_t(const Params& p, int nsplit, int n_layers, cudaStream_t st) {
   using Ly = Layout<D, HQ, QLO>;
   static bool attr[64] = {false};
   int dev = 0;
@@ -649,7 +671,7 @@ int launch_t(const Params& p, int nsplit, cudaStream_t st) {
     attr[dev] = true;
   }
   Launch L_("attend_tc", st);
-  k_attend_tc<D, HQ, QLO><<<dim3(nsplit, p.qb.n_tok), kThreads, Ly::kBytes, st>>>(p);
+  k_attend_tc<D, HQ, QLO><<<dim3(nsplit, p.qb.n_tok, n_layers), kThreads, Ly::kBytes, st>>>(p);
   return cuda_check(cudaGetLastError(), "k_attend_tc");
 }
 
@@ -663,27 +685,35 @@ bool attend_tc_supported(int D, int Hq, int q_dtype) {
   return true;
 }
 
-int launch_attend_tc(const csa2_query_batch* qb, const void* q, int q_dtype, int Hq, const csa2_fp4_cache* kv,
-                     const int32_t* idx, const int32_t* idx_n, int K, const csa2_swa_desc* swa, float scale, void* out,
-                     int out_dtype, float* lse, float* part_o, float* part_ml, int* done, int nsplit,
-                     cudaStream_t st) {
+int launch_attend_tc(const csa2_query_batch* qb, int q_dtype, int Hq, const csa2_fp4_cache* kv, const int32_t* idx,
+                     const int32_t* idx_n, int K, const AttendLayer* layers, int n_layers, float scale, int out_dtype,
+                     float* part_o, float* part_ml, int* done, int nsplit, cudaStream_t st) {
   using namespace attend_tc;
+  if (n_layers < 1 || n_layers > kMaxLayers) return fail(CSA2_ERR_UNSUPPORTED, "1..%d layers per launch", kMaxLayers);
   Params p{};
   p.qb = *qb;
-  p.q = q;
   p.q_f32 = q_dtype == CSA2_F32;
   p.kv = *kv;
   p.idx = idx;
   p.idx_n = idx_n;
   p.K = K;
-  if (swa) {
-    p.swa = *swa;
-    p.has_swa = 1;
+  p.has_swa = layers[0].swa != nullptr;
+  if (p.has_swa) {
+    p.swa_cap = layers[0].swa->cap;
+    p.swa_window = layers[0].swa->window;
+  }
+  for (int l = 0; l < n_layers; ++l) {
+    if ((layers[l].swa != nullptr) != (p.has_swa != 0)) return fail(CSA2_ERR_INVALID_ARG, "mixed sliding-window layers");
+    if (layers[l].swa && (layers[l].swa->cap != p.swa_cap || layers[l].swa->window != p.swa_window))
+      return fail(CSA2_ERR_INVALID_ARG, "sliding-window shapes differ between layers");
+    p.io[l].q = layers[l].q;
+    p.io[l].out = layers[l].out;
+    p.io[l].lse = layers[l].lse;
+    p.io[l].swa_codes = layers[l].swa ? layers[l].swa->codes : nullptr;
+    p.io[l].swa_scale = layers[l].swa ? layers[l].swa->scale : nullptr;
   }
   p.scale = scale;
-  p.out = out;
   p.out_f32 = out_dtype == CSA2_F32;
-  p.lse = lse;
   p.part_o = part_o;
   p.part_ml = part_ml;
   p.done = done;
@@ -691,10 +721,14 @@ int launch_attend_tc(const csa2_query_batch* qb, const void* q, int q_dtype, int
   p.wait_ns = 1000000000ull;
   const int D = kv->dim;
   const bool qlo = p.q_f32 != 0;
-  if (D == 512 && Hq == 64) return qlo ? fail(CSA2_ERR_UNSUPPORTED, "f32 q") : launch_t<512, 64, false>(p, nsplit, st);
-  if (D == 512 && Hq == 16) return qlo ? launch_t<512, 16, true>(p, nsplit, st) : launch_t<512, 16, false>(p, nsplit, st);
-  if (D == 128 && Hq == 64) return qlo ? launch_t<128, 64, true>(p, nsplit, st) : launch_t<128, 64, false>(p, nsplit, st);
-  if (D == 128 && Hq == 16) return qlo ? launch_t<128, 16, true>(p, nsplit, st) : launch_t<128, 16, false>(p, nsplit, st);
+  if (D == 512 && Hq == 64)
+    return qlo ? fail(CSA2_ERR_UNSUPPORTED, "f32 q") : launch_t<512, 64, false>(p, nsplit, n_layers, st);
+  if (D == 512 && Hq == 16)
+    return qlo ? launch_t<512, 16, true>(p, nsplit, n_layers, st) : launch_t<512, 16, false>(p, nsplit, n_layers, st);
+  if (D == 128 && Hq == 64)
+    return qlo ? launch_t<128, 64, true>(p, nsplit, n_layers, st) : launch_t<128, 64, false>(p, nsplit, n_layers, st);
+  if (D == 128 && Hq == 16)
+    return qlo ? launch_t<128, 16, true>(p, nsplit, n_layers, st) : launch_t<128, 16, false>(p, nsplit, n_layers, st);
   return fail(CSA2_ERR_UNSUPPORTED, "attend_tc shape");
 }
 

@@ -19,10 +19,16 @@ int launch_rescore_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8
                       const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n, int P, float* scores,
                       cudaStream_t st);
 bool attend_tc_supported(int D, int Hq, int q_dtype);
-int launch_attend_tc(const csa2_query_batch* qb, const void* q, int q_dtype, int Hq, const csa2_fp4_cache* kv,
-                     const int32_t* idx, const int32_t* idx_n, int K, const csa2_swa_desc* swa, float scale, void* out,
-                     int out_dtype, float* lse, float* part_o, float* part_ml, int* done, int nsplit,
-                     cudaStream_t st);
+// one layer of a multi-layer attention launch (layers share the index list)
+struct AttendLayer {
+  const void* q;
+  void* out;
+  float* lse;
+  const csa2_swa_desc* swa;
+};
+int launch_attend_tc(const csa2_query_batch* qb, int q_dtype, int Hq, const csa2_fp4_cache* kv, const int32_t* idx,
+                     const int32_t* idx_n, int K, const AttendLayer* layers, int n_layers, float scale, int out_dtype,
+                     float* part_o, float* part_ml, int* done, int nsplit, cudaStream_t st);
 
 // Launch bookkeeping: counts every kernel launch and, while the profiler is
 // enabled, brackets it with CUDA events on its stream.

@@ -542,13 +542,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(bar_acce + 8 * u);
-        float acc = 0.0f;
+        // four independent chains; weights read as float4 (broadcast)
+        float a4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
         for (int g = 0; g < 4; ++g)
           if (g < ng) {
 #pragma unroll
-            for (int k = 0; k < 16; ++k) acc = fmaf(wj[g * 16 + k], fmaxf(__uint_as_float(r[g][k]), 0.0f), acc);
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const float4 w4 = *reinterpret_cast<const float4*>(wj + g * 16 + k4 * 4);
+              a4[0] = fmaf(w4.x, fmaxf(__uint_as_float(r[g][k4 * 4 + 0]), 0.0f), a4[0]);
+              a4[1] = fmaf(w4.y, fmaxf(__uint_as_float(r[g][k4 * 4 + 1]), 0.0f), a4[1]);
+              a4[2] = fmaf(w4.z, fmaxf(__uint_as_float(r[g][k4 * 4 + 2]), 0.0f), a4[2]);
+              a4[3] = fmaf(w4.w, fmaxf(__uint_as_float(r[g][k4 * 4 + 3]), 0.0f), a4[3]);
+            }
           }
+        const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
         if (kRescore) {
           // pool entry i = tile*128 + row: position pool[i/8]*8 + i%8
           const int i = ti.tile * kTile + row;
