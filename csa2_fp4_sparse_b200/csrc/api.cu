@@ -128,6 +128,7 @@ static size_t index_ws(const csa2_query_batch* qb, int P) {
   Carve c{nullptr, 0};
   c.take((size_t)qb->n_tok * n_blocks_max(qb) * 4);  // block scores
   c.take((size_t)qb->n_tok * P * kBlock * 4);        // pool position scores
+  c.take((size_t)kNumSmsNominal * sizeof(SelGroup)); // split-selection scratch
   return c.used + 256;
 }
 
@@ -139,7 +140,6 @@ static int n_att_splits(int K, const csa2_swa_desc* swa, int* n_sp) {
 // tensor-core attention: split partials exist only while the launch has fewer
 // than 148 (token, layer) pairs, so at most 296 partial slots are ever used
 constexpr int64_t kMaxPartialSlots = 296;
-constexpr int kMaxAttLayers = 8;
 
 static size_t attend_ws(const csa2_query_batch* qb, int Hq, int D, int K, const csa2_swa_desc* swa) {
   int n_sp;
@@ -153,15 +153,27 @@ static size_t attend_ws(const csa2_query_batch* qb, int Hq, int D, int K, const 
 }
 
 // ---------------------------------------------------------------- launches
-int launch_quantize(const float* x, int64_t n_rows, int dim, const int64_t* slot, uint8_t* codes, uint8_t* scales,
-                    cudaStream_t st) {
+// n_src sources of rows_per_src rows each, quantised into consecutive rows
+static int launch_quantize_multi(const float* const* xs, int n_src, int64_t rows_per_src, int dim,
+                                 const int64_t* slot, uint8_t* codes, uint8_t* scales, cudaStream_t st) {
+  const int64_t n_rows = (int64_t)n_src * rows_per_src;
   if (n_rows == 0) return CSA2_OK;
+  if (n_src < 1 || n_src > kQuantSrc || (slot && n_src != 1))
+    return fail(CSA2_ERR_UNSUPPORTED, "1..%d quantisation sources", kQuantSrc);
+  QuantSrc src{};
+  for (int i = 0; i < n_src; ++i) src.x[i] = xs[i];
+  src.rows_per_src = rows_per_src;
   int64_t work = n_rows * (dim / 8);
   int64_t grid = (work + 255) / 256;
   if (grid > 148 * 32) grid = 148 * 32;
   Launch L_("quantize_fp4", st);
-  k_quantize_fp4<<<(int)grid, 256, 0, st>>>(x, n_rows, dim, slot, codes, scales, status_ptr());
+  k_quantize_fp4<<<(int)grid, 256, 0, st>>>(src, n_rows, dim, slot, codes, scales, status_ptr());
   return cuda_check(cudaGetLastError(), "k_quantize_fp4");
+}
+
+int launch_quantize(const float* x, int64_t n_rows, int dim, const int64_t* slot, uint8_t* codes, uint8_t* scales,
+                    cudaStream_t st) {
+  return launch_quantize_multi(&x, 1, n_rows, dim, slot, codes, scales, st);
 }
 
 template <int DI>
@@ -208,19 +220,92 @@ int launch_scan(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs
   return launch_scan_simt<64>(qb, qc, qs, w, H, kc, bs, ld, st);
 }
 
+// n_sel selector layers (queries [n_sel][T][H][...], weights w[i], scores
+// [n_sel][T][8P]); the tensor-core path takes up to 8 in one launch
+static int launch_rescore_multi(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs,
+                                const float* const* w, int n_sel, int H, const csa2_fp4_cache* kc,
+                                const int32_t* pool, const int32_t* pool_n, int P, float* scores, cudaStream_t st) {
+  if (use_scan_tc(qb, H)) return launch_rescore_tc(qb, qc, qs, w, n_sel, H, kc, pool, pool_n, P, scores, st);
+  const int T = qb->n_tok, dI = kc->dim;
+  for (int i = 0; i < n_sel; ++i) {
+    const uint8_t* c = qc + (size_t)i * T * H * (dI / 2);
+    const uint8_t* s = qs + (size_t)i * T * H * (dI / 32);
+    float* o = scores + (size_t)i * T * P * kBlock;
+    int rc = dI == 128 ? launch_rescore_simt<128>(qb, c, s, w[i], H, kc, pool, pool_n, P, o, st)
+                       : launch_rescore_simt<64>(qb, c, s, w[i], H, kc, pool, pool_n, P, o, st);
+    if (rc) return rc;
+  }
+  return CSA2_OK;
+}
+
 int launch_rescore(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
                    const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n, int P, float* scores,
                    cudaStream_t st) {
-  if (use_scan_tc(qb, H)) return launch_rescore_tc(qb, qc, qs, w, H, kc, pool, pool_n, P, scores, st);
-  if (kc->dim == 128) return launch_rescore_simt<128>(qb, qc, qs, w, H, kc, pool, pool_n, P, scores, st);
-  return launch_rescore_simt<64>(qb, qc, qs, w, H, kc, pool, pool_n, P, scores, st);
+  return launch_rescore_multi(qb, qc, qs, &w, 1, H, kc, pool, pool_n, P, scores, st);
+}
+
+// CTAs per (selector, token) group: with fewer groups than SMs, long
+// candidate lists are split (about 2048 candidates a CTA) so that the whole
+// grid still fits on the GPU at one CTA per SM (the launch is cooperative)
+static int select_splits(int64_t groups, int n_max) {
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+      sms = std::min(v, kNumSmsNominal);
+    else
+      sms = 1;
+  }
+  if (groups >= sms) return 1;
+  int64_t s = (n_max + 2047) / 2048;
+  s = std::min<int64_t>(s, sms / groups);
+  s = std::min<int64_t>(s, kSelMaxSplit);
+  return (int)std::max<int64_t>(s, 1);
+}
+
+// n_sel score matrices [n_sel][T][ld] -> lists [n_sel][T][k_out], counts
+// [n_sel][T].  grp: kNumSmsNominal SelGroup records of scratch, or NULL (one
+// CTA per group)
+static int launch_select_multi(const csa2_query_batch* qb, const float* score, int64_t ld, int mode,
+                               const int32_t* pool, const int32_t* pool_n, int P, int k_out, int32_t* out,
+                               int32_t* out_n, int n_sel, SelGroup* grp, cudaStream_t st) {
+  if (qb->n_tok > 65535 || n_sel > 65535) return fail(CSA2_ERR_UNSUPPORTED, "more than 65535 query tokens");
+  const int64_t groups = (int64_t)qb->n_tok * n_sel;
+  const int n_max = mode == 0 ? n_blocks_max(qb) : P * kBlock;
+  const int S = grp ? select_splits(groups, n_max) : 1;
+  SelParams sp{};
+  sp.qb = *qb;
+  sp.score = score;
+  sp.ld = ld;
+  sp.mode = mode;
+  sp.pool = pool;
+  sp.pool_n = pool_n;
+  sp.P = P;
+  sp.k_out = k_out;
+  sp.out = out;
+  sp.out_n = out_n;
+  sp.grp = grp;
+  sp.status = status_ptr();
+  sp.wait_ns = 1000000000ull;
+  const dim3 grid(S, qb->n_tok, n_sel);
+  if (S > 1) {
+    if (int rc = cuda_check(cudaMemsetAsync(grp, 0, (size_t)groups * sizeof(SelGroup), st), "clear select scratch"))
+      return rc;
+    Launch L_(mode == 0 ? "select_blocks" : "select_positions", st);
+    void* args[] = {&sp};
+    return cuda_check(cudaLaunchCooperativeKernel((const void*)k_select, grid, dim3(kSelThreads), args, 0, st),
+                      "k_select (cooperative)");
+  }
+  Launch L_(mode == 0 ? "select_blocks" : "select_positions", st);
+  k_select<<<grid, kSelThreads, 0, st>>>(sp);
+  return cuda_check(cudaGetLastError(), "k_select");
 }
 
 int launch_select(const csa2_query_batch* qb, const float* score, int64_t ld, int mode, const int32_t* pool,
-                  const int32_t* pool_n, int P, int k_out, int32_t* out, int32_t* out_n, cudaStream_t st) {
-  Launch L_(mode == 0 ? "select_blocks" : "select_positions", st);
-  k_select_topk2<<<qb->n_tok, kSel2Threads, 0, st>>>(*qb, score, ld, mode, pool, pool_n, P, k_out, out, out_n);
-  return cuda_check(cudaGetLastError(), "k_select_topk");
+                  const int32_t* pool_n, int P, int k_out, int32_t* out, int32_t* out_n, SelGroup* grp,
+                  cudaStream_t st) {
+  return launch_select_multi(qb, score, ld, mode, pool, pool_n, P, k_out, out, out_n, 1, grp, st);
 }
 
 // CSA2_ATTEND_IMPL=simt selects the CUDA-core attention (comparison runs).
@@ -233,11 +318,11 @@ static bool use_attend_tc(int D, int Hq, int q_dtype) {
   return env == 1 && attend_tc_supported(D, Hq, q_dtype);
 }
 
-// Attention of n_layers layers that share one index list (one launch on the
-// tensor-core path).  ws: attend_ws() bytes.
-int launch_attend_layers(const csa2_query_batch* qb, int q_dtype, int Hq, const csa2_fp4_cache* kv,
-                         const int32_t* idx, const int32_t* idx_n, int K, const AttendLayer* layers, int n_layers,
-                         float scale, int out_dtype, void* ws, cudaStream_t st) {
+// Attention of n_layers (<= kMaxAttLayers) layers, each with its own index
+// list (one launch on the tensor-core path).  ws: attend_ws() bytes.
+int launch_attend_layers(const csa2_query_batch* qb, int q_dtype, int Hq, const csa2_fp4_cache* kv, int K,
+                         const AttendLayer* layers, int n_layers, float scale, int out_dtype, void* ws,
+                         cudaStream_t st) {
   const int D = kv->dim;
   const csa2_swa_desc* swa = layers[0].swa;
   int n_sp;
@@ -257,8 +342,8 @@ int launch_attend_layers(const csa2_query_batch* qb, int q_dtype, int Hq, const 
     if (nsplit > 1) {
       if (int rc = cuda_check(cudaMemsetAsync(done, 0, (size_t)pairs * 4, st), "clear split counters")) return rc;
     }
-    return launch_attend_tc(qb, q_dtype, Hq, kv, idx, idx_n, K, layers, n_layers, scale, out_dtype, part_o, part_ml,
-                            done, nsplit, st);
+    return launch_attend_tc(qb, q_dtype, Hq, kv, K, layers, n_layers, scale, out_dtype, part_o, part_ml, done,
+                            nsplit, st);
   }
   // CUDA-core path, one layer at a time
   for (int l = 0; l < n_layers; ++l) {
@@ -274,10 +359,12 @@ int launch_attend_layers(const csa2_query_batch* qb, int q_dtype, int Hq, const 
           cudaFuncSetAttribute(k_attend_simt<512>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
           attr = true;
         }
-        k_attend_simt<512><<<grid, 256, smem, st>>>(*qb, layers[l].q, q_dtype, Hq, *kv, idx, idx_n, K, sw, n_sp,
+        k_attend_simt<512><<<grid, 256, smem, st>>>(*qb, layers[l].q, q_dtype, Hq, *kv, layers[l].idx,
+                                                    layers[l].idx_n, K, sw, n_sp,
                                                     scale, part_o, part_ml, ns, status_ptr());
       } else {
-        k_attend_simt<128><<<grid, 256, smem, st>>>(*qb, layers[l].q, q_dtype, Hq, *kv, idx, idx_n, K, sw, n_sp,
+        k_attend_simt<128><<<grid, 256, smem, st>>>(*qb, layers[l].q, q_dtype, Hq, *kv, layers[l].idx,
+                                                    layers[l].idx_n, K, sw, n_sp,
                                                     scale, part_o, part_ml, ns, status_ptr());
       }
     }
@@ -292,8 +379,8 @@ int launch_attend_layers(const csa2_query_batch* qb, int q_dtype, int Hq, const 
 int launch_attend(const csa2_query_batch* qb, const void* q, int q_dtype, int Hq, const csa2_fp4_cache* kv,
                   const int32_t* idx, const int32_t* idx_n, int K, const csa2_swa_desc* swa, float scale, void* out,
                   int out_dtype, float* lse, void* ws, cudaStream_t st) {
-  AttendLayer one{q, out, lse, swa};
-  return launch_attend_layers(qb, q_dtype, Hq, kv, idx, idx_n, K, &one, 1, scale, out_dtype, ws, st);
+  AttendLayer one{idx, idx_n, q, out, lse, swa};
+  return launch_attend_layers(qb, q_dtype, Hq, kv, K, &one, 1, scale, out_dtype, ws, st);
 }
 
 }  // namespace csa2
@@ -390,11 +477,12 @@ int csa2_index_full(const csa2_query_batch* qb, const uint8_t* q_codes, const ui
   const int64_t ld = n_blocks_max(qb);
   float* bs = static_cast<float*>(c.take((size_t)qb->n_tok * ld * 4));
   float* sc = static_cast<float*>(c.take((size_t)qb->n_tok * P * kBlock * 4));
+  SelGroup* grp = static_cast<SelGroup*>(c.take((size_t)kNumSmsNominal * sizeof(SelGroup)));
   if (blockscore) bs = blockscore;
   if (int rc = launch_scan(qb, q_codes, q_scales, w, H_I, k_idx, bs, ld, st)) return rc;
-  if (int rc = launch_select(qb, bs, ld, 0, nullptr, nullptr, P, P, pool, pool_n, st)) return rc;
+  if (int rc = launch_select(qb, bs, ld, 0, nullptr, nullptr, P, P, pool, pool_n, grp, st)) return rc;
   if (int rc = launch_rescore(qb, q_codes, q_scales, w, H_I, k_idx, pool, pool_n, P, sc, st)) return rc;
-  return launch_select(qb, sc, (int64_t)P * kBlock, 1, pool, pool_n, P, K, idx, idx_n, st);
+  return launch_select(qb, sc, (int64_t)P * kBlock, 1, pool, pool_n, P, K, idx, idx_n, grp, st);
 }
 
 int csa2_index_reindex(const csa2_query_batch* qb, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
@@ -410,8 +498,9 @@ int csa2_index_reindex(const csa2_query_batch* qb, const uint8_t* q_codes, const
   Carve c{static_cast<uint8_t*>(workspace), workspace_bytes};
   c.take((size_t)qb->n_tok * n_blocks_max(qb) * 4);
   float* sc = static_cast<float*>(c.take((size_t)qb->n_tok * P * kBlock * 4));
+  SelGroup* grp = static_cast<SelGroup*>(c.take((size_t)kNumSmsNominal * sizeof(SelGroup)));
   if (int rc = launch_rescore(qb, q_codes, q_scales, w, H_I, k_idx, pool, pool_n, P, sc, st)) return rc;
-  return launch_select(qb, sc, (int64_t)P * kBlock, 1, pool, pool_n, P, K, idx, idx_n, st);
+  return launch_select(qb, sc, (int64_t)P * kBlock, 1, pool, pool_n, P, K, idx, idx_n, grp, st);
 }
 
 static int check_attend(const csa2_query_batch* qb, const void* q, int q_dtype, int Hq, const csa2_fp4_cache* kv,
@@ -449,17 +538,30 @@ int csa2_attend_reuse(const csa2_query_batch* qb, const void* q, int32_t q_dtype
 }
 
 // ---------------------------------------------------------------- stack
+// Selector layers (FULL, REINDEX) each produce one index list; a REUSE layer
+// attends over the list of the nearest selector before it.
+static int count_selectors(const csa2_stack_desc* d) {
+  int n = 0;
+  for (int l = 0; l < d->n_layers; ++l) n += d->layers[l].mode != CSA2_MODE_REUSE;
+  return n;
+}
+
 static size_t stack_ws(const csa2_stack_desc* d, size_t* sub_off) {
   const csa2_query_batch* qb = &d->qb;
-  const int dI = d->k_idx.dim;
+  const int dI = d->k_idx.dim, T = qb->n_tok;
+  const int ns = count_selectors(d);
   Carve c{nullptr, 0};
-  c.take((size_t)qb->n_tok * d->H_I * (dI / 2));   // quantised indexer query codes
-  c.take((size_t)qb->n_tok * d->H_I * (dI / 32));  // and scales
-  c.take((size_t)qb->n_tok * d->P * 4);            // pool
-  c.take((size_t)qb->n_tok * 4);                   // pool_n
-  c.take((size_t)qb->n_tok * d->K * 4);            // idx
-  c.take((size_t)qb->n_tok * 4);                   // idx_n
-  size_t sub = std::max(index_ws(qb, d->P), (size_t)0);
+  c.take((size_t)ns * T * d->H_I * (dI / 2));   // quantised indexer queries, every selector
+  c.take((size_t)ns * T * d->H_I * (dI / 32));  // and their scales
+  c.take((size_t)T * d->P * 4);                 // pool
+  c.take((size_t)T * 4);                        // pool_n
+  c.take((size_t)ns * T * d->K * 4);            // index lists, every selector
+  c.take((size_t)ns * T * 4);                   // list lengths
+  Carve ix{nullptr, 0};
+  ix.take((size_t)T * n_blocks_max(qb) * 4);                             // block scores
+  ix.take((size_t)std::min(ns, kMaxSel) * T * d->P * kBlock * 4);        // pool position scores
+  ix.take((size_t)kNumSmsNominal * sizeof(SelGroup));                    // split-selection scratch
+  size_t sub = ix.used + 256;
   bool any_swa = false;
   int win = 0;
   for (int l = 0; l < d->n_layers; ++l)
@@ -486,6 +588,12 @@ int csa2_stack_workspace_size(const csa2_stack_desc* d, size_t* bytes) {
   return CSA2_OK;
 }
 
+static int copy_i32(const int32_t* src, int32_t* dst, int64_t n, cudaStream_t st) {
+  Launch L_("copy", st);
+  k_copy_i32<<<64, 256, 0, st>>>(src, dst, n);
+  return cuda_check(cudaGetLastError(), "copy");
+}
+
 int csa2_decode_stack(const csa2_stack_desc* d, void* workspace, size_t workspace_bytes, void* stream) {
   t_err[0] = 0;
   if (!d) return fail(CSA2_ERR_INVALID_ARG, "desc is NULL");
@@ -510,14 +618,16 @@ int csa2_decode_stack(const csa2_stack_desc* d, void* workspace, size_t workspac
   if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256 || workspace_bytes < need)
     return fail(CSA2_ERR_WORKSPACE, "workspace too small or misaligned (need %zu)", need);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int T = qb->n_tok, dI = d->k_idx.dim;
+  const int T = qb->n_tok, dI = d->k_idx.dim, NL = d->n_layers;
+  const int n_sel = count_selectors(d);
+  const size_t q_codes_sz = (size_t)T * d->H_I * (dI / 2), q_scales_sz = (size_t)T * d->H_I * (dI / 32);
   Carve c{static_cast<uint8_t*>(workspace), workspace_bytes};
-  uint8_t* qc = static_cast<uint8_t*>(c.take((size_t)T * d->H_I * (dI / 2)));
-  uint8_t* qsc = static_cast<uint8_t*>(c.take((size_t)T * d->H_I * (dI / 32)));
+  uint8_t* qc = static_cast<uint8_t*>(c.take(n_sel * q_codes_sz));
+  uint8_t* qsc = static_cast<uint8_t*>(c.take(n_sel * q_scales_sz));
   int32_t* pool = static_cast<int32_t*>(c.take((size_t)T * d->P * 4));
   int32_t* pool_n = static_cast<int32_t*>(c.take((size_t)T * 4));
-  int32_t* idx = static_cast<int32_t*>(c.take((size_t)T * d->K * 4));
-  int32_t* idx_n = static_cast<int32_t*>(c.take((size_t)T * 4));
+  int32_t* idx = static_cast<int32_t*>(c.take((size_t)n_sel * T * d->K * 4));
+  int32_t* idx_n = static_cast<int32_t*>(c.take((size_t)n_sel * T * 4));
   uint8_t* sub = static_cast<uint8_t*>(workspace) + sub_off;
   size_t sub_bytes = workspace_bytes - sub_off;
   const float scale = d->softmax_scale > 0.0f ? d->softmax_scale : 1.0f / std::sqrt((float)d->kv.dim);
@@ -532,45 +642,69 @@ int csa2_decode_stack(const csa2_stack_desc* d, void* workspace, size_t workspac
     if (!d->new_slot_kv) return fail(CSA2_ERR_INVALID_ARG, "new_kv needs new_slot_kv");
     if (int rc = launch_quantize(d->new_kv, T, d->kv.dim, d->new_slot_kv, d->kv.codes, d->kv.scales, st)) return rc;
   }
-  const int32_t* cur_idx = idx;
-  const int32_t* cur_idx_n = idx_n;
-  int l = 0;
-  while (l < d->n_layers) {
-    const csa2_layer_desc& L = d->layers[l];
-    if (L.mode != CSA2_MODE_REUSE) {
-      if (int rc = launch_quantize(L.iq, (int64_t)T * d->H_I, dI, nullptr, qc, qsc, st)) return rc;
-      Carve s{sub, sub_bytes};
-      const int64_t ld = n_blocks_max(qb);
-      float* bs = static_cast<float*>(s.take((size_t)T * ld * 4));
-      float* sc = static_cast<float*>(s.take((size_t)T * d->P * kBlock * 4));
-      if (L.mode == CSA2_MODE_FULL) {
-        if (int rc = launch_scan(qb, qc, qsc, L.iw, d->H_I, &d->k_idx, bs, ld, st)) return rc;
-        if (int rc = launch_select(qb, bs, ld, 0, nullptr, nullptr, d->P, d->P, pool, pool_n, st)) return rc;
-        if (L.pool_out) {
-          Launch L_("copy", st);
-          k_copy_i32<<<64, 256, 0, st>>>(pool, L.pool_out, (int64_t)T * d->P);
-          if (int rc = cuda_check(cudaGetLastError(), "copy pool")) return rc;
-        }
-      }
-      if (int rc = launch_rescore(qb, qc, qsc, L.iw, d->H_I, &d->k_idx, pool, pool_n, d->P, sc, st)) return rc;
-      if (int rc = launch_select(qb, sc, (int64_t)d->P * kBlock, 1, pool, pool_n, d->P, d->K, idx, idx_n, st))
+  // selector layers in order, and each layer's selector
+  std::vector<int> sel_layer;
+  std::vector<int> layer_sel(NL);
+  for (int l = 0; l < NL; ++l) {
+    if (d->layers[l].mode != CSA2_MODE_REUSE) sel_layer.push_back(l);
+    layer_sel[l] = (int)sel_layer.size() - 1;
+  }
+  // every selector's indexer queries, up to kQuantSrc per launch
+  for (int s0 = 0; s0 < n_sel; s0 += kQuantSrc) {
+    const int n = std::min(kQuantSrc, n_sel - s0);
+    const float* xs[kQuantSrc];
+    for (int i = 0; i < n; ++i) xs[i] = d->layers[sel_layer[s0 + i]].iq;
+    if (int rc = launch_quantize_multi(xs, n, (int64_t)T * d->H_I, dI, nullptr, qc + s0 * q_codes_sz,
+                                       qsc + s0 * q_scales_sz, st))
+      return rc;
+  }
+  Carve sc_c{sub, sub_bytes};
+  const int64_t ld = n_blocks_max(qb);
+  float* bs = static_cast<float*>(sc_c.take((size_t)T * ld * 4));
+  float* sc = static_cast<float*>(sc_c.take((size_t)std::min(n_sel, kMaxSel) * T * d->P * kBlock * 4));
+  SelGroup* grp = static_cast<SelGroup*>(sc_c.take((size_t)kNumSmsNominal * sizeof(SelGroup)));
+  // each FULL layer builds the pool that it and the REINDEX layers after it
+  // rescore; the rescoring and position selection of consecutive selectors
+  // run up to kMaxSel at a time
+  int s = 0;
+  while (s < n_sel) {
+    const csa2_layer_desc& F = d->layers[sel_layer[s]];
+    if (F.mode == CSA2_MODE_FULL) {
+      if (int rc = launch_scan(qb, qc + s * q_codes_sz, qsc + s * q_scales_sz, F.iw, d->H_I, &d->k_idx, bs, ld, st))
         return rc;
-      if (L.idx_out) {
-        Launch L_("copy", st);
-        k_copy_i32<<<64, 256, 0, st>>>(idx, L.idx_out, (int64_t)T * d->K);
-        if (int rc = cuda_check(cudaGetLastError(), "copy idx")) return rc;
-      }
+      if (int rc = launch_select(qb, bs, ld, 0, nullptr, nullptr, d->P, d->P, pool, pool_n, grp, st)) return rc;
+      if (F.pool_out)
+        if (int rc = copy_i32(pool, F.pool_out, (int64_t)T * d->P, st)) return rc;
     }
-    // this layer and the Reuse layers after it share the index list: one launch
+    int n = 1;
+    while (s + n < n_sel && n < kMaxSel && d->layers[sel_layer[s + n]].mode != CSA2_MODE_FULL) ++n;
+    const float* ws[kMaxSel];
+    for (int i = 0; i < n; ++i) ws[i] = d->layers[sel_layer[s + i]].iw;
+    if (int rc = launch_rescore_multi(qb, qc + s * q_codes_sz, qsc + s * q_scales_sz, ws, n, d->H_I, &d->k_idx, pool,
+                                      pool_n, d->P, sc, st))
+      return rc;
+    if (int rc = launch_select_multi(qb, sc, (int64_t)d->P * kBlock, 1, pool, pool_n, d->P, d->K,
+                                     idx + (size_t)s * T * d->K, idx_n + (size_t)s * T, n, grp, st))
+      return rc;
+    for (int i = 0; i < n; ++i)
+      if (int32_t* o = d->layers[sel_layer[s + i]].idx_out)
+        if (int rc = copy_i32(idx + (size_t)(s + i) * T * d->K, o, (int64_t)T * d->K, st)) return rc;
+    s += n;
+  }
+  // attention of every layer: consecutive layers alike in having a sliding
+  // window or not, up to kMaxAttLayers per launch
+  int l = 0;
+  while (l < NL) {
     AttendLayer group[kMaxAttLayers];
     int ng = 0;
-    do {
+    const bool has_swa = d->layers[l].swa != nullptr;
+    while (l < NL && ng < kMaxAttLayers && (d->layers[l].swa != nullptr) == has_swa) {
       const csa2_layer_desc& G = d->layers[l];
-      group[ng++] = AttendLayer{G.q, G.out, G.lse, G.swa};
+      const int si = layer_sel[l];
+      group[ng++] = AttendLayer{idx + (size_t)si * T * d->K, idx_n + (size_t)si * T, G.q, G.out, G.lse, G.swa};
       ++l;
-    } while (l < d->n_layers && d->layers[l].mode == CSA2_MODE_REUSE && ng < kMaxAttLayers);
-    if (int rc = launch_attend_layers(qb, d->q_dtype, d->Hq, &d->kv, cur_idx, cur_idx_n, d->K, group, ng, scale,
-                                      d->out_dtype, sub, st))
+    }
+    if (int rc = launch_attend_layers(qb, d->q_dtype, d->Hq, &d->kv, d->K, group, ng, scale, d->out_dtype, sub, st))
       return rc;
   }
   return CSA2_OK;

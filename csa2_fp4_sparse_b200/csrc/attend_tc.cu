@@ -37,9 +37,11 @@ constexpr int kThreads = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;  // P stays <= 2^8 between rescales (fp16-safe)
 
-constexpr int kMaxLayers = 8;  // layers sharing one index list, attended in one launch (grid.z)
+constexpr int kMaxLayers = 32;  // layers attended in one launch (grid.z), each with its own index list
 
 struct LayerIO {
+  const int32_t* idx;    // [T][K] selected Main KV positions of this layer's selector
+  const int32_t* idx_n;  // [T]
   const void* q;
   void* out;
   float* lse;
@@ -51,8 +53,6 @@ struct Params {
   csa2_query_batch qb;
   int q_f32;
   csa2_fp4_cache kv;
-  const int32_t* idx;
-  const int32_t* idx_n;
   int K;
   int has_swa, swa_cap, swa_window;
   float scale;
@@ -141,7 +141,7 @@ __device__ __forceinline__ int reduced_head(int lane, int i) {
 }
 
 template <int D, int HQ, bool QLO>
-__global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
+__global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant__ Params P) {
   using Ly = Layout<D, HQ, QLO>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tok = blockIdx.y, split = blockIdx.x, nsplit = gridDim.x, layer = blockIdx.z;
-  const LayerIO io = P.io[layer];
+  const LayerIO& io = P.io[layer];  // read from parameter space where used
   const int64_t slot0 = ((int64_t)layer * P.qb.n_tok + tok) * nsplit;  // this token's partial slots
   const int b = __ldg(P.qb.tok_seq + tok);
   const int64_t p = __ldg(P.qb.tok_pos + tok);
@@ -238,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_holder;
 
-  const int n_sel = min(__ldg(P.idx_n + tok), P.K);
+  const int n_sel = min(__ldg(io.idx_n + tok), P.K);
   const int n_sp = (n_sel + kRows - 1) / kRows;
   int64_t w_lo = 0;
   int n_w = 0;
@@ -274,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const Params P) {
       if (!swa_chunk) {
         const int j = chunk * kRows + r;
         if (j < n_sel) {
-          const int32_t t = __ldg(P.idx + (int64_t)tok * P.K + j);
+          const int32_t t = __ldg(io.idx + (int64_t)tok * P.K + j);
           if (t >= 0 && t <= p) {
             row = cache_row(P.kv, b, t);
             if (row < 0 || row >= P.kv.n_rows) row = -1;
@@ -685,17 +685,15 @@ bool attend_tc_supported(int D, int Hq, int q_dtype) {
   return true;
 }
 
-int launch_attend_tc(const csa2_query_batch* qb, int q_dtype, int Hq, const csa2_fp4_cache* kv, const int32_t* idx,
-                     const int32_t* idx_n, int K, const AttendLayer* layers, int n_layers, float scale, int out_dtype,
-                     float* part_o, float* part_ml, int* done, int nsplit, cudaStream_t st) {
+int launch_attend_tc(const csa2_query_batch* qb, int q_dtype, int Hq, const csa2_fp4_cache* kv, int K,
+                     const AttendLayer* layers, int n_layers, float scale, int out_dtype, float* part_o,
+                     float* part_ml, int* done, int nsplit, cudaStream_t st) {
   using namespace attend_tc;
   if (n_layers < 1 || n_layers > kMaxLayers) return fail(CSA2_ERR_UNSUPPORTED, "1..%d layers per launch", kMaxLayers);
   Params p{};
   p.qb = *qb;
   p.q_f32 = q_dtype == CSA2_F32;
   p.kv = *kv;
-  p.idx = idx;
-  p.idx_n = idx_n;
   p.K = K;
   p.has_swa = layers[0].swa != nullptr;
   if (p.has_swa) {
@@ -706,6 +704,8 @@ int launch_attend_tc(const csa2_query_batch* qb, int q_dtype, int Hq, const csa2
     if ((layers[l].swa != nullptr) != (p.has_swa != 0)) return fail(CSA2_ERR_INVALID_ARG, "mixed sliding-window layers");
     if (layers[l].swa && (layers[l].swa->cap != p.swa_cap || layers[l].swa->window != p.swa_window))
       return fail(CSA2_ERR_INVALID_ARG, "sliding-window shapes differ between layers");
+    p.io[l].idx = layers[l].idx;
+    p.io[l].idx_n = layers[l].idx_n;
     p.io[l].q = layers[l].q;
     p.io[l].out = layers[l].out;
     p.io[l].lse = layers[l].lse;

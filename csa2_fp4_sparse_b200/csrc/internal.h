@@ -15,20 +15,26 @@ int* status_ptr();
 int launch_scan_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
                    const csa2_fp4_cache* kc, float* bs, int64_t ld, cudaStream_t st);
 
-int launch_rescore_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
-                      const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n, int P, float* scores,
-                      cudaStream_t st);
+int launch_rescore_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* const* w,
+                      int n_sel, int H, const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n, int P,
+                      float* scores, cudaStream_t st);
 bool attend_tc_supported(int D, int Hq, int q_dtype);
-// one layer of a multi-layer attention launch (layers share the index list)
+// one layer of a multi-layer attention launch
 struct AttendLayer {
+  const int32_t* idx;    // [T][K] positions chosen by this layer's selector
+  const int32_t* idx_n;  // [T]
   const void* q;
   void* out;
   float* lse;
   const csa2_swa_desc* swa;
 };
-int launch_attend_tc(const csa2_query_batch* qb, int q_dtype, int Hq, const csa2_fp4_cache* kv, const int32_t* idx,
-                     const int32_t* idx_n, int K, const AttendLayer* layers, int n_layers, float scale, int out_dtype,
-                     float* part_o, float* part_ml, int* done, int nsplit, cudaStream_t st);
+constexpr int kMaxAttLayers = 32;  // layers per attention launch
+constexpr int kMaxSel = 8;         // selector layers per rescoring launch
+constexpr int kNumSmsNominal = 148;  // B200 SMs: sizes the split-selection scratch
+struct SelGroup;
+int launch_attend_tc(const csa2_query_batch* qb, int q_dtype, int Hq, const csa2_fp4_cache* kv, int K,
+                     const AttendLayer* layers, int n_layers, float scale, int out_dtype, float* part_o,
+                     float* part_ml, int* done, int nsplit, cudaStream_t st);
 
 // Launch bookkeeping: counts every kernel launch and, while the profiler is
 // enabled, brackets it with CUDA events on its stream.

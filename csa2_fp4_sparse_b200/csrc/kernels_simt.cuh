@@ -13,7 +13,15 @@ namespace csa2 {
 // grid, found by comparing |x| with scale * {.25,.75,1.25,1.75,2.5,3.5,5}
 // (products exact in fp32), ties to the even code.
 // ============================================================================
-__global__ void __launch_bounds__(256) k_quantize_fp4(const float* __restrict__ x, int64_t n_rows, int dim,
+// up to kQuantSrc row-major sources of rows_per_src rows each, quantised as
+// one matrix of n_src * rows_per_src rows (sources concatenated in order)
+constexpr int kQuantSrc = 8;
+struct QuantSrc {
+  const float* x[kQuantSrc];
+  int64_t rows_per_src;
+};
+
+__global__ void __launch_bounds__(256) k_quantize_fp4(const __grid_constant__ QuantSrc src, int64_t n_rows, int dim,
                                                       const int64_t* __restrict__ slot, uint8_t* __restrict__ codes,
                                                       uint8_t* __restrict__ scales, int* status) {
   const int64_t per_row = dim / 8;
@@ -29,8 +37,9 @@ __global__ void __launch_bounds__(256) k_quantize_fp4(const float* __restrict__ 
     if (active) {
       r = i / per_row;
       c8 = i - r * per_row;
-      const float4* src = reinterpret_cast<const float4*>(x + r * dim + c8 * 8);
-      float4 a = __ldg(src), b = __ldg(src + 1);
+      const int64_t si = r / src.rows_per_src;
+      const float4* xp = reinterpret_cast<const float4*>(src.x[si] + (r - si * src.rows_per_src) * dim + c8 * 8);
+      float4 a = __ldg(xp), b = __ldg(xp + 1);
       v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
       v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 #pragma unroll
@@ -190,113 +199,6 @@ __global__ void __launch_bounds__(128) k_rescore_simt(csa2_query_batch qb, const
     }
   }
   if (i < P * kBlock) scores[(int64_t)tok * P * kBlock + i] = s;
-}
-
-// ============================================================================
-// Top-k selection without a global sort: radix select of the k-th largest key
-// (4 passes of 8 bits over the candidates of one query token), then a stable
-// collect in index order (ties to the lower index) written ascending.
-// mode 0: candidates are block ids 0..n-1 (n = visible blocks of the token).
-// mode 1: candidate i is pool position pool[i/8]*8+i%8 (n = pool_n*8).
-// One CTA of 1024 threads per query token.
-// ============================================================================
-constexpr int kSelThreads = 1024;
-
-__global__ void __launch_bounds__(kSelThreads) k_select_topk(csa2_query_batch qb, const float* __restrict__ score,
-                                                             int64_t ld, int mode, const int32_t* __restrict__ pool,
-                                                             const int32_t* __restrict__ pool_n, int P, int k_out,
-                                                             int32_t* __restrict__ out, int32_t* __restrict__ out_n) {
-  __shared__ int hist[256];
-  __shared__ int scan_scratch[32];
-  __shared__ uint32_t sh_prefix, sh_mask;
-  __shared__ int sh_remaining;
-  const int tok = blockIdx.x;
-  const int64_t p = __ldg(qb.tok_pos + tok);
-  int n;
-  if (mode == 0)
-    n = (int)((p + kBlock) / kBlock);
-  else
-    n = min(__ldg(pool_n + tok), P) * kBlock;
-  const float* sc = score + (int64_t)tok * ld;
-
-  // valid candidates
-  int nv_local = 0;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) nv_local += score_key(sc[i]) != 0u;
-  int n_valid;
-  block_exclusive_scan(nv_local, scan_scratch, &n_valid);
-  const int k_eff = min(k_out, n_valid);
-  if (threadIdx.x == 0) {
-    sh_prefix = 0;
-    sh_mask = 0;
-    sh_remaining = k_eff;
-  }
-  __syncthreads();
-  if (k_eff > 0 && k_eff < n_valid) {
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-      for (int j = threadIdx.x; j < 256; j += blockDim.x) hist[j] = 0;
-      __syncthreads();
-      const uint32_t prefix = sh_prefix, mask = sh_mask;
-      for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        uint32_t key = score_key(sc[i]);
-        if (key != 0u && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
-      }
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        int rem = sh_remaining, cum = 0, d = 255;
-        for (; d > 0; --d) {
-          if (cum + hist[d] >= rem) break;
-          cum += hist[d];
-        }
-        sh_remaining = rem - cum;
-        sh_prefix = prefix | ((uint32_t)d << shift);
-        sh_mask = mask | (255u << shift);
-      }
-      __syncthreads();
-    }
-  }
-  // threshold key T and the number of candidates equal to T to take
-  const bool take_all = (k_eff == n_valid);
-  const uint32_t T = sh_prefix;
-  const int need_eq = sh_remaining;
-  // each thread owns a contiguous segment of candidate indices
-  const int seg = (n + blockDim.x - 1) / blockDim.x;
-  const int lo = min(n, (int)threadIdx.x * seg), hi = min(n, lo + seg);
-  int gt = 0, eq = 0;
-  for (int i = lo; i < hi; ++i) {
-    uint32_t key = score_key(sc[i]);
-    if (key == 0u) continue;
-    if (take_all || key > T)
-      ++gt;
-    else if (key == T)
-      ++eq;
-  }
-  int eq_total;
-  int eq_before = block_exclusive_scan(eq, scan_scratch, &eq_total);
-  int take_eq = take_all ? 0 : max(0, min(eq, need_eq - eq_before));
-  int sel_total;
-  int off = block_exclusive_scan(gt + take_eq, scan_scratch, &sel_total);
-  int32_t* o = out + (int64_t)tok * k_out;
-  int taken_eq = 0;
-  for (int i = lo; i < hi; ++i) {
-    uint32_t key = score_key(sc[i]);
-    if (key == 0u) continue;
-    bool sel = take_all || key > T;
-    if (!sel && key == T && taken_eq < take_eq) {
-      sel = true;
-      ++taken_eq;
-    }
-    if (sel) {
-      int32_t id;
-      if (mode == 0)
-        id = i;
-      else
-        id = __ldg(pool + (int64_t)tok * P + i / kBlock) * kBlock + (i % kBlock);
-      o[off++] = id;
-    }
-  }
-  for (int j = sel_total + threadIdx.x; j < k_out; j += blockDim.x) o[j] = -1;
-  if (threadIdx.x == 0) out_n[tok] = sel_total;
 }
 
 // ============================================================================

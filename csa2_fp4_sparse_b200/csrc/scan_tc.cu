@@ -78,9 +78,10 @@ static_assert(kOffB % 1024 == 0, "B tiles must be 1024-aligned");
 
 struct Params {
   csa2_query_batch qb;
-  const uint8_t* q_codes;
-  const uint8_t* q_scales;
-  const float* w;
+  const uint8_t* q_codes;   // [n_sel][T][H][d_I/2]
+  const uint8_t* q_scales;  // [n_sel][T][H][d_I/32]
+  const float* w[kMaxSel];  // per selector [T][H]
+  int n_sel;                // rescore: selector layers (scan: 1)
   int H, N, DI;
   int64_t n_rows;
   int page_size, max_pages;
@@ -99,12 +100,12 @@ struct Params {
 // a query token (rescore: its own pool).  Tiles are 128 positions.
 template <bool kRescore>
 __device__ __forceinline__ int n_groups(const Params& P) {
-  return kRescore ? P.qb.n_tok : P.qb.n_seq;
+  return kRescore ? P.n_sel * P.qb.n_tok : P.qb.n_seq;
 }
 
 template <bool kRescore>
 __device__ __forceinline__ int group_tiles(const Params& P, int g) {
-  if (kRescore) return (min(__ldg(P.pool_n + g), P.pool_cap) + 15) / 16;
+  if (kRescore) return (min(__ldg(P.pool_n + g % P.qb.n_tok), P.pool_cap) + 15) / 16;
   return (__ldg(P.qb.seq_len + g) + kTile - 1) / kTile;
 }
 
@@ -112,9 +113,9 @@ __device__ __forceinline__ int group_tiles(const Params& P, int g) {
 template <bool kRescore>
 __device__ __forceinline__ void group_info(const Params& P, int g, int* tok0, int* W, int* b) {
   if (kRescore) {
-    *tok0 = g;
+    *tok0 = g % P.qb.n_tok;  // group = (selector, token)
     *W = 1;
-    *b = __ldg(P.qb.tok_seq + g);
+    *b = __ldg(P.qb.tok_seq + *tok0);
   } else {
     *tok0 = __ldg(P.qb.tok_start + g);
     *W = __ldg(P.qb.tok_start + g + 1) - *tok0;
@@ -182,7 +183,7 @@ __device__ __forceinline__ bool warp_wait_or_abort(uint32_t bar, uint32_t parity
 template <bool kRescore>
 __global__ void __launch_bounds__(kThreads, 1)
     k_index_tc(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales,
-               const Params P) {
+               const __grid_constant__ Params P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -355,6 +356,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           W = kMaxW;
         }
         if (mw == 0 && !*abort) {
+          // query rows of this group: selector * T + token (scan: the sequence's tokens)
+          const int64_t qrow0 = kRescore ? (int64_t)(cur_b / P.qb.n_tok) * P.qb.n_tok + tok0 : tok0;
           int64_t* pos_s = reinterpret_cast<int64_t*>(smem + kOffPos);
           if (lane < W) pos_s[lane] = __ldg(P.qb.tok_pos + tok0 + lane);
           // B operand: query codes, swizzled like the TMA-written A tiles
@@ -365,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int ch = e % chunks_per_row;
             uint4 v = make_uint4(0, 0, 0, 0);
             if (n < P.H)
-              v = __ldg(reinterpret_cast<const uint4*>(P.q_codes + ((int64_t)(tok0 + j) * P.H + n) * row_bytes) + ch);
+              v = __ldg(reinterpret_cast<const uint4*>(P.q_codes + ((int64_t)(qrow0 + j) * P.H + n) * row_bytes) + ch);
             const int sch = (P.DI == 128) ? (ch ^ ((n >> 1) & 3)) : (ch ^ ((n >> 2) & 1));
             *reinterpret_cast<uint4*>(smem + kOffB + j * 4096 + n * row_bytes + sch * 16) = v;
           }
@@ -378,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int n = m1 * 32 + m0;
               uint32_t a = 0, b2 = 0;
               if (n < P.H) {
-                const uint8_t* sp = P.q_scales + ((int64_t)(tok0 + j) * P.H + n) * spr + 2 * ks;
+                const uint8_t* sp = P.q_scales + ((int64_t)(qrow0 + j) * P.H + n) * spr + 2 * ks;
                 a = __ldg(sp);
                 b2 = __ldg(sp + 1);
               }
@@ -515,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         W = min(W, kMaxW);
         for (int e = ept; e < W * 64; e += 128) {
           const int j = e / 64, h = e % 64;
-          w_g[e] = h < P.H ? __ldg(P.w + (int64_t)(tok0 + j) * P.H + h) : 0.0f;
+          w_g[e] = h < P.H ? __ldg(P.w[kRescore ? cur_b / P.qb.n_tok : 0] + (int64_t)(tok0 + j) * P.H + h) : 0.0f;
         }
         if (ept < W) pos_g[ept] = __ldg(P.qb.tok_pos + tok0 + ept);
         tc::named_sync(1 + wg, 128);
@@ -563,7 +566,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int np = min(__ldg(P.pool_n + tok), P.pool_cap);
           const int32_t blk = (i / kBlock) < np ? __ldg(P.pool + (int64_t)tok * P.pool_cap + i / kBlock) : -1;
           const int64_t pos = (int64_t)blk * kBlock + (i % kBlock);
-          if (i < P.pool_cap * kBlock) P.out[(int64_t)tok * P.ld + i] = (blk >= 0 && pos <= p) ? acc : -INFINITY;
+          const int64_t orow = (int64_t)(cur_b / P.qb.n_tok) * P.qb.n_tok + tok;  // selector * T + token
+          if (i < P.pool_cap * kBlock) P.out[orow * P.ld + i] = (blk >= 0 && pos <= p) ? acc : -INFINITY;
         } else {
           const int64_t t = t0 + row;
           float sc = (t <= p) ? acc : -INFINITY;
@@ -642,9 +646,9 @@ static int num_sms() {
 }
 
 template <bool kRescore>
-static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
-                           const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n, int pool_cap,
-                           float* out, int64_t ld, cudaStream_t st) {
+static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* const* w,
+                           int n_sel, int H, const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n,
+                           int pool_cap, float* out, int64_t ld, cudaStream_t st) {
   using namespace scan_tc;
   if (!kRescore && qb->max_q_per_seq > kMaxW)
     return fail(CSA2_ERR_UNSUPPORTED, "scan: more than %d query tokens per sequence", kMaxW);
@@ -657,7 +661,9 @@ static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const 
   p.qb = *qb;
   p.q_codes = qc;
   p.q_scales = qs;
-  p.w = w;
+  if (n_sel < 1 || n_sel > kMaxSel) return fail(CSA2_ERR_UNSUPPORTED, "1..%d selector layers per launch", kMaxSel);
+  for (int i = 0; i < n_sel; ++i) p.w[i] = w[i];
+  p.n_sel = n_sel;
   p.H = H;
   p.N = (H + 15) / 16 * 16;
   p.DI = kc->dim;
@@ -690,13 +696,15 @@ static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const 
 
 int launch_scan_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
                    const csa2_fp4_cache* kc, float* bs, int64_t ld, cudaStream_t st) {
-  return launch_index_tc<false>(qb, qc, qs, w, H, kc, nullptr, nullptr, 0, bs, ld, st);
+  return launch_index_tc<false>(qb, qc, qs, &w, 1, H, kc, nullptr, nullptr, 0, bs, ld, st);
 }
 
-int launch_rescore_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
-                      const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n, int P, float* scores,
-                      cudaStream_t st) {
-  return launch_index_tc<true>(qb, qc, qs, w, H, kc, pool, pool_n, P, scores, (int64_t)P * kBlock, st);
+// n_sel selector layers at once: queries [n_sel][T][H][...], weights w[sel],
+// scores [n_sel][T][8P]
+int launch_rescore_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* const* w,
+                      int n_sel, int H, const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n, int P,
+                      float* scores, cudaStream_t st) {
+  return launch_index_tc<true>(qb, qc, qs, w, n_sel, H, kc, pool, pool_n, P, scores, (int64_t)P * kBlock, st);
 }
 
 }  // namespace csa2

@@ -1,375 +1,353 @@
-// select.cuh -- top-k selection without a global sort (block top-P pool and
-// pool top-K positions).  One CTA of 1024 threads per query token.
+// select.cuh -- top-k selection without a global sort: the block top-P pool
+// (mode 0) and the pool's top-K positions (mode 1), for one or several
+// selector layers at once.
 //
-//   keys      order-preserving unsigned images of the fp32 scores (score_key);
-//             invalid candidates map to 0 and are never selected
-//   pass A    range [min, max] and count of the valid scores;
-//   pass B    4096-bin linear histogram over that range (monotone in the
-//             score, so bins are ordered); the bin where the count from the
-//             top reaches k holds the k-th largest score;
-//   pass C    that bin's keys are gathered into shared memory (few in
-//             practice) and its exact k-th key is found by byte-wise radix
-//             steps there (or on global memory if they do not fit);
-//   output    every warp owns a contiguous id range: it counts its selections,
-//             a scan over the 32 warps gives each its output offset, and ties
-//             at the k-th key go to the lowest ids (warp ranges are in id
-//             order); ids are written ascending.
+// The candidates of one (selector, token) group are split over S CTAs
+// (gridDim.x).  Scores become order-preserving unsigned keys (score_key);
+// invalid candidates map to 0 and are never selected.
+//
+//   range     count, smallest and largest valid key of the group;
+//   rounds    the key range [base, base + range] is cut into at most 4096 bins
+//             of 2^shift keys; the bin where the count from the top reaches
+//             the number still wanted holds the k-th largest key, and the next
+//             round cuts only that bin.  A 32-bit key needs at most three
+//             rounds; a round ends the search early when the whole bin is
+//             taken or its width is one key;
+//   output    keys above the threshold key, and the lowest-id ties at it,
+//             written in ascending id order: every CTA owns a contiguous id
+//             segment, every warp a contiguous 512-id stretch of each tile.
+//
+// With S > 1 the group's CTAs merge their counts and histograms in global
+// memory (SelGroup, zeroed before the launch) between group barriers; such
+// launches are cooperative, so all CTAs of the grid are resident together and
+// every barrier wait ends (each is also bounded in time and reports
+// CSA2_ERR_TIMEOUT through the status word).
 #pragma once
 
 #include "common.cuh"
 
 namespace csa2 {
 
-constexpr int kSel2Threads = 1024;
-constexpr int kSelCand = 6144;  // shared candidate capacity
+constexpr int kSelThreads = 512;
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kSelPer = 16;                      // keys per thread per tile
+constexpr int kSelTile = kSelThreads * kSelPer;  // 8192 ids per tile
+constexpr int kSelWarpSpan = 32 * kSelPer;       // 512 ids per warp per tile
+constexpr int kSelBins = 4096;
+constexpr int kSelRounds = 3;
+constexpr int kSelMaxSplit = 64;
 
-struct SelShared {
-  int hist[256];
-  int wsum[32];
-  int wsum2[32];
-  uint32_t cand_key[kSelCand];
-  int cand_n;
-  uint32_t prefix;
-  int remaining;
-  int n_valid;
+struct SelGroup {
+  uint32_t bar;                  // barrier arrivals (S per barrier)
+  uint32_t kmin_inv;             // max over CTAs of ~(smallest valid key)
+  uint32_t kmax;                 // largest valid key
+  int32_t count;                 // valid candidates
+  int32_t cta_gt[kSelMaxSplit];  // per CTA: keys above the threshold
+  int32_t cta_eq[kSelMaxSplit];  // per CTA: keys equal to it
+  int32_t hist[kSelRounds][kSelBins];
 };
 
-__device__ __forceinline__ void hist_add(int* hist, uint32_t digit, bool active) {
-  const uint32_t am = __ballot_sync(0xffffffffu, active);
-  if (!active) return;
-  const uint32_t peers = __match_any_sync(am, digit);
-  if ((__ffs(peers) - 1) == (int)(threadIdx.x & 31)) atomicAdd(&hist[digit], __popc(peers));
-}
-
-// after a histogram: pick the byte where the count from the top reaches `remaining`
-__device__ __forceinline__ void pick_digit(SelShared& S, int shift) {
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    // warp 0: suffix sums over 256 bins, 8 bins per lane
-    const int lane = threadIdx.x;
-    int c[8], tot = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      c[i] = S.hist[255 - (lane * 8 + i)];  // descending digit order
-      tot += c[i];
-    }
-    int incl = tot;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int before = incl - tot;  // keys with a larger digit than this lane's first bin
-    const int rem = S.remaining;
-    int found = -1, above = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (found < 0 && before + c[i] >= rem) {
-        found = 255 - (lane * 8 + i);
-        above = before;
-      }
-      before += c[i];
-    }
-    const uint32_t mask = __ballot_sync(0xffffffffu, found >= 0);
-    const int src = __ffs(mask) - 1;
-    found = __shfl_sync(0xffffffffu, found, src);
-    above = __shfl_sync(0xffffffffu, above, src);
-    if (lane == 0) {
-      S.prefix |= (uint32_t)found << shift;
-      S.remaining = rem - above;
-    }
-  }
-  __syncthreads();
-}
+struct SelParams {
+  csa2_query_batch qb;
+  const float* score;  // [n_sel][T][ld]
+  int64_t ld;
+  int mode;
+  const int32_t* pool;    // [T][P] (mode 1)
+  const int32_t* pool_n;  // [T]
+  int P;
+  int k_out;
+  int32_t* out;    // [n_sel][T][k_out]
+  int32_t* out_n;  // [n_sel][T]
+  SelGroup* grp;   // [n_sel][T] when gridDim.x > 1
+  int* status;
+  uint64_t wait_ns;
+};
 
 // candidate i -> output id
 __device__ __forceinline__ int32_t sel_id(int mode, int i, const int32_t* pool_row) {
   return mode == 0 ? i : __ldg(pool_row + i / kBlock) * kBlock + (i % kBlock);
 }
 
-// key of candidate i (0 past the end)
-__device__ __forceinline__ uint32_t key_at(const float* sc, int i, int n) { return i < n ? score_key(sc[i]) : 0u; }
-
-// visit every candidate: f(i, key) for i in [0, n), several loads in flight per thread
-template <typename F>
-__device__ __forceinline__ void for_keys(const float* sc, int n, F&& f) {
-  constexpr int kU = 8;
-  for (int base = 0; base < n; base += kSel2Threads * kU) {
-    uint32_t k[kU];
-#pragma unroll
-    for (int u = 0; u < kU; ++u) k[u] = key_at(sc, base + u * kSel2Threads + threadIdx.x, n);
-#pragma unroll
-    for (int u = 0; u < kU; ++u) f(base + u * kSel2Threads + threadIdx.x, k[u]);
-  }
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
 }
 
-// block-wide float min/max and int sum (all threads get the result)
-struct MinMaxCount {
-  float mn, mx;
-  int cnt;
-};
-
-__device__ __forceinline__ MinMaxCount block_minmax_count(MinMaxCount v, float* smf, int* smi) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o; o >>= 1) {
-    v.mn = fminf(v.mn, __shfl_xor_sync(0xffffffffu, v.mn, o));
-    v.mx = fmaxf(v.mx, __shfl_xor_sync(0xffffffffu, v.mx, o));
-    v.cnt += __shfl_xor_sync(0xffffffffu, v.cnt, o);
-  }
+// barrier of the S CTAs of one group: returns false (and sets the status)
+// when the wait ran past its limit
+__device__ __forceinline__ bool group_barrier(uint32_t* bar, uint32_t target, uint64_t wait_ns, int* status,
+                                              int* flag_s) {
   __syncthreads();
-  if (lane == 0) {
-    smf[wid] = v.mn;
-    smf[32 + wid] = v.mx;
-    smi[wid] = v.cnt;
-  }
-  __syncthreads();
-  MinMaxCount r{smf[0], smf[32], smi[0]};
-  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) {
-    r.mn = fminf(r.mn, smf[w]);
-    r.mx = fmaxf(r.mx, smf[32 + w]);
-    r.cnt += smi[w];
-  }
-  return r;
-}
-
-constexpr int kLinBins = 4096;
-
-struct SelShared2 {
-  int hist[kLinBins];
-  float redf[64];
-  int redi[32];
-  int wsum[32];
-  int wsum2[32];
-  uint32_t cand_key[kSelCand];
-  int cand_n;
-  int bstar, above;
-  uint32_t prefix;
-  int remaining;
-};
-
-// linear bin of a valid score within [mn, mx] (monotone non-decreasing in s)
-__device__ __forceinline__ int lin_bin(float s, float mn, float scale) {
-  int b = (int)__fmul_rn(__fsub_rn(s, mn), scale);
-  return b < 0 ? 0 : (b >= kLinBins ? kLinBins - 1 : b);
-}
-
-// warp 0: the byte where the count from the top of hist[256] reaches *remaining;
-// updates *prefix and *remaining (callers synchronise around it)
-__device__ __forceinline__ void warp_pick_byte(const int* hist, uint32_t* prefix, int* remaining, int shift) {
-  const int lane = threadIdx.x & 31;
-  int c[8], tot = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    c[i] = hist[255 - (lane * 8 + i)];
-    tot += c[i];
-  }
-  int incl = tot;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  int before = incl - tot;
-  const int rem = *remaining;
-  int found = -1, above = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    if (found < 0 && before + c[i] >= rem) {
-      found = 255 - (lane * 8 + i);
-      above = before;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(bar, 1u);
+    const uint64_t t0 = globaltimer_ns();
+    int ok = 1;
+    while (ld_acquire_u32(bar) < target) {
+      if (globaltimer_ns() - t0 > wait_ns) {
+        set_status(status, CSA2_ERR_TIMEOUT);
+        ok = 0;
+        break;
+      }
+      __nanosleep(64);
     }
-    before += c[i];
+    __threadfence();
+    *flag_s = ok;
   }
-  const uint32_t mask = __ballot_sync(0xffffffffu, found >= 0);
-  const int src = mask ? __ffs(mask) - 1 : 31;
-  found = __shfl_sync(0xffffffffu, found, src);
-  above = __shfl_sync(0xffffffffu, above, src);
-  if (found < 0) found = 0;
-  if (lane == 0) {
-    *prefix |= (uint32_t)found << shift;
-    *remaining = rem - above;
-  }
+  __syncthreads();
+  return *flag_s != 0;
 }
 
-// radix step over the shared candidates: fixes the byte at `shift` of the
-// remaining-th largest key among candidates matching S.prefix above it
-__device__ __forceinline__ void cand_radix_step(SelShared2& S, int nc, int shift) {
-  for (int i = threadIdx.x; i < 256; i += kSel2Threads) S.hist[i] = 0;
-  __syncthreads();
-  const uint32_t hi_mask = shift >= 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
-  const uint32_t pre = S.prefix;
-  for (int i = threadIdx.x; i < nc; i += kSel2Threads) {
-    const uint32_t key = S.cand_key[i];
-    if ((key & hi_mask) == (pre & hi_mask)) atomicAdd(&S.hist[(key >> shift) & 255u], 1);
+// one tile of a CTA's segment: lane l of warp w holds ids
+// tile + w*512 + j*32 + l (j < 16); keys past the segment end are 0
+__device__ __forceinline__ void sel_load_tile(const float* sc, int tile, int hi, uint32_t (&k)[kSelPer]) {
+  const int base = tile + (threadIdx.x >> 5) * kSelWarpSpan + (threadIdx.x & 31);
+  float v[kSelPer];
+#pragma unroll
+  for (int j = 0; j < kSelPer; ++j) {
+    const int i = base + j * 32;
+    v[j] = i < hi ? __ldg(sc + i) : -INFINITY;
   }
-  __syncthreads();
-  if (threadIdx.x < 32) warp_pick_byte(S.hist, &S.prefix, &S.remaining, shift);
-  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kSelPer; ++j) k[j] = score_key(v[j]);
 }
 
-__global__ void __launch_bounds__(kSel2Threads, 1) k_select_topk2(csa2_query_batch qb, const float* __restrict__ score,
-                                                               int64_t ld, int mode, const int32_t* __restrict__ pool,
-                                                               const int32_t* __restrict__ pool_n, int P, int k_out,
-                                                               int32_t* __restrict__ out, int32_t* __restrict__ out_n) {
-  __shared__ SelShared2 S;
-  const int tok = blockIdx.x;
+__global__ void __launch_bounds__(kSelThreads) k_select(const __grid_constant__ SelParams P) {
+  __shared__ int hist[kSelBins];
+  __shared__ int red[3][kSelWarps];
+  __shared__ uint32_t redu[2][kSelWarps];
+  __shared__ int wgt[kSelWarps], weq[kSelWarps];
+  __shared__ int flag_s;
+
+  const int S = gridDim.x, s = blockIdx.x, tok = blockIdx.y;
+  const int T = P.qb.n_tok;
+  const int64_t g = (int64_t)blockIdx.z * T + tok;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int64_t p = __ldg(qb.tok_pos + tok);
-  const int n = mode == 0 ? (int)((p + kBlock) / kBlock) : min(__ldg(pool_n + tok), P) * kBlock;
-  const float* sc = score + (int64_t)tok * ld;
-  const int32_t* pool_row = pool + (int64_t)tok * P;
+  const int64_t p = __ldg(P.qb.tok_pos + tok);
+  const int n = P.mode == 0 ? (int)((p + kBlock) / kBlock) : min(__ldg(P.pool_n + tok), P.P) * kBlock;
+  const float* sc = P.score + g * P.ld;
+  const int32_t* pool_row = P.pool + (int64_t)tok * P.P;
+  SelGroup* G = S > 1 ? P.grp + g : nullptr;
+  uint32_t n_bar = 0;
 
-  // pass A: range and count of the valid scores
-  MinMaxCount v{INFINITY, -INFINITY, 0};
-  for_keys(sc, n, [&](int i, uint32_t key) {
-    if (key != 0u) {
-      const float f = sc[i];
-      v.mn = fminf(v.mn, f);
-      v.mx = fmaxf(v.mx, f);
-      v.cnt += 1;
+  // this CTA's segment, in tiles of 8192 ids; the first tile stays in registers
+  const int seg = (n + S - 1) / S;
+  const int lo = min(n, s * seg), hi = min(n, lo + seg);
+  uint32_t k0[kSelPer];
+  sel_load_tile(sc, lo, hi, k0);
+  auto visit = [&](auto&& f) {
+#pragma unroll
+    for (int j = 0; j < kSelPer; ++j) f(k0[j]);
+    for (int t = lo + kSelTile; t < hi; t += kSelTile) {
+      uint32_t k[kSelPer];
+      sel_load_tile(sc, t, hi, k);
+#pragma unroll
+      for (int j = 0; j < kSelPer; ++j) f(k[j]);
+    }
+  };
+
+  // ---- range and count of the valid keys
+  int cnt = 0;
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  visit([&](uint32_t key) {
+    if (key) {
+      ++cnt;
+      kmin = min(kmin, key);
+      kmax = max(kmax, key);
     }
   });
-  const MinMaxCount r = block_minmax_count(v, S.redf, S.redi);
-  const int n_valid = r.cnt;
-  const int k_eff = min(k_out, n_valid);
-  const bool take_all = k_eff == n_valid;
-  uint32_t T = 0;
+  cnt = __reduce_add_sync(0xffffffffu, cnt);
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  if (lane == 0) {
+    red[0][wid] = cnt;
+    redu[0][wid] = kmin;
+    redu[1][wid] = kmax;
+  }
+  __syncthreads();
+  {
+    const int c = lane < kSelWarps ? red[0][lane] : 0;
+    const uint32_t mn = lane < kSelWarps ? redu[0][lane] : 0xFFFFFFFFu;
+    const uint32_t mx = lane < kSelWarps ? redu[1][lane] : 0u;
+    cnt = __reduce_add_sync(0xffffffffu, c);
+    kmin = __reduce_min_sync(0xffffffffu, mn);
+    kmax = __reduce_max_sync(0xffffffffu, mx);
+  }
+  if (G) {
+    if (threadIdx.x == 0) {
+      atomicAdd(&G->count, cnt);
+      atomicMax(&G->kmin_inv, ~kmin);
+      atomicMax(&G->kmax, kmax);
+    }
+    if (!group_barrier(&G->bar, S * ++n_bar, P.wait_ns, P.status, &flag_s)) return;
+    cnt = __ldcg(&G->count);
+    kmin = ~__ldcg(&G->kmin_inv);
+    kmax = __ldcg(&G->kmax);
+  }
+
+  // ---- threshold: selected = valid keys > thr, plus the first need_eq ties at thr
+  const int k_eff = min(P.k_out, cnt);
+  uint32_t thr = 0;
   int need_eq = 0;
-  if (!take_all && r.mx == r.mn) {
-    T = score_key(r.mx);  // every valid score ties: the lowest ids win
-    need_eq = k_eff;
-  } else if (!take_all) {
-    // pass B: linear histogram over [mn, mx]
-    const float mn = r.mn, scale = (float)kLinBins / (r.mx - r.mn);
-    for (int i = threadIdx.x; i < kLinBins; i += kSel2Threads) S.hist[i] = 0;
-    __syncthreads();
-    for_keys(sc, n, [&](int i, uint32_t key) {
-      if (key != 0u) atomicAdd(&S.hist[lin_bin(sc[i], mn, scale)], 1);
-    });
-    __syncthreads();
-    // threshold bin: suffix sums from the top, 4 bins per thread
-    {
-      constexpr int kPerT = kLinBins / kSel2Threads;
-      const int hb = kLinBins - 1 - threadIdx.x * kPerT;  // this thread's highest bin
+  if (k_eff < cnt) {
+    uint32_t base = kmin, range = kmax - kmin;
+    int remaining = k_eff;
+    for (int r = 0; r < kSelRounds; ++r) {
+      if (range == 0) {  // every remaining candidate has key == base
+        thr = base;
+        need_eq = remaining;
+        break;
+      }
+      const int bits = 32 - __clz(range);
+      const int shift = bits > 12 ? bits - 12 : 0;
+      for (int b = threadIdx.x; b < kSelBins; b += kSelThreads) hist[b] = 0;
+      __syncthreads();
+      visit([&](uint32_t key) {
+        const uint32_t d = key - base;
+        if (key && key >= base && d <= range) atomicAdd(&hist[d >> shift], 1);
+      });
+      __syncthreads();
+      if (G) {
+        for (int b = threadIdx.x; b < kSelBins; b += kSelThreads)
+          if (hist[b]) atomicAdd(&G->hist[r][b], hist[b]);
+        if (!group_barrier(&G->bar, S * ++n_bar, P.wait_ns, P.status, &flag_s)) return;
+        for (int b = threadIdx.x; b < kSelBins; b += kSelThreads) hist[b] = __ldcg(&G->hist[r][b]);
+        __syncthreads();
+      }
+      // bin where the count from the top reaches `remaining`: 8 bins a thread
+      // (thread 0 holds the top bins), then a block scan of the thread sums
+      constexpr int kPerT = kSelBins / kSelThreads;
+      const int top = kSelBins - 1 - threadIdx.x * kPerT;
       int c[kPerT], tot = 0;
 #pragma unroll
       for (int j = 0; j < kPerT; ++j) {
-        c[j] = S.hist[hb - j];
+        c[j] = hist[top - j];
         tot += c[j];
       }
-      int total;
-      const int before = block_exclusive_scan(tot, S.wsum, &total);
-      int cum = before;
+      int incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (lane == 31) red[1][wid] = incl;
+      if (threadIdx.x == 0) red[2][0] = -1;
+      __syncthreads();
+      int before = incl - tot;
+      for (int w = 0; w < wid; ++w) before += red[1][w];
 #pragma unroll
       for (int j = 0; j < kPerT; ++j) {
-        if (cum < k_eff && cum + c[j] >= k_eff) {
-          S.bstar = hb - j;
-          S.above = cum;
+        if (before < remaining && before + c[j] >= remaining) {  // exactly one thread
+          red[2][0] = top - j;
+          red[2][1] = before;
+          red[2][2] = c[j];
         }
-        cum += c[j];
+        before += c[j];
+      }
+      __syncthreads();
+      const int bstar = red[2][0], above = red[2][1], in_bin = red[2][2];
+      __syncthreads();  // red[] and hist[] are reused
+      if (bstar < 0) {  // only with inconsistent counts; every CTA of the group sees the same
+        set_status(P.status, CSA2_ERR_RANGE);
+        return;
+      }
+      remaining -= above;
+      base += (uint32_t)bstar << shift;
+      range = min(range - ((uint32_t)bstar << shift), shift ? (1u << shift) - 1u : 0u);
+      if (in_bin == remaining) {  // the whole bin is taken
+        thr = base - 1u;
+        need_eq = 0;
+        break;
+      }
+      if (shift == 0) {  // one key per bin
+        thr = base;
+        need_eq = remaining;
+        break;
       }
     }
-    __syncthreads();
-    const int bstar = S.bstar;
-    // pass C: gather the keys of the threshold bin
-    if (threadIdx.x == 0) S.cand_n = 0;
-    __syncthreads();
-    for_keys(sc, n, [&](int i, uint32_t key) {
-      if (key != 0u && lin_bin(sc[i], mn, scale) == bstar) {
-        const int slot = atomicAdd(&S.cand_n, 1);
-        if (slot < kSelCand) S.cand_key[slot] = key;
-      }
-    });
-    __syncthreads();
-    const int nc = S.cand_n;
-    if (threadIdx.x == 0) {
-      S.prefix = 0;
-      S.remaining = k_eff - S.above;
-    }
-    __syncthreads();
-    if (nc <= kSelCand) {
-      for (int shift = 24; shift >= 0; shift -= 8) cand_radix_step(S, nc, shift);
-    } else {
-      // more threshold-bin members than fit: resolve the bytes on global memory
-      for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = threadIdx.x; i < 256; i += kSel2Threads) S.hist[i] = 0;
-        __syncthreads();
-        const uint32_t hi_mask = shift >= 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
-        const uint32_t pre = S.prefix;
-        for_keys(sc, n, [&](int i, uint32_t key) {
-          if (key != 0u && lin_bin(sc[i], mn, scale) == bstar && (key & hi_mask) == (pre & hi_mask))
-            atomicAdd(&S.hist[(key >> shift) & 255u], 1);
-        });
-        __syncthreads();
-        if (threadIdx.x < 32) warp_pick_byte(S.hist, &S.prefix, &S.remaining, shift);
-        __syncthreads();
-      }
-    }
-    T = S.prefix;
-    need_eq = S.remaining;
   }
-  // output: warp w owns ids [w*span, (w+1)*span)
-  const int span = (n + 31) / 32;
-  const int lo = min(n, wid * span), hi = min(n, lo + span);
+
+  // ---- output: this CTA's counts, then its place among the group's CTAs
+  auto is_gt = [&](uint32_t key) { return key != 0u && key > thr; };
+  auto is_eq = [&](uint32_t key) { return need_eq > 0 && key != 0u && key == thr; };
   int gt = 0, eq = 0;
-  for (int b0 = lo; b0 < hi; b0 += 32 * 8) {
-    uint32_t k8[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) k8[u] = key_at(sc, b0 + u * 32 + lane, hi);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const uint32_t key = k8[u];
-      const bool g = key != 0u && (take_all || key > T);
-      const bool e = !take_all && key != 0u && key == T;
-      gt += __popc(__ballot_sync(0xffffffffu, g));
-      eq += __popc(__ballot_sync(0xffffffffu, e));
-    }
-  }
+  visit([&](uint32_t key) {
+    gt += is_gt(key);
+    eq += is_eq(key);
+  });
+  gt = __reduce_add_sync(0xffffffffu, gt);
+  eq = __reduce_add_sync(0xffffffffu, eq);
   if (lane == 0) {
-    S.wsum[wid] = gt;
-    S.wsum2[wid] = eq;
+    red[0][wid] = gt;
+    red[1][wid] = eq;
   }
   __syncthreads();
-  // exclusive prefix over the 32 warps (each lane of a warp reads one warp's sum)
-  int eq_before = __shfl_sync(0xffffffffu, 0, 0);
-  {
-    const int v = lane < wid ? S.wsum2[lane] : 0;
-    eq_before = __reduce_add_sync(0xffffffffu, v);
-  }
-  const int take_eq = max(0, min(eq, need_eq - eq_before));
-  __syncthreads();
-  if (lane == 0) S.wsum2[wid] = take_eq;
-  __syncthreads();
-  int out_before;
-  {
-    const int v = lane < wid ? S.wsum[lane] + S.wsum2[lane] : 0;
-    out_before = __reduce_add_sync(0xffffffffu, v);
-  }
-  int32_t* o = out + (int64_t)tok * k_out;
-  int written = out_before, eq_taken = 0;
-  for (int b0 = lo; b0 < hi; b0 += 32 * 8) {
-    uint32_t k8[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) k8[u] = key_at(sc, b0 + u * 32 + lane, hi);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = b0 + u * 32 + lane;
-      const uint32_t key = k8[u];
-      const bool g = key != 0u && (take_all || key > T);
-      const bool e = !take_all && key != 0u && key == T;
-      const uint32_t em = __ballot_sync(0xffffffffu, e);
-      const int e_rank = __popc(em & ((1u << lane) - 1u));
-      const bool sel = g || (e && eq_taken + e_rank < take_eq);
-      const uint32_t sm = __ballot_sync(0xffffffffu, sel);
-      if (sel) o[written + __popc(sm & ((1u << lane) - 1u))] = sel_id(mode, i, pool_row);
-      written += __popc(sm);
-      eq_taken = min(take_eq, eq_taken + __popc(em));
+  gt = __reduce_add_sync(0xffffffffu, lane < kSelWarps ? red[0][lane] : 0);
+  eq = __reduce_add_sync(0xffffffffu, lane < kSelWarps ? red[1][lane] : 0);
+  int run_out = 0, run_eq = 0;  // selections and ties in the group's CTAs before this one
+  if (G) {
+    if (threadIdx.x == 0) {
+      G->cta_gt[s] = gt;
+      G->cta_eq[s] = eq;
+    }
+    if (!group_barrier(&G->bar, S * ++n_bar, P.wait_ns, P.status, &flag_s)) return;
+    for (int c = 0; c < s; ++c) {
+      const int e = __ldcg(&G->cta_eq[c]);
+      run_out += __ldcg(&G->cta_gt[c]) + max(0, min(e, need_eq - run_eq));
+      run_eq += e;
     }
   }
-  __syncthreads();
-  for (int j = k_eff + threadIdx.x; j < k_out; j += kSel2Threads) o[j] = -1;
-  if (threadIdx.x == 0) out_n[tok] = k_eff;
+  int32_t* o = P.out + g * P.k_out;
+  for (int t = lo; t < hi; t += kSelTile) {
+    uint32_t k[kSelPer];
+    if (t == lo) {
+#pragma unroll
+      for (int j = 0; j < kSelPer; ++j) k[j] = k0[j];
+    } else {
+      sel_load_tile(sc, t, hi, k);
+    }
+    int wg = 0, we = 0;
+#pragma unroll
+    for (int j = 0; j < kSelPer; ++j) {
+      wg += __popc(__ballot_sync(0xffffffffu, is_gt(k[j])));
+      we += __popc(__ballot_sync(0xffffffffu, is_eq(k[j])));
+    }
+    if (lane == 0) {
+      wgt[wid] = wg;
+      weq[wid] = we;
+    }
+    __syncthreads();
+    // selections and ties of the warps before this one in the tile
+    int out_before = run_out, eq_before = run_eq;
+    for (int w = 0; w < wid; ++w) {
+      out_before += wgt[w] + max(0, min(weq[w], need_eq - eq_before));
+      eq_before += weq[w];
+    }
+    int written = out_before, ties = eq_before;
+    const int base = t + wid * kSelWarpSpan + lane;
+#pragma unroll
+    for (int j = 0; j < kSelPer; ++j) {
+      const bool gsel = is_gt(k[j]);
+      const bool e = is_eq(k[j]);
+      const uint32_t em = __ballot_sync(0xffffffffu, e);
+      const int e_rank = ties + __popc(em & ((1u << lane) - 1u));
+      const bool take = gsel || (e && e_rank < need_eq);
+      const uint32_t sm = __ballot_sync(0xffffffffu, take);
+      if (take) o[written + __popc(sm & ((1u << lane) - 1u))] = sel_id(P.mode, base + j * 32, pool_row);
+      written += __popc(sm);
+      ties += __popc(em);
+    }
+    for (int w = 0; w < kSelWarps; ++w) {  // the tile's totals
+      run_out += wgt[w] + max(0, min(weq[w], need_eq - run_eq));
+      run_eq += weq[w];
+    }
+    __syncthreads();
+  }
+  if (s == 0) {
+    for (int j = k_eff + threadIdx.x; j < P.k_out; j += kSelThreads) o[j] = -1;
+    if (threadIdx.x == 0) P.out_n[g] = k_eff;
+  }
 }
 
 }  // namespace csa2

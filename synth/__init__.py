@@ -1,4 +1,4 @@
-"""Seeded synthetic inputs shared by the tests, the oracle checks and the benchmark.
+"""Seeded synthetic inputs shared by the tests, the CPU reference checks and the benchmark.
 
 Every element is a pure function of (seed, stream, row, col) defined in
 ``csa2_synth.h`` and produced bit-identically on the host (``libsynth_host.so``)

@@ -138,7 +138,7 @@ class Workload:
         ps = self.cfg.page_size
         return self.page_table[b][pos // ps].astype(np.int64) * ps + pos % ps
 
-    # --- host views used by the oracle checks ------------------------------
+    # --- host views used by the CPU reference checks ------------------------------
     def iq_f32(self, layer: int, tok: int) -> np.ndarray:
         c = self.cfg
         return self.iq[layer].rows_f32(0, tok, 1).reshape(c.H_I, c.d_I)
