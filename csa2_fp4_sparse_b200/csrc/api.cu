@@ -333,12 +333,13 @@ int launch_attend_layers(const csa2_query_batch* qb, int q_dtype, int Hq, const 
   float* part_ml = static_cast<float*>(c.take((size_t)slots * Hq * 2 * 4));
   int* done = static_cast<int*>(c.take((size_t)qb->n_tok * kMaxAttLayers * 4));
   if (use_attend_tc(D, Hq, q_dtype)) {
-    // 128-row chunks; with fewer than 148 (token, layer) pairs one token's
-    // chunks are spread over up to 4 CTAs, whose partials the last one merges
-    const int chunks = (K + 127) / 128 + (swa ? (swa->window + 127) / 128 : 0);
+    // 64-row chunks; with fewer than 148 (token, layer) pairs one token's
+    // chunks are spread over up to 4 CTAs (one wave of one CTA per SM), whose
+    // partials the last one merges
+    const int chunks = (K + 63) / 64 + (swa ? (swa->window + 63) / 64 : 0);
     const int64_t pairs = (int64_t)qb->n_tok * n_layers;
     int nsplit = 1;
-    if (pairs < 148) nsplit = (int)std::min<int64_t>(std::min(chunks, 4), (148 + pairs - 1) / pairs);
+    if (pairs < 148) nsplit = (int)std::max<int64_t>(1, std::min<int64_t>(std::min(chunks, 4), 148 / pairs));
     if (nsplit > 1) {
       if (int rc = cuda_check(cudaMemsetAsync(done, 0, (size_t)pairs * 4, st), "clear split counters")) return rc;
     }

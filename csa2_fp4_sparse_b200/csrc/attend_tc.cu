@@ -9,35 +9,45 @@
 //         and, when given, the window rows e4m3(c_t) * s_t
 //   o_h = sum_t softmax(z)_t * v_t      (one softmax over both sets)
 //
-// One CTA per (query token, split); each walks its 128-row chunks of the key
-// set.  Per chunk:
-//   1. all 8 warps gather the chunk's rows and dequantise them exactly to
-//      fp16 (E2M1 x E4M3 products, or E4M3 window codes) into a 128B-swizzled
-//      shared tile [64-element d-block][row][128 B];
-//   2. one thread issues S^T = K q^T on tcgen05 (kind::f16, M = 128 rows,
-//      N = heads, K = D) into TMEM;
-//   3. warps 0..3 (one row each) scale and mask S^T, reduce per-head maxima and
-//      sums across rows with a halving shuffle transpose, keep a running
-//      (log2) max that only moves when a chunk exceeds it by more than 2^8
-//      (then the TMEM output accumulator is rescaled), and write
-//      P = 2^(z - m) as fp16 rows into shared memory (window rows carry their
-//      per-token scale into P);
-//   4. one thread issues O^T += V^T P^T (M = 128 latent dims per tile, N =
-//      heads, K = 128 rows) reading the same dequantised tile as V.
-// The epilogue divides by the row sum and writes the output (or the split's
-// unnormalised partial with its max and sum for the merge kernel).
+// One CTA per (split, query token, layer) walks its 64-row chunks of the key
+// set through a warp-specialised pipeline with two shared-memory K/V tiles:
+//   warps 4..11  loaders: gather the chunk's rows (codes of the next chunk are
+//                already in flight while the current one is converted) and
+//                dequantise them exactly to fp16 (E2M1 x E4M3 products, or
+//                E4M3 window codes) into a 128B-swizzled tile
+//                [64-element d-block][row][128 B];
+//   warp 12      issues S = Q K^T on tcgen05 (kind::f16, M = 64 heads, N = 64
+//                rows, K = D) into one of two TMEM score buffers;
+//   warps 0..3   softmax, one thread per head (M = 64 keeps head h in TMEM lane
+//                32*(h/16) + h%16): running (log2) max that only moves when a
+//                chunk exceeds it by more than 2^8 (then the output
+//                accumulator is rescaled), P = 2^(z - m) written as fp16 rows
+//                [head][row] (window rows carry their per-token scale into P);
+//   warp 13      issues O^T += V^T P^T (M = 128 latent dims per tile, N =
+//                heads, K = 64 rows) reading the same tile as V; its commit
+//                frees the tile and the P buffer.
+// The epilogue divides by the row sum, stages the output in shared memory and
+// writes it with 16-byte stores (or the split's unnormalised partial with its
+// max and sum; the last split of a token merges them).  Every wait is bounded.
 #include "internal.h"
 #include "tc_common.cuh"
 
 namespace csa2 {
 namespace attend_tc {
 
-constexpr int kRows = 128;
-constexpr int kThreads = 256;
+constexpr int kRows = 64;       // rows per chunk (MMA N of S, K of PV)
+constexpr int kMq = 64;         // MMA M of S: heads, padded to 64
+constexpr int kSoftWarps = 4;   // warps 0..3
+constexpr int kLoadWarps = 8;   // warps 4..11
+constexpr int kWarpS = 12;      // S issuer
+constexpr int kWarpPV = 13;     // PV issuer
+constexpr int kThreads = 448;
+constexpr int kLoadThreads = kLoadWarps * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;  // P stays <= 2^8 between rescales (fp16-safe)
 
 constexpr int kMaxLayers = 32;  // layers attended in one launch (grid.z), each with its own index list
+constexpr int kMaxRows = 2048;  // K: selected rows per query token
 
 struct LayerIO {
   const int32_t* idx;    // [T][K] selected Main KV positions of this layer's selector
@@ -67,78 +77,64 @@ struct Params {
 
 template <int D, int HQ, bool QLO>
 struct Layout {
-  static constexpr int kKB = D / 64;   // 64-element d-blocks
-  static constexpr int kMT = D / 128;  // PV M tiles
-  static constexpr int kPRow = HQ * 2; // bytes per P row
-  static constexpr uint32_t kOffK = 0;
-  static constexpr uint32_t kOffQ = kOffK + kRows * D * 2;
-  static constexpr uint32_t kOffQlo = kOffQ + HQ * D * 2;
-  static constexpr uint32_t kOffP = kOffQlo + (QLO ? HQ * D * 2 : 0);
-  static constexpr uint32_t kOffRed = kOffP + kRows * kPRow;     // [4][HQ] f32
-  static constexpr uint32_t kOffM = kOffRed + 4 * HQ * 4;        // running max (log2) [HQ]
-  static constexpr uint32_t kOffL = kOffM + HQ * 4;              // running sum [HQ]
-  static constexpr uint32_t kOffRs = kOffL + HQ * 4;             // row scale [128] f32
-  static constexpr uint32_t kOffValid = kOffRs + kRows * 4;      // row valid [128] i32
-  static constexpr uint32_t kOffRows = kOffValid + kRows * 4;    // gathered row index [128] i64
-  static constexpr uint32_t kOffMu = kOffRows + kRows * 8;       // max used for this chunk [HQ]
-  static constexpr uint32_t kOffCorr = kOffMu + HQ * 4;          // rescale factor [HQ]
-  static constexpr uint32_t kOffBar = kOffCorr + HQ * 4;         // 3 mbarriers (S, PV, drain)
-  static constexpr uint32_t kOffMisc = kOffBar + 24;             // tmem base, abort, rescale flag
+  static constexpr int kKB = D / 64;                    // 64-element d-blocks
+  static constexpr int kMT = D / 128;                   // PV M tiles
+  static constexpr int kUnitsRow = D / 32;              // 32-element units per row
+  static constexpr int kPer = kRows * kUnitsRow / kLoadThreads;  // units per loader thread per chunk
+  static constexpr uint32_t kTile = kRows * D * 2;      // fp16 K/V tile
+  // Q [kb][HQ][128 B]; the S MMA reads kMq rows per d-block, so the last
+  // d-block's rows past HQ land in a pad inside the region
+  static constexpr uint32_t kQBytes = HQ * D * 2 + (kMq - HQ) * 128;
+  static constexpr uint32_t kPBytes = HQ * kRows * 2;   // P [head][row] fp16
+  static constexpr uint32_t kOffTile = 0;               // [2][kTile]
+  static constexpr uint32_t kOffQ = kOffTile + 2 * kTile;
+  static constexpr uint32_t kOffQlo = kOffQ + (kQBytes + 1023) / 1024 * 1024;
+  static constexpr uint32_t kOffP = kOffQlo + (QLO ? (kQBytes + 1023) / 1024 * 1024 : 0);  // [2][kPBytes]
+  static constexpr uint32_t kOffRows = kOffP + 2 * ((kPBytes + 1023) / 1024 * 1024);       // [kMaxRows] i32 cache rows
+  static constexpr uint32_t kOffRs = kOffRows + kMaxRows * 4;                              // [2][kRows] f32
+  static constexpr uint32_t kOffCorr = kOffRs + 2 * kRows * 4;  // [kMq] f32
+  static constexpr uint32_t kOffL = kOffCorr + kMq * 4;         // [kMq] f32 final row sums
+  static constexpr uint32_t kOffM = kOffL + kMq * 4;            // [kMq] f32 final maxima (log2)
+  static constexpr uint32_t kOffBar = kOffM + kMq * 4;          // 9 mbarriers
+  static constexpr uint32_t kOffMisc = kOffBar + 9 * 8;         // tmem base, abort, last-split flag
   static constexpr uint32_t kBytes = kOffMisc + 16 + 1024;
-  static constexpr int kChains = kKB < 4 ? kKB : 4;  // S = K q^T split over this many issuing threads
-  static constexpr uint32_t kColS = 0;                // chain c accumulates at kColS + c * HQ
-  static constexpr uint32_t kColO = 256;              // O^T tile mt at kColO + mt * HQ
-  static_assert(kChains * HQ <= 256 && kMT * HQ <= 256, "TMEM budget");
+  static constexpr uint32_t kColS = 0;    // score buffer b at kColS + b * kRows
+  static constexpr uint32_t kColO = 256;  // O^T tile mt at kColO + mt * HQ
+  static_assert(kPer >= 1 && kRows * kUnitsRow % kLoadThreads == 0, "loader unit split");
+  static_assert(kMT * HQ <= 256 && 2 * kRows <= 256, "TMEM budget");
+  static_assert((uint32_t)HQ * D * 4 <= 2 * kTile, "epilogue staging fits in the tiles");
 };
+
+// swizzled byte offset of 16-byte chunk c of row r for 128-byte rows
+__device__ __forceinline__ uint32_t swz128(uint32_t r, uint32_t c) { return r * 128 + ((c ^ (r & 7)) << 4); }
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// swizzled byte offset of 16-byte chunk c of row r for rows of `rb` bytes
-__device__ __forceinline__ uint32_t swz(uint32_t r, uint32_t c, uint32_t rb) {
-  uint32_t x = rb == 128 ? (r & 7) : rb == 64 ? ((r >> 1) & 3) : ((r >> 2) & 1);
-  return r * rb + ((c ^ x) << 4);
+// named barrier over the softmax warps with an OR over `pred`
+__device__ __forceinline__ bool soft_sync_or(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.or.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred)
+      : "memory");
+  return r != 0;
 }
 
-// reduce v[0..N) across the 32 lanes of a warp by repeated halving; afterwards
-// lane L holds, in v[0..max(1,N/32)), the warp-wide result for heads
-// N >= 32: 2L.. (N/32 of them, here N = 64 -> heads 2L, 2L+1);
-// N < 32: head L / (32/N) (lanes sharing a head hold the same value)
-template <int N, bool MAX>
-__device__ __forceinline__ void warp_transpose_reduce(float (&v)[N], int lane) {
-  int size = N;
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
-    if (size > 1) {
-      const bool up = (lane & o) != 0;
-      const int half = size / 2;
-#pragma unroll
-      for (int i = 0; i < N / 2; ++i) {
-        if (i < half) {
-          float send = up ? v[i] : v[i + half];
-          float keep = up ? v[i + half] : v[i];
-          float got = __shfl_xor_sync(0xffffffffu, send, o);
-          v[i] = MAX ? fmaxf(keep, got) : keep + got;
-        }
-      }
-      size = half;
-    } else {
-      float got = __shfl_xor_sync(0xffffffffu, v[0], o);
-      v[0] = MAX ? fmaxf(v[0], got) : v[0] + got;
-    }
-  }
-}
-
-template <int HQ>
-__device__ __forceinline__ int reduced_head(int lane, int i) {
-  if constexpr (HQ >= 32) {
-    return lane * (HQ / 32) + i;
-  } else {
-    return lane / (32 / HQ);
-  }
-}
+// one loader thread's share of a chunk: kPer units of 32 elements
+template <int kPer>
+struct Pref {
+  uint4 c[kPer];     // FP4 codes (16 B), or the first 16 of a window unit's 32 FP8 codes
+  uint32_t s[kPer];  // E4M3 scale byte of an FP4 unit
+  float rs[kPer];    // softmax row scale (units starting a row): 1 sparse, s_t window, -1 no row
+  int32_t wrow[kPer];  // window unit: its row (the second 16 bytes are read at conversion)
+};
 
 template <int D, int HQ, bool QLO>
 __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant__ Params P) {
@@ -146,18 +142,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t bar_s = sbase + Ly::kOffBar, bar_pv = bar_s + 8, bar_drain = bar_s + 16;
+  const uint32_t bar_kv_full = sbase + Ly::kOffBar;       // [2] loaders -> S issuer (count kLoadWarps)
+  const uint32_t bar_kv_empty = bar_kv_full + 16;         // [2] PV commit -> loaders, softmax rescale, epilogue
+  const uint32_t bar_s_full = bar_kv_empty + 16;          // [2] S commit -> softmax
+  const uint32_t bar_p_full = bar_s_full + 16;            // [2] softmax -> PV issuer (count kSoftWarps)
+  const uint32_t bar_drain = bar_p_full + 16;             // issuers' final commits (count 2)
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(smem + Ly::kOffMisc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + Ly::kOffMisc + 4);
-  volatile int* any_rescale = reinterpret_cast<volatile int*>(smem + Ly::kOffMisc + 8);
-  float* mu_s = reinterpret_cast<float*>(smem + Ly::kOffMu);
+  float* rs_s = reinterpret_cast<float*>(smem + Ly::kOffRs);
   float* corr_s = reinterpret_cast<float*>(smem + Ly::kOffCorr);
-  float* red = reinterpret_cast<float*>(smem + Ly::kOffRed);
-  float* m_s = reinterpret_cast<float*>(smem + Ly::kOffM);
   float* l_s = reinterpret_cast<float*>(smem + Ly::kOffL);
-  float* rs = reinterpret_cast<float*>(smem + Ly::kOffRs);
-  int* valid = reinterpret_cast<int*>(smem + Ly::kOffValid);
-  int64_t* rows_s = reinterpret_cast<int64_t*>(smem + Ly::kOffRows);
+  float* m_s = reinterpret_cast<float*>(smem + Ly::kOffM);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tok = blockIdx.y, split = blockIdx.x, nsplit = gridDim.x, layer = blockIdx.z;
@@ -167,11 +162,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
   const int64_t p = __ldg(P.qb.tok_pos + tok);
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_s, Ly::kChains);
-    mbar_init(bar_pv, Ly::kMT);
-    mbar_init(bar_drain, 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_kv_full + 8 * i, kLoadWarps);
+      mbar_init(bar_kv_empty + 8 * i, 1);
+      mbar_init(bar_s_full + 8 * i, 1);
+      mbar_init(bar_p_full + 8 * i, kSoftWarps);
+    }
+    mbar_init(bar_drain, 2);
     *abort = 0;
-    *any_rescale = 0;
     tc::fence_barrier_init();
   }
   if (warp == 0) {
@@ -179,65 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
     tc::tmem_relinquish();
     tc::fence_before_sync();
   }
-  for (int h = threadIdx.x; h < HQ; h += kThreads) {
-    m_s[h] = -INFINITY;
-    l_s[h] = 0.0f;
-  }
-  // query -> fp16 (K-major, 128B swizzle); f32 queries also keep the residual.
-  // Loads are issued in batches of 8 independent 16-byte reads per thread.
-  {
-    constexpr int kUnitsQ = HQ * D / 8;  // 8 consecutive d per unit
-    constexpr int kBatch = 8;
-    for (int e0 = 0; e0 < kUnitsQ; e0 += kThreads * kBatch) {
-      float f[kBatch][8];
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int e = e0 + u * kThreads + threadIdx.x;
-        if (e >= kUnitsQ) continue;
-        const int h = e / (D / 8), c8 = e % (D / 8);
-        const int64_t off = ((int64_t)tok * HQ + h) * D + c8 * 8;
-        if (P.q_f32) {
-          const float4* s4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(io.q) + off);
-          float4 a = __ldg(s4), bb = __ldg(s4 + 1);
-          f[u][0] = a.x; f[u][1] = a.y; f[u][2] = a.z; f[u][3] = a.w;
-          f[u][4] = bb.x; f[u][5] = bb.y; f[u][6] = bb.z; f[u][7] = bb.w;
-        } else {
-          uint4 w4 = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(io.q) + off));
-          const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            f[u][2 * k] = __uint_as_float(ww[k] << 16);
-            f[u][2 * k + 1] = __uint_as_float(ww[k] & 0xFFFF0000u);
-          }
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int e = e0 + u * kThreads + threadIdx.x;
-        if (e >= kUnitsQ) continue;
-        const int h = e / (D / 8), c8 = e % (D / 8);
-        const int kb = c8 / 8, c = c8 % 8;
-        uint4 hi, lo;
-        uint32_t* hp = &hi.x;
-        uint32_t* lp = &lo.x;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          __half2 h2 = __floats2half2_rn(f[u][2 * k], f[u][2 * k + 1]);
-          hp[k] = *reinterpret_cast<uint32_t*>(&h2);
-          float2 back = __half22float2(h2);
-          lp[k] = pack_half2(f[u][2 * k] - back.x, f[u][2 * k + 1] - back.y);
-        }
-        const uint32_t o = kb * (HQ * 128) + swz(h, c, 128);
-        *reinterpret_cast<uint4*>(smem + Ly::kOffQ + o) = hi;
-        if (QLO) *reinterpret_cast<uint4*>(smem + Ly::kOffQlo + o) = lo;
-      }
-    }
-  }
-  tc::fence_proxy_async_smem();
-  __syncthreads();
-  tc::fence_after_sync();
-  const uint32_t tmem = *tmem_holder;
-
+  // this CTA's chunks: c = split + nsplit * i (sparse chunks first, then window chunks)
   const int n_sel = min(__ldg(io.idx_n + tok), P.K);
   const int n_sp = (n_sel + kRows - 1) / kRows;
   int64_t w_lo = 0;
@@ -248,382 +188,513 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
     n_w = (int)(p - w_lo + 1);
   }
   const int n_chunks = n_sp + (n_w + kRows - 1) / kRows;
-  const uint32_t idesc_s = tc::idesc_f16(128, HQ, 0, 0);
-  const uint32_t idesc_pv = tc::idesc_f16(128, HQ, 1, 1);
-  const tc::SmemLayout p_sw = HQ == 64 ? tc::kSwizzle128B : HQ == 32 ? tc::kSwizzle64B : tc::kSwizzle32B;
-
-  int it = 0;
-  for (int chunk = split; chunk < n_chunks; chunk += nsplit, ++it) {
-    if (it > 0) {  // the previous chunk's PV still reads the tile (thread 0 probes, the rest park)
-      if (threadIdx.x == 0 && !mbar_wait_bounded(bar_pv, (it - 1) & 1, P.wait_ns)) {
-        set_status(P.status, CSA2_ERR_TIMEOUT);
-        *abort = 1;
-      }
-      __syncthreads();
-      if (*abort) break;
-      tc::fence_after_sync();
+  const int n_mine = split < n_chunks ? (n_chunks - split + nsplit - 1) / nsplit : 0;
+  const int n_mine_sp = split < n_sp ? (n_sp - split + nsplit - 1) / nsplit : 0;
+  int32_t* rows_s = reinterpret_cast<int32_t*>(smem + Ly::kOffRows);
+  // the cache rows of this CTA's sparse chunks (index list, then page table),
+  // every load of a stage in flight together
+  constexpr int kRowPer = (kMaxRows + kThreads - 1) / kThreads;
+  int32_t tv[kRowPer];
+#pragma unroll
+  for (int u = 0; u < kRowPer; ++u) {
+    const int e = threadIdx.x + u * kThreads;
+    tv[u] = -2;  // no entry
+    if (e < n_mine_sp * kRows) {
+      const int j = (split + (e / kRows) * nsplit) * kRows + e % kRows;
+      tv[u] = j < n_sel ? __ldg(io.idx + (int64_t)tok * P.K + j) : -2;
     }
-    // ---- 1. gather + dequantise the chunk into the K/V tile
-    const bool swa_chunk = chunk >= n_sp;
-    // row addresses first (one index load per row), so the code loads below
-    // are independent of each other and all in flight together
-    if (threadIdx.x < kRows) {
-      const int r = threadIdx.x;
-      int64_t row = -1;
-      float scale_r = 1.0f;
-      if (!swa_chunk) {
-        const int j = chunk * kRows + r;
-        if (j < n_sel) {
-          const int32_t t = __ldg(io.idx + (int64_t)tok * P.K + j);
-          if (t >= 0 && t <= p) {
-            row = cache_row(P.kv, b, t);
-            if (row < 0 || row >= P.kv.n_rows) row = -1;
-          }
-          if (row < 0) set_status(P.status, CSA2_ERR_RANGE);
-        }
+  }
+  // query -> fp16 [kb][h][128 B] (K-major, 128B swizzle); f32 queries also
+  // keep the fp16 residual.  All threads, all loads in flight together.
+  {
+    constexpr int kUnitsQ = HQ * D / 8;  // 8 consecutive d per unit
+    constexpr int kQPer = (kUnitsQ + kThreads - 1) / kThreads;
+    constexpr int kQB = kQPer < 3 ? kQPer : 3;  // units in flight per batch
+#pragma unroll 1
+    for (int u0 = 0; u0 < kQPer; u0 += kQB) {
+    // raw query units: 8 bf16 (one uint4) or, with f32 queries (QLO), 8 f32
+    uint4 raw[kQB][QLO ? 2 : 1];
+#pragma unroll
+    for (int u = 0; u < kQB; ++u) {
+      const int e = (u0 + u) * kThreads + threadIdx.x;
+      if (e >= kUnitsQ) continue;
+      const int h = e / (D / 8), c8 = e % (D / 8);
+      const int64_t off = ((int64_t)tok * HQ + h) * D + c8 * 8;
+      if constexpr (QLO) {
+        const uint4* s4 = reinterpret_cast<const uint4*>(reinterpret_cast<const float*>(io.q) + off);
+        raw[u][0] = __ldg(s4);
+        raw[u][QLO ? 1 : 0] = __ldg(s4 + 1);
       } else {
-        const int64_t t = w_lo + (int64_t)(chunk - n_sp) * kRows + r;
-        if (t <= p) {
-          row = (int64_t)b * P.swa_cap + t % P.swa_cap;
-          scale_r = __ldg(io.swa_scale + row);
-        } else {
-          scale_r = 0.0f;
-        }
+        raw[u][0] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(io.q) + off));
       }
-      rows_s[r] = row;
-      valid[r] = row >= 0;
-      rs[r] = scale_r;
     }
-    __syncthreads();
-    if (!swa_chunk) {
-      constexpr int kUnits = D / 32;  // 16-byte code units (32 values, one scale) per row
-      constexpr int kPer = kRows * kUnits / kThreads;
-      uint4 cw[kPer];
-      uint32_t sb[kPer];
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int u = threadIdx.x + i * kThreads;
-        const int r = u / kUnits, g = u % kUnits;
-        const int64_t row = rows_s[r];
-        if (row >= 0) {
-          cw[i] = __ldg(reinterpret_cast<const uint4*>(P.kv.codes + row * (D / 2)) + g);
-          sb[i] = __ldg(P.kv.scales + row * (D / 32) + g);
-        } else {
-          cw[i] = make_uint4(0, 0, 0, 0);
-          sb[i] = 0;
-        }
-      }
+    for (int u = 0; u < kQB; ++u) {
+      const int e = (u0 + u) * kThreads + threadIdx.x;
+      if (e >= kUnitsQ) continue;
+      const int h = e / (D / 8), c8 = e % (D / 8);
+      const int kb = c8 / 8, c = c8 % 8;
+      float f[8];
+      if constexpr (QLO) {
+        const uint32_t ww[8] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w,
+                                raw[u][QLO ? 1 : 0].x, raw[u][QLO ? 1 : 0].y, raw[u][QLO ? 1 : 0].z,
+                                raw[u][QLO ? 1 : 0].w};
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int u = threadIdx.x + i * kThreads;
-        const int r = u / kUnits, g = u % kUnits;
-        const __half sh = __float2half_rn(e4m3_to_f32(sb[i]));
-        const __half2 s2 = __halves2half2(sh, sh);
-        const uint32_t words[4] = {cw[i].x, cw[i].y, cw[i].z, cw[i].w};
-        uint32_t outw[16];
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-#pragma unroll
-          for (int bb = 0; bb < 4; ++bb) {
-            uint32_t h2 = tc::e2m1x2_to_f16x2((words[k] >> (8 * bb)) & 0xFFu);
-            __half2 v = __hmul2(*reinterpret_cast<__half2*>(&h2), s2);
-            outw[k * 4 + bb] = *reinterpret_cast<uint32_t*>(&v);
-          }
-        // 32 values = d in [32g, 32g+32): d-block g/2, 16-byte chunks (g%2)*4 .. +4
-        const int kb = g / 2, c0 = (g % 2) * 4;
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          *reinterpret_cast<uint4*>(smem + Ly::kOffK + kb * (kRows * 128) + swz(r, c0 + k, 128)) =
-              make_uint4(outw[4 * k], outw[4 * k + 1], outw[4 * k + 2], outw[4 * k + 3]);
-      }
-    } else {
-      constexpr int kUnits = D / 16;  // 16 FP8 codes per unit
-      constexpr int kPer = kRows * kUnits / kThreads;
-      uint4 cw[kPer];
-#pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int u = threadIdx.x + i * kThreads;
-        const int r = u / kUnits, g = u % kUnits;
-        const int64_t row = rows_s[r];
-        cw[i] = row >= 0 ? __ldg(reinterpret_cast<const uint4*>(io.swa_codes + row * D) + g) : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int u = threadIdx.x + i * kThreads;
-        const int r = u / kUnits, g = u % kUnits;
-        const uint32_t words[4] = {cw[i].x, cw[i].y, cw[i].z, cw[i].w};
-        uint32_t outw[8];
+        for (int k = 0; k < 8; ++k) f[k] = __uint_as_float(ww[k]);
+      } else {
+        const uint32_t ww[4] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          outw[2 * k] = tc::e4m3x2_to_f16x2(words[k] & 0xFFFFu);
-          outw[2 * k + 1] = tc::e4m3x2_to_f16x2(words[k] >> 16);
+          f[2 * k] = __uint_as_float(ww[k] << 16);
+          f[2 * k + 1] = __uint_as_float(ww[k] & 0xFFFF0000u);
         }
-        const int kb = g / 4, c0 = (g % 4) * 2;
-#pragma unroll
-        for (int k = 0; k < 2; ++k)
-          *reinterpret_cast<uint4*>(smem + Ly::kOffK + kb * (kRows * 128) + swz(r, c0 + k, 128)) =
-              make_uint4(outw[4 * k], outw[4 * k + 1], outw[4 * k + 2], outw[4 * k + 3]);
       }
-    }
-    tc::fence_proxy_async_smem();
-    __syncthreads();
-
-    // ---- 2. S^T = K q^T, the K chain split over kChains issuing threads
-    //         (chain c: d-blocks c, c + kChains, ...; its own accumulator)
-    if (warp == 0 && lane < Ly::kChains) {
-      tc::fence_after_sync();
-      const int c = lane;
-#pragma unroll 1
-      for (int kb = c; kb < Ly::kKB; kb += Ly::kChains)
+      uint4 hi, lo;
+      uint32_t* hp = &hi.x;
+      uint32_t* lp = &lo.x;
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t ad = tc::smem_desc(sbase + Ly::kOffK + kb * (kRows * 128) + ks * 32, 16, 1024, tc::kSwizzle128B);
-          const uint64_t bd = tc::smem_desc(sbase + Ly::kOffQ + kb * (HQ * 128) + ks * 32, 16, 1024, tc::kSwizzle128B);
-          tc::mma_f16(tmem + Ly::kColS + c * HQ, ad, bd, idesc_s, (kb != c || ks) ? 1u : 0u);
-          if (QLO) {
-            const uint64_t bl =
-                tc::smem_desc(sbase + Ly::kOffQlo + kb * (HQ * 128) + ks * 32, 16, 1024, tc::kSwizzle128B);
-            tc::mma_f16(tmem + Ly::kColS + c * HQ, ad, bl, idesc_s, 1u);
+      for (int k = 0; k < 4; ++k) {
+        __half2 h2 = __floats2half2_rn(f[2 * k], f[2 * k + 1]);
+        hp[k] = *reinterpret_cast<uint32_t*>(&h2);
+        const float2 back = __half22float2(h2);
+        lp[k] = pack_half2(f[2 * k] - back.x, f[2 * k + 1] - back.y);
+      }
+      const uint32_t o = kb * (HQ * 128) + swz128(h, c);
+      *reinterpret_cast<uint4*>(smem + Ly::kOffQ + o) = hi;
+      if (QLO) *reinterpret_cast<uint4*>(smem + Ly::kOffQlo + o) = lo;
+    }
+    }
+  }
+  {
+    int64_t pg[kRowPer];
+#pragma unroll
+    for (int u = 0; u < kRowPer; ++u) {
+      const int32_t t = tv[u];
+      pg[u] = 0;
+      if (t >= 0 && t <= p)
+        pg[u] = P.kv.page_table ? (int64_t)__ldg(P.kv.page_table + (int64_t)b * P.kv.max_pages + t / P.kv.page_size)
+                                : __ldg(P.kv.seq_base + b);
+    }
+#pragma unroll
+    for (int u = 0; u < kRowPer; ++u) {
+      const int e = threadIdx.x + u * kThreads;
+      const int32_t t = tv[u];
+      if (t == -2) {
+        if (e < n_mine_sp * kRows) rows_s[e] = -1;
+        continue;
+      }
+      int64_t row = -1;
+      if (t >= 0 && t <= p) {
+        row = P.kv.page_table ? pg[u] * P.kv.page_size + t % P.kv.page_size : pg[u] + t;
+        if (row < 0 || row >= P.kv.n_rows) row = -1;
+      }
+      if (row < 0) set_status(P.status, CSA2_ERR_RANGE);
+      rows_s[e] = (int32_t)row;
+    }
+  }
+  tc::fence_proxy_async_smem();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp >= kSoftWarps && warp < kSoftWarps + kLoadWarps) {
+    // ------------------------------------------------------------ loaders
+    const int lt = threadIdx.x - kSoftWarps * 32;  // 0..255
+    Pref<Ly::kPer> cur, nxt;
+    // codes (and, for units that start a row, the softmax row scale) of local chunk i
+    auto load_codes = [&](int i, Pref<Ly::kPer>& pf) {
+      const int c = split + i * nsplit;
+      const bool sparse = c < n_sp;
+#pragma unroll
+      for (int k = 0; k < Ly::kPer; ++k) {
+        const int u = lt + k * kLoadThreads;
+        const int r = u / Ly::kUnitsRow, g = u % Ly::kUnitsRow;
+        int64_t row = -1;
+        if (sparse) {
+          row = rows_s[i * kRows + r];
+        } else {
+          const int64_t t = w_lo + (int64_t)(c - n_sp) * kRows + r;
+          if (t <= p) row = (int64_t)b * P.swa_cap + t % P.swa_cap;
+        }
+        pf.c[k] = make_uint4(0, 0, 0, 0);
+        pf.s[k] = 0;
+        pf.rs[k] = -1.0f;
+        pf.wrow[k] = (int32_t)row;
+        if (row < 0) continue;
+        if (sparse) {
+          pf.c[k] = __ldg(reinterpret_cast<const uint4*>(P.kv.codes + row * (D / 2)) + g);
+          pf.s[k] = __ldg(P.kv.scales + row * (D / 32) + g);
+          pf.rs[k] = 1.0f;
+        } else {
+          pf.c[k] = __ldg(reinterpret_cast<const uint4*>(io.swa_codes + row * D) + 2 * g);
+          if (g == 0) pf.rs[k] = __ldg(io.swa_scale + row);
+        }
+      }
+    };
+    if (n_mine > 0) load_codes(0, cur);
+    for (int i = 0; i < n_mine; ++i) {
+      const int c = split + i * nsplit, bf = i & 1;
+      // the next chunk's codes go in flight before this chunk is converted
+      if (i + 1 < n_mine) load_codes(i + 1, nxt);
+      bool ok = __shfl_sync(0xffffffffu, (int)!*abort, 0) != 0;
+      // the tile is free once PV(i - 2) has completed
+      if (i >= 2 && ok) {
+        if (!mbar_wait_warp(bar_kv_empty + 8 * bf, ((i >> 1) - 1) & 1, P.wait_ns)) {
+          if (lane == 0) {
+            set_status(P.status, CSA2_ERR_TIMEOUT);
+            *abort = 1;
           }
+          ok = false;
         }
-      tc::commit(bar_s);
+      }
+      if (ok) {
+        uint8_t* tile = smem + Ly::kOffTile + bf * Ly::kTile;
+        const bool sparse = c < n_sp;
+#pragma unroll
+        for (int k = 0; k < Ly::kPer; ++k) {
+          const int u = lt + k * kLoadThreads;
+          const int r = u / Ly::kUnitsRow, g = u % Ly::kUnitsRow;
+          // 32 values = d in [32g, 32g+32): d-block g/2, 16-byte chunks (g%2)*4 .. +4
+          const int kb = g / 2, c0 = (g % 2) * 4;
+          uint32_t outw[16];
+          if (sparse) {
+            const __half sh = __float2half_rn(e4m3_to_f32(cur.s[k]));
+            const __half2 s2 = __halves2half2(sh, sh);
+            const uint32_t words[4] = {cur.c[k].x, cur.c[k].y, cur.c[k].z, cur.c[k].w};
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+#pragma unroll
+              for (int bb = 0; bb < 4; ++bb) {
+                uint32_t h2 = tc::e2m1x2_to_f16x2((words[w] >> (8 * bb)) & 0xFFu);
+                __half2 v = __hmul2(*reinterpret_cast<__half2*>(&h2), s2);
+                outw[w * 4 + bb] = *reinterpret_cast<uint32_t*>(&v);
+              }
+          } else {
+            const uint4 c1 = cur.wrow[k] >= 0
+                                 ? __ldg(reinterpret_cast<const uint4*>(io.swa_codes + (int64_t)cur.wrow[k] * D) + 2 * g + 1)
+                                 : make_uint4(0, 0, 0, 0);
+            const uint32_t words[8] = {cur.c[k].x, cur.c[k].y, cur.c[k].z, cur.c[k].w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+              outw[2 * w] = tc::e4m3x2_to_f16x2(words[w] & 0xFFFFu);
+              outw[2 * w + 1] = tc::e4m3x2_to_f16x2(words[w] >> 16);
+            }
+          }
+#pragma unroll
+          for (int w = 0; w < 4; ++w)
+            *reinterpret_cast<uint4*>(tile + kb * (kRows * 128) + swz128(r, c0 + w)) =
+                make_uint4(outw[4 * w], outw[4 * w + 1], outw[4 * w + 2], outw[4 * w + 3]);
+          if (g == 0) rs_s[bf * kRows + r] = cur.rs[k];  // one thread per row
+        }
+        tc::fence_proxy_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar_kv_full + 8 * bf);
+      cur = nxt;
     }
+  } else if (warp == kWarpS) {
+    // ------------------------------------------------------------ S = Q K^T
+    const uint32_t idesc = tc::idesc_f16(kMq, kRows, 0, 0);
+    for (int i = 0; i < n_mine; ++i) {
+      const int bf = i & 1;
+      if (lane == 0 && !*abort) {
+        if (!mbar_wait_bounded(bar_kv_full + 8 * bf, (i >> 1) & 1, P.wait_ns)) {
+          set_status(P.status, CSA2_ERR_TIMEOUT);
+          *abort = 1;
+        } else {
+          tc::fence_after_sync();
+          const uint32_t tile = sbase + Ly::kOffTile + bf * Ly::kTile;
+#pragma unroll 1
+          for (int kb = 0; kb < Ly::kKB; ++kb)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t ad = tc::smem_desc(sbase + Ly::kOffQ + kb * (HQ * 128) + ks * 32, 16, 1024, tc::kSwizzle128B);
+              const uint64_t bd = tc::smem_desc(tile + kb * (kRows * 128) + ks * 32, 16, 1024, tc::kSwizzle128B);
+              tc::mma_f16(tmem + Ly::kColS + bf * kRows, ad, bd, idesc, (kb | ks) ? 1u : 0u);
+              if (QLO) {
+                const uint64_t al =
+                    tc::smem_desc(sbase + Ly::kOffQlo + kb * (HQ * 128) + ks * 32, 16, 1024, tc::kSwizzle128B);
+                tc::mma_f16(tmem + Ly::kColS + bf * kRows, al, bd, idesc, 1u);
+              }
+            }
+          tc::commit(bar_s_full + 8 * bf);
+        }
+      }
+      __syncwarp();
+    }
+    if (lane == 0) tc::commit(bar_drain);
     __syncwarp();
-
-    // ---- 3. softmax over the rows (warps 0..3: one row per thread)
-    if (warp < 4) {
-      if (!mbar_wait_warp(bar_s, it & 1, P.wait_ns)) {
-        set_status(P.status, CSA2_ERR_TIMEOUT);
-        *abort = 1;
+  } else if (warp == kWarpPV) {
+    // ------------------------------------------------------------ O^T += V^T P^T
+    const uint32_t idesc = tc::idesc_f16(128, HQ, 1, 0);
+    for (int i = 0; i < n_mine; ++i) {
+      const int bf = i & 1;
+      if (lane == 0 && !*abort) {
+        if (!mbar_wait_bounded(bar_p_full + 8 * bf, (i >> 1) & 1, P.wait_ns)) {
+          set_status(P.status, CSA2_ERR_TIMEOUT);
+          *abort = 1;
+        } else {
+          tc::fence_after_sync();
+          const uint32_t tile = sbase + Ly::kOffTile + bf * Ly::kTile;
+          const uint32_t pb = sbase + Ly::kOffP + bf * ((Ly::kPBytes + 1023) / 1024 * 1024);
+#pragma unroll 1
+          for (int mt = 0; mt < Ly::kMT; ++mt)
+#pragma unroll
+            for (int ks = 0; ks < kRows / 16; ++ks) {
+              const uint64_t ad =
+                  tc::smem_desc(tile + (2 * mt) * (kRows * 128) + ks * 2048, kRows * 128, 1024, tc::kSwizzle128B);
+              const uint64_t bd = tc::smem_desc(pb + ks * 32, 16, 1024, tc::kSwizzle128B);
+              tc::mma_f16(tmem + Ly::kColO + mt * HQ, ad, bd, idesc, (i > 0 || ks > 0) ? 1u : 0u);
+            }
+          tc::commit(bar_kv_empty + 8 * bf);
+        }
+      }
+      __syncwarp();
+    }
+    if (lane == 0) tc::commit(bar_drain);
+    __syncwarp();
+  } else if (warp < kSoftWarps) {
+    // ------------------------------------------------------------ softmax
+    // thread = head h = 16 * warp + lane (lanes 16..31 carry no head)
+    const int h = 16 * warp + lane;
+    const bool act = lane < 16 && h < HQ;
+    const uint32_t s_lane = tmem + ((uint32_t)(warp * 32) << 16);
+    const float zs = P.scale * kLog2e;
+    float m = -INFINITY, l = 0.0f;
+    for (int i = 0; i < n_mine; ++i) {
+      const int bf = i & 1;
+      bool ok = __shfl_sync(0xffffffffu, (int)!*abort, 0) != 0;
+      if (ok && !mbar_wait_warp(bar_s_full + 8 * bf, (i >> 1) & 1, P.wait_ns)) {
+        if (lane == 0) {
+          set_status(P.status, CSA2_ERR_TIMEOUT);
+          *abort = 1;
+        }
+        ok = false;
       }
       tc::fence_after_sync();
-      const int r = warp * 32 + lane;
-      const bool rv = valid[r] != 0;
-      const float zscale = P.scale * kLog2e * rs[r];  // log2-domain score scale (window rows: * s_t)
-      constexpr int kPer = HQ >= 32 ? HQ / 32 : 1;
-      const uint32_t s_addr = tmem + ((uint32_t)(warp * 32) << 16) + Ly::kColS;
-      // the chunk's scores (sum of the chains), scaled to the log2 domain
-      // (window rows: * s_t); invalid rows -inf
-      auto load_scores = [&](float (&z)[HQ]) {
+      const float* rsb = rs_s + bf * kRows;
+      const uint32_t s_col = s_lane + Ly::kColS + bf * kRows;
+      // pass 1: the chunk's maximum (log2 domain; window rows scaled by s_t)
+      float cm = -INFINITY;
+      if (ok) {
 #pragma unroll
-        for (int g = 0; g < HQ / 16; ++g) {
-          uint32_t v[Ly::kChains][16];
-#pragma unroll
-          for (int c = 0; c < Ly::kChains; ++c) tc::ld_32x32b_x16(s_addr + c * HQ + g * 16, v[c]);
+        for (int g = 0; g < kRows / 16; ++g) {
+          uint32_t v[16];
+          tc::ld_32x32b_x16(s_col + g * 16, v);
           tc::ld_wait();
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
-            float acc = __uint_as_float(v[0][k]);
-#pragma unroll
-            for (int c = 1; c < Ly::kChains; ++c) acc += __uint_as_float(v[c][k]);
-            z[g * 16 + k] = rv ? acc * zscale : -INFINITY;
+            const float rsj = rsb[g * 16 + k];
+            if (rsj >= 0.0f) cm = fmaxf(cm, __uint_as_float(v[k]) * (zs * rsj));
           }
         }
-      };
-      // per-head maximum of this chunk
-      {
-        float mx[HQ];
-        load_scores(mx);
-        warp_transpose_reduce<HQ, true>(mx, lane);
-#pragma unroll
-        for (int i = 0; i < kPer; ++i) red[warp * HQ + reduced_head<HQ>(lane, i)] = mx[i];
       }
-      tc::named_sync(1, 128);
       // running max: moves only when the chunk exceeds it by more than 2^8
-      if (threadIdx.x < HQ) {
-        const int h = threadIdx.x;
-        const float cm = fmaxf(fmaxf(red[h], red[HQ + h]), fmaxf(red[2 * HQ + h], red[3 * HQ + h]));
-        const float mo = m_s[h];
-        float mu = mo;
-        if (mo == -INFINITY || cm > mo + kRescaleLog2) mu = cm;
-        mu_s[h] = mu;
-        corr_s[h] = (mo == -INFINITY || mu == mo) ? 1.0f : exp2f(mo - mu);
-        if (mo != -INFINITY && mu != mo) *any_rescale = 1;
-      }
-      tc::named_sync(1, 128);
-      // rescale the output accumulator of earlier chunks (rare)
-      if (*any_rescale && it > 0) {
+      float mu = m;
+      if (m == -INFINITY || cm > m + kRescaleLog2) mu = cm;
+      const bool resc = act && m != -INFINITY && mu != m;
+      const float corr = resc ? exp2f(m - mu) : 1.0f;
+      if (act) corr_s[h] = corr;
+      const bool any = soft_sync_or(resc);  // also publishes corr_s
+      if (any && i > 0 && ok) {
+        // rescale the output accumulator of earlier chunks (rare): PV(i - 1)
+        // must have completed first
+        if (!mbar_wait_warp(bar_kv_empty + 8 * ((i - 1) & 1), ((i - 1) >> 1) & 1, P.wait_ns)) {
+          if (lane == 0) {
+            set_status(P.status, CSA2_ERR_TIMEOUT);
+            *abort = 1;
+          }
+        } else {
+          tc::fence_after_sync();
 #pragma unroll 1
-        for (int mt = 0; mt < Ly::kMT; ++mt)
+          for (int mt = 0; mt < Ly::kMT; ++mt)
 #pragma unroll
-          for (int g = 0; g < HQ / 16; ++g) {
-            const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16) + Ly::kColO + mt * HQ + g * 16;
-            uint32_t v[16];
-            tc::ld_32x32b_x16(ta, v);
-            tc::ld_wait();
+            for (int g = 0; g < HQ / 16; ++g) {
+              const uint32_t ta = s_lane + Ly::kColO + mt * HQ + g * 16;
+              uint32_t v[16];
+              tc::ld_32x32b_x16(ta, v);
+              tc::ld_wait();
 #pragma unroll
-            for (int k = 0; k < 16; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * corr_s[g * 16 + k]);
-            tc::st_32x32b_x16(ta, v);
-          }
-        tc::st_wait();
-      }
-      // P = 2^(z - m) as fp16 rows [row][head]; window rows carry s_t into P.
-      // z[] is reused for the weights entering the row sum.
-      uint8_t* prow = smem + Ly::kOffP;
-      const float rsr = rs[r];
-      float z[HQ];
-      load_scores(z);
-#pragma unroll
-      for (int c = 0; c < HQ / 8; ++c) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int h0 = c * 8 + 2 * k;
-          const float m0 = mu_s[h0], m1 = mu_s[h0 + 1];
-          float e0 = (m0 == -INFINITY) ? 0.0f : exp2f(z[h0] - m0);
-          float e1 = (m1 == -INFINITY) ? 0.0f : exp2f(z[h0 + 1] - m1);
-          __half2 w2 = __floats2half2_rn(e0 * rsr, e1 * rsr);
-          pk[k] = *reinterpret_cast<uint32_t*>(&w2);
-          if (rsr == 1.0f) {  // sparse rows: sum exactly the fp16 weights the PV product uses
-            float2 back = __half22float2(w2);
-            e0 = back.x;
-            e1 = back.y;
-          }
-          z[h0] = e0;
-          z[h0 + 1] = e1;
+              for (int k = 0; k < 16; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * corr_s[g * 16 + k]);
+              tc::st_32x32b_x16(ta, v);
+            }
+          tc::st_wait();
         }
-        *reinterpret_cast<uint4*>(prow + swz(r, c, Ly::kPRow)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
-      warp_transpose_reduce<HQ, false>(z, lane);
+      // pass 2: P = 2^(z - m) as fp16 [head][row]; window rows carry s_t into P.
+      // The TMEM loads are warp-collective: every lane issues them (ok is
+      // warp-uniform), only the lanes that carry a head write P.
+      if (ok) {
+        uint8_t* prow = smem + Ly::kOffP + bf * ((Ly::kPBytes + 1023) / 1024 * 1024);
+        float sum = 0.0f;
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int h = reduced_head<HQ>(lane, i);
-        bool writer = true;
-        if constexpr (HQ < 32) writer = (lane % (32 / HQ)) == 0;
-        if (writer) red[warp * HQ + h] = z[i];
+        for (int g = 0; g < kRows / 16; ++g) {
+          uint32_t v[16];
+          tc::ld_32x32b_x16(s_col + g * 16, v);
+          tc::ld_wait();
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int jj = cc * 8 + 2 * k, j0 = g * 16 + jj;
+              const float r0 = rsb[j0], r1 = rsb[j0 + 1];
+              const float z0 = r0 >= 0.0f ? __uint_as_float(v[jj]) * (zs * r0) : -INFINITY;
+              const float z1 = r1 >= 0.0f ? __uint_as_float(v[jj + 1]) * (zs * r1) : -INFINITY;
+              float e0 = (mu == -INFINITY) ? 0.0f : exp2f(z0 - mu);
+              float e1 = (mu == -INFINITY) ? 0.0f : exp2f(z1 - mu);
+              const float w0 = r0 > 0.0f ? r0 : 0.0f, w1 = r1 > 0.0f ? r1 : 0.0f;
+              __half2 w2 = __floats2half2_rn(e0 * w0, e1 * w1);
+              pk[k] = *reinterpret_cast<uint32_t*>(&w2);
+              // sparse rows: sum exactly the fp16 weights the PV product uses
+              const float2 back = __half22float2(w2);
+              if (r0 == 1.0f) e0 = back.x;
+              if (r1 == 1.0f) e1 = back.y;
+              sum += e0 + e1;
+            }
+            if (act) *reinterpret_cast<uint4*>(prow + swz128(h, g * 2 + cc)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+        if (act) {
+          l = l * corr + sum;
+          m = mu;
+        }
       }
-      tc::named_sync(1, 128);
-      if (threadIdx.x < HQ) {
-        const int h = threadIdx.x;
-        l_s[h] = l_s[h] * corr_s[h] + (red[h] + red[HQ + h]) + (red[2 * HQ + h] + red[3 * HQ + h]);
-        m_s[h] = mu_s[h];
-      }
-      if (threadIdx.x == 0) *any_rescale = 0;
       tc::fence_proxy_async_smem();
       tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar_p_full + 8 * bf);
     }
-    __syncthreads();
-    if (*abort) break;
-
-    // ---- 4. O^T += V^T P^T, one M tile (128 latent dims) per issuing thread
-    if (warp == 0 && lane < Ly::kMT) {
-      tc::fence_after_sync();
-      const int mt = lane;
-#pragma unroll
-      for (int ks = 0; ks < kRows / 16; ++ks) {
-        const uint64_t ad =
-            tc::smem_desc(sbase + Ly::kOffK + (2 * mt) * (kRows * 128) + ks * 2048, kRows * 128, 1024, tc::kSwizzle128B);
-        const uint64_t bd = tc::smem_desc(sbase + Ly::kOffP + ks * 16 * Ly::kPRow, 8 * Ly::kPRow, 8 * Ly::kPRow, p_sw);
-        tc::mma_f16(tmem + Ly::kColO + mt * HQ, ad, bd, idesc_pv, (it > 0 || ks > 0) ? 1u : 0u);
-      }
-      tc::commit(bar_pv);
+    if (act) {
+      l_s[h] = l;
+      m_s[h] = m;
     }
-    __syncwarp();
   }
-  // ---- epilogue
-  if (it > 0 && !*abort && threadIdx.x == 0) {
-    if (!mbar_wait_bounded(bar_pv, (it - 1) & 1, P.wait_ns)) {
+  // ---- epilogue: every warp; the tiles are free once the last PV completed
+  if (threadIdx.x == 0 && n_mine > 0 && !*abort) {
+    const int il = n_mine - 1;
+    if (!mbar_wait_bounded(bar_kv_empty + 8 * (il & 1), (il >> 1) & 1, P.wait_ns)) {
       set_status(P.status, CSA2_ERR_TIMEOUT);
       *abort = 1;
     }
   }
   __syncthreads();
   tc::fence_after_sync();
-  const bool have = it > 0 && !*abort;
-  if (warp < 4) {
-#pragma unroll 1
-    for (int mt = 0; mt < Ly::kMT; ++mt) {
-      const int d = mt * 128 + warp * 32 + lane;
+  const bool have = n_mine > 0 && !*abort;
+  // O^T (TMEM lanes = latent dims) -> staging [h][d] in the tile region:
+  // fp32 partials (split mode) or the normalised output in the output dtype
+  {
+    const bool f32_stage = nsplit > 1 || P.out_f32;
+    float* st32 = reinterpret_cast<float*>(smem + Ly::kOffTile);
+    __nv_bfloat16* st16 = reinterpret_cast<__nv_bfloat16*>(smem + Ly::kOffTile);
+    const int q = warp & 3;
+    const int nw_q = (kThreads / 32 - q + 3) / 4;  // warps sharing this lane quarter
+    const int wi = warp >> 2;
+    constexpr int kItems = Ly::kMT * (HQ / 16);
+    for (int item = wi; item < kItems; item += nw_q) {
+      const int mt = item / (HQ / 16), g = item % (HQ / 16);
+      const int d = mt * 128 + q * 32 + lane;
+      uint32_t v[16];
+      if (have) {
+        tc::ld_32x32b_x16(tmem + ((uint32_t)(q * 32) << 16) + Ly::kColO + mt * HQ + g * 16, v);
+        tc::ld_wait();
+      }
 #pragma unroll
-      for (int g = 0; g < HQ / 16; ++g) {
-        uint32_t v[16];
-        if (have) {
-          tc::ld_32x32b_x16(tmem + ((uint32_t)(warp * 32) << 16) + Ly::kColO + mt * HQ + g * 16, v);
-          tc::ld_wait();
+      for (int k = 0; k < 16; ++k) {
+        const int hh = g * 16 + k;
+        float o = have ? __uint_as_float(v[k]) : 0.0f;
+        if (nsplit == 1) {
+          const float lh = l_s[hh];
+          o = (have && lh > 0.0f) ? o / lh : 0.0f;
         }
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const int h = g * 16 + k;
-          const float o = have ? __uint_as_float(v[k]) : 0.0f;
-          if (nsplit == 1) {
-            const float l = l_s[h];
-            const float val = l > 0.0f ? o / l : 0.0f;
-            const int64_t oi = ((int64_t)tok * HQ + h) * D + d;
-            if (P.out_f32)
-              reinterpret_cast<float*>(io.out)[oi] = val;
-            else
-              reinterpret_cast<__nv_bfloat16*>(io.out)[oi] = __float2bfloat16_rn(val);
-          } else {
-            P.part_o[((slot0 + split) * HQ + h) * D + d] = o;
-          }
-        }
+        if (f32_stage)
+          st32[hh * D + d] = o;
+        else
+          st16[hh * D + d] = __float2bfloat16_rn(o);
       }
     }
-    if (threadIdx.x < HQ) {
-      const int h = threadIdx.x;
-      const float l = have ? l_s[h] : 0.0f;
-      const float m2 = have ? m_s[h] : -INFINITY;
-      if (nsplit == 1) {
-        if (io.lse) io.lse[(int64_t)tok * HQ + h] = l > 0.0f ? (m2 + log2f(l)) * 0.6931471805599453f : -INFINITY;
+    __syncthreads();
+    // staging -> global, 16-byte stores over the contiguous [HQ][D] block
+    if (nsplit == 1) {
+      if (P.out_f32) {
+        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(io.out) + (int64_t)tok * HQ * D);
+        const float4* src = reinterpret_cast<const float4*>(st32);
+        for (int e = threadIdx.x; e < HQ * D / 4; e += kThreads) dst[e] = src[e];
       } else {
-        float* ml = P.part_ml + ((slot0 + split) * HQ + h) * 2;
-        ml[0] = l > 0.0f ? m2 * 0.6931471805599453f : -INFINITY;
-        ml[1] = l;
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(io.out) + (int64_t)tok * HQ * D);
+        const uint4* src = reinterpret_cast<const uint4*>(st16);
+        for (int e = threadIdx.x; e < HQ * D / 8; e += kThreads) dst[e] = src[e];
+      }
+    } else {
+      float4* dst = reinterpret_cast<float4*>(P.part_o + (slot0 + split) * HQ * D);
+      const float4* src = reinterpret_cast<const float4*>(st32);
+      for (int e = threadIdx.x; e < HQ * D / 4; e += kThreads) dst[e] = src[e];
+    }
+    if (threadIdx.x < HQ) {
+      const int hh = threadIdx.x;
+      const float lh = have ? l_s[hh] : 0.0f;
+      const float m2 = have ? m_s[hh] : -INFINITY;
+      if (nsplit == 1) {
+        if (io.lse) io.lse[(int64_t)tok * HQ + hh] = lh > 0.0f ? (m2 + log2f(lh)) * 0.6931471805599453f : -INFINITY;
+      } else {
+        float* ml = P.part_ml + ((slot0 + split) * HQ + hh) * 2;
+        ml[0] = lh > 0.0f ? m2 * 0.6931471805599453f : -INFINITY;
+        ml[1] = lh;
       }
     }
   }
   // split mode: the last CTA of this token to finish merges the partials
   // (log-sum-exp weights) and restores the arrival counter to zero
   if (nsplit > 1) {
-    __shared__ int s_last;
+    volatile int* s_last = reinterpret_cast<volatile int*>(smem + Ly::kOffMisc + 8);
     __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) s_last = atomicAdd(P.done + (int64_t)layer * P.qb.n_tok + tok, 1) == nsplit - 1;
+    if (threadIdx.x == 0) *s_last = atomicAdd(P.done + (int64_t)layer * P.qb.n_tok + tok, 1) == nsplit - 1;
     __syncthreads();
-    if (s_last) {
+    if (*s_last) {
       __threadfence();
-      float* wgt = red;  // [nsplit][HQ] weights, reusing the reduction scratch (nsplit <= 4 here)
-      for (int h = threadIdx.x; h < HQ; h += kThreads) {
+      float* wgt = reinterpret_cast<float*>(smem + Ly::kOffTile);  // [nsplit][HQ] weights (tiles are free)
+      for (int hh = threadIdx.x; hh < HQ; hh += kThreads) {
         float M = -INFINITY;
         for (int sp = 0; sp < nsplit; ++sp) {
-          const float* ml = P.part_ml + ((slot0 + sp) * HQ + h) * 2;
+          const float* ml = P.part_ml + ((slot0 + sp) * HQ + hh) * 2;
           if (__ldcg(ml + 1) > 0.0f) M = fmaxf(M, __ldcg(ml));
         }
         float L = 0.0f;
         for (int sp = 0; sp < nsplit; ++sp) {
-          const float* ml = P.part_ml + ((slot0 + sp) * HQ + h) * 2;
-          const float l = __ldcg(ml + 1);
-          const float a = l > 0.0f ? __expf(__ldcg(ml) - M) : 0.0f;
-          wgt[sp * HQ + h] = a;
-          L += a * l;
+          const float* ml = P.part_ml + ((slot0 + sp) * HQ + hh) * 2;
+          const float lv = __ldcg(ml + 1);
+          const float a = lv > 0.0f ? __expf(__ldcg(ml) - M) : 0.0f;
+          wgt[sp * HQ + hh] = a;
+          L += a * lv;
         }
         const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-        for (int sp = 0; sp < nsplit; ++sp) wgt[sp * HQ + h] *= inv;
-        if (io.lse) io.lse[(int64_t)tok * HQ + h] = L > 0.0f ? M + logf(L) : -INFINITY;
+        for (int sp = 0; sp < nsplit; ++sp) wgt[sp * HQ + hh] *= inv;
+        if (io.lse) io.lse[(int64_t)tok * HQ + hh] = L > 0.0f ? M + logf(L) : -INFINITY;
       }
       __syncthreads();
-      // 16-byte loads, all splits of 4 groups in flight per thread (nsplit <= 4)
+      // 16-byte loads, all splits of 2 groups in flight per thread (nsplit <= 4)
       constexpr int kTot4 = HQ * D / 4;
       const float4* po = reinterpret_cast<const float4*>(P.part_o) + slot0 * kTot4;
-      for (int e0 = threadIdx.x; e0 < kTot4; e0 += kThreads * 4) {
-        float4 v[4][4];
+      for (int e0 = threadIdx.x; e0 < kTot4; e0 += kThreads * 2) {
+        float4 v[2][4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int u = 0; u < 2; ++u)
 #pragma unroll
           for (int sp = 0; sp < 4; ++sp) {
             const int e = e0 + u * kThreads;
             v[u][sp] = (sp < nsplit && e < kTot4) ? __ldcg(po + (int64_t)sp * kTot4 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
           }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 2; ++u) {
           const int e = e0 + u * kThreads;
           if (e >= kTot4) continue;
-          const int h = (e * 4) / D;
+          const int hh = (e * 4) / D;
           float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
           for (int sp = 0; sp < 4; ++sp) {
             if (sp >= nsplit) continue;
-            const float wv = wgt[sp * HQ + h];
+            const float wv = wgt[sp * HQ + hh];
             a.x += wv * v[u][sp].x;
             a.y += wv * v[u][sp].y;
             a.z += wv * v[u][sp].z;
@@ -645,8 +716,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
     }
   }
   // no MMA of ours may be in flight when TMEM is released
-  if (warp == 0 && lane < 4) tc::commit(bar_drain);  // every issuing thread
-  __syncwarp();
   if (threadIdx.x == 0) {
     if (!mbar_wait_bounded(bar_drain, 0, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
   }
@@ -668,6 +737,12 @@ int launch_t(const Params& p, int nsplit, int n_layers, cudaStream_t st) {
                                                  Ly::kBytes),
                             "attend smem attribute"))
       return rc;
+    int fit = 0;
+    if (int rc = cuda_check(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, k_attend_tc<D, HQ, QLO>, kThreads,
+                                                                          Ly::kBytes),
+                            "attend occupancy"))
+      return rc;
+    if (fit < 1) return fail(CSA2_ERR_UNSUPPORTED, "attention kernel does not fit on an SM");
     attr[dev] = true;
   }
   Launch L_("attend_tc", st);
@@ -690,6 +765,9 @@ int launch_attend_tc(const csa2_query_batch* qb, int q_dtype, int Hq, const csa2
                      float* part_ml, int* done, int nsplit, cudaStream_t st) {
   using namespace attend_tc;
   if (n_layers < 1 || n_layers > kMaxLayers) return fail(CSA2_ERR_UNSUPPORTED, "1..%d layers per launch", kMaxLayers);
+  if (nsplit < 1 || nsplit > 4) return fail(CSA2_ERR_UNSUPPORTED, "1..4 attention splits");
+  if (K < 1 || K > kMaxRows) return fail(CSA2_ERR_UNSUPPORTED, "K must be 1..%d", kMaxRows);
+  if (kv->n_rows >= (int64_t(1) << 31)) return fail(CSA2_ERR_UNSUPPORTED, "Main KV too large for 32-bit rows");
   Params p{};
   p.qb = *qb;
   p.q_f32 = q_dtype == CSA2_F32;

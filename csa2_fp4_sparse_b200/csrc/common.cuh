@@ -86,15 +86,23 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 }
 
 // Waits for the phase with the given parity to complete; gives up after
-// limit_ns and returns false (the caller records CSA2_ERR_TIMEOUT).  Waiting
-// threads are suspended by the hardware between probes (they take no issue
-// slots from the warps doing work); the clock is read once per probe.
+// about limit_ns and returns false (the caller records CSA2_ERR_TIMEOUT).
+// Waiting threads are suspended by the hardware between probes (they take no
+// issue slots from the warps doing work).  The global timer is read only
+// every 64th probe: its reads go through a narrow pipe that a few dozen
+// waiting warps reading it on every probe would saturate.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
+  uint64_t t0 = 0;
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
-    if (globaltimer_ns() - t0 > limit_ns) return false;
+    if ((i & 63) == 0) {
+      const uint64_t now = globaltimer_ns();
+      if (i == 64)
+        t0 = now;
+      else if (now - t0 > limit_ns)
+        return false;
+    }
   }
 }
 

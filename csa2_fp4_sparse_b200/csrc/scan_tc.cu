@@ -13,19 +13,19 @@
 //   warp 0      TMA producer: tiles of 128 positions of the FP4 indexer K cache
 //               (codes with the 64B/32B swizzle the MMA expects, plus the raw
 //               E4M3 scales) into a 12-stage shared-memory ring;
-//   warps 10,12 scale-factor warps (alternate tiles): rearrange each landed tile's scales into
+//   warp 19     scale-factor warp (two tiles per pass): rearrange each landed tile's scales into
 //               the tensor-core scale-factor layout (each per-32 E4M3 scale
 //               written twice, as the block-scaled MMA takes one UE4M3 scale
 //               per 16 elements) and copies them to TMEM (tcgen05.cp); a
 //               commit hands the stage to the MMA warp, so the copy never
 //               queues behind that warp's earlier MMAs;
-//   warps 1, 11 MMA issuers (alternate tiles, one epilogue warpgroup each):
+//   warps 1, 18 MMA issuers (alternate tiles, two epilogue warpgroups each):
 //               issue tcgen05.mma kind::mxf4nvf4 (M = 128 positions, N = heads,
 //               K = 64 per instruction) per query token into a ring of TMEM
 //               accumulators; commits release the smem stage and hand the
 //               accumulator to the epilogue;
-//   warps 2..9  epilogue, two warpgroups (warps 2..5 for MMA warp 1's tiles,
-//               6..9 for warp 11's):
+//   warps 2..17 epilogue, four warpgroups: warpgroup e takes the accumulator
+//               jobs of MMA warp (e & 1) whose job count has parity e >> 1:
 //               TMEM -> registers (one position per thread), ReLU, weighted
 //               head sum, block max over 8 lanes, block-score store.
 // The key cache is streamed from HBM exactly once per sequence for all of its
@@ -47,11 +47,12 @@ constexpr int kTile = 128;      // positions per tile = MMA M
 constexpr int kChunk = 64;      // rows per TMA box
 constexpr int kAccUnits = 4;    // TMEM accumulator ring, 64 columns each
 constexpr int kMaxW = 8;        // query tokens of one sequence per tile
-constexpr int kThreads = 416;   // 13 warps: producer, 2 MMA issuers, 2 epilogue warpgroups, 2 scale-factor warps
-constexpr int kSfWarp = 10;     // scale-factor warps 10 and 12 take alternate tiles
-constexpr int kSfWarpB = 12;
-constexpr int kMmaWarpB = 11;   // second MMA issuer (the first is warp 1); they take alternate tiles
-constexpr int kUnitsPer = kAccUnits / 2;  // accumulator units of each MMA issuer
+constexpr int kEpiWG = 4;       // epilogue warpgroups (warps 2..17)
+constexpr int kThreads = 640;   // 20 warps: producer, 2 MMA issuers, 4 epilogue warpgroups, scale-factor warp
+constexpr int kMmaWarpB = 18;   // second MMA issuer (the first is warp 1); they take alternate tiles
+constexpr int kSfWarp = 19;     // scale-factor warp
+constexpr int kUnitsPer = kAccUnits / 2;  // accumulator units of each MMA issuer (one per epilogue warpgroup)
+static_assert(kUnitsPer * 2 == kEpiWG, "one accumulator unit per epilogue warpgroup");
 constexpr uint32_t kColAcc = 0;
 constexpr uint32_t kColSfa = kAccUnits * 64;              // 256
 constexpr uint32_t kColSfb = kColSfa + kStages * 8;      // 352
@@ -68,9 +69,9 @@ constexpr uint32_t kOffRaw = kOffA + kStages * 8192;      // [kStages][2048]
 constexpr uint32_t kOffSfa = kOffRaw + kStages * kRawStage;  // [kStages][2][512]
 constexpr uint32_t kOffB = kOffSfa + kStages * 1024;      // [kMaxW][64 rows][64 B]
 constexpr uint32_t kOffSfb = kOffB + kMaxW * 4096;        // [kMaxW][2][512]
-constexpr uint32_t kOffW = kOffSfb + kMaxW * 1024;        // [2 warpgroups][kMaxW][64] f32
-constexpr uint32_t kOffPos = kOffW + 2 * kMaxW * 64 * 4;  // [3][kMaxW] i64 query positions (MMA warp, 2 epilogue warpgroups)
-constexpr uint32_t kOffBar = kOffPos + 3 * kMaxW * 8;     // mbarriers
+constexpr uint32_t kOffW = kOffSfb + kMaxW * 1024;        // [kEpiWG][kMaxW][64] f32
+constexpr uint32_t kOffPos = kOffW + kEpiWG * kMaxW * 64 * 4;  // [1 + kEpiWG][kMaxW] i64 query positions (MMA warps, epilogue warpgroups)
+constexpr uint32_t kOffBar = kOffPos + (1 + kEpiWG) * kMaxW * 8;  // mbarriers
 constexpr uint32_t kNumBars = 3 * kStages + 2 * kAccUnits + 5;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;     // tmem base, abort flag
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;     // + alignment slack
@@ -347,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           warp_wait_or_abort(my_drain, drain_n & 1, P, abort);
           ++drain_n;
         }
-        tc::named_sync(3, 64);  // both issuers drained
+        tc::named_sync(5, 64);  // both issuers drained
         cur_b = ti.b;
         int bseq;
         group_info<kRescore>(P, cur_b, &tok0, &W, &bseq);
@@ -405,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++sfb_n;
           (void)ok;
         }
-        tc::named_sync(4, 64);  // new queries and positions in place
+        tc::named_sync(6, 64);  // new queries and positions in place
         tc::fence_after_sync();
       }
       if ((int)(it & 1) != mw || *abort) continue;  // the other issuer's tile (or nothing left to do)
@@ -446,58 +447,79 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait_bounded(my_drain, drain_n & 1, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
     }
     __syncwarp();
-  } else if (warp == kSfWarp || warp == kSfWarpB) {
+  } else if (warp == kSfWarp) {
     // ------------------------------------------------------------ scale factors
     // raw [row][spr] -> [m0 (32)][m1 (4)][k (4)] per 64-element K step, each
-    // per-32 scale written twice (the MMA takes one scale per 16 elements)
+    // per-32 scale written twice (the MMA takes one scale per 16 elements);
+    // two tiles per pass, so the fixed costs of a pass (proxy fence, copy
+    // issue) are shared
     TileIter<kRescore> ti;
     ti.init(P, wb, we);
     int64_t it = 0;
     constexpr int kBoxRows = kRescore ? kBlock : kChunk;
     constexpr uint32_t kSlot = kRescore ? kRawStage / 16 : kRawStage / 2;
-    const int sfw = warp == kSfWarp ? 0 : 1;
-    for (; ti.valid(); ti.next(P), ++it) {
-      if ((int)(it & 1) != sfw) continue;  // the other scale-factor warp's tile
-      const int s = (int)(it % kStages);
-      const uint32_t n = (uint32_t)(it / kStages);
-      if (!warp_wait_or_abort(bar_full + 8 * s, n & 1, P, abort)) break;
-      const uint8_t* raw = smem + kOffRaw + s * kRawStage;
-      uint32_t wv[4];
+    while (ti.valid()) {
+      const int nt = ti.left >= 2 ? 2 : 1;
+      uint32_t wv[2][4];
+      bool ok = true;
 #pragma unroll
-      for (int m1 = 0; m1 < 4; ++m1) {
-        const int r = m1 * 32 + lane;
-        const uint8_t* src = raw + (r / kBoxRows) * kSlot + (r % kBoxRows) * spr;
-        wv[m1] = (spr == 4) ? *reinterpret_cast<const uint32_t*>(src) : (uint32_t)*reinterpret_cast<const uint16_t*>(src);
+      for (int k = 0; k < 2; ++k) {
+        if (k >= nt) break;
+        const int s = (int)((it + k) % kStages);
+        const uint32_t n = (uint32_t)((it + k) / kStages);
+        if (!warp_wait_or_abort(bar_full + 8 * s, n & 1, P, abort)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* raw = smem + kOffRaw + s * kRawStage;
+#pragma unroll
+        for (int m1 = 0; m1 < 4; ++m1) {
+          const int r = m1 * 32 + lane;
+          const uint8_t* src = raw + (r / kBoxRows) * kSlot + (r % kBoxRows) * spr;
+          wv[k][m1] =
+              (spr == 4) ? *reinterpret_cast<const uint32_t*>(src) : (uint32_t)*reinterpret_cast<const uint16_t*>(src);
+        }
       }
-      for (int ks = 0; ks < ksteps; ++ks) {
-        const uint32_t sel = ks == 0 ? 0x1100u : 0x3322u;
-        *reinterpret_cast<uint4*>(smem + kOffSfa + (s * 2 + ks) * 512 + lane * 16) =
-            make_uint4(__byte_perm(wv[0], 0, sel), __byte_perm(wv[1], 0, sel), __byte_perm(wv[2], 0, sel),
-                       __byte_perm(wv[3], 0, sel));
+      if (!ok) break;
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        if (k >= nt) break;
+        const int s = (int)((it + k) % kStages);
+        for (int ks = 0; ks < ksteps; ++ks) {
+          const uint32_t sel = ks == 0 ? 0x1100u : 0x3322u;
+          *reinterpret_cast<uint4*>(smem + kOffSfa + (s * 2 + ks) * 512 + lane * 16) =
+              make_uint4(__byte_perm(wv[k][0], 0, sel), __byte_perm(wv[k][1], 0, sel),
+                         __byte_perm(wv[k][2], 0, sel), __byte_perm(wv[k][3], 0, sel));
+        }
       }
       tc::fence_proxy_async_smem();
       __syncwarp();
       // copy to TMEM from this warp, so the copy is not queued behind the MMA
-      // warp's earlier MMAs; the commit hands the stage over once it landed
+      // warps' earlier MMAs; each commit hands its stage over once it landed
       if (lane == 0) {
         tc::fence_after_sync();
-        for (int ks = 0; ks < ksteps; ++ks)
-          tc::cp_32x128b_warpx4(tmem + kColSfa + s * 8 + ks * 4,
-                                tc::smem_desc(sbase + kOffSfa + (s * 2 + ks) * 512, 16, 128, tc::kSwizzleNone));
-        tc::commit(bar_sfr + 8 * s);
+        for (int k = 0; k < nt; ++k) {
+          const int s = (int)((it + k) % kStages);
+          for (int ks = 0; ks < ksteps; ++ks)
+            tc::cp_32x128b_warpx4(tmem + kColSfa + s * 8 + ks * 4,
+                                  tc::smem_desc(sbase + kOffSfa + (s * 2 + ks) * 512, 16, 128, tc::kSwizzleNone));
+          tc::commit(bar_sfr + 8 * s);
+        }
       }
       __syncwarp();
+      for (int k = 0; k < nt; ++k) ti.next(P);
+      it += nt;
     }
     // drain: our copies must have landed before teardown
     if (lane == 0) {
-      const uint32_t dr = sfw == 0 ? bar_drain2 : bar_drain_c;
-      tc::commit(dr);
-      if (!mbar_wait_bounded(dr, 0, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
+      tc::commit(bar_drain2);
+      if (!mbar_wait_bounded(bar_drain2, 0, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int wg = (warp - 2) / 4;        // warpgroup 0: warps 2..5, 1: warps 6..9
+    const int wg = (warp - 2) / 4;        // warpgroup: warps 2+4wg .. 5+4wg
+    const int mw = wg & 1, sub = wg >> 1; // its MMA issuer and job parity
     const int quarter = warp & 3;         // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
     const int ept = threadIdx.x - 64 - wg * 128;  // 0..127 within the warpgroup
@@ -506,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     TileIter<kRescore> ti;
     ti.init(P, wb, we);
     int64_t it = 0;
-    int cnt = 0;  // jobs of this warpgroup's issuer
+    int cnt = 0;  // jobs of this warpgroup's issuer (all parities)
     int cur_b = -1, W = 0, tok0 = 0;
     // no early exit: the four warps of the warpgroup meet at named barriers
     for (; ti.valid(); ti.next(P), ++it) {
@@ -523,42 +545,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ept < W) pos_g[ept] = __ldg(P.qb.tok_pos + tok0 + ept);
         tc::named_sync(1 + wg, 128);
       }
-      if ((int)(it & 1) != wg || *abort) continue;  // the other issuer's tile (or nothing left to do)
+      if ((int)(it & 1) != mw || *abort) continue;  // the other issuer's tile (or nothing left to do)
       const int64_t t0 = (int64_t)ti.tile * kTile;
       for (int j = 0; j < W; ++j) {
         const int tok = tok0 + j;
         const int64_t p = pos_g[j];
         if (!kRescore && t0 > p) continue;
-        const int u = wg + 2 * (cnt % kUnitsPer);
-        const uint32_t m = (uint32_t)(cnt / kUnitsPer);
-        ++cnt;
+        const int job = cnt++;
+        if (job % kUnitsPer != sub) continue;  // the other warpgroup of this issuer
+        const int u = mw + 2 * sub;
+        const uint32_t m = (uint32_t)(job / kUnitsPer);
         if (!warp_wait_or_abort(bar_accf + 8 * u, m & 1, P, abort)) break;
         tc::fence_after_sync();
         const float* wj = w_g + j * 64;
         const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + kColAcc + u * 64;
-        uint32_t r[4][16];
         const int ng = P.N / 16;
-#pragma unroll
-        for (int g = 0; g < 4; ++g)
-          if (g < ng) tc::ld_32x32b_x16(taddr + g * 16, r[g]);
-        tc::ld_wait();
-        tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(bar_acce + 8 * u);
-        // four independent chains; weights read as float4 (broadcast)
+        // two halves of 32 columns (register budget); four independent chains,
+        // weights read as float4 (broadcast)
         float a4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-        for (int g = 0; g < 4; ++g)
-          if (g < ng) {
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t r[2][16];
 #pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) {
-              const float4 w4 = *reinterpret_cast<const float4*>(wj + g * 16 + k4 * 4);
-              a4[0] = fmaf(w4.x, fmaxf(__uint_as_float(r[g][k4 * 4 + 0]), 0.0f), a4[0]);
-              a4[1] = fmaf(w4.y, fmaxf(__uint_as_float(r[g][k4 * 4 + 1]), 0.0f), a4[1]);
-              a4[2] = fmaf(w4.z, fmaxf(__uint_as_float(r[g][k4 * 4 + 2]), 0.0f), a4[2]);
-              a4[3] = fmaf(w4.w, fmaxf(__uint_as_float(r[g][k4 * 4 + 3]), 0.0f), a4[3]);
-            }
+          for (int g = 0; g < 2; ++g)
+            if (hf * 2 + g < ng) tc::ld_32x32b_x16(taddr + (hf * 2 + g) * 16, r[g]);
+          tc::ld_wait();
+          if (hf == 1) {  // the accumulator is free once the last load has landed
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar_acce + 8 * u);
           }
+#pragma unroll
+          for (int g = 0; g < 2; ++g)
+            if (hf * 2 + g < ng) {
+#pragma unroll
+              for (int k4 = 0; k4 < 4; ++k4) {
+                const float4 w4 = *reinterpret_cast<const float4*>(wj + (hf * 2 + g) * 16 + k4 * 4);
+                a4[0] = fmaf(w4.x, fmaxf(__uint_as_float(r[g][k4 * 4 + 0]), 0.0f), a4[0]);
+                a4[1] = fmaf(w4.y, fmaxf(__uint_as_float(r[g][k4 * 4 + 1]), 0.0f), a4[1]);
+                a4[2] = fmaf(w4.z, fmaxf(__uint_as_float(r[g][k4 * 4 + 2]), 0.0f), a4[2]);
+                a4[3] = fmaf(w4.w, fmaxf(__uint_as_float(r[g][k4 * 4 + 3]), 0.0f), a4[3]);
+              }
+            }
+        }
         const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
         if (kRescore) {
           // pool entry i = tile*128 + row: position pool[i/8]*8 + i%8
@@ -687,6 +716,12 @@ static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const 
             cudaFuncSetAttribute(k_index_tc<kRescore>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes),
             "index smem attribute"))
       return rc;
+    int fit = 0;  // one CTA of kThreads threads at this register count must fit on an SM
+    if (int rc = cuda_check(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, k_index_tc<kRescore>, kThreads,
+                                                                          kSmemBytes),
+                            "index occupancy"))
+      return rc;
+    if (fit < 1) return fail(CSA2_ERR_UNSUPPORTED, "index kernel does not fit on an SM");
     attr_done[dev] = true;
   }
   Launch L_(kRescore ? "rescore_tc" : "scan_tc", st);

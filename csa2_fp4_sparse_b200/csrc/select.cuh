@@ -84,8 +84,8 @@ __device__ __forceinline__ bool group_barrier(uint32_t* bar, uint32_t target, ui
     atomicAdd(bar, 1u);
     const uint64_t t0 = globaltimer_ns();
     int ok = 1;
-    while (ld_acquire_u32(bar) < target) {
-      if (globaltimer_ns() - t0 > wait_ns) {
+    for (uint32_t i = 1; ld_acquire_u32(bar) < target; ++i) {
+      if ((i & 15) == 0 && globaltimer_ns() - t0 > wait_ns) {  // the timer is read every 16th probe
         set_status(status, CSA2_ERR_TIMEOUT);
         ok = 0;
         break;
