@@ -113,6 +113,14 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// 2^x on the special-function unit (PTX ex2.approx.ftz: relative error below
+// 2^-22; -inf -> +0)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // named barrier over the softmax warps with an OR over `pred`
 __device__ __forceinline__ bool soft_sync_or(bool pred) {
   uint32_t r;
@@ -332,22 +340,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
       }
     };
     if (n_mine > 0) load_codes(0, cur);
+    bool dead = false;  // uniform over the loader warps: a wait gave up
     for (int i = 0; i < n_mine; ++i) {
       const int c = split + i * nsplit, bf = i & 1;
       // the next chunk's codes go in flight before this chunk is converted
       if (i + 1 < n_mine) load_codes(i + 1, nxt);
-      bool ok = __shfl_sync(0xffffffffu, (int)!*abort, 0) != 0;
-      // the tile is free once PV(i - 2) has completed
-      if (i >= 2 && ok) {
-        if (!mbar_wait_warp(bar_kv_empty + 8 * bf, ((i >> 1) - 1) & 1, P.wait_ns)) {
-          if (lane == 0) {
+      // the tile is free once PV(i - 2) has completed: one loader thread
+      // probes, the others park on named barrier 2
+      if (i >= 2 && !dead) {
+        if (!mbar_wait_group(bar_kv_empty + 8 * bf, ((i >> 1) - 1) & 1, P.wait_ns, lt == 0, *abort != 0, 2,
+                             kLoadThreads)) {
+          if (lt == 0) {
             set_status(P.status, CSA2_ERR_TIMEOUT);
             *abort = 1;
           }
-          ok = false;
+          dead = true;
         }
       }
-      if (ok) {
+      if (!dead) {
         uint8_t* tile = smem + Ly::kOffTile + bf * Ly::kTile;
         const bool sparse = c < n_sp;
 #pragma unroll
@@ -403,19 +413,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
           *abort = 1;
         } else {
           tc::fence_after_sync();
-          const uint32_t tile = sbase + Ly::kOffTile + bf * Ly::kTile;
-#pragma unroll 1
+          // descriptors advance by adding (byte offset >> 4) to the start
+          // address field (shared addresses stay below 2^18: no carry out)
+          const uint64_t a0 = tc::smem_desc(sbase + Ly::kOffQ, 16, 1024, tc::kSwizzle128B);
+          const uint64_t al0 = tc::smem_desc(sbase + Ly::kOffQlo, 16, 1024, tc::kSwizzle128B);
+          const uint64_t b0 = tc::smem_desc(sbase + Ly::kOffTile + bf * Ly::kTile, 16, 1024, tc::kSwizzle128B);
+          const uint32_t dcol = tmem + Ly::kColS + bf * kRows;
+#pragma unroll
           for (int kb = 0; kb < Ly::kKB; ++kb)
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
-              const uint64_t ad = tc::smem_desc(sbase + Ly::kOffQ + kb * (HQ * 128) + ks * 32, 16, 1024, tc::kSwizzle128B);
-              const uint64_t bd = tc::smem_desc(tile + kb * (kRows * 128) + ks * 32, 16, 1024, tc::kSwizzle128B);
-              tc::mma_f16(tmem + Ly::kColS + bf * kRows, ad, bd, idesc, (kb | ks) ? 1u : 0u);
-              if (QLO) {
-                const uint64_t al =
-                    tc::smem_desc(sbase + Ly::kOffQlo + kb * (HQ * 128) + ks * 32, 16, 1024, tc::kSwizzle128B);
-                tc::mma_f16(tmem + Ly::kColS + bf * kRows, al, bd, idesc, 1u);
-              }
+              const uint64_t ao = (uint64_t)((kb * (HQ * 128) + ks * 32) >> 4);
+              const uint64_t bd = b0 + (uint64_t)((kb * (kRows * 128) + ks * 32) >> 4);
+              tc::mma_f16(dcol, a0 + ao, bd, idesc, (kb | ks) ? 1u : 0u);
+              if (QLO) tc::mma_f16(dcol, al0 + ao, bd, idesc, 1u);
             }
           tc::commit(bar_s_full + 8 * bf);
         }
@@ -435,15 +446,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
           *abort = 1;
         } else {
           tc::fence_after_sync();
-          const uint32_t tile = sbase + Ly::kOffTile + bf * Ly::kTile;
-          const uint32_t pb = sbase + Ly::kOffP + bf * ((Ly::kPBytes + 1023) / 1024 * 1024);
-#pragma unroll 1
+          const uint64_t a0 =
+              tc::smem_desc(sbase + Ly::kOffTile + bf * Ly::kTile, kRows * 128, 1024, tc::kSwizzle128B);
+          const uint64_t b0 =
+              tc::smem_desc(sbase + Ly::kOffP + bf * ((Ly::kPBytes + 1023) / 1024 * 1024), 16, 1024, tc::kSwizzle128B);
+#pragma unroll
           for (int mt = 0; mt < Ly::kMT; ++mt)
 #pragma unroll
             for (int ks = 0; ks < kRows / 16; ++ks) {
-              const uint64_t ad =
-                  tc::smem_desc(tile + (2 * mt) * (kRows * 128) + ks * 2048, kRows * 128, 1024, tc::kSwizzle128B);
-              const uint64_t bd = tc::smem_desc(pb + ks * 32, 16, 1024, tc::kSwizzle128B);
+              const uint64_t ad = a0 + (uint64_t)(((2 * mt) * (kRows * 128) + ks * 2048) >> 4);
+              const uint64_t bd = b0 + (uint64_t)((ks * 32) >> 4);
               tc::mma_f16(tmem + Ly::kColO + mt * HQ, ad, bd, idesc, (i > 0 || ks > 0) ? 1u : 0u);
             }
           tc::commit(bar_kv_empty + 8 * bf);
@@ -461,19 +473,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
     const uint32_t s_lane = tmem + ((uint32_t)(warp * 32) << 16);
     const float zs = P.scale * kLog2e;
     float m = -INFINITY, l = 0.0f;
+    bool dead = false;  // uniform over the softmax warps: a wait gave up
     for (int i = 0; i < n_mine; ++i) {
       const int bf = i & 1;
-      bool ok = __shfl_sync(0xffffffffu, (int)!*abort, 0) != 0;
-      if (ok && !mbar_wait_warp(bar_s_full + 8 * bf, (i >> 1) & 1, P.wait_ns)) {
-        if (lane == 0) {
+      // one thread probes, the other softmax threads park on named barrier 1
+      const bool ok = !dead && mbar_wait_group(bar_s_full + 8 * bf, (i >> 1) & 1, P.wait_ns, threadIdx.x == 0,
+                                               *abort != 0, 1, 128);
+      if (!ok && !dead) {
+        if (threadIdx.x == 0 && !*abort) {
           set_status(P.status, CSA2_ERR_TIMEOUT);
           *abort = 1;
         }
-        ok = false;
+        dead = true;
       }
       tc::fence_after_sync();
       const float* rsb = rs_s + bf * kRows;
       const uint32_t s_col = s_lane + Ly::kColS + bf * kRows;
+      // every row a valid sparse row (row scale 1): the common case, no per-row scale
+      const bool plain = __all_sync(0xffffffffu, rsb[lane] == 1.0f && rsb[lane + 32] == 1.0f);
       // pass 1: the chunk's maximum (log2 domain; window rows scaled by s_t)
       float cm = -INFINITY;
       if (ok) {
@@ -482,12 +499,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
           uint32_t v[16];
           tc::ld_32x32b_x16(s_col + g * 16, v);
           tc::ld_wait();
+          if (plain) {
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const float rsj = rsb[g * 16 + k];
-            if (rsj >= 0.0f) cm = fmaxf(cm, __uint_as_float(v[k]) * (zs * rsj));
+            for (int k = 0; k < 16; ++k) cm = fmaxf(cm, __uint_as_float(v[k]));
+          } else {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const float rsj = rsb[g * 16 + k];
+              if (rsj >= 0.0f) cm = fmaxf(cm, __uint_as_float(v[k]) * rsj);
+            }
           }
         }
+        cm *= zs;  // zs > 0: scaling after the maximum is the same maximum
       }
       // running max: moves only when the chunk exceeds it by more than 2^8
       float mu = m;
@@ -499,8 +522,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
       if (any && i > 0 && ok) {
         // rescale the output accumulator of earlier chunks (rare): PV(i - 1)
         // must have completed first
-        if (!mbar_wait_warp(bar_kv_empty + 8 * ((i - 1) & 1), ((i - 1) >> 1) & 1, P.wait_ns)) {
-          if (lane == 0) {
+        if (!mbar_wait_group(bar_kv_empty + 8 * ((i - 1) & 1), ((i - 1) >> 1) & 1, P.wait_ns, threadIdx.x == 0,
+                             *abort != 0, 1, 128)) {
+          if (threadIdx.x == 0 && !*abort) {
             set_status(P.status, CSA2_ERR_TIMEOUT);
             *abort = 1;
           }
@@ -523,9 +547,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
       }
       // pass 2: P = 2^(z - m) as fp16 [head][row]; window rows carry s_t into P.
       // The TMEM loads are warp-collective: every lane issues them (ok is
-      // warp-uniform), only the lanes that carry a head write P.
+      // uniform), only the lanes that carry a head write P.
       if (ok) {
         uint8_t* prow = smem + Ly::kOffP + bf * ((Ly::kPBytes + 1023) / 1024 * 1024);
+        const float nmu = mu == -INFINITY ? 0.0f : -mu;
         float sum = 0.0f;
 #pragma unroll
         for (int g = 0; g < kRows / 16; ++g) {
@@ -538,19 +563,29 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const int jj = cc * 8 + 2 * k, j0 = g * 16 + jj;
-              const float r0 = rsb[j0], r1 = rsb[j0 + 1];
-              const float z0 = r0 >= 0.0f ? __uint_as_float(v[jj]) * (zs * r0) : -INFINITY;
-              const float z1 = r1 >= 0.0f ? __uint_as_float(v[jj + 1]) * (zs * r1) : -INFINITY;
-              float e0 = (mu == -INFINITY) ? 0.0f : exp2f(z0 - mu);
-              float e1 = (mu == -INFINITY) ? 0.0f : exp2f(z1 - mu);
-              const float w0 = r0 > 0.0f ? r0 : 0.0f, w1 = r1 > 0.0f ? r1 : 0.0f;
-              __half2 w2 = __floats2half2_rn(e0 * w0, e1 * w1);
-              pk[k] = *reinterpret_cast<uint32_t*>(&w2);
-              // sparse rows: sum exactly the fp16 weights the PV product uses
-              const float2 back = __half22float2(w2);
-              if (r0 == 1.0f) e0 = back.x;
-              if (r1 == 1.0f) e1 = back.y;
-              sum += e0 + e1;
+              if (plain) {
+                // e = 2^(s * zs - mu); the fp16 weight is what PV uses and what the sum adds
+                const float e0 = ex2_approx(fmaf(__uint_as_float(v[jj]), zs, nmu));
+                const float e1 = ex2_approx(fmaf(__uint_as_float(v[jj + 1]), zs, nmu));
+                __half2 w2 = __floats2half2_rn(e0, e1);
+                pk[k] = *reinterpret_cast<uint32_t*>(&w2);
+                const float2 back = __half22float2(w2);
+                sum += back.x + back.y;
+              } else {
+                const float r0 = rsb[j0], r1 = rsb[j0 + 1];
+                const float z0 = r0 >= 0.0f ? __uint_as_float(v[jj]) * (zs * r0) : -INFINITY;
+                const float z1 = r1 >= 0.0f ? __uint_as_float(v[jj + 1]) * (zs * r1) : -INFINITY;
+                float e0 = (mu == -INFINITY) ? 0.0f : ex2_approx(z0 + nmu);
+                float e1 = (mu == -INFINITY) ? 0.0f : ex2_approx(z1 + nmu);
+                const float w0 = r0 > 0.0f ? r0 : 0.0f, w1 = r1 > 0.0f ? r1 : 0.0f;
+                __half2 w2 = __floats2half2_rn(e0 * w0, e1 * w1);
+                pk[k] = *reinterpret_cast<uint32_t*>(&w2);
+                // sparse rows: sum exactly the fp16 weights the PV product uses
+                const float2 back = __half22float2(w2);
+                if (r0 == 1.0f) e0 = back.x;
+                if (r1 == 1.0f) e1 = back.y;
+                sum += e0 + e1;
+              }
             }
             if (act) *reinterpret_cast<uint4*>(prow + swz128(h, g * 2 + cc)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
@@ -568,6 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
     if (act) {
       l_s[h] = l;
       m_s[h] = m;
+      corr_s[h] = l > 0.0f ? 1.0f / l : 0.0f;  // reciprocal row sum for the epilogue
     }
   }
   // ---- epilogue: every warp; the tiles are free once the last PV completed
@@ -603,32 +639,34 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
       for (int k = 0; k < 16; ++k) {
         const int hh = g * 16 + k;
         float o = have ? __uint_as_float(v[k]) : 0.0f;
-        if (nsplit == 1) {
-          const float lh = l_s[hh];
-          o = (have && lh > 0.0f) ? o / lh : 0.0f;
-        }
+        if (nsplit == 1) o = have ? o * corr_s[hh] : 0.0f;
         if (f32_stage)
           st32[hh * D + d] = o;
         else
           st16[hh * D + d] = __float2bfloat16_rn(o);
       }
     }
+    tc::fence_proxy_async_smem();  // the staging is read by the bulk copy
     __syncthreads();
-    // staging -> global, 16-byte stores over the contiguous [HQ][D] block
-    if (nsplit == 1) {
-      if (P.out_f32) {
-        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(io.out) + (int64_t)tok * HQ * D);
-        const float4* src = reinterpret_cast<const float4*>(st32);
-        for (int e = threadIdx.x; e < HQ * D / 4; e += kThreads) dst[e] = src[e];
-      } else {
-        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(io.out) + (int64_t)tok * HQ * D);
-        const uint4* src = reinterpret_cast<const uint4*>(st16);
-        for (int e = threadIdx.x; e < HQ * D / 8; e += kThreads) dst[e] = src[e];
+    // staging -> global: the contiguous [HQ][D] block in one bulk copy (16-byte
+    // stores by every thread when the destination is not 16-byte aligned)
+    uint8_t* dst = nsplit > 1 ? reinterpret_cast<uint8_t*>(P.part_o + (slot0 + split) * HQ * D)
+                              : reinterpret_cast<uint8_t*>(io.out) + (int64_t)tok * HQ * D * (P.out_f32 ? 4 : 2);
+    const uint32_t bytes = (uint32_t)HQ * D * (f32_stage ? 4 : 2);
+    if ((reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+      if (threadIdx.x == 0) {
+        for (uint32_t off = 0; off < bytes; off += 32768)
+          tc::bulk_store(dst + off, sbase + Ly::kOffTile + off, min(32768u, bytes - off));
+        tc::bulk_commit();
+        tc::bulk_wait_all();
+        tc::fence_proxy_async_global();  // before the split-arrival atomic below
       }
     } else {
-      float4* dst = reinterpret_cast<float4*>(P.part_o + (slot0 + split) * HQ * D);
-      const float4* src = reinterpret_cast<const float4*>(st32);
-      for (int e = threadIdx.x; e < HQ * D / 4; e += kThreads) dst[e] = src[e];
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(smem + Ly::kOffTile);
+      for (uint32_t e = threadIdx.x; e < bytes / 4; e += kThreads) {
+        const uint32_t v = src[e];
+        memcpy(dst + 4 * e, &v, 4);
+      }
     }
     if (threadIdx.x < HQ) {
       const int hh = threadIdx.x;

@@ -106,6 +106,32 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
+// Named barrier `id` over `n` threads (multiple of 32) that also returns the
+// AND of `pred` over them.
+__device__ __forceinline__ bool named_sync_and(uint32_t id, uint32_t n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+// Group-wide wait: one thread of the group (`leader`) probes the mbarrier,
+// the others are parked on the named barrier `id` (hardware barriers take no
+// issue slots and no probe bandwidth); every thread gets the result.  With
+// `skip` the leader does not probe and the group gets false.
+__device__ __forceinline__ bool mbar_wait_group(uint32_t bar, uint32_t parity, uint64_t limit_ns, bool leader,
+                                                bool skip, uint32_t id, uint32_t n) {
+  bool ok = true;
+  if (leader) ok = !skip && mbar_wait_bounded(bar, parity, limit_ns);
+  return named_sync_and(id, n, ok);
+}
+
 // Warp-wide wait: only lane 0 probes the barrier (the other lanes are parked
 // at the shuffle and take no issue slots); every lane gets the result.
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, uint64_t limit_ns) {

@@ -13,7 +13,7 @@
 //   warp 0      TMA producer: tiles of 128 positions of the FP4 indexer K cache
 //               (codes with the 64B/32B swizzle the MMA expects, plus the raw
 //               E4M3 scales) into a 12-stage shared-memory ring;
-//   warp 19     scale-factor warp (two tiles per pass): rearrange each landed tile's scales into
+//   warps 19,20 scale-factor warps (alternate passes of two tiles): rearrange each landed tile's scales into
 //               the tensor-core scale-factor layout (each per-32 E4M3 scale
 //               written twice, as the block-scaled MMA takes one UE4M3 scale
 //               per 16 elements) and copies them to TMEM (tcgen05.cp); a
@@ -48,9 +48,9 @@ constexpr int kChunk = 64;      // rows per TMA box
 constexpr int kAccUnits = 4;    // TMEM accumulator ring, 64 columns each
 constexpr int kMaxW = 8;        // query tokens of one sequence per tile
 constexpr int kEpiWG = 4;       // epilogue warpgroups (warps 2..17)
-constexpr int kThreads = 640;   // 20 warps: producer, 2 MMA issuers, 4 epilogue warpgroups, scale-factor warp
+constexpr int kThreads = 672;   // 21 warps: producer, 2 MMA issuers, 4 epilogue warpgroups, 2 scale-factor warps
 constexpr int kMmaWarpB = 18;   // second MMA issuer (the first is warp 1); they take alternate tiles
-constexpr int kSfWarp = 19;     // scale-factor warp
+constexpr int kSfWarp = 19;     // scale-factor warps 19 and 20 take alternate passes of two tiles
 constexpr int kUnitsPer = kAccUnits / 2;  // accumulator units of each MMA issuer (one per epilogue warpgroup)
 static_assert(kUnitsPer * 2 == kEpiWG, "one accumulator unit per epilogue warpgroup");
 constexpr uint32_t kColAcc = 0;
@@ -261,10 +261,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int64_t g0 = 0; g0 < total; g0 += G) {
       const bool act = has_slot && ti.valid();
       const int s = (int)(it % kStages);
-      const uint32_t n = (uint32_t)(it / kStages);
-      if (act && bx == 0) {
-        if (wait_or_abort(bar_empty + 8 * s, (n & 1) ^ 1, P, abort)) tc::mbar_arrive_expect_tx(bar_full + 8 * s, tx);
+      // lane 0 alone waits for the group's stages (they free up in order);
+      // the first lane of each tile then arms its stage
+      if (lane == 0) {
+        for (int k = 0; k < G && g0 + k < total; ++k) {
+          const int64_t tk = g0 + k;
+          if (!wait_or_abort(bar_empty + 8 * (int)(tk % kStages), ((uint32_t)(tk / kStages) & 1) ^ 1, P, abort)) break;
+        }
       }
+      __syncwarp();
+      if (act && bx == 0 && !*abort) tc::mbar_arrive_expect_tx(bar_full + 8 * s, tx);
       __syncwarp();  // every stage of this group armed before any copy lands
       if (act && !*abort) {
         if (ti.b != cur_g) {
@@ -447,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait_bounded(my_drain, drain_n & 1, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
     }
     __syncwarp();
-  } else if (warp == kSfWarp) {
+  } else if (warp == kSfWarp || warp == kSfWarp + 1) {
     // ------------------------------------------------------------ scale factors
     // raw [row][spr] -> [m0 (32)][m1 (4)][k (4)] per 64-element K step, each
     // per-32 scale written twice (the MMA takes one scale per 16 elements);
@@ -458,8 +464,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     int64_t it = 0;
     constexpr int kBoxRows = kRescore ? kBlock : kChunk;
     constexpr uint32_t kSlot = kRescore ? kRawStage / 16 : kRawStage / 2;
+    const int sfw = warp - kSfWarp;
+    int64_t pass = 0;
     while (ti.valid()) {
       const int nt = ti.left >= 2 ? 2 : 1;
+      if ((int)(pass++ & 1) != sfw) {  // the other scale-factor warp's pass
+        for (int k = 0; k < nt; ++k) ti.next(P);
+        it += nt;
+        continue;
+      }
       uint32_t wv[2][4];
       bool ok = true;
 #pragma unroll
@@ -512,8 +525,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // drain: our copies must have landed before teardown
     if (lane == 0) {
-      tc::commit(bar_drain2);
-      if (!mbar_wait_bounded(bar_drain2, 0, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
+      const uint32_t dr = sfw == 0 ? bar_drain2 : bar_drain_c;
+      tc::commit(dr);
+      if (!mbar_wait_bounded(dr, 0, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
     }
     __syncwarp();
   } else {
@@ -530,6 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int64_t it = 0;
     int cnt = 0;  // jobs of this warpgroup's issuer (all parities)
     int cur_b = -1, W = 0, tok0 = 0;
+    bool dead = false;  // warpgroup-uniform: a wait of this warpgroup gave up
     // no early exit: the four warps of the warpgroup meet at named barriers
     for (; ti.valid(); ti.next(P), ++it) {
       if (ti.b != cur_b) {
@@ -545,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ept < W) pos_g[ept] = __ldg(P.qb.tok_pos + tok0 + ept);
         tc::named_sync(1 + wg, 128);
       }
-      if ((int)(it & 1) != mw || *abort) continue;  // the other issuer's tile (or nothing left to do)
+      if ((int)(it & 1) != mw || dead) continue;  // the other issuer's tile (or nothing left to do)
       const int64_t t0 = (int64_t)ti.tile * kTile;
       for (int j = 0; j < W; ++j) {
         const int tok = tok0 + j;
@@ -555,7 +570,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (job % kUnitsPer != sub) continue;  // the other warpgroup of this issuer
         const int u = mw + 2 * sub;
         const uint32_t m = (uint32_t)(job / kUnitsPer);
-        if (!warp_wait_or_abort(bar_accf + 8 * u, m & 1, P, abort)) break;
+        // one prober per warpgroup; the other warps park on the named barrier
+        if (!mbar_wait_group(bar_accf + 8 * u, m & 1, P.wait_ns, ept == 0, *abort != 0, 1 + wg, 128)) {
+          if (ept == 0 && !*abort) {
+            set_status(P.status, CSA2_ERR_TIMEOUT);
+            *abort = 1;
+          }
+          dead = true;
+          break;
+        }
         tc::fence_after_sync();
         const float* wj = w_g + j * 64;
         const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + kColAcc + u * 64;

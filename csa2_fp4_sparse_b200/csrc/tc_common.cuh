@@ -44,6 +44,21 @@ __device__ __forceinline__ void tma_load_1d(uint32_t dst, const void* tmap, uint
       : "memory");
 }
 
+// bulk copy shared -> global (untiled; both addresses 16-byte aligned, size a
+// multiple of 16), tracked by this thread's bulk groups
+__device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// every bulk group of this thread complete (writes performed)
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// order this thread's async-proxy global writes with its later generic-proxy operations
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // generic-proxy shared-memory writes -> visible to the async proxy (tcgen05.cp / mma reads)
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

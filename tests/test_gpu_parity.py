@@ -143,6 +143,18 @@ def test_stack_config1_full_size():
     _check_all(w, dw, range(w.T))
 
 
+@pytest.mark.parametrize("i", [2, 3, 4, 5])
+def test_stack_full_size_sampled(i):
+    """The full-size workloads the benchmark times (same kernels and grids),
+    graded on sampled query tokens: the first, the last and two seeded picks,
+    every layer of each."""
+    from synth.workloads import CONFIGS
+    w, dw = _run_stack(CONFIGS[i])
+    rng = np.random.default_rng(100 + i)
+    toks = sorted(set([0, w.T - 1] + rng.choice(w.T, size=min(2, w.T), replace=False).tolist()))
+    _check_all(w, dw, toks)
+
+
 @pytest.mark.parametrize("case", [
     dict(i=2, B=2, lengths=("fixed", 5000)),
     dict(i=2, B=3, lengths=("list", [8, 9, 1000])),                        # tiny contexts, partial blocks
