@@ -12,18 +12,22 @@
 // Design (one persistent CTA per SM, warp-specialised):
 //   warp 0      TMA producer: tiles of 128 positions of the FP4 indexer K cache
 //               (codes with the 64B/32B swizzle the MMA expects, plus the raw
-//               E4M3 scales) into a 12-stage shared-memory ring;
-//   warps 19,20 scale-factor warps (alternate passes of two tiles): rearrange each landed tile's scales into
-//               the tensor-core scale-factor layout (each per-32 E4M3 scale
-//               written twice, as the block-scaled MMA takes one UE4M3 scale
-//               per 16 elements) and copies them to TMEM (tcgen05.cp); a
-//               commit hands the stage to the MMA warp, so the copy never
-//               queues behind that warp's earlier MMAs;
+//               E4M3 scales) into a shared-memory ring of 17 stages (15 when
+//               rescoring);
+//   warps 19,20 scale-factor warps (alternate passes of two tiles):
+//               rearrange each landed tile's scales into the tensor-core
+//               scale-factor layout (each per-32 E4M3 scale written twice, as
+//               the block-scaled MMA takes one UE4M3 scale per 16 elements)
+//               and copy it to TMEM (tcgen05.cp); a commit hands the stage to
+//               the MMA warp;
 //   warps 1, 18 MMA issuers (alternate tiles, two epilogue warpgroups each):
-//               issue tcgen05.mma kind::mxf4nvf4 (M = 128 positions, N = heads,
-//               K = 64 per instruction) per query token into a ring of TMEM
-//               accumulators; commits release the smem stage and hand the
-//               accumulator to the epilogue;
+//               issue tcgen05.mma kind::mxf4nvf4 (M = 128 positions, N =
+//               heads, K = 64 per instruction) per query token into a ring of
+//               TMEM accumulators (2 units per issuer); one commit per job hands
+//               the accumulator to the epilogue, one per tile returns the
+//               stage to the producer.  A tcgen05 instruction costs its
+//               issuing thread 100-200 cycles, so the copies are issued by the
+//               scale-factor warps, not here;
 //   warps 2..17 epilogue, four warpgroups: warpgroup e takes the accumulator
 //               jobs of MMA warp (e & 1) whose job count has parity e >> 1:
 //               TMEM -> registers (one position per thread), ReLU, weighted
@@ -42,40 +46,47 @@
 namespace csa2 {
 namespace scan_tc {
 
-constexpr int kStages = 12;
 constexpr int kTile = 128;      // positions per tile = MMA M
 constexpr int kChunk = 64;      // rows per TMA box
-constexpr int kAccUnits = 4;    // TMEM accumulator ring, 64 columns each
+constexpr int kAccUnits = 4;    // TMEM accumulator ring, 64 columns each (2 per MMA issuer)
 constexpr int kMaxW = 8;        // query tokens of one sequence per tile
 constexpr int kEpiWG = 4;       // epilogue warpgroups (warps 2..17)
 constexpr int kThreads = 672;   // 21 warps: producer, 2 MMA issuers, 4 epilogue warpgroups, 2 scale-factor warps
 constexpr int kMmaWarpB = 18;   // second MMA issuer (the first is warp 1); they take alternate tiles
 constexpr int kSfWarp = 19;     // scale-factor warps 19 and 20 take alternate passes of two tiles
-constexpr int kUnitsPer = kAccUnits / 2;  // accumulator units of each MMA issuer (one per epilogue warpgroup)
-static_assert(kUnitsPer * 2 == kEpiWG, "one accumulator unit per epilogue warpgroup");
+constexpr int kUnitsPer = kAccUnits / 2;  // accumulator units of each MMA issuer
 constexpr uint32_t kColAcc = 0;
-constexpr uint32_t kColSfa = kAccUnits * 64;              // 256
-constexpr uint32_t kColSfb = kColSfa + kStages * 8;      // 352
-static_assert(kColSfb + kMaxW * 8 <= 512, "TMEM budget");
 constexpr uint32_t kTmemCols = 512;
 
-// shared-memory map (offsets from a 1024-aligned base)
-constexpr uint32_t kOffA = 0;                             // [kStages][8192]
-// raw scales: every TMA box gets its own 128-byte-aligned slot (TMA writes
-// shared memory at 128-byte-aligned addresses): scan 2 boxes at 1024-byte
-// slots, rescoring 16 boxes at 128-byte slots
-constexpr uint32_t kRawStage = 2048;
-constexpr uint32_t kOffRaw = kOffA + kStages * 8192;      // [kStages][2048]
-constexpr uint32_t kOffSfa = kOffRaw + kStages * kRawStage;  // [kStages][2][512]
-constexpr uint32_t kOffB = kOffSfa + kStages * 1024;      // [kMaxW][64 rows][64 B]
-constexpr uint32_t kOffSfb = kOffB + kMaxW * 4096;        // [kMaxW][2][512]
-constexpr uint32_t kOffW = kOffSfb + kMaxW * 1024;        // [kEpiWG][kMaxW][64] f32
-constexpr uint32_t kOffPos = kOffW + kEpiWG * kMaxW * 64 * 4;  // [1 + kEpiWG][kMaxW] i64 query positions (MMA warps, epilogue warpgroups)
-constexpr uint32_t kOffBar = kOffPos + (1 + kEpiWG) * kMaxW * 8;  // mbarriers
-constexpr uint32_t kNumBars = 3 * kStages + 2 * kAccUnits + 5;
-constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;     // tmem base, abort flag
-constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;     // + alignment slack
-static_assert(kOffB % 1024 == 0, "B tiles must be 1024-aligned");
+// Shared-memory and TMEM map.  A tile's stage stays occupied from its load
+// to the completion of its MMAs (~8-9 K cycles: load latency under full HBM
+// load, scale-factor pass, MMA), so the ring is as deep as shared memory
+// allows: 17 stages for the scan, 15 for the rescoring (whose raw-scale slot
+// holds 16 gathered boxes).
+template <bool kRescore>
+struct Ly {
+  static constexpr int kStages = kRescore ? 15 : 17;
+  // raw scales: every TMA box gets its own 128-byte-aligned slot (TMA writes
+  // shared memory at 128-byte-aligned addresses): scan 2 boxes at 256-byte
+  // slots, rescoring 16 boxes at 128-byte slots
+  static constexpr uint32_t kRawStage = kRescore ? 2048 : 512;
+  static constexpr uint32_t kColSfa = kAccUnits * 64;            // key scale factors, 8 columns per stage
+  static constexpr uint32_t kColSfb = kColSfa + kStages * 8;     // query scale factors, 8 columns per token
+  static_assert(kColSfb + kMaxW * 8 <= kTmemCols, "TMEM budget");
+  static constexpr uint32_t kOffA = 0;                                   // [kStages][8192]
+  static constexpr uint32_t kOffRaw = kOffA + kStages * 8192;            // [kStages][kRawStage]
+  static constexpr uint32_t kOffSfa = kOffRaw + kStages * kRawStage;     // [kStages][2][512]
+  static constexpr uint32_t kOffB = (kOffSfa + kStages * 1024 + 1023) / 1024 * 1024;  // [kMaxW][64 rows][64 B]
+  static constexpr uint32_t kOffSfb = kOffB + kMaxW * 4096;              // [kMaxW][2][512]
+  static constexpr uint32_t kOffW = kOffSfb + kMaxW * 1024;              // [kEpiWG][kMaxW][64] f32
+  static constexpr uint32_t kOffPos = kOffW + kEpiWG * kMaxW * 64 * 4;   // [1 + kEpiWG][kMaxW] i64 query positions
+  static constexpr uint32_t kOffBar = kOffPos + (1 + kEpiWG) * kMaxW * 8;  // mbarriers
+  static constexpr uint32_t kNumBars = 3 * kStages + 2 * kAccUnits + 5;
+  static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;           // tmem base, abort flag
+  static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;           // + alignment slack
+  static_assert(kOffB % 1024 == 0, "B tiles must be 1024-aligned");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
 
 struct Params {
   csa2_query_batch qb;
@@ -185,6 +196,12 @@ template <bool kRescore>
 __global__ void __launch_bounds__(kThreads, 1)
     k_index_tc(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales,
                const __grid_constant__ Params P) {
+  using L = Ly<kRescore>;
+  constexpr int kStages = L::kStages;
+  constexpr uint32_t kRawStage = L::kRawStage;
+  constexpr uint32_t kOffA = L::kOffA, kOffRaw = L::kOffRaw, kOffSfa = L::kOffSfa, kOffB = L::kOffB,
+                     kOffSfb = L::kOffSfb, kOffW = L::kOffW, kOffPos = L::kOffPos, kOffBar = L::kOffBar,
+                     kOffMisc = L::kOffMisc, kColSfa = L::kColSfa, kColSfb = L::kColSfb;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -247,7 +264,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int32_t oob_x = (int32_t)(((P.n_rows * spr) + 15) / 16 * 16);
     constexpr int boxes = kRescore ? 16 : 2;
     constexpr int rows_per_box = kTile / boxes;
-    constexpr int G = (32 / boxes) < 8 ? (32 / boxes) : 8;  // <= kStages: no lane waits on a tile of its own group
+    // tiles per group: a group is issued once all its stages are free, so a
+    // small group keeps most of the ring in flight
+    constexpr int G = (32 / boxes) < 4 ? (32 / boxes) : 4;
     const int lt = lane / boxes, bx = lane % boxes;
     const bool has_slot = lane < G * boxes;
     TileIter<kRescore> ti;
@@ -261,16 +280,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int64_t g0 = 0; g0 < total; g0 += G) {
       const bool act = has_slot && ti.valid();
       const int s = (int)(it % kStages);
-      // lane 0 alone waits for the group's stages (they free up in order);
-      // the first lane of each tile then arms its stage
-      if (lane == 0) {
-        for (int k = 0; k < G && g0 + k < total; ++k) {
-          const int64_t tk = g0 + k;
-          if (!wait_or_abort(bar_empty + 8 * (int)(tk % kStages), ((uint32_t)(tk / kStages) & 1) ^ 1, P, abort)) break;
-        }
+      const uint32_t n = (uint32_t)(it / kStages);
+      // the first lane of each tile waits for its stage and arms it (one warp
+      // instruction probes the stages of all the group's tiles at once)
+      if (act && bx == 0) {
+        if (wait_or_abort(bar_empty + 8 * s, (n & 1) ^ 1, P, abort)) tc::mbar_arrive_expect_tx(bar_full + 8 * s, tx);
       }
-      __syncwarp();
-      if (act && bx == 0 && !*abort) tc::mbar_arrive_expect_tx(bar_full + 8 * s, tx);
       __syncwarp();  // every stage of this group armed before any copy lands
       if (act && !*abort) {
         if (ti.b != cur_g) {
@@ -340,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     TileIter<kRescore> ti;
     ti.init(P, wb, we);
     int64_t it = 0;
-    int cnt = 0;  // jobs issued by this warp
+    int cnt = 0;   // jobs issued by this warp
     uint32_t drain_n = 0, sfb_n = 0;
     int cur_b = -1, W = 0, tok0 = 0;
     // No early exit from this loop: both issuers must meet at the same named
@@ -422,11 +437,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         okw = wait_or_abort(bar_sfr + 8 * s, n & 1, P, abort);  // tile landed, scale factors in TMEM
         tc::fence_after_sync();
+        const uint32_t sfa = tmem + kColSfa + (uint32_t)s * 8;
         const int64_t* pos_s = reinterpret_cast<const int64_t*>(smem + kOffPos);
         const int64_t t0 = (int64_t)ti.tile * kTile;
         for (int j = 0; j < W && okw; ++j) {
           if (!kRescore && t0 > pos_s[j]) continue;
-          const int u = mw + 2 * (cnt % kUnitsPer);
+          const int u = mw * kUnitsPer + cnt % kUnitsPer;
           const uint32_t m = (uint32_t)(cnt / kUnitsPer);
           if (!wait_or_abort(bar_acce + 8 * u, (m & 1) ^ 1, P, abort)) {
             okw = false;
@@ -436,12 +452,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int ks = 0; ks < ksteps; ++ks) {
             const uint64_t ad = tc::smem_desc(sbase + kOffA + s * 8192 + ks * 32, 16, sbo, sw);
             const uint64_t bd = tc::smem_desc(sbase + kOffB + j * 4096 + ks * 32, 16, sbo, sw);
-            tc::mma_mxf4nvf4(tmem + kColAcc + u * 64, ad, bd, idesc, tmem + kColSfa + s * 8 + ks * 4,
-                             tmem + kColSfb + j * 8 + ks * 4, ks > 0 ? 1u : 0u);
+            tc::mma_mxf4nvf4(tmem + kColAcc + u * 64, ad, bd, idesc, sfa + ks * 4, tmem + kColSfb + j * 8 + ks * 4,
+                             ks > 0 ? 1u : 0u);
           }
           tc::commit(bar_accf + 8 * u);
           ++cnt;
         }
+        // the stage goes back to the producer as soon as the MMAs that read
+        // it complete
         if (okw) tc::commit(bar_empty + 8 * s);
       }
       cnt = __shfl_sync(0xffffffffu, cnt, 0);
@@ -507,8 +525,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc::fence_proxy_async_smem();
       __syncwarp();
-      // copy to TMEM from this warp, so the copy is not queued behind the MMA
-      // warps' earlier MMAs; each commit hands its stage over once it landed
+      // copy to TMEM from this warp (tcgen05 instructions cost their issuing
+      // thread 100-200 cycles each, so they are spread over the warps that
+      // have time); the commit hands the stage over once the copy landed
       if (lane == 0) {
         tc::fence_after_sync();
         for (int k = 0; k < nt; ++k) {
@@ -567,8 +586,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t p = pos_g[j];
         if (!kRescore && t0 > p) continue;
         const int job = cnt++;
-        if (job % kUnitsPer != sub) continue;  // the other warpgroup of this issuer
-        const int u = mw + 2 * sub;
+        if ((job & 1) != sub) continue;  // the other warpgroup of this issuer
+        const int u = mw * kUnitsPer + job % kUnitsPer;
         const uint32_t m = (uint32_t)(job / kUnitsPer);
         // one prober per warpgroup; the other warps park on the named barrier
         if (!mbar_wait_group(bar_accf + 8 * u, m & 1, P.wait_ns, ept == 0, *abort != 0, 1 + wg, 128)) {
@@ -736,19 +755,20 @@ static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const 
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
     if (int rc = cuda_check(
-            cudaFuncSetAttribute(k_index_tc<kRescore>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes),
+            cudaFuncSetAttribute(k_index_tc<kRescore>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Ly<kRescore>::kSmemBytes),
             "index smem attribute"))
       return rc;
     int fit = 0;  // one CTA of kThreads threads at this register count must fit on an SM
     if (int rc = cuda_check(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, k_index_tc<kRescore>, kThreads,
-                                                                          kSmemBytes),
+                                                                          Ly<kRescore>::kSmemBytes),
                             "index occupancy"))
       return rc;
     if (fit < 1) return fail(CSA2_ERR_UNSUPPORTED, "index kernel does not fit on an SM");
     attr_done[dev] = true;
   }
   Launch L_(kRescore ? "rescore_tc" : "scan_tc", st);
-  k_index_tc<kRescore><<<num_sms(), kThreads, kSmemBytes, st>>>(tmc, tms, p);
+  k_index_tc<kRescore><<<num_sms(), kThreads, Ly<kRescore>::kSmemBytes, st>>>(tmc, tms, p);
   return cuda_check(cudaGetLastError(), "k_index_tc");
 }
 
