@@ -16,10 +16,14 @@
 //                dequantise them exactly to fp16 (E2M1 x E4M3 products, or
 //                E4M3 window codes) into a 128B-swizzled tile
 //                [64-element d-block][row][128 B];
-//   warp 12      issues S = Q K^T on tcgen05 (kind::f16, M = 64 heads, N = 64
-//                rows, K = D) into one of two TMEM score buffers;
-//   warps 0..3   softmax, one thread per head (M = 64 keeps head h in TMEM lane
-//                32*(h/16) + h%16): running (log2) max that only moves when a
+//   warps 12,14  issue S = Q K^T on tcgen05 (kind::f16, M = 64 heads, N = 64
+//                rows, K = D) into one of two TMEM score buffers (alternate
+//                chunks: each MMA costs its issuing thread ~110 cycles);
+//   warps 0..3   softmax, two threads per head (M = 64 keeps head h in TMEM
+//                lane 32*(h/16) + h%16; the 16x32bx2 load gives lanes t and
+//                t+16 of a warp the two halves of head t's scores): one pass
+//                per chunk against the running (log2) max, which only moves
+//                (with a second pass) when a
 //                chunk exceeds it by more than 2^8 (then the output
 //                accumulator is rescaled), P = 2^(z - m) written as fp16 rows
 //                [head][row] (window rows carry their per-token scale into P);
@@ -39,12 +43,14 @@ constexpr int kRows = 64;       // rows per chunk (MMA N of S, K of PV)
 constexpr int kMq = 64;         // MMA M of S: heads, padded to 64
 constexpr int kSoftWarps = 4;   // warps 0..3
 constexpr int kLoadWarps = 8;   // warps 4..11
-constexpr int kWarpS = 12;      // S issuer
+constexpr int kWarpS = 12;      // S issuers: warp 12 (even chunks) and warp 14 (odd chunks); a
+                                // tcgen05.mma costs its issuing thread ~110 cycles
+constexpr int kWarpS2 = 14;
 constexpr int kWarpPV = 13;     // PV issuer
-constexpr int kThreads = 448;
+constexpr int kThreads = 480;
 constexpr int kLoadThreads = kLoadWarps * 32;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRescaleLog2 = 8.0f;  // P stays <= 2^8 between rescales (fp16-safe)
+constexpr float kRescaleLog2 = 15.0f;  // P = 2^(z - m) stays <= 2^15 between rescales (fp16 holds it)
 
 constexpr int kMaxLayers = 32;  // layers attended in one launch (grid.z), each with its own index list
 constexpr int kMaxRows = 2048;  // K: selected rows per query token
@@ -176,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
       mbar_init(bar_s_full + 8 * i, 1);
       mbar_init(bar_p_full + 8 * i, kSoftWarps);
     }
-    mbar_init(bar_drain, 2);
+    mbar_init(bar_drain, 3);  // two S issuers and the PV issuer
     *abort = 0;
     tc::fence_barrier_init();
   }
@@ -402,10 +408,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
       if (lane == 0) tc::mbar_arrive(bar_kv_full + 8 * bf);
       cur = nxt;
     }
-  } else if (warp == kWarpS) {
+  } else if (warp == kWarpS || warp == kWarpS2) {
     // ------------------------------------------------------------ S = Q K^T
     const uint32_t idesc = tc::idesc_f16(kMq, kRows, 0, 0);
-    for (int i = 0; i < n_mine; ++i) {
+    const int par = warp == kWarpS ? 0 : 1;
+    for (int i = par; i < n_mine; i += 2) {
       const int bf = i & 1;
       if (lane == 0 && !*abort) {
         if (!mbar_wait_bounded(bar_kv_full + 8 * bf, (i >> 1) & 1, P.wait_ns)) {
@@ -467,13 +474,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
     __syncwarp();
   } else if (warp < kSoftWarps) {
     // ------------------------------------------------------------ softmax
-    // thread = head h = 16 * warp + lane (lanes 16..31 carry no head)
-    const int h = 16 * warp + lane;
-    const bool act = lane < 16 && h < HQ;
+    // head h = 16 * warp + (lane & 15); lane half `hf` takes rows [32 hf, 32 hf + 32)
+    // of each chunk (the 16x32bx2 TMEM load hands them over)
+    const int hf = lane >> 4;
+    const int h = 16 * warp + (lane & 15);
+    const bool act = h < HQ;
     const uint32_t s_lane = tmem + ((uint32_t)(warp * 32) << 16);
     const float zs = P.scale * kLog2e;
-    float m = -INFINITY, l = 0.0f;
-    bool dead = false;  // uniform over the softmax warps: a wait gave up
+    float m = -INFINITY, l = 0.0f;  // l: this half's rows
+    bool dead = false;              // uniform over the softmax warps: a wait gave up
     for (int i = 0; i < n_mine; ++i) {
       const int bf = i & 1;
       // one thread probes, the other softmax threads park on named barrier 1
@@ -487,37 +496,85 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
         dead = true;
       }
       tc::fence_after_sync();
-      const float* rsb = rs_s + bf * kRows;
+      const float* rsb = rs_s + bf * kRows + 32 * hf;  // this half's rows
       const uint32_t s_col = s_lane + Ly::kColS + bf * kRows;
       // every row a valid sparse row (row scale 1): the common case, no per-row scale
-      const bool plain = __all_sync(0xffffffffu, rsb[lane] == 1.0f && rsb[lane + 32] == 1.0f);
-      // pass 1: the chunk's maximum (log2 domain; window rows scaled by s_t)
-      float cm = -INFINITY;
-      if (ok) {
+      const bool plain = __all_sync(0xffffffffu, rs_s[bf * kRows + lane] == 1.0f && rs_s[bf * kRows + lane + 32] == 1.0f);
+      // P = 2^(z - mu) as fp16 [head][row] for this half's 32 rows, their sum,
+      // and the largest z seen; window rows carry s_t into P.  The TMEM loads
+      // are warp-collective: every lane issues them (ok is uniform), only the
+      // lanes that carry a head write P.
+      uint8_t* prow = smem + Ly::kOffP + bf * ((Ly::kPBytes + 1023) / 1024 * 1024);
+      auto p_pass = [&](float mu_, float& sum_, float& zmax_) {
+        const float nmu = mu_ == -INFINITY ? 0.0f : -mu_;
+        sum_ = 0.0f;
+        zmax_ = -INFINITY;
 #pragma unroll
-        for (int g = 0; g < kRows / 16; ++g) {
+        for (int g = 0; g < 2; ++g) {
           uint32_t v[16];
-          tc::ld_32x32b_x16(s_col + g * 16, v);
+          tc::ld_16x32bx2_x16<32>(s_col + g * 16, v);
           tc::ld_wait();
-          if (plain) {
 #pragma unroll
-            for (int k = 0; k < 16; ++k) cm = fmaxf(cm, __uint_as_float(v[k]));
-          } else {
+          for (int cc = 0; cc < 2; ++cc) {
+            uint32_t pk[4];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              const float rsj = rsb[g * 16 + k];
-              if (rsj >= 0.0f) cm = fmaxf(cm, __uint_as_float(v[k]) * rsj);
+            for (int k = 0; k < 4; ++k) {
+              const int jj = cc * 8 + 2 * k, j0 = g * 16 + jj;
+              if (plain) {
+                const float z0 = __uint_as_float(v[jj]) * zs, z1 = __uint_as_float(v[jj + 1]) * zs;
+                zmax_ = fmaxf(zmax_, fmaxf(z0, z1));
+                const float e0 = mu_ == -INFINITY ? 0.0f : ex2_approx(z0 + nmu);
+                const float e1 = mu_ == -INFINITY ? 0.0f : ex2_approx(z1 + nmu);
+                __half2 w2 = __floats2half2_rn(e0, e1);
+                pk[k] = *reinterpret_cast<uint32_t*>(&w2);
+                // the fp16 weights are what PV uses and what the sum adds
+                const float2 back = __half22float2(w2);
+                sum_ += back.x + back.y;
+              } else {
+                const float r0 = rsb[j0], r1 = rsb[j0 + 1];
+                const float z0 = r0 >= 0.0f ? __uint_as_float(v[jj]) * (zs * r0) : -INFINITY;
+                const float z1 = r1 >= 0.0f ? __uint_as_float(v[jj + 1]) * (zs * r1) : -INFINITY;
+                zmax_ = fmaxf(zmax_, fmaxf(z0, z1));
+                float e0 = (mu_ == -INFINITY) ? 0.0f : ex2_approx(z0 + nmu);
+                float e1 = (mu_ == -INFINITY) ? 0.0f : ex2_approx(z1 + nmu);
+                const float w0 = r0 > 0.0f ? r0 : 0.0f, w1 = r1 > 0.0f ? r1 : 0.0f;
+                __half2 w2 = __floats2half2_rn(e0 * w0, e1 * w1);
+                pk[k] = *reinterpret_cast<uint32_t*>(&w2);
+                // sparse rows: sum exactly the fp16 weights the PV product uses
+                const float2 back = __half22float2(w2);
+                if (r0 == 1.0f) e0 = back.x;
+                if (r1 == 1.0f) e1 = back.y;
+                sum_ += e0 + e1;
+              }
             }
+            // 16-byte chunk of 8 rows: rows 32 hf + 16 g + 8 cc ..
+            if (act)
+              *reinterpret_cast<uint4*>(prow + swz128(h, 4 * hf + 2 * g + cc)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
         }
-        cm *= zs;  // zs > 0: scaling after the maximum is the same maximum
+        zmax_ = fmaxf(zmax_, __shfl_xor_sync(0xffffffffu, zmax_, 16));  // both halves of the head
+      };
+      float mu = m, sum = 0.0f;
+      if (ok) {
+        // a head without a running max yet starts from this chunk's maximum
+        const bool first = __any_sync(0xffffffffu, act && m == -INFINITY);
+        float zmax;
+        if (first) {
+          p_pass(-INFINITY, sum, zmax);  // max only (no weights: every e is 0)
+          if (m == -INFINITY) mu = zmax;
+        }
+        p_pass(mu, sum, zmax);
+        // the running max moves only when the chunk exceeds it by more than
+        // 2^15 (rare after the first chunk): the chunk is redone
+        const bool redo = act && mu != -INFINITY && zmax > mu + kRescaleLog2;
+        if (__any_sync(0xffffffffu, redo)) {
+          if (redo) mu = zmax;
+          p_pass(mu, sum, zmax);
+        }
       }
-      // running max: moves only when the chunk exceeds it by more than 2^8
-      float mu = m;
-      if (m == -INFINITY || cm > m + kRescaleLog2) mu = cm;
       const bool resc = act && m != -INFINITY && mu != m;
       const float corr = resc ? exp2f(m - mu) : 1.0f;
-      if (act) corr_s[h] = corr;
+      if (act && hf == 0) corr_s[h] = corr;
       const bool any = soft_sync_or(resc);  // also publishes corr_s
       if (any && i > 0 && ok) {
         // rescale the output accumulator of earlier chunks (rare): PV(i - 1)
@@ -545,65 +602,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
           tc::st_wait();
         }
       }
-      // pass 2: P = 2^(z - m) as fp16 [head][row]; window rows carry s_t into P.
-      // The TMEM loads are warp-collective: every lane issues them (ok is
-      // uniform), only the lanes that carry a head write P.
-      if (ok) {
-        uint8_t* prow = smem + Ly::kOffP + bf * ((Ly::kPBytes + 1023) / 1024 * 1024);
-        const float nmu = mu == -INFINITY ? 0.0f : -mu;
-        float sum = 0.0f;
-#pragma unroll
-        for (int g = 0; g < kRows / 16; ++g) {
-          uint32_t v[16];
-          tc::ld_32x32b_x16(s_col + g * 16, v);
-          tc::ld_wait();
-#pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int jj = cc * 8 + 2 * k, j0 = g * 16 + jj;
-              if (plain) {
-                // e = 2^(s * zs - mu); the fp16 weight is what PV uses and what the sum adds
-                const float e0 = ex2_approx(fmaf(__uint_as_float(v[jj]), zs, nmu));
-                const float e1 = ex2_approx(fmaf(__uint_as_float(v[jj + 1]), zs, nmu));
-                __half2 w2 = __floats2half2_rn(e0, e1);
-                pk[k] = *reinterpret_cast<uint32_t*>(&w2);
-                const float2 back = __half22float2(w2);
-                sum += back.x + back.y;
-              } else {
-                const float r0 = rsb[j0], r1 = rsb[j0 + 1];
-                const float z0 = r0 >= 0.0f ? __uint_as_float(v[jj]) * (zs * r0) : -INFINITY;
-                const float z1 = r1 >= 0.0f ? __uint_as_float(v[jj + 1]) * (zs * r1) : -INFINITY;
-                float e0 = (mu == -INFINITY) ? 0.0f : ex2_approx(z0 + nmu);
-                float e1 = (mu == -INFINITY) ? 0.0f : ex2_approx(z1 + nmu);
-                const float w0 = r0 > 0.0f ? r0 : 0.0f, w1 = r1 > 0.0f ? r1 : 0.0f;
-                __half2 w2 = __floats2half2_rn(e0 * w0, e1 * w1);
-                pk[k] = *reinterpret_cast<uint32_t*>(&w2);
-                // sparse rows: sum exactly the fp16 weights the PV product uses
-                const float2 back = __half22float2(w2);
-                if (r0 == 1.0f) e0 = back.x;
-                if (r1 == 1.0f) e1 = back.y;
-                sum += e0 + e1;
-              }
-            }
-            if (act) *reinterpret_cast<uint4*>(prow + swz128(h, g * 2 + cc)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          }
-        }
-        if (act) {
-          l = l * corr + sum;
-          m = mu;
-        }
+      if (ok && act) {
+        l = l * corr + sum;
+        m = mu;
       }
       tc::fence_proxy_async_smem();
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(bar_p_full + 8 * bf);
     }
-    if (act) {
-      l_s[h] = l;
+    const float lt = l + __shfl_xor_sync(0xffffffffu, l, 16);  // both halves of the head
+    if (act && hf == 0) {
+      l_s[h] = lt;
       m_s[h] = m;
-      corr_s[h] = l > 0.0f ? 1.0f / l : 0.0f;  // reciprocal row sum for the epilogue
+      corr_s[h] = lt > 0.0f ? 1.0f / lt : 0.0f;  // reciprocal row sum for the epilogue
     }
   }
   // ---- epilogue: every warp; the tiles are free once the last PV completed
