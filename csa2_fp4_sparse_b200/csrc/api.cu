@@ -153,27 +153,33 @@ static size_t attend_ws(const csa2_query_batch* qb, int Hq, int D, int K, const 
 }
 
 // ---------------------------------------------------------------- launches
-// n_src sources of rows_per_src rows each, quantised into consecutive rows
-static int launch_quantize_multi(const float* const* xs, int n_src, int64_t rows_per_src, int dim,
-                                 const int64_t* slot, uint8_t* codes, uint8_t* scales, cudaStream_t st) {
-  const int64_t n_rows = (int64_t)n_src * rows_per_src;
-  if (n_rows == 0) return CSA2_OK;
-  if (n_src < 1 || n_src > kQuantSrc || (slot && n_src != 1))
-    return fail(CSA2_ERR_UNSUPPORTED, "1..%d quantisation sources", kQuantSrc);
-  QuantSrc src{};
-  for (int i = 0; i < n_src; ++i) src.x[i] = xs[i];
-  src.rows_per_src = rows_per_src;
-  int64_t work = n_rows * (dim / 8);
-  int64_t grid = (work + 255) / 256;
+// every job of `J` (jobs with no rows dropped) in one launch
+static int launch_quantize_jobs(QuantJobs& J, cudaStream_t st) {
+  const int64_t total = J.begin[J.n];
+  if (total == 0) return CSA2_OK;
+  int64_t grid = (total + 255) / 256;
   if (grid > 148 * 32) grid = 148 * 32;
   Launch L_("quantize_fp4", st);
-  k_quantize_fp4<<<(int)grid, 256, 0, st>>>(src, n_rows, dim, slot, codes, scales, status_ptr());
+  k_quantize_fp4<<<(int)grid, 256, 0, st>>>(J, status_ptr());
   return cuda_check(cudaGetLastError(), "k_quantize_fp4");
+}
+
+// appends a job of `rows` rows to J (returns false when J is full)
+static bool add_quant_job(QuantJobs& J, const float* x, int64_t rows, int dim, const int64_t* slot, uint8_t* codes,
+                          uint8_t* scales) {
+  if (rows <= 0) return true;
+  if (J.n >= kQuantJobs) return false;
+  J.job[J.n] = QuantJob{x, slot, codes, scales, dim};
+  J.begin[J.n + 1] = J.begin[J.n] + rows * (dim / 8);
+  ++J.n;
+  return true;
 }
 
 int launch_quantize(const float* x, int64_t n_rows, int dim, const int64_t* slot, uint8_t* codes, uint8_t* scales,
                     cudaStream_t st) {
-  return launch_quantize_multi(&x, 1, n_rows, dim, slot, codes, scales, st);
+  QuantJobs J{};
+  add_quant_job(J, x, n_rows, dim, slot, codes, scales);
+  return launch_quantize_jobs(J, st);
 }
 
 template <int DI>
@@ -633,16 +639,6 @@ int csa2_decode_stack(const csa2_stack_desc* d, void* workspace, size_t workspac
   size_t sub_bytes = workspace_bytes - sub_off;
   const float scale = d->softmax_scale > 0.0f ? d->softmax_scale : 1.0f / std::sqrt((float)d->kv.dim);
 
-  // append this step's keys and Main KV rows
-  if (d->new_k_idx) {
-    if (!d->new_slot_k_idx) return fail(CSA2_ERR_INVALID_ARG, "new_k_idx needs new_slot_k_idx");
-    if (int rc = launch_quantize(d->new_k_idx, T, dI, d->new_slot_k_idx, d->k_idx.codes, d->k_idx.scales, st))
-      return rc;
-  }
-  if (d->new_kv) {
-    if (!d->new_slot_kv) return fail(CSA2_ERR_INVALID_ARG, "new_kv needs new_slot_kv");
-    if (int rc = launch_quantize(d->new_kv, T, d->kv.dim, d->new_slot_kv, d->kv.codes, d->kv.scales, st)) return rc;
-  }
   // selector layers in order, and each layer's selector
   std::vector<int> sel_layer;
   std::vector<int> layer_sel(NL);
@@ -650,14 +646,23 @@ int csa2_decode_stack(const csa2_stack_desc* d, void* workspace, size_t workspac
     if (d->layers[l].mode != CSA2_MODE_REUSE) sel_layer.push_back(l);
     layer_sel[l] = (int)sel_layer.size() - 1;
   }
-  // every selector's indexer queries, up to kQuantSrc per launch
-  for (int s0 = 0; s0 < n_sel; s0 += kQuantSrc) {
-    const int n = std::min(kQuantSrc, n_sel - s0);
-    const float* xs[kQuantSrc];
-    for (int i = 0; i < n; ++i) xs[i] = d->layers[sel_layer[s0 + i]].iq;
-    if (int rc = launch_quantize_multi(xs, n, (int64_t)T * d->H_I, dI, nullptr, qc + s0 * q_codes_sz,
-                                       qsc + s0 * q_scales_sz, st))
-      return rc;
+  if (d->new_k_idx && !d->new_slot_k_idx) return fail(CSA2_ERR_INVALID_ARG, "new_k_idx needs new_slot_k_idx");
+  if (d->new_kv && !d->new_slot_kv) return fail(CSA2_ERR_INVALID_ARG, "new_kv needs new_slot_kv");
+  // this step's appended keys and Main KV rows and every selector's indexer
+  // queries: one quantisation launch (more when there are many selectors)
+  {
+    QuantJobs J{};
+    if (d->new_k_idx) add_quant_job(J, d->new_k_idx, T, dI, d->new_slot_k_idx, d->k_idx.codes, d->k_idx.scales);
+    if (d->new_kv) add_quant_job(J, d->new_kv, T, d->kv.dim, d->new_slot_kv, d->kv.codes, d->kv.scales);
+    for (int si = 0; si < n_sel; ++si) {
+      const float* x = d->layers[sel_layer[si]].iq;
+      if (!add_quant_job(J, x, (int64_t)T * d->H_I, dI, nullptr, qc + si * q_codes_sz, qsc + si * q_scales_sz)) {
+        if (int rc = launch_quantize_jobs(J, st)) return rc;
+        J = QuantJobs{};
+        add_quant_job(J, x, (int64_t)T * d->H_I, dI, nullptr, qc + si * q_codes_sz, qsc + si * q_scales_sz);
+      }
+    }
+    if (int rc = launch_quantize_jobs(J, st)) return rc;
   }
   Carve sc_c{sub, sub_bytes};
   const int64_t ld = n_blocks_max(qb);

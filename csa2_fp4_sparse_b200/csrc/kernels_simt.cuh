@@ -13,19 +13,27 @@ namespace csa2 {
 // grid, found by comparing |x| with scale * {.25,.75,1.25,1.75,2.5,3.5,5}
 // (products exact in fp32), ties to the even code.
 // ============================================================================
-// up to kQuantSrc row-major sources of rows_per_src rows each, quantised as
-// one matrix of n_src * rows_per_src rows (sources concatenated in order)
-constexpr int kQuantSrc = 8;
-struct QuantSrc {
-  const float* x[kQuantSrc];
-  int64_t rows_per_src;
+// Quantisation jobs of one launch: each a row-major fp32 matrix [rows][dim]
+// written as codes [row][dim/2] + scales [row][dim/32], rows remapped through
+// `slot` when given (cache append).  A thread takes 8 consecutive elements
+// ("unit"); job j owns units [begin[j], begin[j+1]), multiples of 4, so the 4
+// threads of a 32-element scale group never straddle two jobs.
+constexpr int kQuantJobs = 12;
+struct QuantJob {
+  const float* x;
+  const int64_t* slot;
+  uint8_t* codes;
+  uint8_t* scales;
+  int dim;
+};
+struct QuantJobs {
+  QuantJob job[kQuantJobs];
+  int64_t begin[kQuantJobs + 1];
+  int n;
 };
 
-__global__ void __launch_bounds__(256) k_quantize_fp4(const __grid_constant__ QuantSrc src, int64_t n_rows, int dim,
-                                                      const int64_t* __restrict__ slot, uint8_t* __restrict__ codes,
-                                                      uint8_t* __restrict__ scales, int* status) {
-  const int64_t per_row = dim / 8;
-  const int64_t total = n_rows * per_row;
+__global__ void __launch_bounds__(256) k_quantize_fp4(const __grid_constant__ QuantJobs J, int* status) {
+  const int64_t total = J.begin[J.n];
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t base = (int64_t)blockIdx.x * blockDim.x; base < total; base += stride) {
     int64_t i = base + threadIdx.x;
@@ -34,11 +42,14 @@ __global__ void __launch_bounds__(256) k_quantize_fp4(const __grid_constant__ Qu
     float amax = 0.0f;
     bool bad = false;
     int64_t r = 0, c8 = 0;
+    int jb = 0;
     if (active) {
-      r = i / per_row;
-      c8 = i - r * per_row;
-      const int64_t si = r / src.rows_per_src;
-      const float4* xp = reinterpret_cast<const float4*>(src.x[si] + (r - si * src.rows_per_src) * dim + c8 * 8);
+      while (jb + 1 < J.n && i >= J.begin[jb + 1]) ++jb;
+      const int64_t per_row = J.job[jb].dim / 8;
+      const int64_t li = i - J.begin[jb];
+      r = li / per_row;
+      c8 = li - r * per_row;
+      const float4* xp = reinterpret_cast<const float4*>(J.job[jb].x + r * J.job[jb].dim + c8 * 8);
       float4 a = __ldg(xp), b = __ldg(xp + 1);
       v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
       v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
@@ -54,7 +65,9 @@ __global__ void __launch_bounds__(256) k_quantize_fp4(const __grid_constant__ Qu
     int badq = __shfl_xor_sync(0xffffffffu, (int)bad, 1) | (int)bad;
     badq |= __shfl_xor_sync(0xffffffffu, badq, 2);
     if (!active) continue;
-    int64_t orow = slot ? __ldg(slot + r) : r;
+    const QuantJob& jo = J.job[jb];
+    const int dim = jo.dim;
+    int64_t orow = jo.slot ? __ldg(jo.slot + r) : r;
     uint32_t packed = 0;
     uint8_t sc = 0;
     if (!badq) {
@@ -75,8 +88,8 @@ __global__ void __launch_bounds__(256) k_quantize_fp4(const __grid_constant__ Qu
     } else {
       set_status(status, CSA2_ERR_NONFINITE);
     }
-    *reinterpret_cast<uint32_t*>(codes + orow * (dim / 2) + c8 * 4) = packed;
-    if ((c8 & 3) == 0) scales[orow * (dim / 32) + c8 / 4] = sc;
+    *reinterpret_cast<uint32_t*>(jo.codes + orow * (dim / 2) + c8 * 4) = packed;
+    if ((c8 & 3) == 0) jo.scales[orow * (dim / 32) + c8 / 4] = sc;
   }
 }
 
