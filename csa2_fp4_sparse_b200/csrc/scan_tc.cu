@@ -10,7 +10,10 @@
 // the whole visible context and keeps blocks of 8 positions).
 //
 // Design (one persistent CTA per SM, warp-specialised):
-//   warp 0      TMA producer: tiles of 128 positions of the FP4 indexer K cache
+//   warp 0      TMA producer (rescoring: warps 0, 21, 22 on alternate groups
+//               of tiles, as a TMA instruction costs its warp ~110 cycles and
+//               a rescoring tile gathers 32 boxes): tiles of 128 positions of
+//               the FP4 indexer K cache
 //               (codes with the 64B/32B swizzle the MMA expects, plus the raw
 //               E4M3 scales) into a shared-memory ring of 17 stages (15 when
 //               rescoring);
@@ -51,7 +54,9 @@ constexpr int kChunk = 64;      // rows per TMA box
 constexpr int kAccUnits = 4;    // TMEM accumulator ring, 64 columns each (2 per MMA issuer)
 constexpr int kMaxW = 8;        // query tokens of one sequence per tile
 constexpr int kEpiWG = 4;       // epilogue warpgroups (warps 2..17)
-constexpr int kThreads = 672;   // 21 warps: producer, 2 MMA issuers, 4 epilogue warpgroups, 2 scale-factor warps
+constexpr int kThreads = 736;   // 23 warps: 3 producers, 2 MMA issuers, 4 epilogue warpgroups, 2 scale-factor warps
+constexpr int kProducers = 3;   // TMA producer warps 0, 21, 22 when rescoring (a TMA instruction costs its
+                                // warp ~110 cycles and a rescoring tile gathers 32 boxes); the scan uses warp 0
 constexpr int kMmaWarpB = 18;   // second MMA issuer (the first is warp 1); they take alternate tiles
 constexpr int kSfWarp = 19;     // scale-factor warps 19 and 20 take alternate passes of two tiles
 constexpr int kUnitsPer = kAccUnits / 2;  // accumulator units of each MMA issuer
@@ -254,11 +259,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   int64_t wb, we;
   work_range<kRescore>(P, &wb, &we);
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || warp >= kSfWarp + 2) {
+    // ------------------------------------------------------------ producers
     // G tiles per iteration, `boxes` lanes per tile (scan: 2 boxes of 64 rows,
     // rescore: 16 blocks of 8 rows): the lanes of different tiles wait for
-    // their stages and issue their copies concurrently.
+    // their stages and issue their copies concurrently; the producer warps
+    // take alternate groups of G tiles.
+    const int pi = warp == 0 ? 0 : warp - (kSfWarp + 1);
+    constexpr int nprod = kRescore ? kProducers : 1;  // the scan's 4 boxes a tile need one warp
     const uint32_t tx = (uint32_t)kTile * row_bytes + (uint32_t)kTile * spr;
     const int32_t oob_row = (int32_t)P.n_rows;
     const int32_t oob_x = (int32_t)(((P.n_rows * spr) + 15) / 16 * 16);
@@ -271,13 +279,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool has_slot = lane < G * boxes;
     TileIter<kRescore> ti;
     ti.init(P, wb, we);
-    for (int k = 0; k < lt; ++k) ti.next(P);
-    int64_t it = lt;  // this lane's tile
-    const int64_t total = we - wb;
-    int64_t issued = 0;
+    for (int k = 0; k < pi * G + lt; ++k) ti.next(P);
+    int64_t it = pi * G + lt;  // this lane's tile
+    const int64_t total = pi < nprod ? we - wb : 0;
     int cur_g = -1, tok0 = 0, b = 0;
     int64_t base = 0, len = 0;
-    for (int64_t g0 = 0; g0 < total; g0 += G) {
+    for (int64_t g0 = pi * G; g0 < total; g0 += nprod * G) {
       const bool act = has_slot && ti.valid();
       const int s = (int)(it % kStages);
       const uint32_t n = (uint32_t)(it / kStages);
@@ -328,20 +335,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       if (*abort) break;
-      issued = min(total, g0 + G);
-      for (int k = 0; k < G; ++k) ti.next(P);
-      it += G;
+      for (int k = 0; k < nprod * G; ++k) ti.next(P);
+      it += nprod * G;
     }
-    // no copy of ours may be in flight when the CTA leaves
-    if (lane == 0) {
-      const uint64_t lim = *abort ? 1000000ull : P.wait_ns;
-      for (int s = 0; s < kStages && issued > 0; ++s) {
-        int64_t uses = issued / kStages + (s < issued % kStages ? 1 : 0);
-        if (uses == 0) continue;
-        uint32_t last = (uint32_t)(uses - 1);
-        if (!mbar_wait_bounded(bar_full + 8 * s, last & 1, lim)) set_status(P.status, CSA2_ERR_TIMEOUT);
-      }
-    }
+    // copies in flight: the scale-factor warps wait for every tile's landing
+    // before the CTA ends (after a failed wait, see the end of the kernel)
   } else if (warp == 1 || warp == kMmaWarpB) {
     // ------------------------------------------------------------ MMA issuers
     // Both issuers walk every tile (so both see every change of group) and
@@ -649,6 +647,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+  }
+  // after a failed wait some tile loads may still be in flight: give them
+  // time to land before the CTA's shared memory is released (bounded)
+  if (threadIdx.x == 0 && *abort) {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 200000ull) __nanosleep(1000);
   }
   __syncthreads();
   if (warp == 1) {
