@@ -17,8 +17,9 @@
 //                E4M3 window codes) into a 128B-swizzled tile
 //                [64-element d-block][row][128 B];
 //   warps 12,14  issue S = Q K^T on tcgen05 (kind::f16, M = 64 heads, N = 64
-//                rows, K = D) into one of two TMEM score buffers (alternate
-//                chunks: each MMA costs its issuing thread ~110 cycles);
+//                rows, K = D) into one of two TMEM score buffers, each warp
+//                half of the d-blocks into its own accumulator (the softmax
+//                adds the two; an MMA costs its issuing thread ~110 cycles);
 //   warps 0..3   softmax, two threads per head (M = 64 keeps head h in TMEM
 //                lane 32*(h/16) + h%16; the 16x32bx2 load gives lanes t and
 //                t+16 of a warp the two halves of head t's scores): one pass
@@ -27,9 +28,10 @@
 //                chunk exceeds it by more than 2^8 (then the output
 //                accumulator is rescaled), P = 2^(z - m) written as fp16 rows
 //                [head][row] (window rows carry their per-token scale into P);
-//   warp 13      issues O^T += V^T P^T (M = 128 latent dims per tile, N =
-//                heads, K = 64 rows) reading the same tile as V; its commit
-//                frees the tile and the P buffer.
+//   warps 13,15  issue O^T += V^T P^T (M = 128 latent dims per tile, N =
+//                heads, K = 64 rows; half of the latent-dim tiles each)
+//                reading the same tile as V; their commits free the tile and
+//                the P buffer.
 // The epilogue divides by the row sum, stages the output in shared memory and
 // writes it with 16-byte stores (or the split's unnormalised partial with its
 // max and sum; the last split of a token merges them).  Every wait is bounded.
@@ -43,11 +45,12 @@ constexpr int kRows = 64;       // rows per chunk (MMA N of S, K of PV)
 constexpr int kMq = 64;         // MMA M of S: heads, padded to 64
 constexpr int kSoftWarps = 4;   // warps 0..3
 constexpr int kLoadWarps = 8;   // warps 4..11
-constexpr int kWarpS = 12;      // S issuers: warp 12 (even chunks) and warp 14 (odd chunks); a
-                                // tcgen05.mma costs its issuing thread ~110 cycles
+constexpr int kWarpS = 12;      // S issuers: warps 12 and 14 take the two halves of the d-blocks of every
+                                // chunk (a tcgen05.mma costs its issuing thread ~110 cycles)
 constexpr int kWarpS2 = 14;
-constexpr int kWarpPV = 13;     // PV issuer
-constexpr int kThreads = 480;
+constexpr int kWarpPV = 13;     // PV issuers: warps 13 and 15 take the two halves of the latent-dim tiles
+constexpr int kWarpPV2 = 15;
+constexpr int kThreads = 512;
 constexpr int kLoadThreads = kLoadWarps * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 15.0f;  // P = 2^(z - m) stays <= 2^15 between rescales (fp16 holds it)
@@ -104,7 +107,8 @@ struct Layout {
   static constexpr uint32_t kOffBar = kOffM + kMq * 4;          // 9 mbarriers
   static constexpr uint32_t kOffMisc = kOffBar + 9 * 8;         // tmem base, abort, last-split flag
   static constexpr uint32_t kBytes = kOffMisc + 16 + 1024;
-  static constexpr uint32_t kColS = 0;    // score buffer b at kColS + b * kRows
+  static constexpr uint32_t kColS = 0;    // score buffer b, d-block half c at kColS + c * 2 * kRows + b * kRows
+  static constexpr int kPvIss = kMT >= 2 ? 2 : 1;  // PV issuing warps with work
   static constexpr uint32_t kColO = 256;  // O^T tile mt at kColO + mt * HQ
   static_assert(kPer >= 1 && kRows * kUnitsRow % kLoadThreads == 0, "loader unit split");
   static_assert(kMT * HQ <= 256 && 2 * kRows <= 256, "TMEM budget");
@@ -178,11 +182,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar_kv_full + 8 * i, kLoadWarps);
-      mbar_init(bar_kv_empty + 8 * i, 1);
-      mbar_init(bar_s_full + 8 * i, 1);
+      mbar_init(bar_kv_empty + 8 * i, Ly::kPvIss);
+      mbar_init(bar_s_full + 8 * i, 2);
       mbar_init(bar_p_full + 8 * i, kSoftWarps);
     }
-    mbar_init(bar_drain, 3);  // two S issuers and the PV issuer
+    mbar_init(bar_drain, 2 + Ly::kPvIss);  // every issuing warp
     *abort = 0;
     tc::fence_barrier_init();
   }
@@ -411,8 +415,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
   } else if (warp == kWarpS || warp == kWarpS2) {
     // ------------------------------------------------------------ S = Q K^T
     const uint32_t idesc = tc::idesc_f16(kMq, kRows, 0, 0);
-    const int par = warp == kWarpS ? 0 : 1;
-    for (int i = par; i < n_mine; i += 2) {
+    const int half = warp == kWarpS ? 0 : 1;  // d-blocks [half * kKB/2, (half + 1) * kKB/2)
+    for (int i = 0; i < n_mine; ++i) {
       const int bf = i & 1;
       if (lane == 0 && !*abort) {
         if (!mbar_wait_bounded(bar_kv_full + 8 * bf, (i >> 1) & 1, P.wait_ns)) {
@@ -425,14 +429,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
           const uint64_t a0 = tc::smem_desc(sbase + Ly::kOffQ, 16, 1024, tc::kSwizzle128B);
           const uint64_t al0 = tc::smem_desc(sbase + Ly::kOffQlo, 16, 1024, tc::kSwizzle128B);
           const uint64_t b0 = tc::smem_desc(sbase + Ly::kOffTile + bf * Ly::kTile, 16, 1024, tc::kSwizzle128B);
-          const uint32_t dcol = tmem + Ly::kColS + bf * kRows;
+          const uint32_t dcol = tmem + Ly::kColS + half * 2 * kRows + bf * kRows;
+          constexpr int kHalf = Ly::kKB / 2;
 #pragma unroll
-          for (int kb = 0; kb < Ly::kKB; ++kb)
+          for (int k2 = 0; k2 < kHalf; ++k2)
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
+              const int kb = half * kHalf + k2;
               const uint64_t ao = (uint64_t)((kb * (HQ * 128) + ks * 32) >> 4);
               const uint64_t bd = b0 + (uint64_t)((kb * (kRows * 128) + ks * 32) >> 4);
-              tc::mma_f16(dcol, a0 + ao, bd, idesc, (kb | ks) ? 1u : 0u);
+              tc::mma_f16(dcol, a0 + ao, bd, idesc, (k2 | ks) ? 1u : 0u);
               if (QLO) tc::mma_f16(dcol, al0 + ao, bd, idesc, 1u);
             }
           tc::commit(bar_s_full + 8 * bf);
@@ -442,10 +448,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
     }
     if (lane == 0) tc::commit(bar_drain);
     __syncwarp();
-  } else if (warp == kWarpPV) {
+  } else if (warp == kWarpPV || warp == kWarpPV2) {
     // ------------------------------------------------------------ O^T += V^T P^T
     const uint32_t idesc = tc::idesc_f16(128, HQ, 1, 0);
-    for (int i = 0; i < n_mine; ++i) {
+    const int ph = warp == kWarpPV ? 0 : 1;  // latent-dim tiles [ph * kMT/2, (ph + 1) * kMT/2)
+    const int mt0 = Ly::kPvIss == 2 ? ph * (Ly::kMT / 2) : 0;
+    const int mt1 = Ly::kPvIss == 2 ? mt0 + Ly::kMT / 2 : (ph == 0 ? Ly::kMT : 0);
+    for (int i = 0; i < (mt1 > mt0 ? n_mine : 0); ++i) {
       const int bf = i & 1;
       if (lane == 0 && !*abort) {
         if (!mbar_wait_bounded(bar_p_full + 8 * bf, (i >> 1) & 1, P.wait_ns)) {
@@ -457,8 +466,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
               tc::smem_desc(sbase + Ly::kOffTile + bf * Ly::kTile, kRows * 128, 1024, tc::kSwizzle128B);
           const uint64_t b0 =
               tc::smem_desc(sbase + Ly::kOffP + bf * ((Ly::kPBytes + 1023) / 1024 * 1024), 16, 1024, tc::kSwizzle128B);
-#pragma unroll
-          for (int mt = 0; mt < Ly::kMT; ++mt)
+#pragma unroll 1
+          for (int mt = mt0; mt < mt1; ++mt)
 #pragma unroll
             for (int ks = 0; ks < kRows / 16; ++ks) {
               const uint64_t ad = a0 + (uint64_t)(((2 * mt) * (kRows * 128) + ks * 2048) >> 4);
@@ -470,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
       }
       __syncwarp();
     }
-    if (lane == 0) tc::commit(bar_drain);
+    if (lane == 0 && mt1 > mt0) tc::commit(bar_drain);
     __syncwarp();
   } else if (warp < kSoftWarps) {
     // ------------------------------------------------------------ softmax
@@ -510,16 +519,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
         sum_ = 0.0f;
         zmax_ = -INFINITY;
 #pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          uint32_t v[16];
-          tc::ld_16x32bx2_x16<32>(s_col + g * 16, v);
+        for (int g = 0; g < 4; ++g) {
+          uint32_t v[8], v2[8];  // the two d-block halves of S
+          tc::ld_16x32bx2_x8<32>(s_col + g * 8, v);
+          tc::ld_16x32bx2_x8<32>(s_col + 2 * kRows + g * 8, v2);
           tc::ld_wait();
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
+          for (int k = 0; k < 8; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) + __uint_as_float(v2[k]));
+          {
             uint32_t pk[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              const int jj = cc * 8 + 2 * k, j0 = g * 16 + jj;
+              const int jj = 2 * k, j0 = g * 8 + jj;
               if (plain) {
                 const float z0 = __uint_as_float(v[jj]) * zs, z1 = __uint_as_float(v[jj + 1]) * zs;
                 zmax_ = fmaxf(zmax_, fmaxf(z0, z1));
@@ -547,9 +558,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
                 sum_ += e0 + e1;
               }
             }
-            // 16-byte chunk of 8 rows: rows 32 hf + 16 g + 8 cc ..
-            if (act)
-              *reinterpret_cast<uint4*>(prow + swz128(h, 4 * hf + 2 * g + cc)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            // 16-byte chunk of 8 rows: rows 32 hf + 8 g ..
+            if (act) *reinterpret_cast<uint4*>(prow + swz128(h, 4 * hf + g)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
         }
         zmax_ = fmaxf(zmax_, __shfl_xor_sync(0xffffffffu, zmax_, 16));  // both halves of the head

@@ -137,6 +137,14 @@ __device__ __forceinline__ void ld_16x32bx2_x16(uint32_t taddr, uint32_t (&r)[16
       : "r"(taddr), "n"(kOff));
 }
 
+// as ld_16x32bx2_x16, 8 consecutive columns
+template <int kOff>
+__device__ __forceinline__ void ld_16x32bx2_x8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8], %9;"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr), "n"(kOff));
+}
+
 // registers -> TMEM: this warp's 32 lanes x 16 consecutive 32-bit columns
 __device__ __forceinline__ void st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
