@@ -251,7 +251,7 @@ int launch_rescore(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t*
 }
 
 // CTAs per (selector, token) group: with fewer groups than SMs, long
-// candidate lists are split (about 2048 candidates a CTA) so that the whole
+// candidate lists are split (about 8192 candidates a CTA) so that the whole
 // grid still fits on the GPU at one CTA per SM (the launch is cooperative)
 static int select_splits(int64_t groups, int n_max) {
   static int sms = 0;
@@ -264,7 +264,11 @@ static int select_splits(int64_t groups, int n_max) {
       sms = 1;
   }
   if (groups >= sms) return 1;
-  int64_t s = (n_max + 2047) / 2048;
+  // about 8192 candidates per CTA: a selection round costs a CTA the same few
+  // microseconds of barriers and scans whether it holds 2048 or 8192 keys, and
+  // fewer CTAs per group merge fewer histograms
+  constexpr int kSelChunk = 8192;
+  int64_t s = (n_max + kSelChunk - 1) / kSelChunk;
   s = std::min<int64_t>(s, sms / groups);
   s = std::min<int64_t>(s, kSelMaxSplit);
   return (int)std::max<int64_t>(s, 1);
