@@ -222,12 +222,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
       tv[u] = j < n_sel ? __ldg(io.idx + (int64_t)tok * P.K + j) : -2;
     }
   }
+  // cache rows: index -> page -> row (the page loads wait for the index loads)
+  int64_t pg[kRowPer];
+  auto load_pages = [&]() {
+#pragma unroll
+    for (int u = 0; u < kRowPer; ++u) {
+      const int32_t t = tv[u];
+      pg[u] = 0;
+      if (t >= 0 && t <= p)
+        pg[u] = P.kv.page_table ? (int64_t)__ldg(P.kv.page_table + (int64_t)b * P.kv.max_pages + t / P.kv.page_size)
+                                : __ldg(P.kv.seq_base + b);
+    }
+  };
   // query -> fp16 [kb][h][128 B] (K-major, 128B swizzle); f32 queries also
   // keep the fp16 residual.  All threads, all loads in flight together.
   {
     constexpr int kUnitsQ = HQ * D / 8;  // 8 consecutive d per unit
     constexpr int kQPer = (kUnitsQ + kThreads - 1) / kThreads;
-    constexpr int kQB = kQPer < 3 ? kQPer : 3;  // units in flight per batch
+    // units in flight per batch: every unit of a bf16 query, three of an f32 one
+    constexpr int kQB = QLO ? (kQPer < 3 ? kQPer : 3) : kQPer;
 #pragma unroll 1
     for (int u0 = 0; u0 < kQPer; u0 += kQB) {
     // raw query units: 8 bf16 (one uint4) or, with f32 queries (QLO), 8 f32
@@ -246,6 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
         raw[u][0] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(io.q) + off));
       }
     }
+    // the page-table loads go out while the first query batch is in flight
+    if (u0 == 0) load_pages();
 #pragma unroll
     for (int u = 0; u < kQB; ++u) {
       const int e = (u0 + u) * kThreads + threadIdx.x;
@@ -284,15 +299,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
     }
   }
   {
-    int64_t pg[kRowPer];
-#pragma unroll
-    for (int u = 0; u < kRowPer; ++u) {
-      const int32_t t = tv[u];
-      pg[u] = 0;
-      if (t >= 0 && t <= p)
-        pg[u] = P.kv.page_table ? (int64_t)__ldg(P.kv.page_table + (int64_t)b * P.kv.max_pages + t / P.kv.page_size)
-                                : __ldg(P.kv.seq_base + b);
-    }
 #pragma unroll
     for (int u = 0; u < kRowPer; ++u) {
       const int e = threadIdx.x + u * kThreads;
@@ -680,8 +686,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
         for (uint32_t off = 0; off < bytes; off += 32768)
           tc::bulk_store(dst + off, sbase + Ly::kOffTile + off, min(32768u, bytes - off));
         tc::bulk_commit();
-        tc::bulk_wait_all();
-        tc::fence_proxy_async_global();  // before the split-arrival atomic below
+        if (nsplit > 1) {
+          tc::bulk_wait_all();
+          tc::fence_proxy_async_global();  // before the split-arrival atomic below
+        } else {
+          tc::bulk_wait_read();  // final output: only the staging must stay valid
+        }
       }
     } else {
       const uint32_t* src = reinterpret_cast<const uint32_t*>(smem + Ly::kOffTile);
