@@ -80,6 +80,22 @@ def _peaks():
         return 6650.0, 1590.0, "fallback"
 
 
+def algorithmic_flops(w) -> dict:
+    """Multiply-adds x 2 the method needs per decode step: the scan's and the
+    rescoring's q.k over every visible (resp. pooled) position and indexer
+    head, and attention's Q K^T and P V over the selected and window rows."""
+    import numpy as np
+
+    c = w.cfg
+    n_sel = sum(1 for m in w.modes if m in "FR")
+    vis = w.tok_pos.astype(np.int64) + 1
+    pool = np.minimum(np.minimum((vis + 7) // 8, c.P) * 8, vis)
+    rows = np.minimum(vis, c.K) + (np.minimum(vis, c.window) if c.swa else 0)
+    return {"scan": int(vis.sum()) * c.H_I * c.d_I * 2,
+            "rescore": int(pool.sum()) * n_sel * c.H_I * c.d_I * 2,
+            "attend": int(rows.sum()) * len(w.modes) * c.Hq * c.D * 4}
+
+
 def _workload_desc(cfg, w):
     return {
         "workload": f"{cfg.name}: B={cfg.B}, L={'x'.join(str(int(x)) for x in sorted(set(w.lens.tolist())))[:60]}"
@@ -360,9 +376,22 @@ def run_ours(args):
     roof = None
     kernels = {}
     tot_prof = sum(v[1] for v in kstats.values())
+    fl = algorithmic_flops(w)
+    # per kernel: algorithmic bytes (HBM) and tensor FLOPs per step over its time
+    # per step; FP4 MMAs against the measured bf16 peak x 4 (the nominal
+    # 9 / 2.25 PFLOP/s ratio), fp16 MMAs against the measured bf16 peak
+    per_kernel = {"scan": (ab["scan"], fl["scan"], 4.0), "rescore": (ab["rescore"], fl["rescore"], 4.0),
+                  "attend": (ab["attend"] + ab["swa"], fl["attend"], 1.0)}
     for n, (cnt, ms) in sorted(kstats.items(), key=lambda kv: -kv[1][1]):
         kernels[n] = {"launches_per_step": cnt / args.steps, "us_per_step": 1000.0 * ms / args.steps,
                       "share": ms / tot_prof if tot_prof else None}
+        key = next((k for k in per_kernel if n.startswith(k)), None)
+        if key and ms > 0:
+            b, f, ratio = per_kernel[key]
+            sec = ms / args.steps / 1000.0
+            kernels[n].update({"hbm_gbs": b / sec / 1e9, "hbm_frac": b / sec / 1e9 / peak_hbm,
+                               "tensor_tflops": f / sec / 1e12,
+                               "tensor_frac": f / sec / 1e12 / (peak_bf16 * ratio)})
     if scan_name:
         cnt, ms = kstats[scan_name]
         avg_s = ms / cnt / 1000.0
