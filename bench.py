@@ -42,8 +42,8 @@ UNIT = "qtok/s"
 def _args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", type=int, default=4, help="workload number (1..5)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -280,7 +280,8 @@ def run_reference(args):
     from synth.workloads import CONFIGS, make_workload
     cfg = CONFIGS[args.config]
     w = make_workload(cfg)
-    per_step = max(1.0, min(args.cpu_seconds, 6.0))  # the whole --steps run stays within a few minutes
+    # the whole --steps run stays within a few minutes: at most ~150 s of samples
+    per_step = max(1.0, min(args.cpu_seconds, 6.0, 150.0 / max(1, args.steps)))
     for _ in range(args.warmup):
         oracle_sample(args.config, 0.0)
     vals, times = [], []
@@ -360,6 +361,16 @@ def run_ours(args):
     st = C.csa2_get_status(sp)
     assert st == 0, f"device status {st}"
     value = whole_job_rate(tokens_all, args.steps, total_ms)
+    q = np.percentile(np.asarray(step_ms), [10, 50, 90])
+
+    # warm steps (no L2 flush between them): secondary, for comparison only
+    ev_w = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for k in range(args.steps):
+        ev_w[k][0].record(stream)
+        step()
+        ev_w[k][1].record(stream)
+    torch.cuda.synchronize()
+    warm_ms = allmax(sum(a.elapsed_time(b) for a, b in ev_w)) / args.steps
 
     # per-kernel times (second pass, profiler on; same steps)
     C.csa2_profiler_read()
@@ -436,6 +447,8 @@ def run_ours(args):
             "scan_gbs": roof["achieved"] if roof else None,
             "algorithmic_bytes_per_step": ab,
             "step_ms_min_max": [min(step_ms), max(step_ms)],
+            "step_ms_p10_p50_p90": [float(x) for x in q],
+            "warm_ms_per_step": warm_ms,
         }
         print(json.dumps(line), flush=True)
     R.close()
