@@ -52,19 +52,36 @@ class DeviceWorkload:
         self.swa_codes, self.swa_scale = {}, {}
         qdt = torch.float32 if c.q_dtype == "f32" else torch.bfloat16
         odt = torch.float32 if c.out_dtype == "f32" else torch.bfloat16
+        # every per-step input (queries, head weights, new tokens) in one
+        # contiguous device buffer, and every layer's output in one tensor, so
+        # that a step's host copies are one transfer each way
+        n_fr = sum(1 for m in w.modes if m in "FR")
+        qsz = 4 if qdt == torch.float32 else 2
+        parts = [T * c.H_I * c.d_I * 4, T * c.H_I * 4] * n_fr + [T * c.Hq * c.D * qsz] * len(w.modes) + [
+            T * c.d_I * 4, T * c.D * 4]
+        self.inputs_packed = torch.empty(sum((n + 255) // 256 * 256 for n in parts), dtype=torch.uint8, device=dev)
+        self._in_off = 0
+
+        def take(shape, dtype):
+            n = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+            t = self.inputs_packed[self._in_off:self._in_off + n].view(dtype).view(*shape)
+            self._in_off += (n + 255) // 256 * 256
+            return t
+
+        self.out_all = torch.zeros(len(w.modes), T, c.Hq, c.D, dtype=odt, device=dev)
         for l, m in enumerate(w.modes):
             if m in "FR":
-                self.iq[l] = torch.empty(T, c.H_I, c.d_I, dtype=torch.float32, device=dev)
+                self.iq[l] = take((T, c.H_I, c.d_I), torch.float32)
                 w.iq[l].dev_rows_f32(0, 0, T, self.iq[l].data_ptr(), self.stream)
-                self.iw[l] = torch.empty(T, c.H_I, dtype=torch.float32, device=dev)
+                self.iw[l] = take((T, c.H_I), torch.float32)
                 w.iw[l].dev_rows_f32(0, 0, T, self.iw[l].data_ptr(), self.stream)
                 self.idx_out[l] = torch.full((T, c.K), -2, dtype=torch.int32, device=dev)
-            self.q[l] = torch.empty(T, c.Hq, c.D, dtype=qdt, device=dev)
+            self.q[l] = take((T, c.Hq, c.D), qdt)
             if c.q_dtype == "f32":
                 w.qmain[l].dev_rows_f32(0, 0, T, self.q[l].data_ptr(), self.stream)
             else:
                 w.qmain[l].dev_rows_bf16(0, 0, T, self.q[l].data_ptr(), self.stream)
-            self.out[l] = torch.zeros(T, c.Hq, c.D, dtype=odt, device=dev)
+            self.out[l] = self.out_all[l]
             self.lse[l] = torch.zeros(T, c.Hq, dtype=torch.float32, device=dev)
             if c.swa:
                 cap = c.swa_cap
@@ -78,8 +95,9 @@ class DeviceWorkload:
                                            self.swa_scale[l][b * cap:].data_ptr(), self.stream, st=st)
         self.pool_out = torch.full((T, c.P), -2, dtype=torch.int32, device=dev)
         # this step's new tokens (appended by the decode step)
-        self.new_kidx = torch.empty(T, c.d_I, dtype=torch.float32, device=dev)
-        self.new_kv = torch.empty(T, c.D, dtype=torch.float32, device=dev)
+        self.new_kidx = take((T, c.d_I), torch.float32)
+        self.new_kv = take((T, c.D), torch.float32)
+        assert self._in_off == self.inputs_packed.numel()
         sk, sv = w.kidx.device(dev), w.kv.device(dev)
         for b in range(w.B):
             t0, t1 = int(w.tok_start[b]), int(w.tok_start[b + 1])
