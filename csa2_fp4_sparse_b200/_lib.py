@@ -51,7 +51,8 @@ class csa2_stack_desc(ctypes.Structure):
     _fields_ = [("qb", csa2_query_batch), ("k_idx", csa2_fp4_cache), ("kv", csa2_fp4_cache), ("H_I", _i32),
                 ("P", _i32), ("K", _i32), ("Hq", _i32), ("q_dtype", _i32), ("out_dtype", _i32),
                 ("softmax_scale", ctypes.c_float), ("new_k_idx", _vp), ("new_kv", _vp), ("new_slot_k_idx", _vp),
-                ("new_slot_kv", _vp), ("n_layers", _i32), ("layers", ctypes.POINTER(csa2_layer_desc))]
+                ("new_slot_kv", _vp), ("n_layers", _i32), ("layers", ctypes.POINTER(csa2_layer_desc)),
+                ("attend_wait_event", _vp)]
 
 
 _P = ctypes.POINTER

@@ -702,7 +702,12 @@ int csa2_decode_stack(const csa2_stack_desc* d, void* workspace, size_t workspac
     s += n;
   }
   // attention of every layer: consecutive layers alike in having a sliding
-  // window or not, up to kMaxAttLayers per launch
+  // window or not, up to kMaxAttLayers per launch (after the caller's event,
+  // when one is given: only attention reads the Main queries)
+  if (d->attend_wait_event) {
+    const cudaError_t e = cudaStreamWaitEvent(st, static_cast<cudaEvent_t>(d->attend_wait_event), 0);
+    if (e != cudaSuccess) return fail(CSA2_ERR_CUDA, "cudaStreamWaitEvent: %s", cudaGetErrorString(e));
+  }
   int l = 0;
   while (l < NL) {
     AttendLayer group[kMaxAttLayers];

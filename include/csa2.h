@@ -133,6 +133,10 @@ typedef struct csa2_stack_desc {
   const int64_t* new_slot_kv;    /* [T] destination rows in kv */
   int32_t n_layers;
   const csa2_layer_desc* layers; /* host array [n_layers] */
+  void* attend_wait_event;   /* optional cudaEvent_t: the attention launches of the step
+                              * wait for it (e.g. the Main queries copied on another
+                              * stream while the indexer runs); NULL = no wait.  The
+                              * event must have been recorded before the call. */
 } csa2_stack_desc;
 
 /* ---- entry points -------------------------------------------------------- */

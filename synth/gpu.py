@@ -52,13 +52,16 @@ class DeviceWorkload:
         self.swa_codes, self.swa_scale = {}, {}
         qdt = torch.float32 if c.q_dtype == "f32" else torch.bfloat16
         odt = torch.float32 if c.out_dtype == "f32" else torch.bfloat16
-        # every per-step input (queries, head weights, new tokens) in one
-        # contiguous device buffer, and every layer's output in one tensor, so
-        # that a step's host copies are one transfer each way
+        # every per-step input in one contiguous device buffer: first what the
+        # indexer needs (queries and head weights of every selector, the new
+        # tokens), then the Main queries of every layer (read only by
+        # attention); every layer's output in one tensor.  A step's host copies
+        # are then one transfer each way, or two in, the second overlapping the
+        # indexer kernels
         n_fr = sum(1 for m in w.modes if m in "FR")
         qsz = 4 if qdt == torch.float32 else 2
-        parts = [T * c.H_I * c.d_I * 4, T * c.H_I * 4] * n_fr + [T * c.Hq * c.D * qsz] * len(w.modes) + [
-            T * c.d_I * 4, T * c.D * 4]
+        parts = [T * c.H_I * c.d_I * 4, T * c.H_I * 4] * n_fr + [T * c.d_I * 4, T * c.D * 4] + [
+            T * c.Hq * c.D * qsz] * len(w.modes)
         self.inputs_packed = torch.empty(sum((n + 255) // 256 * 256 for n in parts), dtype=torch.uint8, device=dev)
         self._in_off = 0
 
@@ -68,15 +71,24 @@ class DeviceWorkload:
             self._in_off += (n + 255) // 256 * 256
             return t
 
-        self.out_all = torch.zeros(len(w.modes), T, c.Hq, c.D, dtype=odt, device=dev)
         for l, m in enumerate(w.modes):
             if m in "FR":
                 self.iq[l] = take((T, c.H_I, c.d_I), torch.float32)
-                w.iq[l].dev_rows_f32(0, 0, T, self.iq[l].data_ptr(), self.stream)
                 self.iw[l] = take((T, c.H_I), torch.float32)
+        # this step's new tokens (appended by the decode step)
+        self.new_kidx = take((T, c.d_I), torch.float32)
+        self.new_kv = take((T, c.D), torch.float32)
+        self.inputs_index = self.inputs_packed[:self._in_off]
+        for l in range(len(w.modes)):
+            self.q[l] = take((T, c.Hq, c.D), qdt)
+        self.inputs_main_q = self.inputs_packed[self.inputs_index.numel():]
+        assert self._in_off == self.inputs_packed.numel()
+        self.out_all = torch.zeros(len(w.modes), T, c.Hq, c.D, dtype=odt, device=dev)
+        for l, m in enumerate(w.modes):
+            if m in "FR":
+                w.iq[l].dev_rows_f32(0, 0, T, self.iq[l].data_ptr(), self.stream)
                 w.iw[l].dev_rows_f32(0, 0, T, self.iw[l].data_ptr(), self.stream)
                 self.idx_out[l] = torch.full((T, c.K), -2, dtype=torch.int32, device=dev)
-            self.q[l] = take((T, c.Hq, c.D), qdt)
             if c.q_dtype == "f32":
                 w.qmain[l].dev_rows_f32(0, 0, T, self.q[l].data_ptr(), self.stream)
             else:
@@ -94,10 +106,6 @@ class DeviceWorkload:
                     w.swa[l].dev_rows_e4m3(b, lo, L - lo, cap, self.swa_codes[l][b * cap:].data_ptr(),
                                            self.swa_scale[l][b * cap:].data_ptr(), self.stream, st=st)
         self.pool_out = torch.full((T, c.P), -2, dtype=torch.int32, device=dev)
-        # this step's new tokens (appended by the decode step)
-        self.new_kidx = take((T, c.d_I), torch.float32)
-        self.new_kv = take((T, c.D), torch.float32)
-        assert self._in_off == self.inputs_packed.numel()
         sk, sv = w.kidx.device(dev), w.kv.device(dev)
         for b in range(w.B):
             t0, t1 = int(w.tok_start[b]), int(w.tok_start[b + 1])

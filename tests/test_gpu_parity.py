@@ -265,3 +265,35 @@ def test_individual_entry_points_match_stack():
             ref, rlse = oracle.attend(w.qmain_f64(l, tok), ov.kv_rows(b, g), 1 / math.sqrt(c.D))
             grade_attention(out[tok].cpu().numpy(), ref, "f32", "attend")
             np.testing.assert_allclose(lse[tok].cpu().numpy(), rlse, rtol=1e-5, atol=1e-5)
+
+
+def test_stack_attend_wait_event():
+    """Main queries uploaded on a second stream: with attend_wait_event the
+    stack's attention waits for them and gives the outputs of the plain call"""
+    from synth.gpu import DeviceWorkload
+    from synth.workloads import make_workload
+    C = _C()
+    cfg = _small(2, B=2, lengths=("fixed", 6000), n_reindex=1, n_reuse=2)
+    w = make_workload(cfg)
+    dw = DeviceWorkload(w)
+    dw.fill_caches(include_new=True)
+    desc = dw.stack_desc(append=False)
+    ws = dw.stack_workspace(desc)
+    C.check(C.csa2_decode_stack(ctypes.byref(desc), ws.data_ptr(), ws.numel(), _stream()))
+    assert _status() == 0
+    ref = dw.out_all.clone()
+    h_q = dw.inputs_main_q.cpu().pin_memory()
+    dw.inputs_main_q.zero_()
+    dw.out_all.zero_()
+    s2 = torch.cuda.Stream()
+    ready = torch.cuda.Event()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s2):
+        torch.cuda._sleep(2_000_000)  # the copy lands well after the indexer kernels were queued
+        dw.inputs_main_q.copy_(h_q, non_blocking=True)
+        ready.record(s2)
+    desc.attend_wait_event = ready.cuda_event
+    C.check(C.csa2_decode_stack(ctypes.byref(desc), ws.data_ptr(), ws.numel(), _stream()))
+    assert _status() == 0
+    torch.cuda.synchronize()
+    assert torch.equal(dw.out_all, ref)
