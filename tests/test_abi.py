@@ -103,3 +103,32 @@ def test_product_package_does_not_import_oracle():
                 if f.endswith((".py", ".cu", ".cuh", ".h", ".c")):
                     txt = open(os.path.join(dirpath, f), encoding="utf-8").read()
                     assert "oracle" not in txt.lower(), os.path.join(dirpath, f)
+
+
+def test_struct_layouts_match_header(tmp_path):
+    """The ctypes mirrors have the header's sizes and field offsets (a plain C
+    program built with gcc against include/csa2.h prints them)."""
+    import shutil
+    import subprocess
+
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    structs = {name: getattr(C._lib, name) for name in
+               ("csa2_query_batch", "csa2_fp4_cache", "csa2_swa_desc", "csa2_layer_desc", "csa2_stack_desc",
+                "csa2_kernel_stat")}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "csa2.h"', "int main(void) {"]
+    for name, cls in structs.items():
+        lines.append(f'  printf("{name} sizeof %zu\\n", sizeof({name}));')
+        for f in cls._fields_:
+            lines.append(f'  printf("{name} {f[0]} %zu\\n", offsetof({name}, {f[0]}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
+    out = subprocess.check_output([str(exe)], text=True).split("\n")
+    got = {(a, b): int(c) for a, b, c in (l.split() for l in out if l)}
+    for name, cls in structs.items():
+        assert got[(name, "sizeof")] == ctypes.sizeof(cls), name
+        for f in cls._fields_:
+            assert got[(name, f[0])] == getattr(cls, f[0]).offset, (name, f[0])
