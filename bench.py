@@ -51,18 +51,29 @@ def _args():
     return ap.parse_args()
 
 
-def _profiled_traffic(kernel_src: str, summary: str):
-    """DRAM bytes per launch (read + write) from a committed ncu summary, valid
-    only while the kernel's source is the one the counters were taken on
-    (the summary records the first 16 hex digits of its SHA-256)."""
+def source_digest(text: str) -> str:
+    """First 16 hex digits of the SHA-256 of a C/CUDA source with its comments
+    removed and its whitespace collapsed: the code the compiler sees, so that an
+    edit of a comment leaves it unchanged."""
     import hashlib
     import re
+    code = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    code = re.sub(r"//[^\n]*", " ", code)
+    code = " ".join(code.split())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
+
+
+def _profiled_traffic(kernel_src: str, summary: str):
+    """DRAM bytes per launch (read + write) from a committed ncu summary, valid
+    only while the kernel's code is the one the counters were taken on (the
+    summary records its source_digest)."""
+    import re
     try:
-        with open(os.path.join(ROOT, kernel_src), "rb") as f:
-            h = hashlib.sha256(f.read()).hexdigest()[:16]
+        with open(os.path.join(ROOT, kernel_src), encoding="utf-8") as f:
+            h = source_digest(f.read())
         with open(os.path.join(ROOT, summary)) as f:
             txt = f.read()
-        src = re.search(r"source_sha256_16:\s*([0-9a-f]{16})", txt)
+        src = re.search(r"source_digest:\s*([0-9a-f]{16})", txt)
         tr = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", txt)
         if src and tr and src.group(1) == h:
             return int(tr.group(1))

@@ -24,17 +24,18 @@
 //                lane 32*(h/16) + h%16; the 16x32bx2 load gives lanes t and
 //                t+16 of a warp the two halves of head t's scores): one pass
 //                per chunk against the running (log2) max, which only moves
-//                (with a second pass) when a
-//                chunk exceeds it by more than 2^8 (then the output
-//                accumulator is rescaled), P = 2^(z - m) written as fp16 rows
-//                [head][row] (window rows carry their per-token scale into P);
+//                (with a second pass) when a chunk exceeds it by more than
+//                2^15 (then the output accumulator is rescaled); P = 2^(z - m)
+//                written as fp16 rows [head][row] (window rows carry their
+//                per-token scale into P);
 //   warps 13,15  issue O^T += V^T P^T (M = 128 latent dims per tile, N =
 //                heads, K = 64 rows; half of the latent-dim tiles each)
 //                reading the same tile as V; their commits free the tile and
 //                the P buffer.
 // The epilogue divides by the row sum, stages the output in shared memory and
-// writes it with 16-byte stores (or the split's unnormalised partial with its
-// max and sum; the last split of a token merges them).  Every wait is bounded.
+// writes it with bulk copies (4-byte stores when the destination is not 16-byte
+// aligned), or the split's unnormalised partial with its max and sum (the last
+// split of a token merges them).  Every wait is bounded.
 #include "internal.h"
 #include "tc_common.cuh"
 

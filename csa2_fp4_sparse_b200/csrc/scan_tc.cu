@@ -38,8 +38,9 @@
 // The key cache is streamed from HBM exactly once per sequence for all of its
 // query tokens.  In rescoring mode the producer instead gathers the 16 pool
 // blocks of a tile (8 rows each, one swizzle atom per block) for one query
-// token, and the epilogue writes one score per pool position.  All waits are bounded; on timeout the kernel records
-// CSA2_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
+// token, and the epilogue writes one score per pool position.  All waits are
+// bounded; on timeout the kernel records CSA2_ERR_TIMEOUT, drains its own
+// copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 

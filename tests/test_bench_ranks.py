@@ -78,3 +78,26 @@ def test_reference_arm_under_torchrun_world2():
     assert d["impl"] == "reference" and d["unit"] == "qtok/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["unit"] == d["unit"]
+
+
+def test_source_digest_ignores_comments_only():
+    import bench
+
+    a = "int f(int x) {\n  return x + 1;  // one\n}\n/* block\n comment */\n"
+    b = "// header\nint f(int x) {   return x + 1; }\n"
+    c = "int f(int x) {\n  return x + 2;\n}\n"
+    assert bench.source_digest(a) == bench.source_digest(b)
+    assert bench.source_digest(a) != bench.source_digest(c)
+
+
+def test_algorithmic_flops_closed_form():
+    import bench
+    from synth.workloads import CONFIGS, make_workload
+
+    w = make_workload(CONFIGS[4])
+    f = bench.algorithmic_flops(w)
+    c = w.cfg
+    n_pos = 4 * 1048576  # one query token per sequence, every position visible
+    assert f["scan"] == n_pos * c.H_I * c.d_I * 2
+    assert f["rescore"] == 4 * c.P * 8 * 4 * c.H_I * c.d_I * 2  # 4 selectors, full pools
+    assert f["attend"] == 4 * c.K * 20 * c.Hq * c.D * 4
