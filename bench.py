@@ -452,7 +452,7 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "fp4", "data": "synthetic",
-            "config": dict(_workload_desc(cfg, w), parallelism=f"replicas x{world}"),
+            "config": _workload_desc(cfg, w), "parallelism": f"replicas x{world}",
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(n_launch),
             "clocks": clk, "kernels": kernels,
             "scan_gbs": roof["achieved"] if roof else None,

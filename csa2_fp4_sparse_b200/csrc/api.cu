@@ -98,13 +98,20 @@ static int check_batch(const csa2_query_batch* qb) {
   return CSA2_OK;
 }
 
-static int check_cache(const csa2_fp4_cache* c, const char* name) {
+// the cache descriptor, and that a paged cache's table covers every position
+// the batch can address (the kernels index page_table[b][t / page_size]
+// without a bound: a sequence longer than its table row would read the next
+// sequence's pages)
+static int check_cache(const csa2_fp4_cache* c, const char* name, const csa2_query_batch* qb) {
   if (!c) return fail(CSA2_ERR_INVALID_ARG, "%s cache is NULL", name);
   if (!c->codes || !c->scales || c->n_rows < 1) return fail(CSA2_ERR_INVALID_ARG, "%s cache buffers missing", name);
   if (c->dim < 32 || c->dim % 32) return fail(CSA2_ERR_UNSUPPORTED, "%s dim %d not a multiple of 32", name, c->dim);
   if (c->page_table) {
     if (c->page_size < 64 || c->page_size % 64 || c->max_pages < 1)
       return fail(CSA2_ERR_UNSUPPORTED, "%s page_size must be a positive multiple of 64", name);
+    if ((int64_t)qb->max_seq_len > (int64_t)c->max_pages * c->page_size)
+      return fail(CSA2_ERR_INVALID_ARG, "%s: max_seq_len %d exceeds max_pages * page_size = %lld", name,
+                  qb->max_seq_len, (long long)c->max_pages * c->page_size);
   } else if (!c->seq_base) {
     return fail(CSA2_ERR_INVALID_ARG, "%s: unpaged cache needs seq_base", name);
   }
@@ -124,30 +131,27 @@ struct Carve {
 
 static int n_blocks_max(const csa2_query_batch* qb) { return (qb->max_seq_len + kBlock - 1) / kBlock; }
 
+// split-selection scratch: one record per (selector, token) group of a
+// split launch (a launch splits only while it has fewer groups than SMs)
+static size_t select_ws(const csa2_query_batch*, int, int) { return (size_t)kSelMaxGroups * sizeof(SelGroup); }
+
 static size_t index_ws(const csa2_query_batch* qb, int P) {
   Carve c{nullptr, 0};
   c.take((size_t)qb->n_tok * n_blocks_max(qb) * 4);  // block scores
   c.take((size_t)qb->n_tok * P * kBlock * 4);        // pool position scores
-  c.take((size_t)kNumSmsNominal * sizeof(SelGroup)); // split-selection scratch
+  c.take(select_ws(qb, P, 1));                       // split-selection scratch
   return c.used + 256;
 }
 
-static int n_att_splits(int K, const csa2_swa_desc* swa, int* n_sp) {
-  *n_sp = (K + kAttRows - 1) / kAttRows;
-  return *n_sp + (swa ? (swa->window + kAttRows - 1) / kAttRows : 0);
-}
-
-// tensor-core attention: split partials exist only while the launch has fewer
-// than 148 (token, layer) pairs, so at most 296 partial slots are ever used
+// attention: split partials exist only while a launch has fewer than 148
+// (token, layer) pairs, and a pair is split over at most 148 / pairs CTAs, so
+// at most 148 partial slots are ever used (296 kept for headroom)
 constexpr int64_t kMaxPartialSlots = 296;
 
-static size_t attend_ws(const csa2_query_batch* qb, int Hq, int D, int K, const csa2_swa_desc* swa) {
-  int n_sp;
-  int ns = n_att_splits(K, swa, &n_sp);
-  const int64_t slots = std::max<int64_t>((int64_t)qb->n_tok * ns, kMaxPartialSlots);
+static size_t attend_ws(const csa2_query_batch* qb, int Hq, int D) {
   Carve c{nullptr, 0};
-  c.take((size_t)slots * Hq * D * 4);
-  c.take((size_t)slots * Hq * 2 * 4);
+  c.take((size_t)kMaxPartialSlots * Hq * D * 4);
+  c.take((size_t)kMaxPartialSlots * Hq * 2 * 4);
   c.take((size_t)qb->n_tok * kMaxAttLayers * 4);  // split arrival counters
   return c.used + 256;
 }
@@ -182,66 +186,17 @@ int launch_quantize(const float* x, int64_t n_rows, int dim, const int64_t* slot
   return launch_quantize_jobs(J, st);
 }
 
-template <int DI>
-static int launch_scan_simt(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
-                            const csa2_fp4_cache* kc, float* bs, int64_t ld, cudaStream_t st) {
-  size_t smem = (size_t)H * DI * 4 + H * 4;
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k_scan_simt<DI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attr = true;
-  }
-  dim3 grid((qb->max_seq_len + 127) / 128, qb->n_tok);
-  Launch L_("scan_simt", st);
-  k_scan_simt<DI><<<grid, 128, smem, st>>>(*qb, qc, qs, w, H, *kc, bs, ld, status_ptr());
-  return cuda_check(cudaGetLastError(), "k_scan_simt");
-}
-
-template <int DI>
-static int launch_rescore_simt(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
-                               const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n, int P,
-                               float* scores, cudaStream_t st) {
-  size_t smem = (size_t)H * DI * 4 + H * 4;
-  dim3 grid((P * kBlock + 127) / 128, qb->n_tok);
-  Launch L_("rescore_simt", st);
-  k_rescore_simt<DI><<<grid, 128, smem, st>>>(*qb, qc, qs, w, H, *kc, pool, pool_n, P, scores, status_ptr());
-  return cuda_check(cudaGetLastError(), "k_rescore_simt");
-}
-
-// CSA2_SCAN_IMPL=simt selects the CUDA-core scan (comparison runs); the
-// tensor-core scan is the default wherever its shape limits hold.
-static bool use_scan_tc(const csa2_query_batch* qb, int H) {
-  static int env = -1;
-  if (env < 0) {
-    const char* e = getenv("CSA2_SCAN_IMPL");
-    env = (e && strcmp(e, "simt") == 0) ? 0 : 1;
-  }
-  return env == 1 && qb->max_q_per_seq <= 8 && H <= 64;
-}
-
 int launch_scan(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
                 const csa2_fp4_cache* kc, float* bs, int64_t ld, cudaStream_t st) {
-  if (use_scan_tc(qb, H)) return launch_scan_tc(qb, qc, qs, w, H, kc, bs, ld, st);
-  if (kc->dim == 128) return launch_scan_simt<128>(qb, qc, qs, w, H, kc, bs, ld, st);
-  return launch_scan_simt<64>(qb, qc, qs, w, H, kc, bs, ld, st);
+  return launch_scan_tc(qb, qc, qs, w, H, kc, bs, ld, st);
 }
 
 // n_sel selector layers (queries [n_sel][T][H][...], weights w[i], scores
-// [n_sel][T][8P]); the tensor-core path takes up to 8 in one launch
+// [n_sel][T][8P]), up to kMaxSel in one launch
 static int launch_rescore_multi(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs,
                                 const float* const* w, int n_sel, int H, const csa2_fp4_cache* kc,
                                 const int32_t* pool, const int32_t* pool_n, int P, float* scores, cudaStream_t st) {
-  if (use_scan_tc(qb, H)) return launch_rescore_tc(qb, qc, qs, w, n_sel, H, kc, pool, pool_n, P, scores, st);
-  const int T = qb->n_tok, dI = kc->dim;
-  for (int i = 0; i < n_sel; ++i) {
-    const uint8_t* c = qc + (size_t)i * T * H * (dI / 2);
-    const uint8_t* s = qs + (size_t)i * T * H * (dI / 32);
-    float* o = scores + (size_t)i * T * P * kBlock;
-    int rc = dI == 128 ? launch_rescore_simt<128>(qb, c, s, w[i], H, kc, pool, pool_n, P, o, st)
-                       : launch_rescore_simt<64>(qb, c, s, w[i], H, kc, pool, pool_n, P, o, st);
-    if (rc) return rc;
-  }
-  return CSA2_OK;
+  return launch_rescore_tc(qb, qc, qs, w, n_sel, H, kc, pool, pool_n, P, scores, st);
 }
 
 int launch_rescore(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
@@ -259,7 +214,7 @@ static int select_splits(int64_t groups, int n_max) {
     int dev = 0, v = 0;
     if (cudaGetDevice(&dev) == cudaSuccess &&
         cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
-      sms = std::min(v, kNumSmsNominal);
+      sms = std::min(v, kSelMaxGroups);
     else
       sms = 1;
   }
@@ -275,12 +230,13 @@ static int select_splits(int64_t groups, int n_max) {
 }
 
 // n_sel score matrices [n_sel][T][ld] -> lists [n_sel][T][k_out], counts
-// [n_sel][T].  grp: kNumSmsNominal SelGroup records of scratch, or NULL (one
-// CTA per group)
+// [n_sel][T].  scratch: kSelMaxGroups SelGroup records, or NULL (one CTA per
+// group)
 static int launch_select_multi(const csa2_query_batch* qb, const float* score, int64_t ld, int mode,
                                const int32_t* pool, const int32_t* pool_n, int P, int k_out, int32_t* out,
-                               int32_t* out_n, int n_sel, SelGroup* grp, cudaStream_t st) {
+                               int32_t* out_n, int n_sel, void* scratch, cudaStream_t st) {
   if (qb->n_tok > 65535 || n_sel > 65535) return fail(CSA2_ERR_UNSUPPORTED, "more than 65535 query tokens");
+  SelGroup* grp = static_cast<SelGroup*>(scratch);
   const int64_t groups = (int64_t)qb->n_tok * n_sel;
   const int n_max = mode == 0 ? n_blocks_max(qb) : P * kBlock;
   const int S = grp ? select_splits(groups, n_max) : 1;
@@ -313,78 +269,35 @@ static int launch_select_multi(const csa2_query_batch* qb, const float* score, i
 }
 
 int launch_select(const csa2_query_batch* qb, const float* score, int64_t ld, int mode, const int32_t* pool,
-                  const int32_t* pool_n, int P, int k_out, int32_t* out, int32_t* out_n, SelGroup* grp,
+                  const int32_t* pool_n, int P, int k_out, int32_t* out, int32_t* out_n, void* scratch,
                   cudaStream_t st) {
-  return launch_select_multi(qb, score, ld, mode, pool, pool_n, P, k_out, out, out_n, 1, grp, st);
-}
-
-// CSA2_ATTEND_IMPL=simt selects the CUDA-core attention (comparison runs).
-static bool use_attend_tc(int D, int Hq, int q_dtype) {
-  static int env = -1;
-  if (env < 0) {
-    const char* e = getenv("CSA2_ATTEND_IMPL");
-    env = (e && strcmp(e, "simt") == 0) ? 0 : 1;
-  }
-  return env == 1 && attend_tc_supported(D, Hq, q_dtype);
+  return launch_select_multi(qb, score, ld, mode, pool, pool_n, P, k_out, out, out_n, 1, scratch, st);
 }
 
 // Attention of n_layers (<= kMaxAttLayers) layers, each with its own index
-// list (one launch on the tensor-core path).  ws: attend_ws() bytes.
+// list, in one launch.  ws: attend_ws() bytes.
 int launch_attend_layers(const csa2_query_batch* qb, int q_dtype, int Hq, const csa2_fp4_cache* kv, int K,
                          const AttendLayer* layers, int n_layers, float scale, int out_dtype, void* ws,
                          cudaStream_t st) {
   const int D = kv->dim;
   const csa2_swa_desc* swa = layers[0].swa;
-  int n_sp;
-  const int ns = n_att_splits(K, swa, &n_sp);
-  const int64_t slots = std::max<int64_t>((int64_t)qb->n_tok * ns, kMaxPartialSlots);
+  if (!attend_tc_supported(D, Hq, q_dtype)) return fail(CSA2_ERR_UNSUPPORTED, "attention shape D=%d Hq=%d", D, Hq);
   Carve c{static_cast<uint8_t*>(ws), ~size_t(0)};
-  float* part_o = static_cast<float*>(c.take((size_t)slots * Hq * D * 4));
-  float* part_ml = static_cast<float*>(c.take((size_t)slots * Hq * 2 * 4));
+  float* part_o = static_cast<float*>(c.take((size_t)kMaxPartialSlots * Hq * D * 4));
+  float* part_ml = static_cast<float*>(c.take((size_t)kMaxPartialSlots * Hq * 2 * 4));
   int* done = static_cast<int*>(c.take((size_t)qb->n_tok * kMaxAttLayers * 4));
-  if (use_attend_tc(D, Hq, q_dtype)) {
-    // 64-row chunks; with fewer than 148 (token, layer) pairs one token's
-    // chunks are spread over up to 4 CTAs (one wave of one CTA per SM), whose
-    // partials the last one merges
-    const int chunks = (K + 63) / 64 + (swa ? (swa->window + 63) / 64 : 0);
-    const int64_t pairs = (int64_t)qb->n_tok * n_layers;
-    int nsplit = 1;
-    if (pairs < 148) nsplit = (int)std::max<int64_t>(1, std::min<int64_t>(std::min(chunks, 4), 148 / pairs));
-    if (nsplit > 1) {
-      if (int rc = cuda_check(cudaMemsetAsync(done, 0, (size_t)pairs * 4, st), "clear split counters")) return rc;
-    }
-    return launch_attend_tc(qb, q_dtype, Hq, kv, K, layers, n_layers, scale, out_dtype, part_o, part_ml, done,
-                            nsplit, st);
+  // 64-row chunks; with fewer than 148 (token, layer) pairs one token's
+  // chunks are spread over up to 4 CTAs (one wave of one CTA per SM), whose
+  // partials the last one merges
+  const int chunks = (K + 63) / 64 + (swa ? (swa->window + 63) / 64 : 0);
+  const int64_t pairs = (int64_t)qb->n_tok * n_layers;
+  int nsplit = 1;
+  if (pairs < 148) nsplit = (int)std::max<int64_t>(1, std::min<int64_t>(std::min(chunks, 4), 148 / pairs));
+  if (nsplit > 1) {
+    if (int rc = cuda_check(cudaMemsetAsync(done, 0, (size_t)pairs * 4, st), "clear split counters")) return rc;
   }
-  // CUDA-core path, one layer at a time
-  for (int l = 0; l < n_layers; ++l) {
-    csa2_swa_desc sw{};
-    if (layers[l].swa) sw = *layers[l].swa;
-    size_t smem = (size_t)kAttRows * D * 4 + kAttRows * 4;
-    dim3 grid(ns, qb->n_tok);
-    {
-      Launch L_("attend_simt", st);
-      if (D == 512) {
-        static bool attr = false;
-        if (!attr) {
-          cudaFuncSetAttribute(k_attend_simt<512>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-          attr = true;
-        }
-        k_attend_simt<512><<<grid, 256, smem, st>>>(*qb, layers[l].q, q_dtype, Hq, *kv, layers[l].idx,
-                                                    layers[l].idx_n, K, sw, n_sp,
-                                                    scale, part_o, part_ml, ns, status_ptr());
-      } else {
-        k_attend_simt<128><<<grid, 256, smem, st>>>(*qb, layers[l].q, q_dtype, Hq, *kv, layers[l].idx,
-                                                    layers[l].idx_n, K, sw, n_sp,
-                                                    scale, part_o, part_ml, ns, status_ptr());
-      }
-    }
-    if (int rc = cuda_check(cudaGetLastError(), "k_attend_simt")) return rc;
-    Launch L_("merge", st);
-    k_merge<<<dim3(Hq, qb->n_tok), 128, 0, st>>>(part_o, part_ml, ns, Hq, D, layers[l].out, out_dtype, layers[l].lse);
-    if (int rc = cuda_check(cudaGetLastError(), "k_merge")) return rc;
-  }
-  return CSA2_OK;
+  return launch_attend_tc(qb, q_dtype, Hq, kv, K, layers, n_layers, scale, out_dtype, part_o, part_ml, done, nsplit,
+                          st);
 }
 
 int launch_attend(const csa2_query_batch* qb, const void* q, int q_dtype, int Hq, const csa2_fp4_cache* kv,
@@ -444,16 +357,15 @@ int csa2_attend_workspace_size(const csa2_query_batch* qb, int32_t Hq, int32_t D
   t_err[0] = 0;
   if (int rc = check_batch(qb)) return rc;
   if (!bytes || Hq < 1 || D < 32 || K < 1) return fail(CSA2_ERR_INVALID_ARG, "bad arguments");
-  csa2_swa_desc sw{};
-  sw.window = 256;
-  *bytes = attend_ws(qb, Hq, D, K, has_swa ? &sw : nullptr);
+  (void)has_swa;
+  *bytes = attend_ws(qb, Hq, D);
   return CSA2_OK;
 }
 
 static int check_index_common(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w,
                               int H_I, const csa2_fp4_cache* kc, int P, int K) {
   if (int rc = check_batch(qb)) return rc;
-  if (int rc = check_cache(kc, "k_idx")) return rc;
+  if (int rc = check_cache(kc, "k_idx", qb)) return rc;
   if (!qc || !qs || !w) return fail(CSA2_ERR_INVALID_ARG, "indexer query buffers must be non-NULL");
   if (kc->dim != 64 && kc->dim != 128) return fail(CSA2_ERR_UNSUPPORTED, "d_I must be 64 or 128");
   if (H_I < 1 || H_I > 64) return fail(CSA2_ERR_UNSUPPORTED, "H_I must be in [1, 64]");
@@ -488,7 +400,7 @@ int csa2_index_full(const csa2_query_batch* qb, const uint8_t* q_codes, const ui
   const int64_t ld = n_blocks_max(qb);
   float* bs = static_cast<float*>(c.take((size_t)qb->n_tok * ld * 4));
   float* sc = static_cast<float*>(c.take((size_t)qb->n_tok * P * kBlock * 4));
-  SelGroup* grp = static_cast<SelGroup*>(c.take((size_t)kNumSmsNominal * sizeof(SelGroup)));
+  void* grp = c.take(select_ws(qb, P, 1));
   if (blockscore) bs = blockscore;
   if (int rc = launch_scan(qb, q_codes, q_scales, w, H_I, k_idx, bs, ld, st)) return rc;
   if (int rc = launch_select(qb, bs, ld, 0, nullptr, nullptr, P, P, pool, pool_n, grp, st)) return rc;
@@ -509,7 +421,7 @@ int csa2_index_reindex(const csa2_query_batch* qb, const uint8_t* q_codes, const
   Carve c{static_cast<uint8_t*>(workspace), workspace_bytes};
   c.take((size_t)qb->n_tok * n_blocks_max(qb) * 4);
   float* sc = static_cast<float*>(c.take((size_t)qb->n_tok * P * kBlock * 4));
-  SelGroup* grp = static_cast<SelGroup*>(c.take((size_t)kNumSmsNominal * sizeof(SelGroup)));
+  void* grp = c.take(select_ws(qb, P, 1));
   if (int rc = launch_rescore(qb, q_codes, q_scales, w, H_I, k_idx, pool, pool_n, P, sc, st)) return rc;
   return launch_select(qb, sc, (int64_t)P * kBlock, 1, pool, pool_n, P, K, idx, idx_n, grp, st);
 }
@@ -517,13 +429,15 @@ int csa2_index_reindex(const csa2_query_batch* qb, const uint8_t* q_codes, const
 static int check_attend(const csa2_query_batch* qb, const void* q, int q_dtype, int Hq, const csa2_fp4_cache* kv,
                         bool have_idx, int K, const csa2_swa_desc* swa, void* out, int out_dtype) {
   if (int rc = check_batch(qb)) return rc;
-  if (int rc = check_cache(kv, "kv")) return rc;
+  if (int rc = check_cache(kv, "kv", qb)) return rc;
   if (kv->dim != 128 && kv->dim != 512) return fail(CSA2_ERR_UNSUPPORTED, "D must be 128 or 512");
   if (Hq != 16 && Hq != 32 && Hq != 64) return fail(CSA2_ERR_UNSUPPORTED, "Hq must be 16, 32 or 64");
   if (K < 1 || K > 2048) return fail(CSA2_ERR_UNSUPPORTED, "K must be in [1, 2048]");
   if (!q || !have_idx || !out) return fail(CSA2_ERR_INVALID_ARG, "NULL buffer");
   if ((q_dtype != CSA2_F32 && q_dtype != CSA2_BF16) || (out_dtype != CSA2_F32 && out_dtype != CSA2_BF16))
     return fail(CSA2_ERR_INVALID_ARG, "bad dtype");
+  if (q_dtype == CSA2_F32 && kv->dim * Hq > 16384)
+    return fail(CSA2_ERR_UNSUPPORTED, "fp32 queries need D * Hq <= 16384 (use bf16 queries)");
   if (swa) {
     if (!swa->codes || !swa->scale) return fail(CSA2_ERR_INVALID_ARG, "swa buffers missing");
     if (swa->dim != kv->dim) return fail(CSA2_ERR_INVALID_ARG, "swa dim must equal the Main KV dim");
@@ -540,7 +454,7 @@ int csa2_attend_reuse(const csa2_query_batch* qb, const void* q, int32_t q_dtype
                       size_t workspace_bytes, void* stream) {
   t_err[0] = 0;
   if (int rc = check_attend(qb, q, q_dtype, Hq, kv, idx && idx_n, K, swa, out, out_dtype)) return rc;
-  size_t need = attend_ws(qb, Hq, kv->dim, K, swa);
+  size_t need = attend_ws(qb, Hq, kv->dim);
   if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256 || workspace_bytes < need)
     return fail(CSA2_ERR_WORKSPACE, "workspace too small or misaligned (need %zu)", need);
   float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / std::sqrt((float)kv->dim);
@@ -571,18 +485,9 @@ static size_t stack_ws(const csa2_stack_desc* d, size_t* sub_off) {
   Carve ix{nullptr, 0};
   ix.take((size_t)T * n_blocks_max(qb) * 4);                             // block scores
   ix.take((size_t)std::min(ns, kMaxSel) * T * d->P * kBlock * 4);        // pool position scores
-  ix.take((size_t)kNumSmsNominal * sizeof(SelGroup));                    // split-selection scratch
+  ix.take(select_ws(qb, d->P, std::min(ns, kMaxSel)));                  // split-selection scratch
   size_t sub = ix.used + 256;
-  bool any_swa = false;
-  int win = 0;
-  for (int l = 0; l < d->n_layers; ++l)
-    if (d->layers[l].swa) {
-      any_swa = true;
-      win = std::max(win, d->layers[l].swa->window);
-    }
-  csa2_swa_desc sw{};
-  sw.window = win;
-  sub = std::max(sub, attend_ws(qb, d->Hq, d->kv.dim, d->K, any_swa ? &sw : nullptr));
+  sub = std::max(sub, attend_ws(qb, d->Hq, d->kv.dim));
   c.take(0);
   *sub_off = c.used;
   c.take(sub);
@@ -620,7 +525,7 @@ int csa2_decode_stack(const csa2_stack_desc* d, void* workspace, size_t workspac
     if (int rc = check_attend(qb, L.q, d->q_dtype, d->Hq, &d->kv, true, d->K, L.swa, L.out, d->out_dtype))
       return rc;
   }
-  if (int rc = check_cache(&d->k_idx, "k_idx")) return rc;
+  if (int rc = check_cache(&d->k_idx, "k_idx", qb)) return rc;
   if (d->k_idx.dim != 64 && d->k_idx.dim != 128) return fail(CSA2_ERR_UNSUPPORTED, "d_I must be 64 or 128");
   if (d->H_I < 1 || d->H_I > 64 || d->P < 1 || d->P > 4096 || d->K < 1 || d->K > 2048 || d->K > d->P * kBlock)
     return fail(CSA2_ERR_UNSUPPORTED, "H_I/P/K out of the supported range");
@@ -672,7 +577,7 @@ int csa2_decode_stack(const csa2_stack_desc* d, void* workspace, size_t workspac
   const int64_t ld = n_blocks_max(qb);
   float* bs = static_cast<float*>(sc_c.take((size_t)T * ld * 4));
   float* sc = static_cast<float*>(sc_c.take((size_t)std::min(n_sel, kMaxSel) * T * d->P * kBlock * 4));
-  SelGroup* grp = static_cast<SelGroup*>(sc_c.take((size_t)kNumSmsNominal * sizeof(SelGroup)));
+  void* grp = sc_c.take(select_ws(qb, d->P, std::min(n_sel, kMaxSel)));
   // each FULL layer builds the pool that it and the REINDEX layers after it
   // rescore; the rescoring and position selection of consecutive selectors
   // run up to kMaxSel at a time

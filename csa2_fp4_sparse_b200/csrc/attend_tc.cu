@@ -85,7 +85,7 @@ struct Params {
   uint64_t wait_ns;
 };
 
-template <int D, int HQ, bool QLO>
+template <int D, int HQ, bool QLO, bool PLO>
 struct Layout {
   static constexpr int kKB = D / 64;                    // 64-element d-blocks
   static constexpr int kMT = D / 128;                   // PV M tiles
@@ -100,7 +100,9 @@ struct Layout {
   static constexpr uint32_t kOffQ = kOffTile + 2 * kTile;
   static constexpr uint32_t kOffQlo = kOffQ + (kQBytes + 1023) / 1024 * 1024;
   static constexpr uint32_t kOffP = kOffQlo + (QLO ? (kQBytes + 1023) / 1024 * 1024 : 0);  // [2][kPBytes]
-  static constexpr uint32_t kOffRows = kOffP + 2 * ((kPBytes + 1023) / 1024 * 1024);       // [kMaxRows] i32 cache rows
+  // fp32 outputs: the low fp16 part of P (one buffer; see the softmax)
+  static constexpr uint32_t kOffPlo = kOffP + 2 * ((kPBytes + 1023) / 1024 * 1024);
+  static constexpr uint32_t kOffRows = kOffPlo + (PLO ? (kPBytes + 1023) / 1024 * 1024 : 0);  // [kMaxRows] i32 cache rows
   static constexpr uint32_t kOffRs = kOffRows + kMaxRows * 4;                              // [2][kRows] f32
   static constexpr uint32_t kOffCorr = kOffRs + 2 * kRows * 4;  // [kMq] f32
   static constexpr uint32_t kOffL = kOffCorr + kMq * 4;         // [kMq] f32 final row sums
@@ -155,9 +157,9 @@ struct Pref {
   int32_t wrow[kPer];  // window unit: its row (the second 16 bytes are read at conversion)
 };
 
-template <int D, int HQ, bool QLO>
+template <int D, int HQ, bool QLO, bool PLO>
 __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant__ Params P) {
-  using Ly = Layout<D, HQ, QLO>;
+  using Ly = Layout<D, HQ, QLO, PLO>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -286,6 +288,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
       uint4 hi, lo;
       uint32_t* hp = &hi.x;
       uint32_t* lp = &lo.x;
+      // the MMAs take the query in fp16: a value at or beyond 65520 (or a NaN)
+      // has no fp16 form; it is reported and the result is not meaningful
+      bool out_of_range = false;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) out_of_range |= !(fabsf(f[k]) < 65520.0f);
+      if (out_of_range) set_status(P.status, CSA2_ERR_RANGE);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         __half2 h2 = __floats2half2_rn(f[2 * k], f[2 * k + 1]);
@@ -473,6 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
               tc::smem_desc(sbase + Ly::kOffTile + bf * Ly::kTile, kRows * 128, 1024, tc::kSwizzle128B);
           const uint64_t b0 =
               tc::smem_desc(sbase + Ly::kOffP + bf * ((Ly::kPBytes + 1023) / 1024 * 1024), 16, 1024, tc::kSwizzle128B);
+          const uint64_t bl0 = tc::smem_desc(sbase + Ly::kOffPlo, 16, 1024, tc::kSwizzle128B);
 #pragma unroll 1
           for (int mt = mt0; mt < mt1; ++mt)
 #pragma unroll
@@ -480,6 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
               const uint64_t ad = a0 + (uint64_t)(((2 * mt) * (kRows * 128) + ks * 2048) >> 4);
               const uint64_t bd = b0 + (uint64_t)((ks * 32) >> 4);
               tc::mma_f16(tmem + Ly::kColO + mt * HQ, ad, bd, idesc, (i > 0 || ks > 0) ? 1u : 0u);
+              if (PLO) tc::mma_f16(tmem + Ly::kColO + mt * HQ, ad, bl0 + (uint64_t)((ks * 32) >> 4), idesc, 1u);
             }
           tc::commit(bar_kv_empty + 8 * bf);
         }
@@ -521,6 +531,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
       // are warp-collective: every lane issues them (ok is uniform), only the
       // lanes that carry a head write P.
       uint8_t* prow = smem + Ly::kOffP + bf * ((Ly::kPBytes + 1023) / 1024 * 1024);
+      uint8_t* plow = smem + Ly::kOffPlo;
+      // fp32 outputs: P is written as two fp16 parts, hi = fp16(e) and
+      // lo = fp16(e - hi), and PV runs over both (relative error of the
+      // weights ~2^-22 instead of the 2^-12 of one fp16), while the sum adds
+      // the fp32 weights.  The one lo buffer is free once PV(i - 1) is done.
+      if (PLO && i > 0 && ok) {
+        if (!mbar_wait_group(bar_kv_empty + 8 * ((i - 1) & 1), ((i - 1) >> 1) & 1, P.wait_ns, threadIdx.x == 0,
+                             *abort != 0, 1, 128)) {
+          if (threadIdx.x == 0 && !*abort) {
+            set_status(P.status, CSA2_ERR_TIMEOUT);
+            *abort = 1;
+          }
+        }
+      }
       auto p_pass = [&](float mu_, float& sum_, float& zmax_) {
         const float nmu = mu_ == -INFINITY ? 0.0f : -mu_;
         sum_ = 0.0f;
@@ -534,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
 #pragma unroll
           for (int k = 0; k < 8; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) + __uint_as_float(v2[k]));
           {
-            uint32_t pk[4];
+            uint32_t pk[4], pl[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const int jj = 2 * k, j0 = g * 8 + jj;
@@ -545,9 +569,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
                 const float e1 = mu_ == -INFINITY ? 0.0f : ex2_approx(z1 + nmu);
                 __half2 w2 = __floats2half2_rn(e0, e1);
                 pk[k] = *reinterpret_cast<uint32_t*>(&w2);
-                // the fp16 weights are what PV uses and what the sum adds
                 const float2 back = __half22float2(w2);
-                sum_ += back.x + back.y;
+                if (PLO) {
+                  pl[k] = pack_half2(e0 - back.x, e1 - back.y);
+                  sum_ += e0 + e1;
+                } else {
+                  // the fp16 weights are what PV uses and what the sum adds
+                  sum_ += back.x + back.y;
+                }
               } else {
                 const float r0 = rsb[j0], r1 = rsb[j0 + 1];
                 const float z0 = r0 >= 0.0f ? __uint_as_float(v[jj]) * (zs * r0) : -INFINITY;
@@ -558,15 +587,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
                 const float w0 = r0 > 0.0f ? r0 : 0.0f, w1 = r1 > 0.0f ? r1 : 0.0f;
                 __half2 w2 = __floats2half2_rn(e0 * w0, e1 * w1);
                 pk[k] = *reinterpret_cast<uint32_t*>(&w2);
-                // sparse rows: sum exactly the fp16 weights the PV product uses
                 const float2 back = __half22float2(w2);
-                if (r0 == 1.0f) e0 = back.x;
-                if (r1 == 1.0f) e1 = back.y;
+                if (PLO) {
+                  pl[k] = pack_half2(e0 * w0 - back.x, e1 * w1 - back.y);
+                } else {
+                  // sparse rows: sum exactly the fp16 weights the PV product uses
+                  if (r0 == 1.0f) e0 = back.x;
+                  if (r1 == 1.0f) e1 = back.y;
+                }
                 sum_ += e0 + e1;
               }
             }
             // 16-byte chunk of 8 rows: rows 32 hf + 8 g ..
             if (act) *reinterpret_cast<uint4*>(prow + swz128(h, 4 * hf + g)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            if (PLO && act)
+              *reinterpret_cast<uint4*>(plow + swz128(h, 4 * hf + g)) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
           }
         }
         zmax_ = fmaxf(zmax_, __shfl_xor_sync(0xffffffffu, zmax_, 16));  // both halves of the head
@@ -797,19 +832,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
   }
 }
 
-template <int D, int HQ, bool QLO>
+template <int D, int HQ, bool QLO, bool PLO>
 int launch_t(const Params& p, int nsplit, int n_layers, cudaStream_t st) {
-  using Ly = Layout<D, HQ, QLO>;
+  using Ly = Layout<D, HQ, QLO, PLO>;
+  static_assert(Ly::kBytes <= 232448, "attention shared memory");
   static bool attr[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr[dev]) {
-    if (int rc = cuda_check(cudaFuncSetAttribute(k_attend_tc<D, HQ, QLO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (int rc = cuda_check(cudaFuncSetAttribute(k_attend_tc<D, HQ, QLO, PLO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  Ly::kBytes),
                             "attend smem attribute"))
       return rc;
     int fit = 0;
-    if (int rc = cuda_check(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, k_attend_tc<D, HQ, QLO>, kThreads,
+    if (int rc = cuda_check(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, k_attend_tc<D, HQ, QLO, PLO>, kThreads,
                                                                           Ly::kBytes),
                             "attend occupancy"))
       return rc;
@@ -817,16 +853,28 @@ int launch_t(const Params& p, int nsplit, int n_layers, cudaStream_t st) {
     attr[dev] = true;
   }
   Launch L_("attend_tc", st);
-  k_attend_tc<D, HQ, QLO><<<dim3(nsplit, p.qb.n_tok, n_layers), kThreads, Ly::kBytes, st>>>(p);
+  k_attend_tc<D, HQ, QLO, PLO><<<dim3(nsplit, p.qb.n_tok, n_layers), kThreads, Ly::kBytes, st>>>(p);
   return cuda_check(cudaGetLastError(), "k_attend_tc");
+}
+
+// fp32 queries (the fp16 residual copy) exist for D * Hq <= 16384 only
+template <int D, int HQ, bool PLO>
+int launch_q(const Params& p, int nsplit, int n_layers, cudaStream_t st) {
+  if constexpr (D * HQ <= 16384) {
+    return launch_t<D, HQ, true, PLO>(p, nsplit, n_layers, st);
+  } else {
+    (void)p, (void)nsplit, (void)n_layers, (void)st;
+    return fail(CSA2_ERR_UNSUPPORTED, "fp32 queries need D * Hq <= 16384");
+  }
 }
 
 }  // namespace attend_tc
 
-// tensor-core attention is used for (D, Hq) in {(512, 64), (128, 16), (128, 64), (512, 16)};
-// fp32 queries need the residual copy, which fits for D * Hq <= 16384.
+// shapes of the attention kernel: D in {128, 512}, Hq in {16, 32, 64}; fp32
+// queries keep an fp16 residual copy next to the fp16 query, which fits in
+// shared memory for D * Hq <= 16384.
 bool attend_tc_supported(int D, int Hq, int q_dtype) {
-  if (!((D == 512 || D == 128) && (Hq == 64 || Hq == 16))) return false;
+  if (!((D == 512 || D == 128) && (Hq == 64 || Hq == 32 || Hq == 16))) return false;
   if (q_dtype == CSA2_F32 && D * Hq > 16384) return false;
   return true;
 }
@@ -870,14 +918,20 @@ int launch_attend_tc(const csa2_query_batch* qb, int q_dtype, int Hq, const csa2
   p.wait_ns = 1000000000ull;
   const int D = kv->dim;
   const bool qlo = p.q_f32 != 0;
-  if (D == 512 && Hq == 64)
-    return qlo ? fail(CSA2_ERR_UNSUPPORTED, "f32 q") : launch_t<512, 64, false>(p, nsplit, n_layers, st);
-  if (D == 512 && Hq == 16)
-    return qlo ? launch_t<512, 16, true>(p, nsplit, n_layers, st) : launch_t<512, 16, false>(p, nsplit, n_layers, st);
-  if (D == 128 && Hq == 64)
-    return qlo ? launch_t<128, 64, true>(p, nsplit, n_layers, st) : launch_t<128, 64, false>(p, nsplit, n_layers, st);
-  if (D == 128 && Hq == 16)
-    return qlo ? launch_t<128, 16, true>(p, nsplit, n_layers, st) : launch_t<128, 16, false>(p, nsplit, n_layers, st);
+  // fp32 outputs take the two-part P (see the softmax)
+  const bool plo = p.out_f32 != 0;
+#define CSA2_ATT_CASE(d, hq)                                                                                   \
+  if (D == d && Hq == hq) {                                                                                   \
+    if (plo) return qlo ? launch_q<d, hq, true>(p, nsplit, n_layers, st) : launch_t<d, hq, false, true>(p, nsplit, n_layers, st); \
+    return qlo ? launch_q<d, hq, false>(p, nsplit, n_layers, st) : launch_t<d, hq, false, false>(p, nsplit, n_layers, st); \
+  }
+  CSA2_ATT_CASE(512, 64)
+  CSA2_ATT_CASE(512, 32)
+  CSA2_ATT_CASE(512, 16)
+  CSA2_ATT_CASE(128, 64)
+  CSA2_ATT_CASE(128, 32)
+  CSA2_ATT_CASE(128, 16)
+#undef CSA2_ATT_CASE
   return fail(CSA2_ERR_UNSUPPORTED, "attend_tc shape");
 }
 

@@ -30,7 +30,6 @@ struct AttendLayer {
 };
 constexpr int kMaxAttLayers = 32;  // layers per attention launch
 constexpr int kMaxSel = 8;         // selector layers per rescoring launch
-constexpr int kNumSmsNominal = 148;  // B200 SMs: sizes the split-selection scratch
 struct SelGroup;
 int launch_attend_tc(const csa2_query_batch* qb, int q_dtype, int Hq, const csa2_fp4_cache* kv, int K,
                      const AttendLayer* layers, int n_layers, float scale, int out_dtype, float* part_o,

@@ -9,8 +9,6 @@
 // candidate) in a fixed file-scope device array that every GPU which loads the
 // library holds until the process exits.  The call allocates nothing: no
 // cudaMalloc, no cudaFree, no allocating library routine.
-#include <mutex>
-
 #include "common.cuh"
 #include "internal.h"
 
@@ -20,26 +18,15 @@ namespace csa2 {
 constexpr int64_t kNoAllocScratchFloats = int64_t(1) << 20;
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
 
-// device address of the array, looked up once per device with that device
-// current (in host code the symbol is only a host-side stand-in)
+// device address of the array for the current device.  In host code the
+// symbol is only a host-side stand-in, so the address is looked up with that
+// device current, on every call: a cached address would go stale if the
+// device were reset (a new context loads the module again at another
+// address).  The lookup allocates nothing.
 static float* noalloc_scratch_ptr(int* rc) {
-  static std::mutex mu;
-  static float* cache[64] = {nullptr};
-  int dev = 0;
-  *rc = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
-  if (*rc) return nullptr;
-  if (dev < 0 || dev >= 64) {
-    *rc = fail(CSA2_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
-    return nullptr;
-  }
-  std::lock_guard<std::mutex> lk(mu);
-  if (!cache[dev]) {
-    float* p = nullptr;
-    *rc = cuda_check(cudaGetSymbolAddress((void**)&p, g_noalloc_scratch), "cudaGetSymbolAddress(scratch)");
-    if (*rc) return nullptr;
-    cache[dev] = p;
-  }
-  return cache[dev];
+  float* p = nullptr;
+  *rc = cuda_check(cudaGetSymbolAddress((void**)&p, g_noalloc_scratch), "cudaGetSymbolAddress(scratch)");
+  return *rc ? nullptr : p;
 }
 
 int check_index_args(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H_I,
@@ -48,7 +35,7 @@ int launch_rescore(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t*
                    const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n, int P, float* scores,
                    cudaStream_t st);
 int launch_select(const csa2_query_batch* qb, const float* score, int64_t ld, int mode, const int32_t* pool,
-                  const int32_t* pool_n, int P, int k_out, int32_t* out, int32_t* out_n, SelGroup* grp,
+                  const int32_t* pool_n, int P, int k_out, int32_t* out, int32_t* out_n, void* scratch,
                   cudaStream_t st);
 void clear_last_error();
 

@@ -44,6 +44,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+
 #include "internal.h"
 #include "tc_common.cuh"
 
@@ -100,6 +102,7 @@ struct Params {
   const uint8_t* q_scales;  // [n_sel][T][H][d_I/32]
   const float* w[kMaxSel];  // per selector [T][H]
   int n_sel;                // rescore: selector layers (scan: 1)
+  int qchunks;              // scan: groups per sequence, each of up to kMaxW of its query tokens
   int H, N, DI;
   int64_t n_rows;
   int page_size, max_pages;
@@ -114,20 +117,18 @@ struct Params {
   uint64_t wait_ns;
 };
 
-// Work groups: a sequence (scan: all of its query tokens share every tile) or
-// a query token (rescore: its own pool).  Tiles are 128 positions.
+// Work groups: a chunk of up to kMaxW query tokens of one sequence (scan:
+// the chunk's tokens share every tile; sequence b's chunk c is group
+// b * qchunks + c and holds its tokens c*kMaxW ..; a decode step with at most
+// kMaxW tokens per sequence has one chunk per sequence, and longer token runs
+// (verify, chunked prefill) read the keys once per chunk) or a query token
+// (rescore: its own pool).  Tiles are 128 positions.
 template <bool kRescore>
 __device__ __forceinline__ int n_groups(const Params& P) {
-  return kRescore ? P.n_sel * P.qb.n_tok : P.qb.n_seq;
+  return kRescore ? P.n_sel * P.qb.n_tok : P.qb.n_seq * P.qchunks;
 }
 
-template <bool kRescore>
-__device__ __forceinline__ int group_tiles(const Params& P, int g) {
-  if (kRescore) return (min(__ldg(P.pool_n + g % P.qb.n_tok), P.pool_cap) + 15) / 16;
-  return (__ldg(P.qb.seq_len + g) + kTile - 1) / kTile;
-}
-
-// first query token, number of query tokens, sequence of group g
+// first query token, number of query tokens (0: empty chunk), sequence of group g
 template <bool kRescore>
 __device__ __forceinline__ void group_info(const Params& P, int g, int* tok0, int* W, int* b) {
   if (kRescore) {
@@ -135,10 +136,22 @@ __device__ __forceinline__ void group_info(const Params& P, int g, int* tok0, in
     *W = 1;
     *b = __ldg(P.qb.tok_seq + *tok0);
   } else {
-    *tok0 = __ldg(P.qb.tok_start + g);
-    *W = __ldg(P.qb.tok_start + g + 1) - *tok0;
-    *b = g;
+    *b = g / P.qchunks;
+    const int t_end = __ldg(P.qb.tok_start + *b + 1);
+    *tok0 = __ldg(P.qb.tok_start + *b) + (g % P.qchunks) * kMaxW;
+    *W = max(0, min(kMaxW, t_end - *tok0));
   }
+}
+
+// tiles of group g: those holding a position visible to one of its tokens
+template <bool kRescore>
+__device__ __forceinline__ int group_tiles(const Params& P, int g) {
+  if (kRescore) return (min(__ldg(P.pool_n + g % P.qb.n_tok), P.pool_cap) + 15) / 16;
+  int tok0, W, b;
+  group_info<false>(P, g, &tok0, &W, &b);
+  if (W <= 0) return 0;
+  const int64_t vis = min((int64_t)__ldg(P.qb.tok_pos + tok0 + W - 1) + 1, (int64_t)__ldg(P.qb.seq_len + b));
+  return (int)((max(vis, (int64_t)0) + kTile - 1) / kTile);
 }
 
 // this CTA's contiguous range of (group, tile) work in group-major order
@@ -726,8 +739,6 @@ static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const 
                            int n_sel, int H, const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n,
                            int pool_cap, float* out, int64_t ld, cudaStream_t st) {
   using namespace scan_tc;
-  if (!kRescore && qb->max_q_per_seq > kMaxW)
-    return fail(CSA2_ERR_UNSUPPORTED, "scan: more than %d query tokens per sequence", kMaxW);
   if (kc->n_rows * (kc->dim / 32) >= (int64_t(1) << 31)) return fail(CSA2_ERR_UNSUPPORTED, "cache too large for TMA");
   const int box_rows = kRescore ? kBlock : kChunk;
   CUtensorMap tmc, tms;
@@ -740,6 +751,7 @@ static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const 
   if (n_sel < 1 || n_sel > kMaxSel) return fail(CSA2_ERR_UNSUPPORTED, "1..%d selector layers per launch", kMaxSel);
   for (int i = 0; i < n_sel; ++i) p.w[i] = w[i];
   p.n_sel = n_sel;
+  p.qchunks = kRescore ? 1 : std::max(1, (qb->max_q_per_seq + kMaxW - 1) / kMaxW);
   p.H = H;
   p.N = (H + 15) / 16 * 16;
   p.DI = kc->dim;

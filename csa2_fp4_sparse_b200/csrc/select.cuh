@@ -36,6 +36,7 @@ constexpr int kSelWarpSpan = 32 * kSelPer;       // 512 ids per warp per tile
 constexpr int kSelBins = 4096;
 constexpr int kSelRounds = 3;
 constexpr int kSelMaxSplit = 64;
+constexpr int kSelMaxGroups = 148;  // groups of a split launch (fewer than the SMs)
 
 struct SelGroup {
   uint32_t bar;                  // barrier arrivals (S per barrier)

@@ -53,7 +53,8 @@ enum {
   CSA2_ERR_CUDA = -4,         /* a CUDA runtime call failed (message in csa2_last_error) */
   CSA2_ERR_TIMEOUT = -5,      /* device: a bounded wait inside a kernel gave up */
   CSA2_ERR_NONFINITE = -6,    /* device: quantiser input held Inf/NaN (that group is zeroed) */
-  CSA2_ERR_RANGE = -7         /* device: an index/page entry of the inputs was out of range (skipped) */
+  CSA2_ERR_RANGE = -7         /* device: an index/page entry of the inputs was out of range (skipped),
+                               * or a main query value has no fp16 form (|q| >= 65520 or NaN) */
 };
 
 enum { CSA2_F32 = 0, CSA2_BF16 = 1 };                         /* element types of q / out */
@@ -80,8 +81,9 @@ typedef struct csa2_query_batch {
  * per byte (element 2i in the low nibble) in codes[r][dim/2] and one E4M3
  * scale per 32 elements in scales[r][dim/32].  Position t of sequence b lives
  * in row  page_table[b*max_pages + t/page_size]*page_size + t%page_size  when
- * page_table != NULL (page_size must be a multiple of 64), else in row
- * seq_base[b] + t. */
+ * page_table != NULL (page_size must be a multiple of 64, and a table row
+ * must cover the batch: max_pages * page_size >= max_seq_len, else the calls
+ * return CSA2_ERR_INVALID_ARG), else in row seq_base[b] + t. */
 typedef struct csa2_fp4_cache {
   uint8_t* codes;
   uint8_t* scales;
@@ -163,7 +165,9 @@ int csa2_quantize_fp4(const float* x, int64_t n_rows, int32_t dim, const int64_t
  * pool [T][P], pool_n [T], idx [T][K], idx_n [T]; blockscore: optional
  * [T][ceil(max_seq_len/8)] fp32 copy of B_j (entries past a token's last
  * visible block are unspecified).  d_I = k_idx->dim in {64, 128};
- * 1 <= H_I <= 64; 1 <= P <= 4096; 1 <= K <= 2048; K <= 8*P. */
+ * 1 <= H_I <= 64; 1 <= P <= 4096; 1 <= K <= 2048; K <= 8*P.  Any number of
+ * query tokens per sequence: the scan reads the keys once for every 8 of a
+ * sequence's tokens (a decode or verify step with W_b <= 8 reads them once). */
 int csa2_index_full(const csa2_query_batch* qb, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
                     int32_t H_I, const csa2_fp4_cache* k_idx, int32_t P, int32_t K, int32_t* pool, int32_t* pool_n,
                     int32_t* idx, int32_t* idx_n, float* blockscore, void* workspace, size_t workspace_bytes,
@@ -182,9 +186,12 @@ int csa2_index_reindex(const csa2_query_batch* qb, const uint8_t* q_codes, const
  * FP4 Main KV, V = the same latent), concatenated when swa != NULL with the
  * window rows max(0,p_i-window+1)..p_i of the FP8 SWA KV; one softmax over the
  * concatenation; out[i][h] = sum softmax(z)_t * v_t, rounded once to out_dtype.
- * q: [T][Hq][D] q_dtype (CSA2_F32 or CSA2_BF16; magnitudes below 65504);
+ * q: [T][Hq][D] q_dtype (CSA2_F32 or CSA2_BF16); the tensor-core products
+ * take q in fp16 (an fp32 q as an fp16 value plus its fp16 residual), so
+ * |q| must stay below 65520 (else CSA2_ERR_RANGE is recorded);
  * out: [T][Hq][D] out_dtype; lse optional [T][Hq].  D = kv->dim in {128, 512};
- * Hq in {16, 32, 64}; 1 <= K <= 2048. */
+ * Hq in {16, 32, 64}; CSA2_F32 queries need D * Hq <= 16384 (else
+ * CSA2_ERR_UNSUPPORTED); 1 <= K <= 2048. */
 int csa2_attend_reuse(const csa2_query_batch* qb, const void* q, int32_t q_dtype, int32_t Hq, const csa2_fp4_cache* kv,
                       const int32_t* idx, const int32_t* idx_n, int32_t K, const csa2_swa_desc* swa,
                       float softmax_scale, void* out, int32_t out_dtype, float* lse, void* workspace,
@@ -219,17 +226,22 @@ int csa2_version(void);
  * device memory for its KV pool at start-up and forbids later allocations,
  * or a plug-in interface with no workspace argument).  The method described
  * on the pages has no counterpart to this call; it computes exactly what
- * csa2_index_reindex computes, with the same kernels.
+ * csa2_index_reindex computes, with the same kernels, except that its
+ * selection runs one CTA per query token (csa2_index_reindex splits a
+ * token's candidates over several CTAs when there are few tokens), so for
+ * small n_tok it can be slower.
  * Scratch: a fixed file-scope device array of 2^20 fp32 candidate scores
  * (4 MiB) that every GPU loading the library holds until the process exits;
  * requires n_tok * P * 8 <= 2^20, else returns CSA2_ERR_WORKSPACE and
  * launches nothing.  The call allocates nothing (no cudaMalloc, cudaFree or
- * allocating library routine).  The first call on a device looks up the
- * array's device address (cudaGetSymbolAddress) with that device current;
- * make that first call before any stream capture.  Every call shares the one
- * array and leaves its contents behind; each call overwrites every slot it
- * reads, so nothing needs clearing, but calls that overlap on the GPU (other
- * streams, other threads) race on the array and must be serialised. */
+ * allocating library routine).  Every call looks up the array's device
+ * address for the current device (cudaGetSymbolAddress), so the address
+ * stays right after a device reset; the first call on a device also loads
+ * the library's kernels there, so make it before any stream capture.  Every
+ * call shares the one array and leaves its contents behind; each call
+ * overwrites every slot it reads, so nothing needs clearing, but calls that
+ * overlap on the GPU (other streams, other threads) race on the array and
+ * must be serialised. */
 int csa2_index_reindex_noalloc(const csa2_query_batch* qb, const uint8_t* q_codes, const uint8_t* q_scales,
                                const float* w, int32_t H_I, const csa2_fp4_cache* k_idx, const int32_t* pool,
                                const int32_t* pool_n, int32_t P, int32_t K, int32_t* idx, int32_t* idx_n,

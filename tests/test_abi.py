@@ -132,3 +132,47 @@ def test_struct_layouts_match_header(tmp_path):
         assert got[(name, "sizeof")] == ctypes.sizeof(cls), name
         for f in cls._fields_:
             assert got[(name, f[0])] == getattr(cls, f[0]).offset, (name, f[0])
+
+
+def test_paged_cache_must_cover_the_batch():
+    """A paged cache whose table rows cover fewer positions than the batch's
+    longest sequence is refused before any launch (the kernels index the page
+    table without a bound)."""
+    b = _batch(max_seq_len=1000)
+    short = C.csa2_fp4_cache(16, 16, 1 << 20, 128, 64, 16, 15, None)   # 15 * 64 = 960 < 1000
+    enough = C.csa2_fp4_cache(16, 16, 1 << 20, 128, 64, 16, 16, None)  # 1024
+    full = lambda kc: C.csa2_index_full(ctypes.byref(b), 256, 256, 256, 64, ctypes.byref(kc), 2048, 512, 256,  # noqa: E731
+                                        256, 256, 256, None, 256, 1 << 30, None)
+    assert full(short) == C.CSA2_ERR_INVALID_ARG
+    assert "max_pages" in C.csa2_last_error()
+    reindex = lambda kc: C.csa2_index_reindex(ctypes.byref(b), 256, 256, 256, 64, ctypes.byref(kc), 256, 256,  # noqa: E731
+                                              2048, 512, 256, 256, 256, 1 << 30, None)
+    assert reindex(short) == C.CSA2_ERR_INVALID_ARG
+    kv_short = C.csa2_fp4_cache(16, 16, 1 << 20, 512, 64, 16, 15, None)
+    rc = C.csa2_attend_reuse(ctypes.byref(b), 256, C.CSA2_BF16, 64, ctypes.byref(kv_short), 256, 256, 512, None,
+                             0.0, 256, C.CSA2_BF16, None, 256, 1 << 30, None)
+    assert rc == C.CSA2_ERR_INVALID_ARG
+    # the covering table passes the table check: with a too-small workspace
+    # the call stops at the workspace check instead (nothing is launched)
+    rc = C.csa2_index_full(ctypes.byref(b), 256, 256, 256, 64, ctypes.byref(enough), 2048, 512, 256, 256, 256, 256,
+                           None, 256, 10, None)
+    assert rc == C.CSA2_ERR_WORKSPACE
+
+
+def test_attend_shapes():
+    """Hq in {16, 32, 64}, D in {128, 512}; fp32 queries need D * Hq <= 16384"""
+    b = _batch()
+    call = lambda Hq, D, qdt: C.csa2_attend_reuse(  # noqa: E731
+        ctypes.byref(b), 256, qdt, Hq, ctypes.byref(C.csa2_fp4_cache(16, 16, 100, D, 0, None, 0, 16)), 256, 256,
+        512, None, 0.0, 256, C.CSA2_BF16, None, 256, 10, None)
+    for Hq in (16, 32, 64):
+        for D in (128, 512):
+            for qdt in (C.CSA2_BF16, C.CSA2_F32):
+                rc = call(Hq, D, qdt)
+                if qdt == C.CSA2_F32 and D * Hq > 16384:
+                    assert rc == C.CSA2_ERR_UNSUPPORTED, (Hq, D)
+                    assert "fp32" in C.csa2_last_error()
+                else:  # accepted shape: only the (deliberately tiny) workspace is refused
+                    assert rc == C.CSA2_ERR_WORKSPACE, (Hq, D, qdt, C.csa2_last_error())
+    assert call(48, 512, C.CSA2_BF16) == C.CSA2_ERR_UNSUPPORTED
+    assert call(64, 256, C.CSA2_BF16) == C.CSA2_ERR_UNSUPPORTED
