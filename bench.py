@@ -349,6 +349,9 @@ def run_ours(args):
         step()
     st = C.csa2_get_status(sp)
     assert st == 0, f"device status {st}"
+    # measured tensor peaks of the two MMA kinds the step uses (outside the
+    # timed region): block-scaled FP4 (indexer) and fp16 (attention)
+    probe = {"fp4_tflops": C.csa2_tensor_peak(1, 8192, sp), "f16_tflops": C.csa2_tensor_peak(0, 8192, sp)}
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     clocks = ClockSampler(local)
@@ -400,20 +403,23 @@ def run_ours(args):
     tot_prof = sum(v[1] for v in kstats.values())
     fl = algorithmic_flops(w)
     # per kernel: algorithmic bytes (HBM) and tensor FLOPs per step over its time
-    # per step; FP4 MMAs against the measured bf16 peak x 4 (the nominal
-    # 9 / 2.25 PFLOP/s ratio), fp16 MMAs against the measured bf16 peak
-    per_kernel = {"scan": (ab["scan"], fl["scan"], 4.0), "rescore": (ab["rescore"], fl["rescore"], 4.0),
-                  "attend": (ab["attend"] + ab["swa"], fl["attend"], 1.0)}
+    # per step; FP4 MMAs against the FP4 peak measured by the probe above
+    # (tensor_frac; tensor_frac_bf16x4: against the measured bf16 peak x 4, the
+    # nominal 9 / 2.25 PFLOP/s ratio), fp16 MMAs against the measured bf16 peak
+    fp4_peak = probe["fp4_tflops"]
+    per_kernel = {"scan": (ab["scan"], fl["scan"], fp4_peak), "rescore": (ab["rescore"], fl["rescore"], fp4_peak),
+                  "attend": (ab["attend"] + ab["swa"], fl["attend"], peak_bf16)}
     for n, (cnt, ms) in sorted(kstats.items(), key=lambda kv: -kv[1][1]):
         kernels[n] = {"launches_per_step": cnt / args.steps, "us_per_step": 1000.0 * ms / args.steps,
                       "share": ms / tot_prof if tot_prof else None}
         key = next((k for k in per_kernel if n.startswith(k)), None)
         if key and ms > 0:
-            b, f, ratio = per_kernel[key]
+            b, f, tpeak = per_kernel[key]
             sec = ms / args.steps / 1000.0
             kernels[n].update({"hbm_gbs": b / sec / 1e9, "hbm_frac": b / sec / 1e9 / peak_hbm,
-                               "tensor_tflops": f / sec / 1e12,
-                               "tensor_frac": f / sec / 1e12 / (peak_bf16 * ratio)})
+                               "tensor_tflops": f / sec / 1e12, "tensor_frac": f / sec / 1e12 / tpeak})
+            if key != "attend":
+                kernels[n]["tensor_frac_bf16x4"] = f / sec / 1e12 / (4.0 * peak_bf16)
     if scan_name:
         cnt, ms = kstats[scan_name]
         avg_s = ms / cnt / 1000.0
@@ -455,6 +461,7 @@ def run_ours(args):
             "config": _workload_desc(cfg, w), "parallelism": f"replicas x{world}",
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(n_launch),
             "clocks": clk, "kernels": kernels,
+            "tensor_peaks": dict(probe, bf16_measured_tflops=peak_bf16, source=peak_kind),
             "scan_gbs": roof["achieved"] if roof else None,
             "algorithmic_bytes_per_step": ab,
             "step_ms_min_max": [min(step_ms), max(step_ms)],

@@ -77,6 +77,7 @@ _SIGS = {
     "csa2_profiler_enable": [ctypes.c_int],
     "csa2_profiler_read": [_vp, _i32, _vp],
     "csa2_launch_count": [],
+    "csa2_tensor_peak": [_i32, _i32, ctypes.POINTER(ctypes.c_double), _vp],
 }
 
 _lib = None
@@ -144,6 +145,13 @@ def csa2_profiler_read(cap: int = 64) -> dict:
     n = _i32(0)
     check(lib().csa2_profiler_read(arr, cap, ctypes.byref(n)))
     return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms)) for i in range(n.value)}
+
+
+def csa2_tensor_peak(kind: int, iters: int, stream) -> float:
+    """measured dense MMA rate (TFLOP/s) of kind 0 (fp16) or 1 (block-scaled FP4)"""
+    v = ctypes.c_double(0.0)
+    check(lib().csa2_tensor_peak(kind, iters, ctypes.byref(v), stream))
+    return v.value
 
 
 def csa2_last_error() -> str:

@@ -261,6 +261,16 @@ int csa2_profiler_enable(int on);
  * the last read (or enable) into `out`, sets *n_out, and clears them. */
 int csa2_profiler_read(csa2_kernel_stat* out, int32_t cap, int32_t* n_out);
 
+/* Tensor-core peak probe (a measurement hook, not part of the decode step):
+ * every SM issues back-to-back dense M = 128, N = 256 MMAs from fixed
+ * shared-memory operands, kind 0: kind::f16 (the attention products, fp16 in,
+ * fp32 accumulate, K = 16), kind 1: kind::mxf4nvf4 with UE4M3 scales per 16
+ * elements (the indexer products, K = 64); `iters` MMAs per issuing thread
+ * (16 .. 2^20), two issuing threads per SM.  Writes the best of two timed runs
+ * (after a warm-up run) in TFLOP/s (2 M N K per MMA) to *tflops.
+ * Synchronises `stream`. */
+int csa2_tensor_peak(int32_t kind, int32_t iters, double* tflops, void* stream);
+
 /* Number of kernels this process has launched through the library. */
 int64_t csa2_launch_count(void);
 
