@@ -78,6 +78,13 @@ _SIGS = {
     "csa2_profiler_read": [_vp, _i32, _vp],
     "csa2_launch_count": [],
     "csa2_tensor_peak": [_i32, _i32, ctypes.POINTER(ctypes.c_double), _vp],
+    "csa2_cp_candidates": [_vp, _i64, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
+    "csa2_cp_merge": [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
+    "csa2_cp_localize": [_vp, _vp, _i32, _i32, _i64, _i64, _i32, _vp, _vp, _vp],
+    "csa2_cp_pool_scores": [_P(csa2_query_batch), _vp, _vp, _vp, _i32, _i32, _P(csa2_fp4_cache), _vp, _vp, _i32,
+                            _vp, _vp],
+    "csa2_cp_select_positions": [_vp, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _vp],
+    "csa2_cp_attend_merge": [_vp, _vp, _i32, _i64, _i64, _i32, _i32, _i32, _vp, _i32, _vp, _vp],
 }
 
 _lib = None
@@ -129,6 +136,12 @@ csa2_stack_workspace_size = _wrap("csa2_stack_workspace_size")
 csa2_get_status = _wrap("csa2_get_status")
 csa2_version = _wrap("csa2_version")
 csa2_selftest_wait_timeout = _wrap("csa2_selftest_wait_timeout")
+csa2_cp_candidates = _wrap("csa2_cp_candidates")
+csa2_cp_merge = _wrap("csa2_cp_merge")
+csa2_cp_localize = _wrap("csa2_cp_localize")
+csa2_cp_pool_scores = _wrap("csa2_cp_pool_scores")
+csa2_cp_select_positions = _wrap("csa2_cp_select_positions")
+csa2_cp_attend_merge = _wrap("csa2_cp_attend_merge")
 
 
 class csa2_kernel_stat(ctypes.Structure):

@@ -131,10 +131,11 @@ struct Carve {
 
 static int n_blocks_max(const csa2_query_batch* qb) { return (qb->max_seq_len + kBlock - 1) / kBlock; }
 
-// split-selection scratch: one record per (selector, token) group of a
-// split launch (a launch splits only while it has fewer groups than SMs)
+// split-selection scratch: one record per (selector, token) group of a split
+// launch (a launch splits only while it has fewer groups than SMs)
 static size_t select_ws(const csa2_query_batch*, int, int) { return (size_t)kSelMaxGroups * sizeof(SelGroup); }
 
+// block scores, pool position scores, selection scratch
 static size_t index_ws(const csa2_query_batch* qb, int P) {
   Carve c{nullptr, 0};
   c.take((size_t)qb->n_tok * n_blocks_max(qb) * 4);  // block scores
@@ -186,8 +187,8 @@ int launch_quantize(const float* x, int64_t n_rows, int dim, const int64_t* slot
   return launch_quantize_jobs(J, st);
 }
 
-int launch_scan(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
-                const csa2_fp4_cache* kc, float* bs, int64_t ld, cudaStream_t st) {
+static int launch_scan(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
+                         const csa2_fp4_cache* kc, float* bs, int64_t ld, cudaStream_t st) {
   return launch_scan_tc(qb, qc, qs, w, H, kc, bs, ld, st);
 }
 
@@ -368,6 +369,8 @@ static int check_index_common(const csa2_query_batch* qb, const uint8_t* qc, con
   if (int rc = check_cache(kc, "k_idx", qb)) return rc;
   if (!qc || !qs || !w) return fail(CSA2_ERR_INVALID_ARG, "indexer query buffers must be non-NULL");
   if (kc->dim != 64 && kc->dim != 128) return fail(CSA2_ERR_UNSUPPORTED, "d_I must be 64 or 128");
+  if ((kc->n_rows * (kc->dim / 32)) % 16)
+    return fail(CSA2_ERR_UNSUPPORTED, "indexer cache: n_rows * d_I / 32 must be a multiple of 16");
   if (H_I < 1 || H_I > 64) return fail(CSA2_ERR_UNSUPPORTED, "H_I must be in [1, 64]");
   if (P < 1 || P > 4096) return fail(CSA2_ERR_UNSUPPORTED, "P must be in [1, 4096]");
   if (K < 1 || K > 2048 || K > P * kBlock) return fail(CSA2_ERR_UNSUPPORTED, "K must be in [1, min(2048, 8P)]");
@@ -527,6 +530,8 @@ int csa2_decode_stack(const csa2_stack_desc* d, void* workspace, size_t workspac
   }
   if (int rc = check_cache(&d->k_idx, "k_idx", qb)) return rc;
   if (d->k_idx.dim != 64 && d->k_idx.dim != 128) return fail(CSA2_ERR_UNSUPPORTED, "d_I must be 64 or 128");
+  if ((d->k_idx.n_rows * (d->k_idx.dim / 32)) % 16)
+    return fail(CSA2_ERR_UNSUPPORTED, "indexer cache: n_rows * d_I / 32 must be a multiple of 16");
   if (d->H_I < 1 || d->H_I > 64 || d->P < 1 || d->P > 4096 || d->K < 1 || d->K > 2048 || d->K > d->P * kBlock)
     return fail(CSA2_ERR_UNSUPPORTED, "H_I/P/K out of the supported range");
   size_t sub_off;

@@ -7,40 +7,40 @@
 //   s_t = sum_h w[i][h] * max(0, q~_{i,h} . k~_t),   B_j = max_{t in block j} s_t
 // (hierarchical indexer of the DeepSeek-V4.1-Flash pages, dbyun.net article
 // 10794, section "KV Cache 成为这一代架构改造的核心": the first Full layer scans
-// the whole visible context and keeps blocks of 8 positions).
+// the whole visible context and keeps blocks of 8 positions; later layers
+// rescore only the pool).
 //
-// Design (one persistent CTA per SM, warp-specialised):
-//   warp 0      TMA producer (rescoring: warps 0, 21, 22 on alternate groups
-//               of tiles, as a TMA instruction costs its warp ~110 cycles and
-//               a rescoring tile gathers 32 boxes): tiles of 128 positions of
-//               the FP4 indexer K cache
-//               (codes with the 64B/32B swizzle the MMA expects, plus the raw
-//               E4M3 scales) into a shared-memory ring of 17 stages (15 when
-//               rescoring);
-//   warps 19,20 scale-factor warps (alternate passes of two tiles):
-//               rearrange each landed tile's scales into the tensor-core
-//               scale-factor layout (each per-32 E4M3 scale written twice, as
-//               the block-scaled MMA takes one UE4M3 scale per 16 elements)
-//               and copy it to TMEM (tcgen05.cp); a commit hands the stage to
-//               the MMA warp;
-//   warps 1, 18 MMA issuers (alternate tiles, two epilogue warpgroups each):
-//               issue tcgen05.mma kind::mxf4nvf4 (M = 128 positions, N =
-//               heads, K = 64 per instruction) per query token into a ring of
-//               TMEM accumulators (2 units per issuer); one commit per job hands
-//               the accumulator to the epilogue, one per tile returns the
-//               stage to the producer.  A tcgen05 instruction costs its
-//               issuing thread 100-200 cycles, so the copies are issued by the
-//               scale-factor warps, not here;
-//   warps 2..17 epilogue, four warpgroups: warpgroup e takes the accumulator
-//               jobs of MMA warp (e & 1) whose job count has parity e >> 1:
-//               TMEM -> registers (one position per thread), ReLU, weighted
-//               head sum, block max over 8 lanes, block-score store.
-// The key cache is streamed from HBM exactly once per sequence for all of its
-// query tokens.  In rescoring mode the producer instead gathers the 16 pool
-// blocks of a tile (8 rows each, one swizzle atom per block) for one query
-// token, and the epilogue writes one score per pool position.  All waits are
-// bounded; on timeout the kernel records CSA2_ERR_TIMEOUT, drains its own
-// copies and MMAs, frees TMEM and returns.
+// Work: one persistent CTA per SM walks a contiguous range of (group, stage)
+// items.  A stage is 128 positions of the FP4 indexer K cache; a group is up
+// to four "query columns" that share its stages: the scan's group is up to
+// four query tokens of one sequence (one pass over the sequence's keys per
+// group), the rescoring's group is one query token and up to four selector
+// layers (the token's pool is gathered once for all of them).
+//
+// Warp roles (16 warps):
+//   0, 1    TMA producers, alternate stages: the stage's codes (a 128-row box,
+//           two 64-row boxes when pages hold 64 rows, or 16 gathered 8-row
+//           pool blocks) in the 64B/32B swizzle the MMA reads, and the rows'
+//           per-32 E4M3 scales (the scale array seen as rows of 16 bytes);
+//   2, 3    MMA issuers, alternate stages: per query column two
+//           tcgen05.mma.kind::mxf4nvf4.block_scale.block16 (M = 128 positions,
+//           N = heads, K = 64 each) into the column's part of a TMEM
+//           accumulator slot, then one commit per stage, which frees the
+//           stage for the producer and hands the slot to the epilogue;
+//   4 .. 7  scale-factor warps, one per TMEM lane quarter: each writes the
+//           stage's scales in the block-scale layout with tcgen05.st (each
+//           per-32 scale twice: the MMA takes one UE4M3 scale per 16
+//           elements) and arrives on the stage's scale barrier;
+//   8 .. 19 epilogue, three warpgroups taking stages in turn: TMEM -> registers
+//           (one position per thread), ReLU, weighted head sum, block max
+//           over 8 lanes (scan) and the score stores; the slot is released as
+//           soon as its last load has landed.
+// A tcgen05 instruction costs its issuing thread 60-170 cycles and a TMA
+// instruction several hundred, while different warps issue concurrently; the
+// roles above keep every issuing thread's per-stage instruction count small
+// (producer: 2 TMA; MMA: 2 per column + 1 commit; SF warps: one tcgen05.st).
+// All waits are bounded; on timeout the kernel records CSA2_ERR_TIMEOUT,
+// drains its own copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -52,49 +52,37 @@
 namespace csa2 {
 namespace scan_tc {
 
-constexpr int kTile = 128;      // positions per tile = MMA M
-constexpr int kChunk = 64;      // rows per TMA box
-constexpr int kAccUnits = 4;    // TMEM accumulator ring, 64 columns each (2 per MMA issuer)
-constexpr int kMaxW = 8;        // query tokens of one sequence per tile
-constexpr int kEpiWG = 4;       // epilogue warpgroups (warps 2..17)
-constexpr int kThreads = 736;   // 23 warps: 3 producers, 2 MMA issuers, 4 epilogue warpgroups, 2 scale-factor warps
-constexpr int kProducers = 3;   // TMA producer warps 0, 21, 22 when rescoring (a TMA instruction costs its
-                                // warp ~110 cycles and a rescoring tile gathers 32 boxes); the scan uses warp 0
-constexpr int kMmaWarpB = 18;   // second MMA issuer (the first is warp 1); they take alternate tiles
-constexpr int kSfWarp = 19;     // scale-factor warps 19 and 20 take alternate passes of two tiles
-constexpr int kUnitsPer = kAccUnits / 2;  // accumulator units of each MMA issuer
-constexpr uint32_t kColAcc = 0;
+constexpr int kTile = 128;      // positions per stage = MMA M
+constexpr int kStages = 18;     // stage ring: a multiple of every accumulator slot count (1, 2, 3, 6), of the
+                                // producer and MMA warp counts (2) and of the epilogue warpgroups (3)
+constexpr int kMaxWc = 4;       // query columns per group
+constexpr int kEpiWG = 3;       // epilogue warpgroups
+constexpr int kThreads = 32 * (8 + 4 * kEpiWG);
+constexpr int kProd0 = 0;       // producer warps 0, 1
+constexpr int kMma0 = 2;        // MMA warps 2, 3
+constexpr int kSf0 = 4;         // scale-factor warps 4..7 (lane quarters 0..3)
+constexpr int kEpi0 = 8;        // epilogue warpgroups 8..11, 12..15, 16..19
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColSfa = 0;                          // [kStages][8]
+constexpr uint32_t kColSfb = kColSfa + kStages * 8;      // [kMaxWc][8]
+constexpr uint32_t kColAcc = kColSfb + kMaxWc * 8;       // accumulator slots
+constexpr uint32_t kAccCols = kTmemCols - kColAcc;       // 384
 
-// Shared-memory and TMEM map.  A tile's stage stays occupied from its load
-// to the completion of its MMAs (~8-9 K cycles: load latency under full HBM
-// load, scale-factor pass, MMA), so the ring is as deep as shared memory
-// allows: 17 stages for the scan, 15 for the rescoring (whose raw-scale slot
-// holds 16 gathered boxes).
-template <bool kRescore>
-struct Ly {
-  static constexpr int kStages = kRescore ? 15 : 17;
-  // raw scales: every TMA box gets its own 128-byte-aligned slot (TMA writes
-  // shared memory at 128-byte-aligned addresses): scan 2 boxes at 256-byte
-  // slots, rescoring 16 boxes at 128-byte slots
-  static constexpr uint32_t kRawStage = kRescore ? 2048 : 512;
-  static constexpr uint32_t kColSfa = kAccUnits * 64;            // key scale factors, 8 columns per stage
-  static constexpr uint32_t kColSfb = kColSfa + kStages * 8;     // query scale factors, 8 columns per token
-  static_assert(kColSfb + kMaxW * 8 <= kTmemCols, "TMEM budget");
-  static constexpr uint32_t kOffA = 0;                                   // [kStages][8192]
-  static constexpr uint32_t kOffRaw = kOffA + kStages * 8192;            // [kStages][kRawStage]
-  static constexpr uint32_t kOffSfa = kOffRaw + kStages * kRawStage;     // [kStages][2][512]
-  static constexpr uint32_t kOffB = (kOffSfa + kStages * 1024 + 1023) / 1024 * 1024;  // [kMaxW][64 rows][64 B]
-  static constexpr uint32_t kOffSfb = kOffB + kMaxW * 4096;              // [kMaxW][2][512]
-  static constexpr uint32_t kOffW = kOffSfb + kMaxW * 1024;              // [kEpiWG][kMaxW][64] f32
-  static constexpr uint32_t kOffPos = kOffW + kEpiWG * kMaxW * 64 * 4;   // [1 + kEpiWG][kMaxW] i64 query positions
-  static constexpr uint32_t kOffBar = kOffPos + (1 + kEpiWG) * kMaxW * 8;  // mbarriers
-  static constexpr uint32_t kNumBars = 3 * kStages + 2 * kAccUnits + 5;
-  static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;           // tmem base, abort flag
-  static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;           // + alignment slack
-  static_assert(kOffB % 1024 == 0, "B tiles must be 1024-aligned");
-  static_assert(kSmemBytes <= 232448, "shared memory budget");
-};
+// shared-memory map
+constexpr uint32_t kCodeStage = 8192;                    // 128 rows x <= 64 B
+constexpr uint32_t kRawStage = 2048;                     // raw scales: up to 16 boxes at 128-byte slots
+constexpr uint32_t kOffA = 0;                            // [kStages][8192]
+constexpr uint32_t kOffRaw = kOffA + kStages * kCodeStage;
+constexpr uint32_t kOffB = kOffRaw + kStages * kRawStage;  // [kMaxWc][64 rows][64 B]
+constexpr uint32_t kOffSfb = kOffB + kMaxWc * 4096;        // [kMaxWc][2][512]
+constexpr uint32_t kOffW = kOffSfb + kMaxWc * 1024;        // [kEpiWG][kMaxWc][64] f32
+constexpr uint32_t kOffPos = kOffW + kEpiWG * kMaxWc * 64 * 4;  // [kEpiWG][kMaxWc] i64 query positions
+constexpr uint32_t kOffBar = kOffPos + kEpiWG * kMaxWc * 8;
+constexpr uint32_t kNumBars = 3 * kStages + 12 + 3;        // full, done, sf; acc_empty[6][2]; drain[2], sfb
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;      // tmem base, abort flag
+constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;      // + alignment slack
+static_assert(kOffB % 1024 == 0, "B tiles must be 1024-aligned");
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct Params {
   csa2_query_batch qb;
@@ -102,13 +90,15 @@ struct Params {
   const uint8_t* q_scales;  // [n_sel][T][H][d_I/32]
   const float* w[kMaxSel];  // per selector [T][H]
   int n_sel;                // rescore: selector layers (scan: 1)
-  int qchunks;              // scan: groups per sequence, each of up to kMaxW of its query tokens
-  int H, N, DI;
+  int cpg;                  // groups per sequence (scan) or per token (rescore)
+  int H, Nh, DI;            // heads, heads padded to 16 (MMA N per column), key dim
+  int slot_cols, n_slots;   // accumulator slots of (query columns x Nh) columns
+  int box_rows;             // scan: rows per TMA box (128, or 64 for 64-row pages)
   int64_t n_rows;
   int page_size, max_pages;
   const int32_t* page_table;
   const int64_t* seq_base;
-  float* out;        // scan: block scores [T][ld]; rescore: pool-position scores [T][ld]
+  float* out;        // scan: block scores [T][ld]; rescore: pool-position scores [n_sel*T][ld]
   int64_t ld;
   const int32_t* pool;   // rescore: [T][pool_cap] block ids
   const int32_t* pool_n; // rescore: [T]
@@ -117,44 +107,44 @@ struct Params {
   uint64_t wait_ns;
 };
 
-// Work groups: a chunk of up to kMaxW query tokens of one sequence (scan:
-// the chunk's tokens share every tile; sequence b's chunk c is group
-// b * qchunks + c and holds its tokens c*kMaxW ..; a decode step with at most
-// kMaxW tokens per sequence has one chunk per sequence, and longer token runs
-// (verify, chunked prefill) read the keys once per chunk) or a query token
-// (rescore: its own pool).  Tiles are 128 positions.
+// Groups: scan group g = (sequence b, chunk c), c < cpg, holds the sequence's
+// query tokens c*kMaxWc ..; rescore group g = (token t, chunk c), c < cpg,
+// holds selectors c*kMaxWc ..
 template <bool kRescore>
 __device__ __forceinline__ int n_groups(const Params& P) {
-  return kRescore ? P.n_sel * P.qb.n_tok : P.qb.n_seq * P.qchunks;
+  return (kRescore ? P.qb.n_tok : P.qb.n_seq) * P.cpg;
 }
 
-// first query token, number of query tokens (0: empty chunk), sequence of group g
+// group g: first query token, query columns (0: empty chunk), sequence, first selector
 template <bool kRescore>
-__device__ __forceinline__ void group_info(const Params& P, int g, int* tok0, int* W, int* b) {
+__device__ __forceinline__ void group_info(const Params& P, int g, int* tok0, int* W, int* b, int* sel0) {
   if (kRescore) {
-    *tok0 = g % P.qb.n_tok;  // group = (selector, token)
-    *W = 1;
+    *tok0 = g / P.cpg;
+    *sel0 = (g % P.cpg) * kMaxWc;
+    *W = max(0, min(kMaxWc, P.n_sel - *sel0));
     *b = __ldg(P.qb.tok_seq + *tok0);
   } else {
-    *b = g / P.qchunks;
+    *b = g / P.cpg;
+    *sel0 = 0;
     const int t_end = __ldg(P.qb.tok_start + *b + 1);
-    *tok0 = __ldg(P.qb.tok_start + *b) + (g % P.qchunks) * kMaxW;
-    *W = max(0, min(kMaxW, t_end - *tok0));
+    *tok0 = __ldg(P.qb.tok_start + *b) + (g % P.cpg) * kMaxWc;
+    *W = max(0, min(kMaxWc, t_end - *tok0));
   }
 }
 
-// tiles of group g: those holding a position visible to one of its tokens
+// stages of group g: scan, the 128-position tiles holding a position visible
+// to one of its tokens; rescore, the token's pool in 16-block tiles
 template <bool kRescore>
 __device__ __forceinline__ int group_tiles(const Params& P, int g) {
-  if (kRescore) return (min(__ldg(P.pool_n + g % P.qb.n_tok), P.pool_cap) + 15) / 16;
-  int tok0, W, b;
-  group_info<false>(P, g, &tok0, &W, &b);
+  int tok0, W, b, sel0;
+  group_info<kRescore>(P, g, &tok0, &W, &b, &sel0);
   if (W <= 0) return 0;
+  if (kRescore) return (min(__ldg(P.pool_n + tok0), P.pool_cap) + 15) / 16;
   const int64_t vis = min((int64_t)__ldg(P.qb.tok_pos + tok0 + W - 1) + 1, (int64_t)__ldg(P.qb.seq_len + b));
   return (int)((max(vis, (int64_t)0) + kTile - 1) / kTile);
 }
 
-// this CTA's contiguous range of (group, tile) work in group-major order
+// this CTA's contiguous range of (group, stage) work in group-major order
 template <bool kRescore>
 __device__ __forceinline__ void work_range(const Params& P, int64_t* begin, int64_t* end) {
   int64_t total = 0;
@@ -163,7 +153,7 @@ __device__ __forceinline__ void work_range(const Params& P, int64_t* begin, int6
   *end = total * (blockIdx.x + 1) / gridDim.x;
 }
 
-// iterator over the tiles of [begin, end)
+// iterator over the stages of [begin, end)
 template <bool kRescore>
 struct TileIter {
   int b, tile, ntile;  // b: group
@@ -211,32 +201,38 @@ __device__ __forceinline__ bool warp_wait_or_abort(uint32_t bar, uint32_t parity
   return __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
 }
 
+// cache row of position `pos` of sequence b, or -1 when outside the cache
+__device__ __forceinline__ int64_t key_row(const Params& P, int b, int64_t pos, int64_t base) {
+  int64_t row;
+  if (P.page_table) {
+    const int32_t pg = __ldg(P.page_table + (int64_t)b * P.max_pages + pos / P.page_size);
+    row = (int64_t)pg * P.page_size + pos % P.page_size;
+  } else {
+    row = base + pos;
+  }
+  return (row >= 0 && row < P.n_rows) ? row : -1;
+}
+
 template <bool kRescore>
 __global__ void __launch_bounds__(kThreads, 1)
     k_index_tc(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales,
                const __grid_constant__ Params P) {
-  using L = Ly<kRescore>;
-  constexpr int kStages = L::kStages;
-  constexpr uint32_t kRawStage = L::kRawStage;
-  constexpr uint32_t kOffA = L::kOffA, kOffRaw = L::kOffRaw, kOffSfa = L::kOffSfa, kOffB = L::kOffB,
-                     kOffSfb = L::kOffSfb, kOffW = L::kOffW, kOffPos = L::kOffPos, kOffBar = L::kOffBar,
-                     kOffMisc = L::kOffMisc, kColSfa = L::kColSfa, kColSfb = L::kColSfb;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t bar_full = sbase + kOffBar;
-  const uint32_t bar_empty = bar_full + kStages * 8;
-  const uint32_t bar_accf = bar_empty + kStages * 8;
-  const uint32_t bar_acce = bar_accf + kAccUnits * 8;
-  const uint32_t bar_drain = bar_acce + kAccUnits * 8;
-  const uint32_t bar_sfr = bar_drain + 8;
-  const uint32_t bar_drain2 = bar_sfr + 8 * kStages;
-  const uint32_t bar_drain_b = bar_drain2 + 8;
-  const uint32_t bar_sfb = bar_drain_b + 8;
-  const uint32_t bar_drain_c = bar_sfb + 8;
+  const uint32_t bar_full = sbase + kOffBar;          // [kStages] TMA landed
+  const uint32_t bar_done = bar_full + kStages * 8;   // [kStages] MMAs of the stage complete (commit)
+  const uint32_t bar_sf = bar_done + kStages * 8;     // [kStages] scale factors in TMEM (4 warps)
+  // [6 slots][2 MMA warps] accumulator slot read (4 warps): the epilogue
+  // releases a slot on the barrier of the MMA warp that uses it next, so that
+  // every barrier has one waiter and one releaser, both in stage order (a
+  // barrier waited by two warps that take turns could be waited two phases
+  // ahead, where its parity reads as complete)
+  const uint32_t bar_acce = bar_sf + kStages * 8;
+  const uint32_t bar_drain = bar_acce + 12 * 8;       // [2] MMA warps' drains
+  const uint32_t bar_sfb = bar_drain + 2 * 8;         // query scale-factor copies
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(smem + kOffMisc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
-  float* w_s = reinterpret_cast<float*>(smem + kOffW);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row_bytes = P.DI / 2, spr = P.DI / 32, ksteps = P.DI / 64;
@@ -244,24 +240,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(bar_full + 8 * i, 1);
-      mbar_init(bar_empty + 8 * i, 1);
+      mbar_init(bar_done + 8 * i, 1);
+      mbar_init(bar_sf + 8 * i, 4);
     }
-    for (int i = 0; i < kAccUnits; ++i) {
-      mbar_init(bar_accf + 8 * i, 1);
-      mbar_init(bar_acce + 8 * i, 4);
-    }
+    for (int i = 0; i < 12; ++i) mbar_init(bar_acce + 8 * i, 4);
     mbar_init(bar_drain, 1);
-    for (int i = 0; i < kStages; ++i) mbar_init(bar_sfr + 8 * i, 1);
-    mbar_init(bar_drain2, 1);
-    mbar_init(bar_drain_b, 1);
+    mbar_init(bar_drain + 8, 1);
     mbar_init(bar_sfb, 1);
-    mbar_init(bar_drain_c, 1);
     *abort = 0;
     tc::fence_barrier_init();
     tc::tma_prefetch_desc(&tm_codes);
     tc::tma_prefetch_desc(&tm_scales);
   }
-  if (warp == 1) {
+  if (warp == kMma0) {
     tc::tmem_alloc(sbase + kOffMisc, kTmemCols);
     tc::tmem_relinquish();
     tc::fence_before_sync();
@@ -273,127 +264,101 @@ __global__ void __launch_bounds__(kThreads, 1)
   int64_t wb, we;
   work_range<kRescore>(P, &wb, &we);
 
-  if (warp == 0 || warp >= kSfWarp + 2) {
+  if (warp < kMma0) {
     // ------------------------------------------------------------ producers
-    // G tiles per iteration, `boxes` lanes per tile (scan: 2 boxes of 64 rows,
-    // rescore: 16 blocks of 8 rows): the lanes of different tiles wait for
-    // their stages and issue their copies concurrently; the producer warps
-    // take alternate groups of G tiles.
-    const int pi = warp == 0 ? 0 : warp - (kSfWarp + 1);
-    constexpr int nprod = kRescore ? kProducers : 1;  // the scan's 4 boxes a tile need one warp
+    // lane k issues box k of the stage: scan 1 or 2 boxes of 128 / 64 rows,
+    // rescore 16 pool blocks of 8 rows (codes and scales each)
+    const int pw = warp - kProd0;
+    const int box_rows = kRescore ? kBlock : P.box_rows;
+    const int nbox = kRescore ? 16 : kTile / box_rows;
     const uint32_t tx = (uint32_t)kTile * row_bytes + (uint32_t)kTile * spr;
-    const int32_t oob_row = (int32_t)P.n_rows;
-    const int32_t oob_x = (int32_t)(((P.n_rows * spr) + 15) / 16 * 16);
-    constexpr int boxes = kRescore ? 16 : 2;
-    constexpr int rows_per_box = kTile / boxes;
-    // tiles per group: a group is issued once all its stages are free, so a
-    // small group keeps most of the ring in flight
-    constexpr int G = (32 / boxes) < 4 ? (32 / boxes) : 4;
-    const int lt = lane / boxes, bx = lane % boxes;
-    const bool has_slot = lane < G * boxes;
     TileIter<kRescore> ti;
     ti.init(P, wb, we);
-    for (int k = 0; k < pi * G + lt; ++k) ti.next(P);
-    int64_t it = pi * G + lt;  // this lane's tile
-    const int64_t total = pi < nprod ? we - wb : 0;
+    int64_t it = 0;
     int cur_g = -1, tok0 = 0, b = 0;
     int64_t base = 0, len = 0;
-    for (int64_t g0 = pi * G; g0 < total; g0 += nprod * G) {
-      const bool act = has_slot && ti.valid();
+    for (; ti.valid(); ti.next(P), ++it) {
+      if ((int)(it & 1) != pw || *abort) continue;
       const int s = (int)(it % kStages);
       const uint32_t n = (uint32_t)(it / kStages);
-      // the first lane of each tile waits for its stage and arms it (one warp
-      // instruction probes the stages of all the group's tiles at once)
-      if (act && bx == 0) {
-        if (wait_or_abort(bar_empty + 8 * s, (n & 1) ^ 1, P, abort)) tc::mbar_arrive_expect_tx(bar_full + 8 * s, tx);
+      if (lane == 0) {
+        // the stage is free once the MMAs of its previous use completed
+        if (n == 0 || wait_or_abort(bar_done + 8 * s, (n - 1) & 1, P, abort))
+          tc::mbar_arrive_expect_tx(bar_full + 8 * s, tx);
       }
-      __syncwarp();  // every stage of this group armed before any copy lands
-      if (act && !*abort) {
-        if (ti.b != cur_g) {
-          cur_g = ti.b;
-          int W;
-          group_info<kRescore>(P, cur_g, &tok0, &W, &b);
-          len = __ldg(P.qb.seq_len + b);
-          base = P.page_table ? 0 : __ldg(P.seq_base + b);
-        }
+      __syncwarp();
+      if (*abort) continue;
+      if (ti.b != cur_g) {
+        cur_g = ti.b;
+        int W, sel0;
+        group_info<kRescore>(P, cur_g, &tok0, &W, &b, &sel0);
+        len = __ldg(P.qb.seq_len + b);
+        base = P.page_table ? 0 : __ldg(P.seq_base + b);
+      }
+      if (lane < nbox) {
         int64_t pos0 = -1;
         if (kRescore) {
-          const int e = ti.tile * 16 + bx;
+          const int e = ti.tile * 16 + lane;
           const int np = min(__ldg(P.pool_n + tok0), P.pool_cap);
           const int32_t blk = e < np ? __ldg(P.pool + (int64_t)tok0 * P.pool_cap + e) : -1;
           if (blk >= 0) pos0 = (int64_t)blk * kBlock;
         } else {
-          pos0 = (int64_t)ti.tile * kTile + bx * kChunk;
+          pos0 = (int64_t)ti.tile * kTile + lane * box_rows;
           if (pos0 >= len) pos0 = -1;
         }
-        int64_t row0 = -1;
-        if (pos0 >= 0) {
-          if (P.page_table) {
-            const int32_t pg = __ldg(P.page_table + (int64_t)b * P.max_pages + pos0 / P.page_size);
-            row0 = (int64_t)pg * P.page_size + pos0 % P.page_size;
-          } else {
-            row0 = base + pos0;
-          }
-        }
-        int32_t ry = oob_row, sx = oob_x;
-        if (row0 >= 0 && row0 < P.n_rows && ((row0 * spr) & 15) == 0) {
+        const int64_t row0 = pos0 >= 0 ? key_row(P, b, pos0, base) : -1;
+        // out of the cache, or not 16-byte aligned in the scale array: the
+        // box is read out of range (zeros) and the row reported
+        int32_t ry = (int32_t)P.n_rows, sy = (int32_t)(P.n_rows * spr / 16);
+        if (row0 >= 0 && ((row0 * spr) & 15) == 0) {
           ry = (int32_t)row0;
-          sx = (int32_t)(row0 * spr);
-        } else if (row0 >= 0) {
-          set_status(P.status, CSA2_ERR_RANGE);  // misplaced row: read as zeros
+          sy = (int32_t)(row0 * spr / 16);
+        } else if (pos0 >= 0) {
+          set_status(P.status, CSA2_ERR_RANGE);
         }
-        tc::tma_load_2d(sbase + kOffA + s * 8192 + bx * rows_per_box * row_bytes, &tm_codes, bar_full + 8 * s, 0,
+        tc::tma_load_2d(sbase + kOffA + s * kCodeStage + lane * box_rows * row_bytes, &tm_codes, bar_full + 8 * s, 0,
                         ry);
-        tc::tma_load_1d(sbase + kOffRaw + s * kRawStage + bx * (kRawStage / boxes), &tm_scales, bar_full + 8 * s,
-                        sx);
+        const uint32_t slot = kRescore ? 128u : (uint32_t)(box_rows * spr);
+        tc::tma_load_2d(sbase + kOffRaw + s * kRawStage + lane * slot, &tm_scales, bar_full + 8 * s, 0, sy);
       }
       __syncwarp();
-      if (*abort) break;
-      for (int k = 0; k < nprod * G; ++k) ti.next(P);
-      it += nprod * G;
     }
-    // copies in flight: the scale-factor warps wait for every tile's landing
+    // copies in flight: the scale-factor warps wait for every stage's landing
     // before the CTA ends (after a failed wait, see the end of the kernel)
-  } else if (warp == 1 || warp == kMmaWarpB) {
+  } else if (warp < kSf0) {
     // ------------------------------------------------------------ MMA issuers
-    // Both issuers walk every tile (so both see every change of group) and
-    // issue the MMAs of the tiles of their parity; a single issuing thread is
-    // limited by the latency of its barrier tests and MMA issues, two overlap.
-    const int mw = warp == 1 ? 0 : 1;
-    const uint32_t my_drain = mw == 0 ? bar_drain : bar_drain_b;
-    const uint32_t idesc = tc::idesc_mxf4nvf4(128, P.N);
+    // Both walk every stage (both see every change of group) and issue the
+    // MMAs of the stages of their parity.
+    const int mw = warp - kMma0;
+    const uint32_t my_drain = bar_drain + 8 * mw;
+    const uint32_t idesc = tc::idesc_mxf4nvf4(128, P.Nh);
     const tc::SmemLayout sw = (P.DI == 128) ? tc::kSwizzle64B : tc::kSwizzle32B;
     const uint32_t sbo = 8u * row_bytes;  // 8 rows per swizzle atom
     TileIter<kRescore> ti;
     ti.init(P, wb, we);
     int64_t it = 0;
-    int cnt = 0;   // jobs issued by this warp
     uint32_t drain_n = 0, sfb_n = 0;
-    int cur_b = -1, W = 0, tok0 = 0;
-    // No early exit from this loop: both issuers must meet at the same named
-    // barriers, so after a failed wait a warp keeps walking the tiles without
-    // issuing anything (every later wait returns at once once *abort is set).
+    int cur_g = -1, W = 0;
+    // No early exit from this loop: both issuers meet at the same named
+    // barriers; after a failed wait a warp keeps walking without issuing.
     for (; ti.valid(); ti.next(P), ++it) {
-      if (ti.b != cur_b) {
-        if (cur_b >= 0) {  // every MMA reading the old queries must finish first
+      if (ti.b != cur_g) {
+        if (cur_g >= 0) {  // every MMA reading the old queries must finish first
           if (lane == 0) tc::commit(my_drain);
           __syncwarp();
           warp_wait_or_abort(my_drain, drain_n & 1, P, abort);
           ++drain_n;
         }
         tc::named_sync(5, 64);  // both issuers drained
-        cur_b = ti.b;
-        int bseq;
-        group_info<kRescore>(P, cur_b, &tok0, &W, &bseq);
-        if (W > kMaxW) {
-          if (lane == 0 && mw == 0) set_status(P.status, CSA2_ERR_RANGE);
-          W = kMaxW;
-        }
+        cur_g = ti.b;
+        int tok0, b, sel0;
+        group_info<kRescore>(P, cur_g, &tok0, &W, &b, &sel0);
         if (mw == 0 && !*abort) {
-          // query rows of this group: selector * T + token (scan: the sequence's tokens)
-          const int64_t qrow0 = kRescore ? (int64_t)(cur_b / P.qb.n_tok) * P.qb.n_tok + tok0 : tok0;
-          int64_t* pos_s = reinterpret_cast<int64_t*>(smem + kOffPos);
-          if (lane < W) pos_s[lane] = __ldg(P.qb.tok_pos + tok0 + lane);
+          // query rows of this group's columns: scan, its tokens; rescore,
+          // selector (sel0 + j) of its token
+          auto qrow = [&](int j) -> int64_t {
+            return kRescore ? (int64_t)(sel0 + j) * P.qb.n_tok + tok0 : (int64_t)(tok0 + j);
+          };
           // B operand: query codes, swizzled like the TMA-written A tiles
           const int chunks_per_row = row_bytes / 16;
           for (int e = lane; e < W * 64 * chunks_per_row; e += 32) {
@@ -401,8 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int n = (e / chunks_per_row) % 64;
             const int ch = e % chunks_per_row;
             uint4 v = make_uint4(0, 0, 0, 0);
-            if (n < P.H)
-              v = __ldg(reinterpret_cast<const uint4*>(P.q_codes + ((int64_t)(qrow0 + j) * P.H + n) * row_bytes) + ch);
+            if (n < P.H) v = __ldg(reinterpret_cast<const uint4*>(P.q_codes + (qrow(j) * P.H + n) * row_bytes) + ch);
             const int sch = (P.DI == 128) ? (ch ^ ((n >> 1) & 3)) : (ch ^ ((n >> 2) & 1));
             *reinterpret_cast<uint4*>(smem + kOffB + j * 4096 + n * row_bytes + sch * 16) = v;
           }
@@ -415,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int n = m1 * 32 + m0;
               uint32_t a = 0, b2 = 0;
               if (n < P.H) {
-                const uint8_t* sp = P.q_scales + ((int64_t)(qrow0 + j) * P.H + n) * spr + 2 * ks;
+                const uint8_t* sp = P.q_scales + (qrow(j) * P.H + n) * spr + 2 * ks;
                 a = __ldg(sp);
                 b2 = __ldg(sp + 1);
               }
@@ -426,7 +390,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc::fence_proxy_async_smem();
           __syncwarp();
-          bool ok = true;
           if (lane == 0) {
             tc::fence_after_sync();
             for (int j = 0; j < W; ++j)
@@ -434,48 +397,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::cp_32x128b_warpx4(tmem + kColSfb + j * 8 + ks * 4,
                                       tc::smem_desc(sbase + kOffSfb + (j * 2 + ks) * 512, 16, 128, tc::kSwizzleNone));
             tc::commit(bar_sfb);
-            ok = wait_or_abort(bar_sfb, sfb_n & 1, P, abort);  // the copies landed before anyone issues
+            wait_or_abort(bar_sfb, sfb_n & 1, P, abort);  // the copies landed before anyone issues
           }
           ++sfb_n;
-          (void)ok;
         }
-        tc::named_sync(6, 64);  // new queries and positions in place
+        tc::named_sync(6, 64);  // new queries in place
         tc::fence_after_sync();
       }
-      if ((int)(it & 1) != mw || *abort) continue;  // the other issuer's tile (or nothing left to do)
+      if ((int)(it & 1) != mw || *abort) continue;  // the other issuer's stage (or nothing left to do)
       const int s = (int)(it % kStages);
       const uint32_t n = (uint32_t)(it / kStages);
-      bool okw = true;
+      const int slot = (int)(it % P.n_slots);
+      const uint32_t u = (uint32_t)(it / P.n_slots);  // use of the slot
+      // this warp's earlier waits on its barrier of the slot: every use
+      // (even slot count: the slot's stages all have this warp's parity) or
+      // every other use (odd count: the parity of the slot's stages alternates)
+      const uint32_t ph = (P.n_slots & 1) ? (u - 1) >> 1 : u - 1;
       if (lane == 0) {
-        okw = wait_or_abort(bar_sfr + 8 * s, n & 1, P, abort);  // tile landed, scale factors in TMEM
-        tc::fence_after_sync();
-        const uint32_t sfa = tmem + kColSfa + (uint32_t)s * 8;
-        const int64_t* pos_s = reinterpret_cast<const int64_t*>(smem + kOffPos);
-        const int64_t t0 = (int64_t)ti.tile * kTile;
-        for (int j = 0; j < W && okw; ++j) {
-          if (!kRescore && t0 > pos_s[j]) continue;
-          const int u = mw * kUnitsPer + cnt % kUnitsPer;
-          const uint32_t m = (uint32_t)(cnt / kUnitsPer);
-          if (!wait_or_abort(bar_acce + 8 * u, (m & 1) ^ 1, P, abort)) {
-            okw = false;
-            break;
-          }
+        bool ok = wait_or_abort(bar_full + 8 * s, n & 1, P, abort);      // codes landed
+        if (ok) ok = wait_or_abort(bar_sf + 8 * s, n & 1, P, abort);     // scale factors in TMEM
+        if (ok && u > 0) ok = wait_or_abort(bar_acce + 8 * (slot * 2 + mw), ph & 1, P, abort);  // slot read
+        if (ok) {
           tc::fence_after_sync();
-          for (int ks = 0; ks < ksteps; ++ks) {
-            const uint64_t ad = tc::smem_desc(sbase + kOffA + s * 8192 + ks * 32, 16, sbo, sw);
-            const uint64_t bd = tc::smem_desc(sbase + kOffB + j * 4096 + ks * 32, 16, sbo, sw);
-            tc::mma_mxf4nvf4(tmem + kColAcc + u * 64, ad, bd, idesc, sfa + ks * 4, tmem + kColSfb + j * 8 + ks * 4,
-                             ks > 0 ? 1u : 0u);
-          }
-          tc::commit(bar_accf + 8 * u);
-          ++cnt;
+          const uint32_t sfa = tmem + kColSfa + (uint32_t)s * 8;
+          const uint32_t acc = tmem + kColAcc + (uint32_t)(slot * P.slot_cols);
+          for (int j = 0; j < W; ++j)
+            for (int ks = 0; ks < ksteps; ++ks) {
+              const uint64_t ad = tc::smem_desc(sbase + kOffA + s * kCodeStage + ks * 32, 16, sbo, sw);
+              const uint64_t bd = tc::smem_desc(sbase + kOffB + j * 4096 + ks * 32, 16, sbo, sw);
+              tc::mma_mxf4nvf4(acc + j * P.Nh, ad, bd, idesc, sfa + ks * 4, tmem + kColSfb + j * 8 + ks * 4,
+                               ks > 0 ? 1u : 0u);
+            }
+          // one commit: the stage's shared memory and scale factors are free
+          // and the slot holds the scores once these MMAs complete
+          tc::commit(bar_done + 8 * s);
         }
-        // the stage goes back to the producer as soon as the MMAs that read
-        // it complete
-        if (okw) tc::commit(bar_empty + 8 * s);
       }
-      cnt = __shfl_sync(0xffffffffu, cnt, 0);
-      (void)okw;
+      __syncwarp();
     }
     // drain: no MMA or copy of ours in flight at teardown
     if (lane == 0) {
@@ -483,151 +441,115 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait_bounded(my_drain, drain_n & 1, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
     }
     __syncwarp();
-  } else if (warp == kSfWarp || warp == kSfWarp + 1) {
+  } else if (warp < kEpi0) {
     // ------------------------------------------------------------ scale factors
-    // raw [row][spr] -> [m0 (32)][m1 (4)][k (4)] per 64-element K step, each
-    // per-32 scale written twice (the MMA takes one scale per 16 elements);
-    // two tiles per pass, so the fixed costs of a pass (proxy fence, copy
-    // issue) are shared
+    // raw per-32 scales of the stage's rows -> the block-scale layout the
+    // MMA reads (K step ks: per-16 scales (s_2ks, s_2ks, s_2ks+1, s_2ks+1);
+    // lane m0 of every lane quarter holds rows m1*32 + m0 in column m1),
+    // written by this warp into its own lane quarter
+    const int q = warp & 3;
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     TileIter<kRescore> ti;
     ti.init(P, wb, we);
     int64_t it = 0;
-    constexpr int kBoxRows = kRescore ? kBlock : kChunk;
-    constexpr uint32_t kSlot = kRescore ? kRawStage / 16 : kRawStage / 2;
-    const int sfw = warp - kSfWarp;
-    int64_t pass = 0;
-    while (ti.valid()) {
-      const int nt = ti.left >= 2 ? 2 : 1;
-      if ((int)(pass++ & 1) != sfw) {  // the other scale-factor warp's pass
-        for (int k = 0; k < nt; ++k) ti.next(P);
-        it += nt;
-        continue;
-      }
-      uint32_t wv[2][4];
-      bool ok = true;
+    const int box_rows = kRescore ? kBlock : P.box_rows;
+    const int slot_bytes = kRescore ? 128 : box_rows * spr;
+    for (; ti.valid(); ti.next(P), ++it) {
+      const int s = (int)(it % kStages);
+      const uint32_t n = (uint32_t)(it / kStages);
+      if (!warp_wait_or_abort(bar_full + 8 * s, n & 1, P, abort)) break;
+      const uint8_t* raw = smem + kOffRaw + s * kRawStage;
+      uint32_t r[8];
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        if (k >= nt) break;
-        const int s = (int)((it + k) % kStages);
-        const uint32_t n = (uint32_t)((it + k) / kStages);
-        if (!warp_wait_or_abort(bar_full + 8 * s, n & 1, P, abort)) {
-          ok = false;
-          break;
-        }
-        const uint8_t* raw = smem + kOffRaw + s * kRawStage;
-#pragma unroll
-        for (int m1 = 0; m1 < 4; ++m1) {
-          const int r = m1 * 32 + lane;
-          const uint8_t* src = raw + (r / kBoxRows) * kSlot + (r % kBoxRows) * spr;
-          wv[k][m1] =
-              (spr == 4) ? *reinterpret_cast<const uint32_t*>(src) : (uint32_t)*reinterpret_cast<const uint16_t*>(src);
-        }
+      for (int m1 = 0; m1 < 4; ++m1) {
+        const int rw = m1 * 32 + lane;
+        const uint8_t* src = raw + (rw / box_rows) * slot_bytes + (rw % box_rows) * spr;
+        const uint32_t wv =
+            (spr == 4) ? *reinterpret_cast<const uint32_t*>(src) : (uint32_t)*reinterpret_cast<const uint16_t*>(src);
+        r[m1] = __byte_perm(wv, 0, 0x1100u);      // K step 0: scales 0, 1
+        r[4 + m1] = __byte_perm(wv, 0, 0x3322u);  // K step 1: scales 2, 3
       }
-      if (!ok) break;
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        if (k >= nt) break;
-        const int s = (int)((it + k) % kStages);
-        for (int ks = 0; ks < ksteps; ++ks) {
-          const uint32_t sel = ks == 0 ? 0x1100u : 0x3322u;
-          *reinterpret_cast<uint4*>(smem + kOffSfa + (s * 2 + ks) * 512 + lane * 16) =
-              make_uint4(__byte_perm(wv[k][0], 0, sel), __byte_perm(wv[k][1], 0, sel),
-                         __byte_perm(wv[k][2], 0, sel), __byte_perm(wv[k][3], 0, sel));
-        }
+      const uint32_t ta = tmem + lane_base + kColSfa + (uint32_t)s * 8;
+      if (ksteps == 2) {
+        tc::st_32x32b_x8(ta, r);
+      } else {
+        const uint32_t r4[4] = {r[0], r[1], r[2], r[3]};
+        tc::st_32x32b_x4(ta, r4);
       }
-      tc::fence_proxy_async_smem();
+      tc::st_wait();
+      tc::fence_before_sync();
       __syncwarp();
-      // copy to TMEM from this warp (tcgen05 instructions cost their issuing
-      // thread 100-200 cycles each, so they are spread over the warps that
-      // have time); the commit hands the stage over once the copy landed
-      if (lane == 0) {
-        tc::fence_after_sync();
-        for (int k = 0; k < nt; ++k) {
-          const int s = (int)((it + k) % kStages);
-          for (int ks = 0; ks < ksteps; ++ks)
-            tc::cp_32x128b_warpx4(tmem + kColSfa + s * 8 + ks * 4,
-                                  tc::smem_desc(sbase + kOffSfa + (s * 2 + ks) * 512, 16, 128, tc::kSwizzleNone));
-          tc::commit(bar_sfr + 8 * s);
-        }
-      }
-      __syncwarp();
-      for (int k = 0; k < nt; ++k) ti.next(P);
-      it += nt;
+      if (lane == 0) tc::mbar_arrive(bar_sf + 8 * s);
     }
-    // drain: our copies must have landed before teardown
-    if (lane == 0) {
-      const uint32_t dr = sfw == 0 ? bar_drain2 : bar_drain_c;
-      tc::commit(dr);
-      if (!mbar_wait_bounded(dr, 0, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
-    }
-    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int wg = (warp - 2) / 4;        // warpgroup: warps 2+4wg .. 5+4wg
-    const int mw = wg & 1, sub = wg >> 1; // its MMA issuer and job parity
-    const int quarter = warp & 3;         // TMEM lane quarter this warp may access
+    const int wg = (warp - kEpi0) / 4;   // warpgroup: the stages it with it % kEpiWG == wg
+    const int quarter = warp & 3;        // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
-    const int ept = threadIdx.x - 64 - wg * 128;  // 0..127 within the warpgroup
-    float* w_g = w_s + wg * kMaxW * 64;
-    int64_t* pos_g = reinterpret_cast<int64_t*>(smem + kOffPos) + (1 + wg) * kMaxW;
+    const int ept = threadIdx.x - kEpi0 * 32 - wg * 128;  // 0..127 within the warpgroup
+    float* w_g = reinterpret_cast<float*>(smem + kOffW) + wg * kMaxWc * 64;
+    int64_t* pos_g = reinterpret_cast<int64_t*>(smem + kOffPos) + wg * kMaxWc;
     TileIter<kRescore> ti;
     ti.init(P, wb, we);
     int64_t it = 0;
-    int cnt = 0;  // jobs of this warpgroup's issuer (all parities)
-    int cur_b = -1, W = 0, tok0 = 0;
+    int cur_g = -1, W = 0, tok0 = 0, sel0 = 0;
     bool dead = false;  // warpgroup-uniform: a wait of this warpgroup gave up
+    const int ng = P.Nh / 16;
     // no early exit: the four warps of the warpgroup meet at named barriers
     for (; ti.valid(); ti.next(P), ++it) {
-      if (ti.b != cur_b) {
+      if (ti.b != cur_g) {
         tc::named_sync(1 + wg, 128);
-        cur_b = ti.b;
+        cur_g = ti.b;
         int bseq;
-        group_info<kRescore>(P, cur_b, &tok0, &W, &bseq);
-        W = min(W, kMaxW);
+        group_info<kRescore>(P, cur_g, &tok0, &W, &bseq, &sel0);
         for (int e = ept; e < W * 64; e += 128) {
           const int j = e / 64, h = e % 64;
-          w_g[e] = h < P.H ? __ldg(P.w[kRescore ? cur_b / P.qb.n_tok : 0] + (int64_t)(tok0 + j) * P.H + h) : 0.0f;
+          w_g[e] = h < P.H ? __ldg(P.w[kRescore ? sel0 + j : 0] + (int64_t)(kRescore ? tok0 : tok0 + j) * P.H + h)
+                           : 0.0f;
         }
-        if (ept < W) pos_g[ept] = __ldg(P.qb.tok_pos + tok0 + ept);
+        if (ept < W) pos_g[ept] = __ldg(P.qb.tok_pos + (kRescore ? tok0 : tok0 + ept));
         tc::named_sync(1 + wg, 128);
       }
-      if ((int)(it & 1) != mw || dead) continue;  // the other issuer's tile (or nothing left to do)
-      const int64_t t0 = (int64_t)ti.tile * kTile;
-      for (int j = 0; j < W; ++j) {
-        const int tok = tok0 + j;
-        const int64_t p = pos_g[j];
-        if (!kRescore && t0 > p) continue;
-        const int job = cnt++;
-        if ((job & 1) != sub) continue;  // the other warpgroup of this issuer
-        const int u = mw * kUnitsPer + job % kUnitsPer;
-        const uint32_t m = (uint32_t)(job / kUnitsPer);
-        // one prober per warpgroup; the other warps park on the named barrier
-        if (!mbar_wait_group(bar_accf + 8 * u, m & 1, P.wait_ns, ept == 0, *abort != 0, 1 + wg, 128)) {
-          if (ept == 0 && !*abort) {
-            set_status(P.status, CSA2_ERR_TIMEOUT);
-            *abort = 1;
-          }
-          dead = true;
-          break;
+      if ((int)(it % kEpiWG) != wg || dead) continue;  // another warpgroup's stage (or nothing left to do)
+      const int s = (int)(it % kStages);
+      const uint32_t n = (uint32_t)(it / kStages);
+      const int slot = (int)(it % P.n_slots);
+      // one prober per warpgroup; the other warps park on the named barrier
+      if (!mbar_wait_group(bar_done + 8 * s, n & 1, P.wait_ns, ept == 0, *abort != 0, 1 + wg, 128)) {
+        if (ept == 0 && !*abort) {
+          set_status(P.status, CSA2_ERR_TIMEOUT);
+          *abort = 1;
         }
-        tc::fence_after_sync();
+        dead = true;
+        continue;
+      }
+      tc::fence_after_sync();
+      const int64_t t0 = (int64_t)ti.tile * kTile;
+      const uint32_t taddr0 = tmem + ((uint32_t)(quarter * 32) << 16) + kColAcc + (uint32_t)(slot * P.slot_cols);
+      int32_t blk = -1;  // rescore: this thread's pool block
+      if (kRescore) {
+        const int i = ti.tile * kTile + row;
+        const int np = min(__ldg(P.pool_n + tok0), P.pool_cap);
+        blk = (i / kBlock) < np ? __ldg(P.pool + (int64_t)tok0 * P.pool_cap + i / kBlock) : -1;
+      }
+      for (int j = 0; j < W; ++j) {
         const float* wj = w_g + j * 64;
-        const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + kColAcc + u * 64;
-        const int ng = P.N / 16;
-        // two halves of 32 columns (register budget); four independent chains,
-        // weights read as float4 (broadcast)
-        float a4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        const uint32_t taddr = taddr0 + j * P.Nh;
+        // the column's scores in two halves of 32 heads (register budget):
+        // ReLU and weighted sum in packed pairs (two float2 chains)
+        float2 a2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
+          if (hf * 2 >= ng) break;
           uint32_t r[2][16];
 #pragma unroll
           for (int g = 0; g < 2; ++g)
             if (hf * 2 + g < ng) tc::ld_32x32b_x16(taddr + (hf * 2 + g) * 16, r[g]);
           tc::ld_wait();
-          if (hf == 1) {  // the accumulator is free once the last load has landed
-            tc::fence_before_sync();
+          if (j == W - 1 && (hf == 1 || ng <= 2)) {  // the slot is free once its last load has landed:
+            tc::fence_before_sync();                 // for the warp issuing its next use
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(bar_acce + 8 * u);
+            if (lane == 0) tc::mbar_arrive(bar_acce + 8 * (slot * 2 + (int)((it + P.n_slots) & 1)));
           }
 #pragma unroll
           for (int g = 0; g < 2; ++g)
@@ -635,21 +557,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int k4 = 0; k4 < 4; ++k4) {
                 const float4 w4 = *reinterpret_cast<const float4*>(wj + (hf * 2 + g) * 16 + k4 * 4);
-                a4[0] = fmaf(w4.x, fmaxf(__uint_as_float(r[g][k4 * 4 + 0]), 0.0f), a4[0]);
-                a4[1] = fmaf(w4.y, fmaxf(__uint_as_float(r[g][k4 * 4 + 1]), 0.0f), a4[1]);
-                a4[2] = fmaf(w4.z, fmaxf(__uint_as_float(r[g][k4 * 4 + 2]), 0.0f), a4[2]);
-                a4[3] = fmaf(w4.w, fmaxf(__uint_as_float(r[g][k4 * 4 + 3]), 0.0f), a4[3]);
+                const float2 x0 = make_float2(fmaxf(__uint_as_float(r[g][k4 * 4 + 0]), 0.0f),
+                                              fmaxf(__uint_as_float(r[g][k4 * 4 + 1]), 0.0f));
+                const float2 x1 = make_float2(fmaxf(__uint_as_float(r[g][k4 * 4 + 2]), 0.0f),
+                                              fmaxf(__uint_as_float(r[g][k4 * 4 + 3]), 0.0f));
+                a2[0] = __ffma2_rn(make_float2(w4.x, w4.y), x0, a2[0]);
+                a2[1] = __ffma2_rn(make_float2(w4.z, w4.w), x1, a2[1]);
               }
             }
         }
-        const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+        const float acc = (a2[0].x + a2[1].x) + (a2[0].y + a2[1].y);
+        const int64_t p = pos_g[kRescore ? 0 : j];
         if (kRescore) {
           // pool entry i = tile*128 + row: position pool[i/8]*8 + i%8
           const int i = ti.tile * kTile + row;
-          const int np = min(__ldg(P.pool_n + tok), P.pool_cap);
-          const int32_t blk = (i / kBlock) < np ? __ldg(P.pool + (int64_t)tok * P.pool_cap + i / kBlock) : -1;
           const int64_t pos = (int64_t)blk * kBlock + (i % kBlock);
-          const int64_t orow = (int64_t)(cur_b / P.qb.n_tok) * P.qb.n_tok + tok;  // selector * T + token
+          const int64_t orow = (int64_t)(sel0 + j) * P.qb.n_tok + tok0;  // selector * T + token
           if (i < P.pool_cap * kBlock) P.out[orow * P.ld + i] = (blk >= 0 && pos <= p) ? acc : -INFINITY;
         } else {
           const int64_t t = t0 + row;
@@ -657,7 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 1));
           sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 2));
           sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 4));
-          if ((lane & 7) == 0 && t <= p) P.out[(int64_t)tok * P.ld + t / kBlock] = sc;
+          if ((lane & 7) == 0 && t <= p) P.out[(int64_t)(tok0 + j) * P.ld + t / kBlock] = sc;
         }
       }
     }
@@ -669,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     while (globaltimer_ns() - t0 < 200000ull) __nanosleep(1000);
   }
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMma0) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, kTmemCols);
   }
@@ -706,15 +629,18 @@ int make_codes_map(CUtensorMap* m, const uint8_t* codes, int64_t n_rows, int row
   return CSA2_OK;
 }
 
-// scales: 1-D byte array [n_rows * spr], box of box_rows rows
+// scales: the [n_rows][spr] byte array seen as rows of 16 bytes (n_rows * spr
+// a multiple of 16), box of box_rows * spr / 16 such rows (the scales of
+// box_rows cache rows)
 int make_scales_map(CUtensorMap* m, const uint8_t* scales, int64_t n_rows, int spr, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return fail(CSA2_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-  cuuint64_t dims[1] = {(cuuint64_t)(n_rows * spr)};
-  cuuint64_t strides[1] = {0};
-  cuuint32_t box[1] = {(cuuint32_t)(box_rows * spr)};
-  cuuint32_t es[1] = {1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, const_cast<uint8_t*>(scales), dims, strides, box, es,
+  if ((n_rows * spr) % 16) return fail(CSA2_ERR_UNSUPPORTED, "indexer cache rows * d_I/32 must be a multiple of 16");
+  cuuint64_t dims[2] = {16, (cuuint64_t)(n_rows * spr / 16)};
+  cuuint64_t strides[1] = {16};
+  cuuint32_t box[2] = {16, (cuuint32_t)(box_rows * spr / 16)};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(scales), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(CSA2_ERR_CUDA, "cuTensorMapEncodeTiled(scales) failed: %d", (int)r);
@@ -739,8 +665,10 @@ static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const 
                            int n_sel, int H, const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n,
                            int pool_cap, float* out, int64_t ld, cudaStream_t st) {
   using namespace scan_tc;
-  if (kc->n_rows * (kc->dim / 32) >= (int64_t(1) << 31)) return fail(CSA2_ERR_UNSUPPORTED, "cache too large for TMA");
-  const int box_rows = kRescore ? kBlock : kChunk;
+  if (kc->n_rows >= (int64_t(1) << 31)) return fail(CSA2_ERR_UNSUPPORTED, "cache too large for TMA");
+  if (n_sel < 1 || n_sel > kMaxSel) return fail(CSA2_ERR_UNSUPPORTED, "1..%d selector layers per launch", kMaxSel);
+  // scan boxes: 128 rows, or 64 when pages of 64 (or an odd multiple of 64) rows would be crossed
+  const int box_rows = kRescore ? kBlock : (kc->page_table && kc->page_size % 128 != 0 ? 64 : 128);
   CUtensorMap tmc, tms;
   if (int rc = make_codes_map(&tmc, kc->codes, kc->n_rows, kc->dim / 2, box_rows)) return rc;
   if (int rc = make_scales_map(&tms, kc->scales, kc->n_rows, kc->dim / 32, box_rows)) return rc;
@@ -748,13 +676,22 @@ static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const 
   p.qb = *qb;
   p.q_codes = qc;
   p.q_scales = qs;
-  if (n_sel < 1 || n_sel > kMaxSel) return fail(CSA2_ERR_UNSUPPORTED, "1..%d selector layers per launch", kMaxSel);
   for (int i = 0; i < n_sel; ++i) p.w[i] = w[i];
   p.n_sel = n_sel;
-  p.qchunks = kRescore ? 1 : std::max(1, (qb->max_q_per_seq + kMaxW - 1) / kMaxW);
+  // query columns per group and groups per sequence (scan) or token (rescore)
+  const int cols = kRescore ? n_sel : std::max(1, qb->max_q_per_seq);
+  const int wc = std::min(cols, kMaxWc);
+  p.cpg = (cols + kMaxWc - 1) / kMaxWc;
   p.H = H;
-  p.N = (H + 15) / 16 * 16;
+  p.Nh = (H + 15) / 16 * 16;
   p.DI = kc->dim;
+  p.slot_cols = wc * p.Nh;
+  // accumulator slots: as many as fit, a divisor of the stage count (so that a
+  // stage's commit barrier cannot run two phases ahead of a slot's reader)
+  int ns = std::min<int>(6, (int)(kAccCols / p.slot_cols));
+  while (ns > 1 && kStages % ns) --ns;
+  p.n_slots = ns;
+  p.box_rows = box_rows;
   p.n_rows = kc->n_rows;
   p.page_size = kc->page_size;
   p.max_pages = kc->max_pages;
@@ -772,20 +709,19 @@ static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const 
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
     if (int rc = cuda_check(
-            cudaFuncSetAttribute(k_index_tc<kRescore>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Ly<kRescore>::kSmemBytes),
+            cudaFuncSetAttribute(k_index_tc<kRescore>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes),
             "index smem attribute"))
       return rc;
     int fit = 0;  // one CTA of kThreads threads at this register count must fit on an SM
     if (int rc = cuda_check(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, k_index_tc<kRescore>, kThreads,
-                                                                          Ly<kRescore>::kSmemBytes),
+                                                                          kSmemBytes),
                             "index occupancy"))
       return rc;
     if (fit < 1) return fail(CSA2_ERR_UNSUPPORTED, "index kernel does not fit on an SM");
     attr_done[dev] = true;
   }
   Launch L_(kRescore ? "rescore_tc" : "scan_tc", st);
-  k_index_tc<kRescore><<<num_sms(), kThreads, Ly<kRescore>::kSmemBytes, st>>>(tmc, tms, p);
+  k_index_tc<kRescore><<<num_sms(), kThreads, kSmemBytes, st>>>(tmc, tms, p);
   return cuda_check(cudaGetLastError(), "k_index_tc");
 }
 
@@ -795,7 +731,7 @@ int launch_scan_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t*
 }
 
 // n_sel selector layers at once: queries [n_sel][T][H][...], weights w[sel],
-// scores [n_sel][T][8P]
+// scores [n_sel][T][8P]; a token's pool is gathered once for up to four of them
 int launch_rescore_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* const* w,
                       int n_sel, int H, const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n, int P,
                       float* scores, cudaStream_t st) {

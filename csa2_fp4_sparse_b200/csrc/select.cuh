@@ -53,7 +53,7 @@ struct SelParams {
   const float* score;  // [n_sel][T][ld]
   int64_t ld;
   int mode;
-  const int32_t* pool;    // [T][P] (mode 1)
+  const int32_t* pool;    // [T][P] (mode 1), candidate ids [T][P] (mode 2)
   const int32_t* pool_n;  // [T]
   int P;
   int k_out;
@@ -64,8 +64,11 @@ struct SelParams {
   uint64_t wait_ns;
 };
 
-// candidate i -> output id
+// candidate i -> output id: mode 0 the candidate itself (a block), mode 1 the
+// position of pool entry i, mode 2 the id listed for candidate i (merging
+// candidate lists gathered from several ranks)
 __device__ __forceinline__ int32_t sel_id(int mode, int i, const int32_t* pool_row) {
+  if (mode == 2) return __ldg(pool_row + i);
   return mode == 0 ? i : __ldg(pool_row + i / kBlock) * kBlock + (i % kBlock);
 }
 
@@ -126,7 +129,9 @@ __global__ void __launch_bounds__(kSelThreads) k_select(const __grid_constant__ 
   const int64_t g = (int64_t)blockIdx.z * T + tok;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int64_t p = __ldg(P.qb.tok_pos + tok);
-  const int n = P.mode == 0 ? (int)((p + kBlock) / kBlock) : min(__ldg(P.pool_n + tok), P.P) * kBlock;
+  const int n = P.mode == 0   ? (int)((p + kBlock) / kBlock)
+                : P.mode == 1 ? min(__ldg(P.pool_n + tok), P.P) * kBlock
+                              : P.P;  // mode 2: P candidates a token
   const float* sc = P.score + g * P.ld;
   const int32_t* pool_row = P.pool + (int64_t)tok * P.P;
   SelGroup* G = S > 1 ? P.grp + g : nullptr;

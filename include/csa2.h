@@ -164,7 +164,11 @@ int csa2_quantize_fp4(const float* x, int64_t n_rows, int32_t dim, const int64_t
  * q_codes [T][H_I][d_I/2], q_scales [T][H_I][d_I/32], w [T][H_I];
  * pool [T][P], pool_n [T], idx [T][K], idx_n [T]; blockscore: optional
  * [T][ceil(max_seq_len/8)] fp32 copy of B_j (entries past a token's last
- * visible block are unspecified).  d_I = k_idx->dim in {64, 128};
+ * visible block are unspecified).  d_I = k_idx->dim in {64, 128}; the
+ * indexer cache's scale array is read in rows of 16 bytes: n_rows * d_I / 32
+ * must be a multiple of 16 (else CSA2_ERR_UNSUPPORTED) and a row that holds a
+ * position must start a 16-byte row of it (row * d_I / 32 a multiple of 16;
+ * a misplaced row reads as zeros and CSA2_ERR_RANGE is recorded);
  * 1 <= H_I <= 64; 1 <= P <= 4096; 1 <= K <= 2048; K <= 8*P.  Any number of
  * query tokens per sequence: the scan reads the keys once for every 8 of a
  * sequence's tokens (a decode or verify step with W_b <= 8 reads them once). */
@@ -260,6 +264,63 @@ int csa2_profiler_enable(int on);
 /* Synchronises the recorded events, writes up to `cap` per-kernel totals since
  * the last read (or enable) into `out`, sets *n_out, and clears them. */
 int csa2_profiler_read(csa2_kernel_stat* out, int32_t cap, int32_t* n_out);
+
+/* ---- context parallelism: one sequence's positions over G GPUs ------------
+ * Rank r holds positions [lo_r, hi_r) of each sequence (ascending ranges, lo
+ * a multiple of 8) in its own caches and runs the calls above on its slice,
+ * with query positions given relative to lo_r (a query sees its whole slice
+ * when the slice ends before it, -1: nothing).  These calls combine the
+ * ranks' results after the caller's all-gathers (every rank passes the same
+ * gathered buffers, rank-major).  Exact: the global top-k of a set split into
+ * parts lies in the union of the parts' top-k (hierarchical indexer, dbyun.net
+ * article 10794, section "KV Cache 成为这一代架构改造的核心"), and one softmax
+ * over a split key set is the log-sum-exp merge of the parts.  All pointers
+ * are device pointers; every call is asynchronous on `stream`. */
+
+/* A rank's selected local ids ids[T][n] (-1: none) -> (score, global id):
+ * by_id != 0, score = scores[t][ld-strided row][id] (block scores), else
+ * scores[t][i]; global id = id + offset; out_score/out_id [T][n] (-inf / -1
+ * for none). */
+int csa2_cp_candidates(const float* scores, int64_t ld, const int32_t* ids, int32_t n_tok, int32_t n, int32_t by_id,
+                       int32_t offset, float* out_score, int32_t* out_id, void* stream);
+
+/* Gathered candidate lists score/ids [n_ranks][T][n] -> per token the k
+ * best by score (ties to the lower id), ascending, in out[T][k] (-1 padded),
+ * counts out_n[T].  n_ranks * n <= 16384. */
+int csa2_cp_merge(const float* score, const int32_t* ids, int32_t n_ranks, int32_t n_tok, int32_t n, int32_t k,
+                  int32_t* out, int32_t* out_n, void* stream);
+
+/* Global id lists ids[T][k] (ascending, n_in[t] valid) -> this rank's ids
+ * (id - lo for lo <= id < hi): compact != 0, its entries in order, -1 padded,
+ * counts out_n; compact == 0, entry i stays at i (-1 where not its own) and
+ * out_n = n_in. */
+int csa2_cp_localize(const int32_t* ids, const int32_t* n_in, int32_t n_tok, int32_t k, int64_t lo, int64_t hi,
+                     int32_t compact, int32_t* out, int32_t* out_n, void* stream);
+
+/* Pool-position scores of n_sel selector layers (queries [n_sel][T][H_I][..]
+ * FP4, weights w[i] [T][H_I], host array of n_sel device pointers) over
+ * `local_pool` [T][P] (the global pool made local and aligned with
+ * csa2_cp_localize(compact = 0): -1 where another rank owns the block):
+ * scores [n_sel][T][8P], -inf where not this rank's. */
+int csa2_cp_pool_scores(const csa2_query_batch* qb, const uint8_t* q_codes, const uint8_t* q_scales,
+                        const float* const* w, int32_t n_sel, int32_t H_I, const csa2_fp4_cache* k_idx,
+                        const int32_t* local_pool, const int32_t* pool_n, int32_t P, float* scores, void* stream);
+
+/* Gathered pool-position scores [n_ranks][n_sel][T][8P] -> per selector and
+ * token the best K positions of the global pool[T][P] (ties to the lower
+ * position), ascending, in idx[n_sel][T][K] (-1 padded), idx_n[n_sel][T].
+ * P <= 2048. */
+int csa2_cp_select_positions(const float* scores, int32_t n_ranks, int32_t n_sel, int32_t n_tok, const int32_t* pool,
+                             const int32_t* pool_n, int32_t P, int32_t K, int32_t* idx, int32_t* idx_n, void* stream);
+
+/* Gathered attention parts: rank g's part at o_parts + g * o_rank_stride,
+ * [T][Hq][D] fp32 (its csa2_attend_reuse output over its own selected rows),
+ * and lse_parts + g * lse_rank_stride, [T][Hq] (natural log, -inf for an
+ * empty part) -> out [T][Hq][D] in out_dtype and, optionally, lse [T][Hq]
+ * of the union (strides in elements). */
+int csa2_cp_attend_merge(const float* o_parts, const float* lse_parts, int32_t n_ranks, int64_t o_rank_stride,
+                         int64_t lse_rank_stride, int32_t n_tok, int32_t Hq, int32_t D, void* out, int32_t out_dtype,
+                         float* lse, void* stream);
 
 /* Tensor-core peak probe (a measurement hook, not part of the decode step):
  * every SM issues back-to-back dense M = 128, N = 256 MMAs from fixed

@@ -7,9 +7,8 @@ e2m1(code_t) * e4m3(scale_t) (ReLU of a non-negative value), so the planted
 key bytes fix every score exactly and the selections can be compared with the
 oracle's exhaustive top-k id for id: ties at the k-th score take the lowest
 ids.  The patterns cover a single CTA per group, groups split over several
-CTAs, heavy ties, all-equal scores and a pattern that defeats the sampled
-threshold (its high scores sit exactly where the sample looks), which the
-kernel must still select exactly."""
+CTAs, heavy ties, all-equal scores and a structured pattern (high scores on
+an evenly spaced grid of blocks)."""
 import ctypes
 
 import numpy as np
@@ -41,10 +40,11 @@ def _run(code, scale, P, K):
     C = _C()
     L = len(code)
     dI = 64
-    codes = np.zeros((L, dI // 2), np.uint8)
-    codes[:, 0] = np.asarray(code, np.uint8) & 7
-    scales = np.zeros((L, dI // 32), np.uint8)
-    scales[:, 0] = np.asarray(scale, np.uint8)
+    rows = (L + 7) // 8 * 8  # the indexer cache holds a multiple of 8 rows at d_I = 64
+    codes = np.zeros((rows, dI // 2), np.uint8)
+    codes[:L, 0] = np.asarray(code, np.uint8) & 7
+    scales = np.zeros((rows, dI // 32), np.uint8)
+    scales[:L, 0] = np.asarray(scale, np.uint8)
     val = np.array([E2M1[c & 7] for c in code], np.float64) * np.array([oracle.e4m3_value(int(s)) for s in scale])
     dev = "cuda"
     kc_t = torch.from_numpy(codes).to(dev)
@@ -56,7 +56,7 @@ def _run(code, scale, P, K):
     seq_base = torch.tensor([0], dtype=torch.int64, device=dev)
     qb = C.csa2_query_batch(1, 1, L, 1, seq_len.data_ptr(), tok_start.data_ptr(), tok_seq.data_ptr(),
                             tok_pos.data_ptr())
-    kc = C.csa2_fp4_cache(kc_t.data_ptr(), ks_t.data_ptr(), L, dI, 0, None, 0, seq_base.data_ptr())
+    kc = C.csa2_fp4_cache(kc_t.data_ptr(), ks_t.data_ptr(), rows, dI, 0, None, 0, seq_base.data_ptr())
     qcodes = torch.zeros(1, dI // 2, dtype=torch.uint8, device=dev)
     qcodes[0, 0] = 0x2  # element 0 = 1.0
     qscales = torch.zeros(1, dI // 32, dtype=torch.uint8, device=dev)
@@ -124,10 +124,9 @@ def test_all_scores_equal(nb):
     _check(np.full(L, 2), np.full(L, 0x38))
 
 
-def test_sample_defeating_pattern():
-    """high scores exactly at the blocks the evenly spaced sample reads: the
-    sampled threshold sits above the true k-th score, and the kernel falls
-    back to selecting from every key"""
+def test_evenly_spaced_high_blocks():
+    """4096 high blocks on an evenly spaced grid over 40000 (more than P), in
+    eight score levels, over a flat background"""
     nb, ns = 40000, 4096
     L = nb * 8
     code = np.full(L, 1)
