@@ -131,16 +131,41 @@ struct Carve {
 
 static int n_blocks_max(const csa2_query_batch* qb) { return (qb->max_seq_len + kBlock - 1) / kBlock; }
 
-// split-selection scratch: one record per (selector, token) group of a split
-// launch (a launch splits only while it has fewer groups than SMs)
-static size_t select_ws(const csa2_query_batch*, int, int) { return (size_t)kSelMaxGroups * sizeof(SelGroup); }
+// Key counts that seed the selections: kHistBins counts per group, filled by
+// the scoring kernels, zeroed by one memset per call and left zeroed by every
+// selection; the block selection's T groups, then the position selection's
+// n_sel * T groups.
+struct SelPlan {
+  uint32_t* blk = nullptr;
+  uint32_t* pos = nullptr;
+  size_t bytes = 0;
+};
+static SelPlan take_select_scratch(Carve& c, const csa2_query_batch* qb, int, int n_sel) {
+  SelPlan s;
+  const int64_t gb = qb->n_tok, gp = (int64_t)qb->n_tok * n_sel;
+  s.bytes = (size_t)(gb + gp) * kHistBins * 4;
+  auto* z = static_cast<uint32_t*>(c.take(s.bytes));
+  if (z) {
+    s.blk = z;
+    s.pos = z + gb * kHistBins;
+  }
+  return s;
+}
+static size_t select_ws(const csa2_query_batch* qb, int P, int n_sel) {
+  Carve c{nullptr, 0};
+  take_select_scratch(c, qb, P, n_sel);
+  return c.used + 256;
+}
+static int clear_select_counts(const SelPlan& s, cudaStream_t st) {
+  return cuda_check(cudaMemsetAsync(s.blk, 0, s.bytes, st), "clear selection counts");
+}
 
 // block scores, pool position scores, selection scratch
 static size_t index_ws(const csa2_query_batch* qb, int P) {
   Carve c{nullptr, 0};
   c.take((size_t)qb->n_tok * n_blocks_max(qb) * 4);  // block scores
   c.take((size_t)qb->n_tok * P * kBlock * 4);        // pool position scores
-  c.take(select_ws(qb, P, 1));                       // split-selection scratch
+  c.take(select_ws(qb, P, 1));                       // selection scratch
   return c.used + 256;
 }
 
@@ -188,59 +213,123 @@ int launch_quantize(const float* x, int64_t n_rows, int dim, const int64_t* slot
 }
 
 static int launch_scan(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
-                         const csa2_fp4_cache* kc, float* bs, int64_t ld, cudaStream_t st) {
-  return launch_scan_tc(qb, qc, qs, w, H, kc, bs, ld, st);
+                       const csa2_fp4_cache* kc, float* bs, int64_t ld, uint32_t* hist, cudaStream_t st) {
+  return launch_scan_tc(qb, qc, qs, w, H, kc, bs, ld, hist, st);
 }
 
 // n_sel selector layers (queries [n_sel][T][H][...], weights w[i], scores
-// [n_sel][T][8P]), up to kMaxSel in one launch
+// [n_sel][T][8P]), up to kMaxSel in one launch; hist: the groups' key counts
+// for the selection that follows (NULL: none)
 static int launch_rescore_multi(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs,
                                 const float* const* w, int n_sel, int H, const csa2_fp4_cache* kc,
-                                const int32_t* pool, const int32_t* pool_n, int P, float* scores, cudaStream_t st) {
-  return launch_rescore_tc(qb, qc, qs, w, n_sel, H, kc, pool, pool_n, P, scores, st);
+                                const int32_t* pool, const int32_t* pool_n, int P, float* scores, uint32_t* hist,
+                                cudaStream_t st) {
+  return launch_rescore_tc(qb, qc, qs, w, n_sel, H, kc, pool, pool_n, P, scores, hist, st);
 }
 
 int launch_rescore(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
                    const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n, int P, float* scores,
                    cudaStream_t st) {
-  return launch_rescore_multi(qb, qc, qs, &w, 1, H, kc, pool, pool_n, P, scores, st);
+  return launch_rescore_multi(qb, qc, qs, &w, 1, H, kc, pool, pool_n, P, scores, nullptr, st);
 }
 
-// CTAs per (selector, token) group: with fewer groups than SMs, long
-// candidate lists are split (about 8192 candidates a CTA) so that the whole
-// grid still fits on the GPU at one CTA per SM (the launch is cooperative)
-static int select_splits(int64_t groups, int n_max) {
-  static int sms = 0;
-  if (!sms) {
-    int dev = 0, v = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess &&
-        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
-      sms = std::min(v, kSelMaxGroups);
-    else
-      sms = 1;
+// SMs of the current device
+static int num_sms_dev() {
+  static int n[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!n[dev]) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    n[dev] = v > 0 ? v : 148;
   }
-  if (groups >= sms) return 1;
-  // about 8192 candidates per CTA: a selection round costs a CTA the same few
-  // microseconds of barriers and scans whether it holds 2048 or 8192 keys, and
-  // fewer CTAs per group merge fewer histograms
-  constexpr int kSelChunk = 8192;
-  int64_t s = (n_max + kSelChunk - 1) / kSelChunk;
-  s = std::min<int64_t>(s, sms / groups);
-  s = std::min<int64_t>(s, kSelMaxSplit);
-  return (int)std::max<int64_t>(s, 1);
+  return n[dev];
 }
 
-// n_sel score matrices [n_sel][T][ld] -> lists [n_sel][T][k_out], counts
-// [n_sel][T].  scratch: kSelMaxGroups SelGroup records, or NULL (one CTA per
-// group)
 static int launch_select_multi(const csa2_query_batch* qb, const float* score, int64_t ld, int mode,
                                const int32_t* pool, const int32_t* pool_n, int P, int k_out, int32_t* out,
-                               int32_t* out_n, int n_sel, void* scratch, cudaStream_t st) {
+                               int32_t* out_n, int n_sel, cudaStream_t st);
+
+// n_sel score matrices [n_sel][T][ld] -> lists [n_sel][T][k_out], counts
+// [n_sel][T], seeded by the scoring kernel's key counts `hist`
+// (k_select_cluster: the group's candidates split over a cluster of S CTAs
+// while there are fewer groups than SMs)
+static int launch_select_cluster(const csa2_query_batch* qb, const float* score, int64_t ld, int mode,
+                                 const int32_t* pool, const int32_t* pool_n, int P, int k_out, int32_t* out,
+                                 int32_t* out_n, int n_sel, uint32_t* hist, cudaStream_t st) {
   if (qb->n_tok > 65535 || n_sel > 65535) return fail(CSA2_ERR_UNSUPPORTED, "more than 65535 query tokens");
-  SelGroup* grp = static_cast<SelGroup*>(scratch);
   const int64_t groups = (int64_t)qb->n_tok * n_sel;
-  const int n_max = mode == 0 ? n_blocks_max(qb) : P * kBlock;
-  const int S = grp ? select_splits(groups, n_max) : 1;
+  const int n_max = std::max(1, mode == 0 ? n_blocks_max(qb) : P * kBlock);
+  SelCParams sp{};
+  sp.qb = *qb;
+  sp.score = score;
+  sp.ld = ld;
+  sp.mode = mode;
+  sp.pool = pool;
+  sp.pool_n = pool_n;
+  sp.P = P;
+  sp.k_out = k_out;
+  sp.out = out;
+  sp.out_n = out_n;
+  sp.hist = hist;
+  sp.words = (n_max + 31) / 32;
+  sp.cap = std::min(kSelCandCap, n_max);
+  sp.status = status_ptr();
+  const SelCLayout lay(sp.words, sp.cap, mode == 1 ? P : 0);
+  // the group's bitmaps, candidates and pool row in one CTA's shared memory;
+  // longer candidate lists (contexts beyond about 4.7M positions) take the
+  // selection without key counts
+  constexpr int kDynMax = 200 * 1024;
+  if (lay.bytes > (uint32_t)kDynMax)
+    return launch_select_multi(qb, score, ld, mode, pool, pool_n, P, k_out, out, out_n, n_sel, st);
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    if (int rc = cuda_check(cudaFuncSetAttribute(k_select_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 kDynMax),
+                            "select smem attribute"))
+      return rc;
+    if (int rc = cuda_check(
+            cudaFuncSetAttribute(k_select_cluster, cudaFuncAttributeNonPortableClusterSizeAllowed, 1),
+            "select cluster attribute"))
+      return rc;
+    attr_done[dev] = true;
+  }
+  // CTAs per group: about 8192 candidates each, a power of two <= 16, the
+  // whole grid within the SMs, and a cluster shape the GPU can place
+  int S = 1;
+  const int sms = std::min(num_sms_dev(), kSelMaxGroups);
+  if (groups < sms) {
+    int want = (int)std::min<int64_t>({(int64_t)(n_max + 8191) / 8192, 16, sms / groups});
+    while (S * 2 <= want) S *= 2;
+  }
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute at[1];
+  cfg.blockDim = dim3(kSelThreads);
+  cfg.dynamicSmemBytes = lay.bytes;
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  for (;; S /= 2) {
+    cfg.gridDim = dim3(S, qb->n_tok, n_sel);
+    at[0].val.clusterDim.x = S;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    int nc = 0;
+    if (S == 1 || (cudaOccupancyMaxActiveClusters(&nc, k_select_cluster, &cfg) == cudaSuccess && nc >= 1)) break;
+    cudaGetLastError();  // a refused shape is not an error of the call
+  }
+  Launch L_(mode == 0 ? "select_blocks" : "select_positions", st);
+  return cuda_check(cudaLaunchKernelEx(&cfg, k_select_cluster, sp), "k_select_cluster");
+}
+
+// the same without key counts (one CTA per group, k_select's own rounds)
+static int launch_select_multi(const csa2_query_batch* qb, const float* score, int64_t ld, int mode,
+                               const int32_t* pool, const int32_t* pool_n, int P, int k_out, int32_t* out,
+                               int32_t* out_n, int n_sel, cudaStream_t st) {
+  if (qb->n_tok > 65535 || n_sel > 65535) return fail(CSA2_ERR_UNSUPPORTED, "more than 65535 query tokens");
   SelParams sp{};
   sp.qb = *qb;
   sp.score = score;
@@ -252,27 +341,16 @@ static int launch_select_multi(const csa2_query_batch* qb, const float* score, i
   sp.k_out = k_out;
   sp.out = out;
   sp.out_n = out_n;
-  sp.grp = grp;
   sp.status = status_ptr();
-  sp.wait_ns = 1000000000ull;
-  const dim3 grid(S, qb->n_tok, n_sel);
-  if (S > 1) {
-    if (int rc = cuda_check(cudaMemsetAsync(grp, 0, (size_t)groups * sizeof(SelGroup), st), "clear select scratch"))
-      return rc;
-    Launch L_(mode == 0 ? "select_blocks" : "select_positions", st);
-    void* args[] = {&sp};
-    return cuda_check(cudaLaunchCooperativeKernel((const void*)k_select, grid, dim3(kSelThreads), args, 0, st),
-                      "k_select (cooperative)");
-  }
+  const dim3 grid(1, qb->n_tok, n_sel);
   Launch L_(mode == 0 ? "select_blocks" : "select_positions", st);
   k_select<<<grid, kSelThreads, 0, st>>>(sp);
   return cuda_check(cudaGetLastError(), "k_select");
 }
 
 int launch_select(const csa2_query_batch* qb, const float* score, int64_t ld, int mode, const int32_t* pool,
-                  const int32_t* pool_n, int P, int k_out, int32_t* out, int32_t* out_n, void* scratch,
-                  cudaStream_t st) {
-  return launch_select_multi(qb, score, ld, mode, pool, pool_n, P, k_out, out, out_n, 1, scratch, st);
+                  const int32_t* pool_n, int P, int k_out, int32_t* out, int32_t* out_n, cudaStream_t st) {
+  return launch_select_multi(qb, score, ld, mode, pool, pool_n, P, k_out, out, out_n, 1, st);
 }
 
 // Attention of n_layers (<= kMaxAttLayers) layers, each with its own index
@@ -403,12 +481,14 @@ int csa2_index_full(const csa2_query_batch* qb, const uint8_t* q_codes, const ui
   const int64_t ld = n_blocks_max(qb);
   float* bs = static_cast<float*>(c.take((size_t)qb->n_tok * ld * 4));
   float* sc = static_cast<float*>(c.take((size_t)qb->n_tok * P * kBlock * 4));
-  void* grp = c.take(select_ws(qb, P, 1));
+  const SelPlan sp = take_select_scratch(c, qb, P, 1);
   if (blockscore) bs = blockscore;
-  if (int rc = launch_scan(qb, q_codes, q_scales, w, H_I, k_idx, bs, ld, st)) return rc;
-  if (int rc = launch_select(qb, bs, ld, 0, nullptr, nullptr, P, P, pool, pool_n, grp, st)) return rc;
-  if (int rc = launch_rescore(qb, q_codes, q_scales, w, H_I, k_idx, pool, pool_n, P, sc, st)) return rc;
-  return launch_select(qb, sc, (int64_t)P * kBlock, 1, pool, pool_n, P, K, idx, idx_n, grp, st);
+  if (int rc = clear_select_counts(sp, st)) return rc;
+  if (int rc = launch_scan(qb, q_codes, q_scales, w, H_I, k_idx, bs, ld, sp.blk, st)) return rc;
+  if (int rc = launch_select_cluster(qb, bs, ld, 0, nullptr, nullptr, P, P, pool, pool_n, 1, sp.blk, st)) return rc;
+  if (int rc = launch_rescore_multi(qb, q_codes, q_scales, &w, 1, H_I, k_idx, pool, pool_n, P, sc, sp.pos, st))
+    return rc;
+  return launch_select_cluster(qb, sc, (int64_t)P * kBlock, 1, pool, pool_n, P, K, idx, idx_n, 1, sp.pos, st);
 }
 
 int csa2_index_reindex(const csa2_query_batch* qb, const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
@@ -424,9 +504,11 @@ int csa2_index_reindex(const csa2_query_batch* qb, const uint8_t* q_codes, const
   Carve c{static_cast<uint8_t*>(workspace), workspace_bytes};
   c.take((size_t)qb->n_tok * n_blocks_max(qb) * 4);
   float* sc = static_cast<float*>(c.take((size_t)qb->n_tok * P * kBlock * 4));
-  void* grp = c.take(select_ws(qb, P, 1));
-  if (int rc = launch_rescore(qb, q_codes, q_scales, w, H_I, k_idx, pool, pool_n, P, sc, st)) return rc;
-  return launch_select(qb, sc, (int64_t)P * kBlock, 1, pool, pool_n, P, K, idx, idx_n, grp, st);
+  const SelPlan sp = take_select_scratch(c, qb, P, 1);
+  if (int rc = clear_select_counts(sp, st)) return rc;
+  if (int rc = launch_rescore_multi(qb, q_codes, q_scales, &w, 1, H_I, k_idx, pool, pool_n, P, sc, sp.pos, st))
+    return rc;
+  return launch_select_cluster(qb, sc, (int64_t)P * kBlock, 1, pool, pool_n, P, K, idx, idx_n, 1, sp.pos, st);
 }
 
 static int check_attend(const csa2_query_batch* qb, const void* q, int q_dtype, int Hq, const csa2_fp4_cache* kv,
@@ -488,7 +570,7 @@ static size_t stack_ws(const csa2_stack_desc* d, size_t* sub_off) {
   Carve ix{nullptr, 0};
   ix.take((size_t)T * n_blocks_max(qb) * 4);                             // block scores
   ix.take((size_t)std::min(ns, kMaxSel) * T * d->P * kBlock * 4);        // pool position scores
-  ix.take(select_ws(qb, d->P, std::min(ns, kMaxSel)));                  // split-selection scratch
+  ix.take(select_ws(qb, d->P, std::min(ns, kMaxSel)));                  // selection scratch
   size_t sub = ix.used + 256;
   sub = std::max(sub, attend_ws(qb, d->Hq, d->kv.dim));
   c.take(0);
@@ -582,7 +664,8 @@ int csa2_decode_stack(const csa2_stack_desc* d, void* workspace, size_t workspac
   const int64_t ld = n_blocks_max(qb);
   float* bs = static_cast<float*>(sc_c.take((size_t)T * ld * 4));
   float* sc = static_cast<float*>(sc_c.take((size_t)std::min(n_sel, kMaxSel) * T * d->P * kBlock * 4));
-  void* grp = sc_c.take(select_ws(qb, d->P, std::min(n_sel, kMaxSel)));
+  const SelPlan sel = take_select_scratch(sc_c, qb, d->P, std::min(n_sel, kMaxSel));
+  if (int rc = clear_select_counts(sel, st)) return rc;
   // each FULL layer builds the pool that it and the REINDEX layers after it
   // rescore; the rescoring and position selection of consecutive selectors
   // run up to kMaxSel at a time
@@ -590,9 +673,11 @@ int csa2_decode_stack(const csa2_stack_desc* d, void* workspace, size_t workspac
   while (s < n_sel) {
     const csa2_layer_desc& F = d->layers[sel_layer[s]];
     if (F.mode == CSA2_MODE_FULL) {
-      if (int rc = launch_scan(qb, qc + s * q_codes_sz, qsc + s * q_scales_sz, F.iw, d->H_I, &d->k_idx, bs, ld, st))
+      if (int rc = launch_scan(qb, qc + s * q_codes_sz, qsc + s * q_scales_sz, F.iw, d->H_I, &d->k_idx, bs, ld,
+                               sel.blk, st))
         return rc;
-      if (int rc = launch_select(qb, bs, ld, 0, nullptr, nullptr, d->P, d->P, pool, pool_n, grp, st)) return rc;
+      if (int rc = launch_select_cluster(qb, bs, ld, 0, nullptr, nullptr, d->P, d->P, pool, pool_n, 1, sel.blk, st))
+        return rc;
       if (F.pool_out)
         if (int rc = copy_i32(pool, F.pool_out, (int64_t)T * d->P, st)) return rc;
     }
@@ -601,10 +686,10 @@ int csa2_decode_stack(const csa2_stack_desc* d, void* workspace, size_t workspac
     const float* ws[kMaxSel];
     for (int i = 0; i < n; ++i) ws[i] = d->layers[sel_layer[s + i]].iw;
     if (int rc = launch_rescore_multi(qb, qc + s * q_codes_sz, qsc + s * q_scales_sz, ws, n, d->H_I, &d->k_idx, pool,
-                                      pool_n, d->P, sc, st))
+                                      pool_n, d->P, sc, sel.pos, st))
       return rc;
-    if (int rc = launch_select_multi(qb, sc, (int64_t)d->P * kBlock, 1, pool, pool_n, d->P, d->K,
-                                     idx + (size_t)s * T * d->K, idx_n + (size_t)s * T, n, grp, st))
+    if (int rc = launch_select_cluster(qb, sc, (int64_t)d->P * kBlock, 1, pool, pool_n, d->P, d->K,
+                                    idx + (size_t)s * T * d->K, idx_n + (size_t)s * T, n, sel.pos, st))
       return rc;
     for (int i = 0; i < n; ++i)
       if (int32_t* o = d->layers[sel_layer[s + i]].idx_out)

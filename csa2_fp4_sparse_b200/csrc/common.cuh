@@ -180,6 +180,10 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* to
   return warp_before + x - v;
 }
 
+// key counts that seed a selection: bins of the top 12 key bits
+constexpr int kHistBins = 4096;
+constexpr int kHistShift = 20;
+
 // order-preserving map of a score to an unsigned key; invalid (-inf marker)
 // entries map to 0, below every finite score
 __device__ __forceinline__ uint32_t score_key(float f) {

@@ -12,12 +12,14 @@ int fail(int code, const char* fmt, ...);
 int cuda_check(cudaError_t e, const char* what);
 int* status_ptr();
 
+// hist: per (selector, token) group, counts of the stored scores' keys by
+// their top 12 bits (4096 bins, zeroed before the launch), or NULL
 int launch_scan_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
-                   const csa2_fp4_cache* kc, float* bs, int64_t ld, cudaStream_t st);
+                   const csa2_fp4_cache* kc, float* bs, int64_t ld, uint32_t* hist, cudaStream_t st);
 
 int launch_rescore_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* const* w,
                       int n_sel, int H, const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n, int P,
-                      float* scores, cudaStream_t st);
+                      float* scores, uint32_t* hist, cudaStream_t st);
 bool attend_tc_supported(int D, int Hq, int q_dtype);
 // one layer of a multi-layer attention launch
 struct AttendLayer {

@@ -35,8 +35,7 @@ int launch_rescore(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t*
                    const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n, int P, float* scores,
                    cudaStream_t st);
 int launch_select(const csa2_query_batch* qb, const float* score, int64_t ld, int mode, const int32_t* pool,
-                  const int32_t* pool_n, int P, int k_out, int32_t* out, int32_t* out_n, void* scratch,
-                  cudaStream_t st);
+                  const int32_t* pool_n, int P, int k_out, int32_t* out, int32_t* out_n, cudaStream_t st);
 void clear_last_error();
 
 }  // namespace csa2
@@ -63,6 +62,7 @@ extern "C" int csa2_index_reindex_noalloc(const csa2_query_batch* qb, const uint
   // array by an earlier call is ever read: no clearing is needed.
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (int r = launch_rescore(qb, q_codes, q_scales, w, H_I, k_idx, pool, pool_n, P, scores, st)) return r;
-  // no split-selection scratch either: one CTA per query token
-  return launch_select(qb, scores, (int64_t)P * kBlock, 1, pool, pool_n, P, K, idx, idx_n, nullptr, st);
+  // no selection scratch either: one CTA per query token, with its own
+  // histogram rounds over the scores
+  return launch_select(qb, scores, (int64_t)P * kBlock, 1, pool, pool_n, P, K, idx, idx_n, st);
 }

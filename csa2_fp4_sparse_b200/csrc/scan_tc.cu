@@ -103,6 +103,7 @@ struct Params {
   const int32_t* pool;   // rescore: [T][pool_cap] block ids
   const int32_t* pool_n; // rescore: [T]
   int pool_cap;
+  uint32_t* hist;        // key counts by the top 12 bits, [group][kHistBins] (group = selector * T + token), or NULL
   int* status;
   uint64_t wait_ns;
 };
@@ -573,14 +574,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int i = ti.tile * kTile + row;
           const int64_t pos = (int64_t)blk * kBlock + (i % kBlock);
           const int64_t orow = (int64_t)(sel0 + j) * P.qb.n_tok + tok0;  // selector * T + token
-          if (i < P.pool_cap * kBlock) P.out[orow * P.ld + i] = (blk >= 0 && pos <= p) ? acc : -INFINITY;
+          const bool valid = blk >= 0 && pos <= p && i < P.pool_cap * kBlock;
+          if (i < P.pool_cap * kBlock) P.out[orow * P.ld + i] = valid ? acc : -INFINITY;
+          if (P.hist) {  // one count per distinct bin of the warp
+            const uint32_t key = valid ? score_key(acc) : 0u;
+            const uint32_t bin = key ? key >> kHistShift : 0xFFFFFFFFu;
+            const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+            if (key && lane == __ffs(peers) - 1) atomicAdd(P.hist + orow * kHistBins + bin, (uint32_t)__popc(peers));
+          }
         } else {
           const int64_t t = t0 + row;
           float sc = (t <= p) ? acc : -INFINITY;
           sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 1));
           sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 2));
           sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 4));
-          if ((lane & 7) == 0 && t <= p) P.out[(int64_t)(tok0 + j) * P.ld + t / kBlock] = sc;
+          if ((lane & 7) == 0 && t <= p) {
+            P.out[(int64_t)(tok0 + j) * P.ld + t / kBlock] = sc;
+            const uint32_t key = score_key(sc);
+            if (P.hist && key) atomicAdd(P.hist + (int64_t)(tok0 + j) * kHistBins + (key >> kHistShift), 1u);
+          }
         }
       }
     }
@@ -663,7 +675,7 @@ static int num_sms() {
 template <bool kRescore>
 static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* const* w,
                            int n_sel, int H, const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n,
-                           int pool_cap, float* out, int64_t ld, cudaStream_t st) {
+                           int pool_cap, float* out, int64_t ld, uint32_t* hist, cudaStream_t st) {
   using namespace scan_tc;
   if (kc->n_rows >= (int64_t(1) << 31)) return fail(CSA2_ERR_UNSUPPORTED, "cache too large for TMA");
   if (n_sel < 1 || n_sel > kMaxSel) return fail(CSA2_ERR_UNSUPPORTED, "1..%d selector layers per launch", kMaxSel);
@@ -702,6 +714,7 @@ static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const 
   p.pool = pool;
   p.pool_n = pool_n;
   p.pool_cap = pool_cap;
+  p.hist = hist;
   p.status = status_ptr();
   p.wait_ns = 1000000000ull;  // 1 s
   static bool attr_done[64] = {false};
@@ -726,16 +739,16 @@ static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const 
 }
 
 int launch_scan_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
-                   const csa2_fp4_cache* kc, float* bs, int64_t ld, cudaStream_t st) {
-  return launch_index_tc<false>(qb, qc, qs, &w, 1, H, kc, nullptr, nullptr, 0, bs, ld, st);
+                   const csa2_fp4_cache* kc, float* bs, int64_t ld, uint32_t* hist, cudaStream_t st) {
+  return launch_index_tc<false>(qb, qc, qs, &w, 1, H, kc, nullptr, nullptr, 0, bs, ld, hist, st);
 }
 
 // n_sel selector layers at once: queries [n_sel][T][H][...], weights w[sel],
 // scores [n_sel][T][8P]; a token's pool is gathered once for up to four of them
 int launch_rescore_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* const* w,
                       int n_sel, int H, const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n, int P,
-                      float* scores, cudaStream_t st) {
-  return launch_index_tc<true>(qb, qc, qs, w, n_sel, H, kc, pool, pool_n, P, scores, (int64_t)P * kBlock, st);
+                      float* scores, uint32_t* hist, cudaStream_t st) {
+  return launch_index_tc<true>(qb, qc, qs, w, n_sel, H, kc, pool, pool_n, P, scores, (int64_t)P * kBlock, hist, st);
 }
 
 }  // namespace csa2
