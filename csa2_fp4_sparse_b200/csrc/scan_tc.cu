@@ -94,6 +94,8 @@ struct Params {
   int H, Nh, DI;            // heads, heads padded to 16 (MMA N per column), key dim
   int slot_cols, n_slots;   // accumulator slots of (query columns x Nh) columns
   int box_rows;             // scan: rows per TMA box (128, or 64 for 64-row pages)
+  const uint8_t* codes;     // the indexer cache (rescoring gathers it directly)
+  const uint8_t* scales;
   int64_t n_rows;
   int page_size, max_pages;
   const int32_t* page_table;
@@ -240,7 +242,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(bar_full + 8 * i, 1);
+      // scan: one arrival with the TMA byte count; rescoring: the 32 lanes of
+      // the producer warp, each when its copies have landed
+      mbar_init(bar_full + 8 * i, kRescore ? 32 : 1);
       mbar_init(bar_done + 8 * i, 1);
       mbar_init(bar_sf + 8 * i, 4);
     }
@@ -275,16 +279,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tx = (uint32_t)kTile * row_bytes + (uint32_t)kTile * spr;
     TileIter<kRescore> ti;
     ti.init(P, wb, we);
-    int64_t it = 0;
+    int it = 0, s = 0;  // this CTA's stage count, ring stage
+    uint32_t n = 0;     // use of the ring stage
+    auto adv = [&]() {
+      ++it;
+      if (++s == kStages) {
+        s = 0;
+        ++n;
+      }
+    };
     int cur_g = -1, tok0 = 0, b = 0;
     int64_t base = 0, len = 0;
-    for (; ti.valid(); ti.next(P), ++it) {
-      if ((int)(it & 1) != pw || *abort) continue;
-      const int s = (int)(it % kStages);
-      const uint32_t n = (uint32_t)(it / kStages);
+    for (; ti.valid(); ti.next(P), adv()) {
+      if ((it & 1) != pw || *abort) continue;
       if (lane == 0) {
         // the stage is free once the MMAs of its previous use completed
-        if (n == 0 || wait_or_abort(bar_done + 8 * s, (n - 1) & 1, P, abort))
+        if ((n == 0 || wait_or_abort(bar_done + 8 * s, (n - 1) & 1, P, abort)) && !kRescore)
           tc::mbar_arrive_expect_tx(bar_full + 8 * s, tx);
       }
       __syncwarp();
@@ -296,17 +306,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         len = __ldg(P.qb.seq_len + b);
         base = P.page_table ? 0 : __ldg(P.seq_base + b);
       }
-      if (lane < nbox) {
-        int64_t pos0 = -1;
-        if (kRescore) {
+      if (kRescore) {
+        // gather: 16 pool blocks of 8 rows, 16-byte asynchronous copies from
+        // every lane (a TMA instruction per block and array would cost the
+        // warp hundreds of cycles each); codes land in the swizzle the MMA
+        // reads, each block's scales at its 128-byte slot.  Rows outside the
+        // cache are zero-filled.
+        int64_t my_row0 = -1;  // lane e < 16: first cache row of block e
+        if (lane < 16) {
           const int e = ti.tile * 16 + lane;
           const int np = min(__ldg(P.pool_n + tok0), P.pool_cap);
           const int32_t blk = e < np ? __ldg(P.pool + (int64_t)tok0 * P.pool_cap + e) : -1;
-          if (blk >= 0) pos0 = (int64_t)blk * kBlock;
-        } else {
-          pos0 = (int64_t)ti.tile * kTile + lane * box_rows;
-          if (pos0 >= len) pos0 = -1;
+          if (blk >= 0) {
+            const int64_t row0 = key_row(P, b, (int64_t)blk * kBlock, base);
+            if (row0 >= 0 && ((row0 * spr) & 15) == 0) my_row0 = row0;
+            else set_status(P.status, CSA2_ERR_RANGE);
+          }
         }
+        const int cpr = row_bytes / 16;  // 16-byte chunks a code row
+        const uint32_t a_base = sbase + kOffA + s * kCodeStage;
+        for (int c = lane; c < kTile * cpr; c += 32) {
+          const int r = c / cpr, ch = c % cpr;
+          const int64_t row0 = __shfl_sync(0xffffffffu, my_row0, r / kBlock);
+          const int64_t gr = row0 + r % kBlock;
+          const bool in = row0 >= 0 && gr < P.n_rows;
+          const int sch = (P.DI == 128) ? (ch ^ ((r >> 1) & 3)) : (ch ^ ((r >> 2) & 1));
+          tc::cp_async_16(a_base + r * row_bytes + sch * 16, in ? P.codes + gr * row_bytes + ch * 16 : P.codes,
+                          in ? 16u : 0u);
+        }
+        {
+          const int per_blk = kBlock * spr / 16;  // scale chunks a block (2 or 1)
+          const int e = lane / per_blk, h = lane % per_blk;
+          const int64_t row0 = __shfl_sync(0xffffffffu, my_row0, min(e, 31));
+          // bytes of this chunk inside the scale array (a block cut by the
+          // cache's end keeps its first rows; the rest is zero-filled)
+          const int64_t first = row0 + h * (16 / spr);
+          const uint32_t nb = row0 >= 0 ? (uint32_t)max((int64_t)0, min((int64_t)16, (P.n_rows - first) * spr)) : 0u;
+          if (e < 16)
+            tc::cp_async_16(sbase + kOffRaw + s * kRawStage + e * 128 + h * 16,
+                            nb ? P.scales + first * spr : P.scales, nb);
+        }
+        tc::cp_async_arrive_noinc(bar_full + 8 * s);  // the stage completes when all 32 lanes' copies landed
+      } else if (lane < nbox) {
+        int64_t pos0 = -1;
+        pos0 = (int64_t)ti.tile * kTile + lane * box_rows;
+        if (pos0 >= len) pos0 = -1;
         const int64_t row0 = pos0 >= 0 ? key_row(P, b, pos0, base) : -1;
         // out of the cache, or not 16-byte aligned in the scale array: the
         // box is read out of range (zeros) and the row reported
@@ -319,13 +363,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc::tma_load_2d(sbase + kOffA + s * kCodeStage + lane * box_rows * row_bytes, &tm_codes, bar_full + 8 * s, 0,
                         ry);
-        const uint32_t slot = kRescore ? 128u : (uint32_t)(box_rows * spr);
+        const uint32_t slot = (uint32_t)(box_rows * spr);
         tc::tma_load_2d(sbase + kOffRaw + s * kRawStage + lane * slot, &tm_scales, bar_full + 8 * s, 0, sy);
       }
       __syncwarp();
     }
-    // copies in flight: the scale-factor warps wait for every stage's landing
-    // before the CTA ends (after a failed wait, see the end of the kernel)
+    // this thread's copies land before it leaves (the scale-factor warps also
+    // wait for every stage's landing before the CTA ends)
+    if (kRescore) tc::cp_async_wait_all();
   } else if (warp < kSf0) {
     // ------------------------------------------------------------ MMA issuers
     // Both walk every stage (both see every change of group) and issue the
@@ -337,12 +382,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sbo = 8u * row_bytes;  // 8 rows per swizzle atom
     TileIter<kRescore> ti;
     ti.init(P, wb, we);
-    int64_t it = 0;
+    int it = 0, s = 0, slot = 0;  // stage count, ring stage, accumulator slot
+    uint32_t n = 0, u = 0;        // uses of the ring stage and of the slot
+    auto adv = [&]() {
+      ++it;
+      if (++s == kStages) {
+        s = 0;
+        ++n;
+      }
+      if (++slot == P.n_slots) {
+        slot = 0;
+        ++u;
+      }
+    };
     uint32_t drain_n = 0, sfb_n = 0;
     int cur_g = -1, W = 0;
     // No early exit from this loop: both issuers meet at the same named
     // barriers; after a failed wait a warp keeps walking without issuing.
-    for (; ti.valid(); ti.next(P), ++it) {
+    for (; ti.valid(); ti.next(P), adv()) {
       if (ti.b != cur_g) {
         if (cur_g >= 0) {  // every MMA reading the old queries must finish first
           if (lane == 0) tc::commit(my_drain);
@@ -360,35 +417,46 @@ __global__ void __launch_bounds__(kThreads, 1)
           auto qrow = [&](int j) -> int64_t {
             return kRescore ? (int64_t)(sel0 + j) * P.qb.n_tok + tok0 : (int64_t)(tok0 + j);
           };
-          // B operand: query codes, swizzled like the TMA-written A tiles
+          // B operand: query codes, swizzled like the TMA-written A tiles,
+          // in 16-byte asynchronous copies that are all in flight together
+          // (heads past H zero-filled)
           const int chunks_per_row = row_bytes / 16;
           for (int e = lane; e < W * 64 * chunks_per_row; e += 32) {
             const int j = e / (64 * chunks_per_row);
             const int n = (e / chunks_per_row) % 64;
             const int ch = e % chunks_per_row;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (n < P.H) v = __ldg(reinterpret_cast<const uint4*>(P.q_codes + (qrow(j) * P.H + n) * row_bytes) + ch);
             const int sch = (P.DI == 128) ? (ch ^ ((n >> 1) & 3)) : (ch ^ ((n >> 2) & 1));
-            *reinterpret_cast<uint4*>(smem + kOffB + j * 4096 + n * row_bytes + sch * 16) = v;
+            const bool in = n < P.H;
+            tc::cp_async_16(sbase + kOffB + j * 4096 + n * row_bytes + sch * 16,
+                            in ? P.q_codes + (qrow(j) * P.H + n) * row_bytes + ch * 16 : P.q_codes, in ? 16u : 0u);
           }
-          // B scale factors: [m0 (32)][m1 (4)][k (4)] per 64-element K step
-          for (int e = lane; e < W * ksteps * 32; e += 32) {
-            const int j = e / (ksteps * 32), ks = (e / 32) % ksteps, m0 = e % 32;
-            uint32_t v[4];
+          // B scale factors, [m0 (32)][m1 (4)][k (4)] per 64-element K step:
+          // lane m0 first loads the scale words of its heads m1*32 + m0 of
+          // every column (all loads in flight together), then duplicates each
+          // per-32 scale into the per-16 layout
+          uint32_t hw[kMaxWc][4];
+#pragma unroll
+          for (int j = 0; j < kMaxWc; ++j)
 #pragma unroll
             for (int m1 = 0; m1 < 4; ++m1) {
-              const int n = m1 * 32 + m0;
-              uint32_t a = 0, b2 = 0;
-              if (n < P.H) {
-                const uint8_t* sp = P.q_scales + (qrow(j) * P.H + n) * spr + 2 * ks;
-                a = __ldg(sp);
-                b2 = __ldg(sp + 1);
+              const int n = m1 * 32 + lane;
+              hw[j][m1] = 0u;
+              if (j < W && n < P.H) {
+                const uint8_t* sp = P.q_scales + (qrow(j) * P.H + n) * spr;
+                hw[j][m1] = spr == 4 ? __ldg(reinterpret_cast<const uint32_t*>(sp))
+                                     : (uint32_t)__ldg(reinterpret_cast<const uint16_t*>(sp));
               }
-              v[m1] = a | (a << 8) | (b2 << 16) | (b2 << 24);
             }
-            *reinterpret_cast<uint4*>(smem + kOffSfb + (j * 2 + ks) * 512 + m0 * 16) =
-                make_uint4(v[0], v[1], v[2], v[3]);
-          }
+#pragma unroll
+          for (int j = 0; j < kMaxWc; ++j)
+            for (int ks = 0; ks < ksteps; ++ks)
+              if (j < W) {
+                const uint32_t sel = ks == 0 ? 0x1100u : 0x3322u;
+                *reinterpret_cast<uint4*>(smem + kOffSfb + (j * 2 + ks) * 512 + lane * 16) =
+                    make_uint4(__byte_perm(hw[j][0], 0, sel), __byte_perm(hw[j][1], 0, sel),
+                               __byte_perm(hw[j][2], 0, sel), __byte_perm(hw[j][3], 0, sel));
+              }
+          tc::cp_async_wait_all();
           tc::fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
@@ -405,11 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::named_sync(6, 64);  // new queries in place
         tc::fence_after_sync();
       }
-      if ((int)(it & 1) != mw || *abort) continue;  // the other issuer's stage (or nothing left to do)
-      const int s = (int)(it % kStages);
-      const uint32_t n = (uint32_t)(it / kStages);
-      const int slot = (int)(it % P.n_slots);
-      const uint32_t u = (uint32_t)(it / P.n_slots);  // use of the slot
+      if ((it & 1) != mw || *abort) continue;  // the other issuer's stage (or nothing left to do)
       // this warp's earlier waits on its barrier of the slot: every use
       // (even slot count: the slot's stages all have this warp's parity) or
       // every other use (odd count: the parity of the slot's stages alternates)
@@ -420,6 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && u > 0) ok = wait_or_abort(bar_acce + 8 * (slot * 2 + mw), ph & 1, P, abort);  // slot read
         if (ok) {
           tc::fence_after_sync();
+          if (kRescore) tc::fence_proxy_async_smem();  // codes written by cp.async (generic proxy)
           const uint32_t sfa = tmem + kColSfa + (uint32_t)s * 8;
           const uint32_t acc = tmem + kColAcc + (uint32_t)(slot * P.slot_cols);
           for (int j = 0; j < W; ++j)
@@ -452,19 +517,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     TileIter<kRescore> ti;
     ti.init(P, wb, we);
-    int64_t it = 0;
+    int s = 0;
+    uint32_t n = 0;
     const int box_rows = kRescore ? kBlock : P.box_rows;
+    const int bshift = box_rows == 128 ? 7 : (box_rows == 64 ? 6 : 3);  // box_rows is 128, 64 or 8
     const int slot_bytes = kRescore ? 128 : box_rows * spr;
-    for (; ti.valid(); ti.next(P), ++it) {
-      const int s = (int)(it % kStages);
-      const uint32_t n = (uint32_t)(it / kStages);
+    for (; ti.valid(); ti.next(P), (++s == kStages ? (s = 0, ++n) : 0u)) {
       if (!warp_wait_or_abort(bar_full + 8 * s, n & 1, P, abort)) break;
       const uint8_t* raw = smem + kOffRaw + s * kRawStage;
       uint32_t r[8];
 #pragma unroll
       for (int m1 = 0; m1 < 4; ++m1) {
         const int rw = m1 * 32 + lane;
-        const uint8_t* src = raw + (rw / box_rows) * slot_bytes + (rw % box_rows) * spr;
+        const uint8_t* src = raw + (rw >> bshift) * slot_bytes + (rw & (box_rows - 1)) * spr;
         const uint32_t wv =
             (spr == 4) ? *reinterpret_cast<const uint32_t*>(src) : (uint32_t)*reinterpret_cast<const uint16_t*>(src);
         r[m1] = __byte_perm(wv, 0, 0x1100u);      // K step 0: scales 0, 1
@@ -492,12 +557,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     int64_t* pos_g = reinterpret_cast<int64_t*>(smem + kOffPos) + wg * kMaxWc;
     TileIter<kRescore> ti;
     ti.init(P, wb, we);
-    int64_t it = 0;
+    int it = 0, s = 0, slot = 0, wgc = 0;  // stage count, ring stage, slot, warpgroup of the stage
+    uint32_t n = 0;
+    auto adv = [&]() {
+      ++it;
+      if (++s == kStages) {
+        s = 0;
+        ++n;
+      }
+      if (++slot == P.n_slots) slot = 0;
+      if (++wgc == kEpiWG) wgc = 0;
+    };
     int cur_g = -1, W = 0, tok0 = 0, sel0 = 0;
     bool dead = false;  // warpgroup-uniform: a wait of this warpgroup gave up
     const int ng = P.Nh / 16;
     // no early exit: the four warps of the warpgroup meet at named barriers
-    for (; ti.valid(); ti.next(P), ++it) {
+    for (; ti.valid(); ti.next(P), adv()) {
       if (ti.b != cur_g) {
         tc::named_sync(1 + wg, 128);
         cur_g = ti.b;
@@ -511,10 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ept < W) pos_g[ept] = __ldg(P.qb.tok_pos + (kRescore ? tok0 : tok0 + ept));
         tc::named_sync(1 + wg, 128);
       }
-      if ((int)(it % kEpiWG) != wg || dead) continue;  // another warpgroup's stage (or nothing left to do)
-      const int s = (int)(it % kStages);
-      const uint32_t n = (uint32_t)(it / kStages);
-      const int slot = (int)(it % P.n_slots);
+      if (wgc != wg || dead) continue;  // another warpgroup's stage (or nothing left to do)
       // one prober per warpgroup; the other warps park on the named barrier
       if (!mbar_wait_group(bar_done + 8 * s, n & 1, P.wait_ns, ept == 0, *abort != 0, 1 + wg, 128)) {
         if (ept == 0 && !*abort) {
@@ -550,7 +622,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (j == W - 1 && (hf == 1 || ng <= 2)) {  // the slot is free once its last load has landed:
             tc::fence_before_sync();                 // for the warp issuing its next use
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(bar_acce + 8 * (slot * 2 + (int)((it + P.n_slots) & 1)));
+            if (lane == 0) tc::mbar_arrive(bar_acce + 8 * (slot * 2 + ((it + P.n_slots) & 1)));
           }
 #pragma unroll
           for (int g = 0; g < 2; ++g)
@@ -704,6 +776,8 @@ static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const 
   while (ns > 1 && kStages % ns) --ns;
   p.n_slots = ns;
   p.box_rows = box_rows;
+  p.codes = kc->codes;
+  p.scales = kc->scales;
   p.n_rows = kc->n_rows;
   p.page_size = kc->page_size;
   p.max_pages = kc->max_pages;
