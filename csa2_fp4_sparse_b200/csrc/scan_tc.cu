@@ -52,9 +52,7 @@
 namespace csa2 {
 namespace scan_tc {
 
-constexpr int kTile = 128;      // positions per stage = MMA M
-constexpr int kStages = 18;     // stage ring: a multiple of every accumulator slot count (1, 2, 3, 6), of the
-                                // producer and MMA warp counts (2) and of the epilogue warpgroups (3)
+constexpr int kTile = 128;      // positions per MMA tile = MMA M
 constexpr int kMaxWc = 4;       // query columns per group
 constexpr int kEpiWG = 3;       // epilogue warpgroups
 constexpr int kThreads = 32 * (8 + 4 * kEpiWG);
@@ -63,26 +61,32 @@ constexpr int kMma0 = 2;        // MMA warps 2, 3
 constexpr int kSf0 = 4;         // scale-factor warps 4..7 (lane quarters 0..3)
 constexpr int kEpi0 = 8;        // epilogue warpgroups 8..11, 12..15, 16..19
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColSfa = 0;                          // [kStages][8]
-constexpr uint32_t kColSfb = kColSfa + kStages * 8;      // [kMaxWc][8]
-constexpr uint32_t kColAcc = kColSfb + kMaxWc * 8;       // accumulator slots
-constexpr uint32_t kAccCols = kTmemCols - kColAcc;       // 384
 
-// shared-memory map
-constexpr uint32_t kCodeStage = 8192;                    // 128 rows x <= 64 B
-constexpr uint32_t kRawStage = 2048;                     // raw scales: up to 16 boxes at 128-byte slots
-constexpr uint32_t kOffA = 0;                            // [kStages][8192]
-constexpr uint32_t kOffRaw = kOffA + kStages * kCodeStage;
-constexpr uint32_t kOffB = kOffRaw + kStages * kRawStage;  // [kMaxWc][64 rows][64 B]
-constexpr uint32_t kOffSfb = kOffB + kMaxWc * 4096;        // [kMaxWc][2][512]
-constexpr uint32_t kOffW = kOffSfb + kMaxWc * 1024;        // [kEpiWG][kMaxWc][64] f32
-constexpr uint32_t kOffPos = kOffW + kEpiWG * kMaxWc * 64 * 4;  // [kEpiWG][kMaxWc] i64 query positions
-constexpr uint32_t kOffBar = kOffPos + kEpiWG * kMaxWc * 8;
-constexpr uint32_t kNumBars = 3 * kStages + 12 + 3;        // full, done, sf; acc_empty[6][2]; drain[2], sfb
-constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;      // tmem base, abort flag
-constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;      // + alignment slack
-static_assert(kOffB % 1024 == 0, "B tiles must be 1024-aligned");
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+// Shared-memory and TMEM maps for stages of kSub MMA tiles (kSub * 128
+// positions; two tiles a stage halve every per-stage cost per position).
+// The stage ring is even (producer and MMA warps take stages in turn).
+template <int kSub>
+struct Layout {
+  static constexpr int kStages = kSub == 2 ? 10 : 18;
+  static constexpr uint32_t kCodeStage = 8192u * kSub;               // kSub x 128 rows x <= 64 B
+  static constexpr uint32_t kRawStage = kSub == 2 ? 1024u : 2048u;    // raw scales (rescoring: 16 boxes at 128 B)
+  static constexpr uint32_t kColSfa = 0;                             // [kStages][kSub][8]
+  static constexpr uint32_t kColSfb = kColSfa + kStages * 8 * kSub;  // [kMaxWc][8]
+  static constexpr uint32_t kColAcc = kColSfb + kMaxWc * 8;          // accumulator slots
+  static constexpr uint32_t kAccCols = kTmemCols - kColAcc;
+  static constexpr uint32_t kOffA = 0;                               // [kStages][kCodeStage]
+  static constexpr uint32_t kOffRaw = kOffA + kStages * kCodeStage;
+  static constexpr uint32_t kOffB = kOffRaw + kStages * kRawStage;   // [kMaxWc][64 rows][64 B]
+  static constexpr uint32_t kOffSfb = kOffB + kMaxWc * 4096;         // [kMaxWc][2][512]
+  static constexpr uint32_t kOffW = kOffSfb + kMaxWc * 1024;         // [kEpiWG][kMaxWc][64] f32
+  static constexpr uint32_t kOffPos = kOffW + kEpiWG * kMaxWc * 64 * 4;  // [kEpiWG][kMaxWc] i64 query positions
+  static constexpr uint32_t kOffBar = kOffPos + kEpiWG * kMaxWc * 8;
+  static constexpr uint32_t kNumBars = 3 * kStages + 12 + 3;  // full, done, sf; acc_empty[6][2]; drain[2], sfb
+  static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;      // tmem base, abort flag
+  static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;      // + alignment slack
+  static_assert(kOffB % 1024 == 0, "B tiles must be 1024-aligned");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
 
 struct Params {
   csa2_query_batch qb;
@@ -93,7 +97,8 @@ struct Params {
   int cpg;                  // groups per sequence (scan) or per token (rescore)
   int H, Nh, DI;            // heads, heads padded to 16 (MMA N per column), key dim
   int slot_cols, n_slots;   // accumulator slots of (query columns x Nh) columns
-  int box_rows;             // scan: rows per TMA box (128, or 64 for 64-row pages)
+  int box_rows;             // scan: rows per TMA box (256, 128, or 64 for 64-row pages)
+  int rows;                 // positions per stage (kSub * 128)
   const uint8_t* codes;     // the indexer cache (rescoring gathers it directly)
   const uint8_t* scales;
   int64_t n_rows;
@@ -144,7 +149,7 @@ __device__ __forceinline__ int group_tiles(const Params& P, int g) {
   if (W <= 0) return 0;
   if (kRescore) return (min(__ldg(P.pool_n + tok0), P.pool_cap) + 15) / 16;
   const int64_t vis = min((int64_t)__ldg(P.qb.tok_pos + tok0 + W - 1) + 1, (int64_t)__ldg(P.qb.seq_len + b));
-  return (int)((max(vis, (int64_t)0) + kTile - 1) / kTile);
+  return (int)((max(vis, (int64_t)0) + P.rows - 1) / P.rows);
 }
 
 // this CTA's contiguous range of (group, stage) work in group-major order
@@ -216,10 +221,17 @@ __device__ __forceinline__ int64_t key_row(const Params& P, int b, int64_t pos, 
   return (row >= 0 && row < P.n_rows) ? row : -1;
 }
 
-template <bool kRescore>
+template <bool kRescore, int kSub>
 __global__ void __launch_bounds__(kThreads, 1)
     k_index_tc(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales,
                const __grid_constant__ Params P) {
+  using Lay = Layout<kSub>;
+  constexpr int kStages = Lay::kStages;
+  constexpr int kRows = kTile * kSub;  // positions per stage
+  constexpr uint32_t kCodeStage = Lay::kCodeStage, kRawStage = Lay::kRawStage, kColSfa = Lay::kColSfa,
+                     kColSfb = Lay::kColSfb, kColAcc = Lay::kColAcc, kOffA = Lay::kOffA, kOffRaw = Lay::kOffRaw,
+                     kOffB = Lay::kOffB, kOffSfb = Lay::kOffSfb, kOffW = Lay::kOffW, kOffPos = Lay::kOffPos,
+                     kOffBar = Lay::kOffBar, kOffMisc = Lay::kOffMisc;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -275,8 +287,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // rescore 16 pool blocks of 8 rows (codes and scales each)
     const int pw = warp - kProd0;
     const int box_rows = kRescore ? kBlock : P.box_rows;
-    const int nbox = kRescore ? 16 : kTile / box_rows;
-    const uint32_t tx = (uint32_t)kTile * row_bytes + (uint32_t)kTile * spr;
+    const int nbox = kRescore ? 16 : kRows / box_rows;
+    const uint32_t tx = (uint32_t)kRows * row_bytes + (uint32_t)kRows * spr;
     TileIter<kRescore> ti;
     ti.init(P, wb, we);
     int it = 0, s = 0;  // this CTA's stage count, ring stage
@@ -349,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::cp_async_arrive_noinc(bar_full + 8 * s);  // the stage completes when all 32 lanes' copies landed
       } else if (lane < nbox) {
         int64_t pos0 = -1;
-        pos0 = (int64_t)ti.tile * kTile + lane * box_rows;
+        pos0 = (int64_t)ti.tile * kRows + lane * box_rows;
         if (pos0 >= len) pos0 = -1;
         const int64_t row0 = pos0 >= 0 ? key_row(P, b, pos0, base) : -1;
         // out of the cache, or not 16-byte aligned in the scale array: the
@@ -485,15 +497,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) {
           tc::fence_after_sync();
           if (kRescore) tc::fence_proxy_async_smem();  // codes written by cp.async (generic proxy)
-          const uint32_t sfa = tmem + kColSfa + (uint32_t)s * 8;
+          const uint32_t sfa = tmem + kColSfa + (uint32_t)s * 8 * kSub;
           const uint32_t acc = tmem + kColAcc + (uint32_t)(slot * P.slot_cols);
-          for (int j = 0; j < W; ++j)
-            for (int ks = 0; ks < ksteps; ++ks) {
-              const uint64_t ad = tc::smem_desc(sbase + kOffA + s * kCodeStage + ks * 32, 16, sbo, sw);
-              const uint64_t bd = tc::smem_desc(sbase + kOffB + j * 4096 + ks * 32, 16, sbo, sw);
-              tc::mma_mxf4nvf4(acc + j * P.Nh, ad, bd, idesc, sfa + ks * 4, tmem + kColSfb + j * 8 + ks * 4,
-                               ks > 0 ? 1u : 0u);
-            }
+          // tile m of the stage (rows m*128 ..) and query column j into the
+          // slot's part (m * W + j) * Nh
+#pragma unroll
+          for (int m = 0; m < kSub; ++m)
+            for (int j = 0; j < W; ++j)
+              for (int ks = 0; ks < ksteps; ++ks) {
+                const uint64_t ad =
+                    tc::smem_desc(sbase + kOffA + s * kCodeStage + m * kTile * row_bytes + ks * 32, 16, sbo, sw);
+                const uint64_t bd = tc::smem_desc(sbase + kOffB + j * 4096 + ks * 32, 16, sbo, sw);
+                tc::mma_mxf4nvf4(acc + (m * W + j) * P.Nh, ad, bd, idesc, sfa + m * 8 + ks * 4,
+                                 tmem + kColSfb + j * 8 + ks * 4, ks > 0 ? 1u : 0u);
+              }
           // one commit: the stage's shared memory and scale factors are free
           // and the slot holds the scores once these MMAs complete
           tc::commit(bar_done + 8 * s);
@@ -520,27 +537,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     int s = 0;
     uint32_t n = 0;
     const int box_rows = kRescore ? kBlock : P.box_rows;
-    const int bshift = box_rows == 128 ? 7 : (box_rows == 64 ? 6 : 3);  // box_rows is 128, 64 or 8
+    const int bshift = __ffs(box_rows) - 1;  // box_rows is a power of two (256, 128, 64 or 8)
     const int slot_bytes = kRescore ? 128 : box_rows * spr;
     for (; ti.valid(); ti.next(P), (++s == kStages ? (s = 0, ++n) : 0u)) {
       if (!warp_wait_or_abort(bar_full + 8 * s, n & 1, P, abort)) break;
       const uint8_t* raw = smem + kOffRaw + s * kRawStage;
-      uint32_t r[8];
+      // tile m of the stage: rows m*128 + m1*32 + lane, columns m*8 ..
+      uint32_t r[kSub][8];
 #pragma unroll
-      for (int m1 = 0; m1 < 4; ++m1) {
-        const int rw = m1 * 32 + lane;
-        const uint8_t* src = raw + (rw >> bshift) * slot_bytes + (rw & (box_rows - 1)) * spr;
-        const uint32_t wv =
-            (spr == 4) ? *reinterpret_cast<const uint32_t*>(src) : (uint32_t)*reinterpret_cast<const uint16_t*>(src);
-        r[m1] = __byte_perm(wv, 0, 0x1100u);      // K step 0: scales 0, 1
-        r[4 + m1] = __byte_perm(wv, 0, 0x3322u);  // K step 1: scales 2, 3
-      }
-      const uint32_t ta = tmem + lane_base + kColSfa + (uint32_t)s * 8;
+      for (int m = 0; m < kSub; ++m)
+#pragma unroll
+        for (int m1 = 0; m1 < 4; ++m1) {
+          const int rw = m * kTile + m1 * 32 + lane;
+          const uint8_t* src = raw + (rw >> bshift) * slot_bytes + (rw & (box_rows - 1)) * spr;
+          const uint32_t wv = (spr == 4) ? *reinterpret_cast<const uint32_t*>(src)
+                                         : (uint32_t)*reinterpret_cast<const uint16_t*>(src);
+          r[m][m1] = __byte_perm(wv, 0, 0x1100u);      // K step 0: scales 0, 1
+          r[m][4 + m1] = __byte_perm(wv, 0, 0x3322u);  // K step 1: scales 2, 3
+        }
+      const uint32_t ta = tmem + lane_base + kColSfa + (uint32_t)s * 8 * kSub;
       if (ksteps == 2) {
-        tc::st_32x32b_x8(ta, r);
+        if (kSub == 2) {
+          const uint32_t r16[16] = {r[0][0], r[0][1], r[0][2], r[0][3], r[0][4], r[0][5], r[0][6], r[0][7],
+                                    r[kSub - 1][0], r[kSub - 1][1], r[kSub - 1][2], r[kSub - 1][3],
+                                    r[kSub - 1][4], r[kSub - 1][5], r[kSub - 1][6], r[kSub - 1][7]};
+          tc::st_32x32b_x16(ta, r16);
+        } else {
+          tc::st_32x32b_x8(ta, r[0]);
+        }
       } else {
-        const uint32_t r4[4] = {r[0], r[1], r[2], r[3]};
-        tc::st_32x32b_x4(ta, r4);
+#pragma unroll
+        for (int m = 0; m < kSub; ++m) {
+          const uint32_t r4[4] = {r[m][0], r[m][1], r[m][2], r[m][3]};
+          tc::st_32x32b_x4(ta + m * 8, r4);
+        }
       }
       tc::st_wait();
       tc::fence_before_sync();
@@ -597,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       tc::fence_after_sync();
-      const int64_t t0 = (int64_t)ti.tile * kTile;
+      const int64_t t0 = (int64_t)ti.tile * kRows;
       const uint32_t taddr0 = tmem + ((uint32_t)(quarter * 32) << 16) + kColAcc + (uint32_t)(slot * P.slot_cols);
       int32_t blk = -1;  // rescore: this thread's pool block
       if (kRescore) {
@@ -605,9 +635,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int np = min(__ldg(P.pool_n + tok0), P.pool_cap);
         blk = (i / kBlock) < np ? __ldg(P.pool + (int64_t)tok0 * P.pool_cap + i / kBlock) : -1;
       }
-      for (int j = 0; j < W; ++j) {
+      for (int mj = 0; mj < kSub * W; ++mj) {  // tile m = mj / W of the stage, query column j = mj % W
+        const int m = kSub == 1 ? 0 : mj / W, j = kSub == 1 ? mj : mj - m * W;
         const float* wj = w_g + j * 64;
-        const uint32_t taddr = taddr0 + j * P.Nh;
+        const uint32_t taddr = taddr0 + mj * P.Nh;
         // the column's scores in two halves of 32 heads (register budget):
         // ReLU and weighted sum in packed pairs (two float2 chains)
         float2 a2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
@@ -619,7 +650,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int g = 0; g < 2; ++g)
             if (hf * 2 + g < ng) tc::ld_32x32b_x16(taddr + (hf * 2 + g) * 16, r[g]);
           tc::ld_wait();
-          if (j == W - 1 && (hf == 1 || ng <= 2)) {  // the slot is free once its last load has landed:
+          if (mj == kSub * W - 1 && (hf == 1 || ng <= 2)) {  // the slot is free once its last load landed:
             tc::fence_before_sync();                 // for the warp issuing its next use
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar_acce + 8 * (slot * 2 + ((it + P.n_slots) & 1)));
@@ -655,7 +686,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (key && lane == __ffs(peers) - 1) atomicAdd(P.hist + orow * kHistBins + bin, (uint32_t)__popc(peers));
           }
         } else {
-          const int64_t t = t0 + row;
+          const int64_t t = t0 + m * kTile + row;
           float sc = (t <= p) ? acc : -INFINITY;
           sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 1));
           sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 2));
@@ -744,15 +775,21 @@ static int num_sms() {
   return n[dev];
 }
 
-template <bool kRescore>
+template <bool kRescore, int kSub>
 static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* const* w,
                            int n_sel, int H, const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n,
                            int pool_cap, float* out, int64_t ld, uint32_t* hist, cudaStream_t st) {
   using namespace scan_tc;
+  using Lay = Layout<kSub>;
+  constexpr int kRows = kTile * kSub;
   if (kc->n_rows >= (int64_t(1) << 31)) return fail(CSA2_ERR_UNSUPPORTED, "cache too large for TMA");
   if (n_sel < 1 || n_sel > kMaxSel) return fail(CSA2_ERR_UNSUPPORTED, "1..%d selector layers per launch", kMaxSel);
-  // scan boxes: 128 rows, or 64 when pages of 64 (or an odd multiple of 64) rows would be crossed
-  const int box_rows = kRescore ? kBlock : (kc->page_table && kc->page_size % 128 != 0 ? 64 : 128);
+  // scan boxes: a stage's rows, or the largest power of two (>= 64) that
+  // does not cross a page
+  int box_rows = kRows;
+  if (!kRescore && kc->page_table)
+    while (box_rows > 64 && kc->page_size % box_rows != 0) box_rows /= 2;
+  if (kRescore) box_rows = kBlock;
   CUtensorMap tmc, tms;
   if (int rc = make_codes_map(&tmc, kc->codes, kc->n_rows, kc->dim / 2, box_rows)) return rc;
   if (int rc = make_scales_map(&tms, kc->scales, kc->n_rows, kc->dim / 32, box_rows)) return rc;
@@ -769,13 +806,15 @@ static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const 
   p.H = H;
   p.Nh = (H + 15) / 16 * 16;
   p.DI = kc->dim;
-  p.slot_cols = wc * p.Nh;
+  p.slot_cols = kSub * wc * p.Nh;
   // accumulator slots: as many as fit, a divisor of the stage count (so that a
   // stage's commit barrier cannot run two phases ahead of a slot's reader)
-  int ns = std::min<int>(6, (int)(kAccCols / p.slot_cols));
-  while (ns > 1 && kStages % ns) --ns;
+  int ns = std::min<int>(6, (int)(Lay::kAccCols / p.slot_cols));
+  while (ns > 1 && Lay::kStages % ns) --ns;
+  if (ns < 1) return fail(CSA2_ERR_UNSUPPORTED, "index accumulators do not fit in TMEM");
   p.n_slots = ns;
   p.box_rows = box_rows;
+  p.rows = kRows;
   p.codes = kc->codes;
   p.scales = kc->scales;
   p.n_rows = kc->n_rows;
@@ -795,26 +834,29 @@ static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const 
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-    if (int rc = cuda_check(
-            cudaFuncSetAttribute(k_index_tc<kRescore>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes),
-            "index smem attribute"))
+    if (int rc = cuda_check(cudaFuncSetAttribute(k_index_tc<kRescore, kSub>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmemBytes),
+                            "index smem attribute"))
       return rc;
     int fit = 0;  // one CTA of kThreads threads at this register count must fit on an SM
-    if (int rc = cuda_check(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, k_index_tc<kRescore>, kThreads,
-                                                                          kSmemBytes),
+    if (int rc = cuda_check(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, k_index_tc<kRescore, kSub>, kThreads,
+                                                                          Lay::kSmemBytes),
                             "index occupancy"))
       return rc;
     if (fit < 1) return fail(CSA2_ERR_UNSUPPORTED, "index kernel does not fit on an SM");
     attr_done[dev] = true;
   }
   Launch L_(kRescore ? "rescore_tc" : "scan_tc", st);
-  k_index_tc<kRescore><<<num_sms(), kThreads, kSmemBytes, st>>>(tmc, tms, p);
+  k_index_tc<kRescore, kSub><<<num_sms(), kThreads, Lay::kSmemBytes, st>>>(tmc, tms, p);
   return cuda_check(cudaGetLastError(), "k_index_tc");
 }
 
 int launch_scan_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,
                    const csa2_fp4_cache* kc, float* bs, int64_t ld, uint32_t* hist, cudaStream_t st) {
-  return launch_index_tc<false>(qb, qc, qs, &w, 1, H, kc, nullptr, nullptr, 0, bs, ld, hist, st);
+  // one query token per sequence: stages of two MMA tiles (256 positions)
+  if (qb->max_q_per_seq <= 1)
+    return launch_index_tc<false, 2>(qb, qc, qs, &w, 1, H, kc, nullptr, nullptr, 0, bs, ld, hist, st);
+  return launch_index_tc<false, 1>(qb, qc, qs, &w, 1, H, kc, nullptr, nullptr, 0, bs, ld, hist, st);
 }
 
 // n_sel selector layers at once: queries [n_sel][T][H][...], weights w[sel],
@@ -822,7 +864,8 @@ int launch_scan_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t*
 int launch_rescore_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* const* w,
                       int n_sel, int H, const csa2_fp4_cache* kc, const int32_t* pool, const int32_t* pool_n, int P,
                       float* scores, uint32_t* hist, cudaStream_t st) {
-  return launch_index_tc<true>(qb, qc, qs, w, n_sel, H, kc, pool, pool_n, P, scores, (int64_t)P * kBlock, hist, st);
+  return launch_index_tc<true, 1>(qb, qc, qs, w, n_sel, H, kc, pool, pool_n, P, scores, (int64_t)P * kBlock, hist,
+                                  st);
 }
 
 }  // namespace csa2
