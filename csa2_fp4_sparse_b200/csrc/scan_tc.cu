@@ -95,6 +95,7 @@ struct Params {
   const float* w[kMaxSel];  // per selector [T][H]
   int n_sel;                // rescore: selector layers (scan: 1)
   int cpg;                  // groups per sequence (scan) or per token (rescore)
+  int wc;                   // query columns per group (<= kMaxWc)
   int H, Nh, DI;            // heads, heads padded to 16 (MMA N per column), key dim
   int slot_cols, n_slots;   // accumulator slots of (query columns x Nh) columns
   int box_rows;             // scan: rows per TMA box (256, 128, or 64 for 64-row pages)
@@ -116,8 +117,8 @@ struct Params {
 };
 
 // Groups: scan group g = (sequence b, chunk c), c < cpg, holds the sequence's
-// query tokens c*kMaxWc ..; rescore group g = (token t, chunk c), c < cpg,
-// holds selectors c*kMaxWc ..
+// query tokens c*wc ..; rescore group g = (token t, chunk c), c < cpg, holds
+// selectors c*wc ..
 template <bool kRescore>
 __device__ __forceinline__ int n_groups(const Params& P) {
   return (kRescore ? P.qb.n_tok : P.qb.n_seq) * P.cpg;
@@ -128,15 +129,15 @@ template <bool kRescore>
 __device__ __forceinline__ void group_info(const Params& P, int g, int* tok0, int* W, int* b, int* sel0) {
   if (kRescore) {
     *tok0 = g / P.cpg;
-    *sel0 = (g % P.cpg) * kMaxWc;
-    *W = max(0, min(kMaxWc, P.n_sel - *sel0));
+    *sel0 = (g % P.cpg) * P.wc;
+    *W = max(0, min(P.wc, P.n_sel - *sel0));
     *b = __ldg(P.qb.tok_seq + *tok0);
   } else {
     *b = g / P.cpg;
     *sel0 = 0;
     const int t_end = __ldg(P.qb.tok_start + *b + 1);
-    *tok0 = __ldg(P.qb.tok_start + *b) + (g % P.cpg) * kMaxWc;
-    *W = max(0, min(kMaxWc, t_end - *tok0));
+    *tok0 = __ldg(P.qb.tok_start + *b) + (g % P.cpg) * P.wc;
+    *W = max(0, min(P.wc, t_end - *tok0));
   }
 }
 
@@ -801,16 +802,26 @@ static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const 
   p.n_sel = n_sel;
   // query columns per group and groups per sequence (scan) or token (rescore)
   const int cols = kRescore ? n_sel : std::max(1, qb->max_q_per_seq);
-  const int wc = std::min(cols, kMaxWc);
-  p.cpg = (cols + kMaxWc - 1) / kMaxWc;
   p.H = H;
   p.Nh = (H + 15) / 16 * 16;
   p.DI = kc->dim;
+  // accumulator slots for wc query columns per group: as many as fit, a
+  // divisor of the stage count (so that a stage's commit barrier cannot run
+  // two phases ahead of a slot's reader)
+  auto slots_for = [&](int wc) {
+    int ns = std::min<int>(6, (int)(Lay::kAccCols / (uint32_t)(kSub * wc * p.Nh)));
+    while (ns > 1 && Lay::kStages % ns) --ns;
+    return ns;
+  };
+  // the widest group that still leaves two accumulator slots (MMAs of one
+  // stage overlap the epilogue of the previous one); one slot only when even
+  // a single column leaves no second
+  int wc = std::min(cols, kMaxWc);
+  while (wc > 1 && slots_for(wc) < 2) --wc;
+  p.wc = wc;
+  p.cpg = (cols + wc - 1) / wc;
   p.slot_cols = kSub * wc * p.Nh;
-  // accumulator slots: as many as fit, a divisor of the stage count (so that a
-  // stage's commit barrier cannot run two phases ahead of a slot's reader)
-  int ns = std::min<int>(6, (int)(Lay::kAccCols / p.slot_cols));
-  while (ns > 1 && Lay::kStages % ns) --ns;
+  const int ns = slots_for(wc);
   if (ns < 1) return fail(CSA2_ERR_UNSUPPORTED, "index accumulators do not fit in TMEM");
   p.n_slots = ns;
   p.box_rows = box_rows;
