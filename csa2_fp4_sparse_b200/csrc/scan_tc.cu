@@ -261,7 +261,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_done + 8 * i, 1);
       mbar_init(bar_sf + 8 * i, 4);
     }
-    for (int i = 0; i < 12; ++i) mbar_init(bar_acce + 8 * i, 4);
+    // every epilogue unit of a stage (one MMA tile x query column) arrives
+    // from its four warps; a stage with fewer units than the launch's widest
+    // group weights its last unit's arrivals
+    for (int i = 0; i < 12; ++i) mbar_init(bar_acce + 8 * i, 4 * kSub * P.wc);
     mbar_init(bar_drain, 1);
     mbar_init(bar_drain + 8, 1);
     mbar_init(bar_sfb, 1);
@@ -588,7 +591,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     int64_t* pos_g = reinterpret_cast<int64_t*>(smem + kOffPos) + wg * kMaxWc;
     TileIter<kRescore> ti;
     ti.init(P, wb, we);
-    int it = 0, s = 0, slot = 0, wgc = 0;  // stage count, ring stage, slot, warpgroup of the stage
+    // stage count, ring stage, slot, first warpgroup of the stage.  A scan
+    // stage's units (its MMA tiles x query columns) are split between its
+    // warpgroup wgc (the first half) and the next one (the rest), so that the
+    // tiles of one stage are reduced in parallel.  Every warpgroup takes
+    // part in every third stage, so before it waits for a stage's commit it
+    // has seen the commit of a stage of the same MMA warp at most six stages
+    // back: the barrier cannot be a phase behind the one waited for.
+    int it = 0, s = 0, slot = 0, wgc = 0;
     uint32_t n = 0;
     auto adv = [&]() {
       ++it;
@@ -617,7 +627,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ept < W) pos_g[ept] = __ldg(P.qb.tok_pos + (kRescore ? tok0 : tok0 + ept));
         tc::named_sync(1 + wg, 128);
       }
-      if (wgc != wg || dead) continue;  // another warpgroup's stage (or nothing left to do)
+      // units of this stage; rescoring keeps a stage's units on one
+      // warpgroup (its units share the gathered block ids; measured faster)
+      const int nu = kSub * W, half = kRescore ? nu : (nu + 1) / 2;
+      int mj0 = 0, mj1 = 0;  // this warpgroup's units
+      if (wgc == wg) {
+        mj1 = half;
+      } else if (wgc + 1 == wg || wgc + 1 == wg + kEpiWG) {
+        mj0 = half;
+        mj1 = nu;
+      }
+      if (mj0 >= mj1 || dead) continue;  // no unit of this stage (or nothing left to do)
       // one prober per warpgroup; the other warps park on the named barrier
       if (!mbar_wait_group(bar_done + 8 * s, n & 1, P.wait_ns, ept == 0, *abort != 0, 1 + wg, 128)) {
         if (ept == 0 && !*abort) {
@@ -636,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int np = min(__ldg(P.pool_n + tok0), P.pool_cap);
         blk = (i / kBlock) < np ? __ldg(P.pool + (int64_t)tok0 * P.pool_cap + i / kBlock) : -1;
       }
-      for (int mj = 0; mj < kSub * W; ++mj) {  // tile m = mj / W of the stage, query column j = mj % W
+      for (int mj = mj0; mj < mj1; ++mj) {  // unit: tile m = mj / W of the stage, query column j = mj % W
         const int m = kSub == 1 ? 0 : mj / W, j = kSub == 1 ? mj : mj - m * W;
         const float* wj = w_g + j * 64;
         const uint32_t taddr = taddr0 + mj * P.Nh;
@@ -651,10 +671,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int g = 0; g < 2; ++g)
             if (hf * 2 + g < ng) tc::ld_32x32b_x16(taddr + (hf * 2 + g) * 16, r[g]);
           tc::ld_wait();
-          if (mj == kSub * W - 1 && (hf == 1 || ng <= 2)) {  // the slot is free once its last load landed:
-            tc::fence_before_sync();                 // for the warp issuing its next use
+          if (hf == 1 || ng <= 2) {  // this unit's part of the slot is read once its last load landed:
+            tc::fence_before_sync();  // for the warp issuing the slot's next use
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(bar_acce + 8 * (slot * 2 + ((it + P.n_slots) & 1)));
+            if (lane == 0)
+              tc::mbar_arrive_cnt(bar_acce + 8 * (slot * 2 + ((it + P.n_slots) & 1)),
+                                  mj == nu - 1 ? (uint32_t)(1 + kSub * P.wc - nu) : 1u);
           }
 #pragma unroll
           for (int g = 0; g < 2; ++g)
