@@ -67,7 +67,7 @@ constexpr uint32_t kTmemCols = 512;
 // The stage ring is even (producer and MMA warps take stages in turn).
 template <int kSub>
 struct Layout {
-  static constexpr int kStages = kSub == 2 ? 10 : 18;
+  static constexpr int kStages = kSub == 2 ? 6 : 12;
   static constexpr uint32_t kCodeStage = 8192u * kSub;               // kSub x 128 rows x <= 64 B
   static constexpr uint32_t kRawStage = kSub == 2 ? 1024u : 2048u;    // raw scales (rescoring: 16 boxes at 128 B)
   static constexpr uint32_t kColSfa = 0;                             // [kStages][kSub][8]
@@ -839,7 +839,12 @@ static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const 
   // stage overlap the epilogue of the previous one); one slot only when even
   // a single column leaves no second
   int wc = std::min(cols, kMaxWc);
-  while (wc > 1 && slots_for(wc) < 2) --wc;
+  // rescoring with plenty of stages per CTA: the widest group (every pool
+  // block gathered once for up to four selectors) even with one slot; the
+  // gathers, not the epilogue, bound it there
+  const bool wide = kRescore && (int64_t)qb->n_tok * ((int64_t)pool_cap * kBlock / kRows) >= 4ll * num_sms();
+  if (!wide)
+    while (wc > 1 && slots_for(wc) < 2) --wc;
   p.wc = wc;
   p.cpg = (cols + wc - 1) / wc;
   p.slot_cols = kSub * wc * p.Nh;
