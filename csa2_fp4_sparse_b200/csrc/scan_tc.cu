@@ -306,6 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     int cur_g = -1, tok0 = 0, b = 0;
     int64_t base = 0, len = 0;
+    const uint64_t l2_ef = tc::l2_policy_evict_first();
     for (; ti.valid(); ti.next(P), adv()) {
       if ((it & 1) != pw || *abort) continue;
       if (lane == 0) {
@@ -377,10 +378,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (pos0 >= 0) {
           set_status(P.status, CSA2_ERR_RANGE);
         }
-        tc::tma_load_2d(sbase + kOffA + s * kCodeStage + lane * box_rows * row_bytes, &tm_codes, bar_full + 8 * s, 0,
-                        ry);
+        tc::tma_load_2d_hint(sbase + kOffA + s * kCodeStage + lane * box_rows * row_bytes, &tm_codes, bar_full + 8 * s,
+                             0, ry, l2_ef);
         const uint32_t slot = (uint32_t)(box_rows * spr);
-        tc::tma_load_2d(sbase + kOffRaw + s * kRawStage + lane * slot, &tm_scales, bar_full + 8 * s, 0, sy);
+        tc::tma_load_2d_hint(sbase + kOffRaw + s * kRawStage + lane * slot, &tm_scales, bar_full + 8 * s, 0, sy, l2_ef);
       }
       __syncwarp();
     }

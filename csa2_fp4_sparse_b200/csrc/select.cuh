@@ -525,14 +525,16 @@ __global__ void __launch_bounds__(kSelThreads) k_select_cluster(const __grid_con
       if (fits) {
         for (int i = threadIdx.x; i < m; i += kSelThreads) f(cand[i].x, cand[i].y);
       } else {
-        for (int t = 0; t < n; t += kSelTile) {
-          uint32_t k[kSelPer];
-          sel_load_tile(sc, t, n, k);
-          const int wbase = t + wid * kSelWarpSpan + lane;
-#pragma unroll
-          for (int j = 0; j < kSelPer; ++j)
-            if (k[j] != 0u && (k[j] >> kHistShift) == ub1) f(k[j], (uint32_t)(wbase + j * 32));
-        }
+        // (a rare path: rolled, one key at a time)
+        const int wbase = wid * kSelWarpSpan + lane;
+#pragma unroll 1
+        for (int t = 0; t < n; t += kSelTile)
+#pragma unroll 1
+          for (int j = 0; j < kSelPer; ++j) {
+            const int i = t + wbase + j * 32;
+            const uint32_t key = i < n ? score_key(__ldg(sc + i)) : 0u;
+            if (key != 0u && (key >> kHistShift) == ub1) f(key, (uint32_t)i);
+          }
       }
     };
     // digit 2: key bits 19..8
@@ -579,18 +581,21 @@ __global__ void __launch_bounds__(kSelThreads) k_select_cluster(const __grid_con
   __syncthreads();
 
   // ---- C: bitmaps -> ascending ids; position of a selected id = selected
-  // ids before it + min(ties before it, need_eq)
+  // ids before it + min(ties before it, need_eq).  A thread takes wpt
+  // consecutive words (1..8: every thread busy on short lists)
   int32_t* o = P.out + g * P.k_out;
   const int words_n = (n + 31) / 32;
+  const int wpt = min(8, max(1, (words_n + kSelThreads - 1) / kSelThreads));
   int run_sel = 0, run_tie = 0, bad = 0;
-  for (int w0 = 0; w0 < words_n; w0 += kSelThreads * 8) {
-    const int wi = w0 + (int)threadIdx.x * 8;
+  for (int w0 = 0; w0 < words_n; w0 += kSelThreads * wpt) {
+    const int wi = w0 + (int)threadIdx.x * wpt;
     uint32_t sw[8], tw[8];
     int cs = 0, ct = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      sw[j] = wi + j < words_n ? bsel[wi + j] : 0u;
-      tw[j] = (need_eq > 0 && wi + j < words_n) ? btie[wi + j] : 0u;
+      const bool in = j < wpt && wi + j < words_n;
+      sw[j] = in ? bsel[wi + j] : 0u;
+      tw[j] = (need_eq > 0 && in) ? btie[wi + j] : 0u;
       if (wi + j == words_n - 1 && (n & 31)) {  // ids past n: not candidates
         sw[j] &= (1u << (n & 31)) - 1u;
         tw[j] &= (1u << (n & 31)) - 1u;
