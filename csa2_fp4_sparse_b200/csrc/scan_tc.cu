@@ -622,8 +622,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         group_info<kRescore>(P, cur_g, &tok0, &W, &bseq, &sel0);
         for (int e = ept; e < W * 64; e += 128) {
           const int j = e / 64, h = e % 64;
-          w_g[e] = h < P.H ? __ldg(P.w[kRescore ? sel0 + j : 0] + (int64_t)(kRescore ? tok0 : tok0 + j) * P.H + h)
-                           : 0.0f;
+          // half weights: the epilogue's ReLU is s + |s| = 2 max(s, 0)
+          const float* wsrc = P.w[kRescore ? sel0 + j : 0] + (int64_t)(kRescore ? tok0 : tok0 + j) * P.H;
+          w_g[e] = h < P.H ? 0.5f * __ldg(wsrc + h) : 0.0f;
         }
         if (ept < W) pos_g[ept] = __ldg(P.qb.tok_pos + (kRescore ? tok0 : tok0 + ept));
         tc::named_sync(1 + wg, 128);
@@ -662,8 +663,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float* wj = w_g + j * 64;
         const uint32_t taddr = taddr0 + mj * P.Nh;
         // the column's scores in two halves of 32 heads (register budget):
-        // ReLU and weighted sum in packed pairs (two float2 chains)
-        float2 a2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+        // weighted sum in packed pairs (four float2 chains).  ReLU as
+        // s + |s| (an add on the FMA pipe, which the epilogue leaves idle,
+        // instead of a max on the busier ALU pipe) against half weights:
+        // (w/2)(2s) is w*s exactly, so every product is w*max(s, 0)
+        float2 a2[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
+                        make_float2(0.0f, 0.0f)};
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           if (hf * 2 >= ng) break;
@@ -685,16 +690,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int k4 = 0; k4 < 4; ++k4) {
                 const float4 w4 = *reinterpret_cast<const float4*>(wj + (hf * 2 + g) * 16 + k4 * 4);
-                const float2 x0 = make_float2(fmaxf(__uint_as_float(r[g][k4 * 4 + 0]), 0.0f),
-                                              fmaxf(__uint_as_float(r[g][k4 * 4 + 1]), 0.0f));
-                const float2 x1 = make_float2(fmaxf(__uint_as_float(r[g][k4 * 4 + 2]), 0.0f),
-                                              fmaxf(__uint_as_float(r[g][k4 * 4 + 3]), 0.0f));
-                a2[0] = __ffma2_rn(make_float2(w4.x, w4.y), x0, a2[0]);
-                a2[1] = __ffma2_rn(make_float2(w4.z, w4.w), x1, a2[1]);
+                const float s0 = __uint_as_float(r[g][k4 * 4 + 0]), s1 = __uint_as_float(r[g][k4 * 4 + 1]);
+                const float s2 = __uint_as_float(r[g][k4 * 4 + 2]), s3 = __uint_as_float(r[g][k4 * 4 + 3]);
+                const float2 x0 = make_float2(s0 + fabsf(s0), s1 + fabsf(s1));
+                const float2 x1 = make_float2(s2 + fabsf(s2), s3 + fabsf(s3));
+                a2[2 * g] = __ffma2_rn(make_float2(w4.x, w4.y), x0, a2[2 * g]);
+                a2[2 * g + 1] = __ffma2_rn(make_float2(w4.z, w4.w), x1, a2[2 * g + 1]);
               }
             }
         }
-        const float acc = (a2[0].x + a2[1].x) + (a2[0].y + a2[1].y);
+        const float acc = ((a2[0].x + a2[1].x) + (a2[0].y + a2[1].y)) + ((a2[2].x + a2[3].x) + (a2[2].y + a2[3].y));
         const int64_t p = pos_g[kRescore ? 0 : j];
         if (kRescore) {
           // pool entry i = tile*128 + row: position pool[i/8]*8 + i%8

@@ -62,6 +62,10 @@ CONFIGS = {
     5: Config("swa_verify", 5, B=64, H_I=64, d_I=128, P=2048, K=512, Hq=64, D=512, n_reindex=3,
               n_reuse=16, lengths=("loguniform", 4096, 524288), widths=("uniform", 1, 6), swa=True,
               n_needles=32),
+    # chunked prefill: a 256-token chunk appended to each of two 128K
+    # contexts; every chunk token selects its own pool and top-K
+    6: Config("chunked_prefill", 6, B=2, H_I=64, d_I=128, P=2048, K=512, Hq=64, D=512, n_reindex=3,
+              n_reuse=16, lengths=("fixed", 131072), widths=("fixed", 256), n_needles=32),
 }
 
 

@@ -143,7 +143,7 @@ def test_stack_config1_full_size():
     _check_all(w, dw, range(w.T))
 
 
-@pytest.mark.parametrize("i", [2, 3, 4, 5])
+@pytest.mark.parametrize("i", [2, 3, 4, 5, 6])
 def test_stack_full_size_sampled(i):
     """The full-size workloads the benchmark times (same kernels and grids),
     graded on sampled query tokens: the first, the last and two seeded picks,
