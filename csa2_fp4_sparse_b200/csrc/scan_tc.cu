@@ -80,7 +80,11 @@ struct Layout {
   static constexpr uint32_t kOffSfb = kOffB + kMaxWc * 4096;         // [kMaxWc][2][512]
   static constexpr uint32_t kOffW = kOffSfb + kMaxWc * 1024;         // [kEpiWG][kMaxWc][64] f32
   static constexpr uint32_t kOffPos = kOffW + kEpiWG * kMaxWc * 64 * 4;  // [kEpiWG][kMaxWc] i64 query positions
-  static constexpr uint32_t kOffBar = kOffPos + kEpiWG * kMaxWc * 8;
+  // key counts of the current group, [query column][kHistBins] (a two-tile
+  // stage serves one query column)
+  static constexpr int kHistCols = kSub == 2 ? 1 : kMaxWc;
+  static constexpr uint32_t kOffHist = kOffPos + kEpiWG * kMaxWc * 8;
+  static constexpr uint32_t kOffBar = kOffHist + kHistCols * kHistBins * 4;
   static constexpr uint32_t kNumBars = 3 * kStages + 12 + 3;  // full, done, sf; acc_empty[6][2]; drain[2], sfb
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;      // tmem base, abort flag
   static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;      // + alignment slack
@@ -232,7 +236,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kCodeStage = Lay::kCodeStage, kRawStage = Lay::kRawStage, kColSfa = Lay::kColSfa,
                      kColSfb = Lay::kColSfb, kColAcc = Lay::kColAcc, kOffA = Lay::kOffA, kOffRaw = Lay::kOffRaw,
                      kOffB = Lay::kOffB, kOffSfb = Lay::kOffSfb, kOffW = Lay::kOffW, kOffPos = Lay::kOffPos,
-                     kOffBar = Lay::kOffBar, kOffMisc = Lay::kOffMisc;
+                     kOffBar = Lay::kOffBar, kOffMisc = Lay::kOffMisc, kOffHist = Lay::kOffHist;
+  constexpr int kHistCols = Lay::kHistCols;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -278,6 +283,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::tmem_relinquish();
     tc::fence_before_sync();
   }
+  uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + kOffHist);
+  for (int i = threadIdx.x; i < kHistCols * kHistBins; i += kThreads) hist_s[i] = 0u;
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_holder;
@@ -613,10 +620,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     int cur_g = -1, W = 0, tok0 = 0, sel0 = 0;
     bool dead = false;  // warpgroup-uniform: a wait of this warpgroup gave up
     const int ng = P.Nh / 16;
-    // no early exit: the four warps of the warpgroup meet at named barriers
+    // The group's key counts gather in shared memory (per CTA) and go to the
+    // global counts, one atomic per non-empty bin, when the CTA leaves the
+    // group: every SM adding each score to one group's global bins directly
+    // contended on the few bins that hold most scores
+    constexpr int kEpiThreads = 128 * kEpiWG;
+    const int et = threadIdx.x - kEpi0 * 32;  // 0 .. kEpiThreads-1
+    auto flush_counts = [&]() {
+      for (int i = et; i < W * kHistBins; i += kEpiThreads) {
+        const uint32_t v = hist_s[i];
+        if (v) {
+          const int j = i / kHistBins;
+          const int64_t grow = kRescore ? (int64_t)(sel0 + j) * P.qb.n_tok + tok0 : (int64_t)(tok0 + j);
+          atomicAdd(P.hist + grow * kHistBins + (i % kHistBins), v);
+          hist_s[i] = 0u;
+        }
+      }
+    };
+    // no early exit: the warps of the epilogue meet at named barriers
     for (; ti.valid(); ti.next(P), adv()) {
       if (ti.b != cur_g) {
-        tc::named_sync(1 + wg, 128);
+        tc::named_sync(7, kEpiThreads);  // every epilogue warp is done with the old group
+        if (P.hist && cur_g >= 0) {
+          flush_counts();
+          tc::named_sync(7, kEpiThreads);
+        }
         cur_g = ti.b;
         int bseq;
         group_info<kRescore>(P, cur_g, &tok0, &W, &bseq, &sel0);
@@ -659,7 +687,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         blk = (i / kBlock) < np ? __ldg(P.pool + (int64_t)tok0 * P.pool_cap + i / kBlock) : -1;
       }
       for (int mj = mj0; mj < mj1; ++mj) {  // unit: tile m = mj / W of the stage, query column j = mj % W
-        const int m = kSub == 1 ? 0 : mj / W, j = kSub == 1 ? mj : mj - m * W;
+        // two-tile stages only serve one query token per sequence (W = 1)
+        const int m = kSub == 1 ? 0 : mj, j = kSub == 1 ? mj : 0;
         const float* wj = w_g + j * 64;
         const uint32_t taddr = taddr0 + mj * P.Nh;
         // the column's scores in two halves of 32 heads (register budget):
@@ -708,11 +737,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int64_t orow = (int64_t)(sel0 + j) * P.qb.n_tok + tok0;  // selector * T + token
           const bool valid = blk >= 0 && pos <= p && i < P.pool_cap * kBlock;
           if (i < P.pool_cap * kBlock) P.out[orow * P.ld + i] = valid ? acc : -INFINITY;
-          if (P.hist) {  // one count per distinct bin of the warp
-            const uint32_t key = valid ? score_key(acc) : 0u;
-            const uint32_t bin = key ? key >> kHistShift : 0xFFFFFFFFu;
-            const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-            if (key && lane == __ffs(peers) - 1) atomicAdd(P.hist + orow * kHistBins + bin, (uint32_t)__popc(peers));
+          if (P.hist && valid) {
+            const uint32_t key = score_key(acc);
+            if (key) atomicAdd(hist_s + j * kHistBins + (key >> kHistShift), 1u);
           }
         } else {
           const int64_t t = t0 + m * kTile + row;
@@ -723,11 +750,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if ((lane & 7) == 0 && t <= p) {
             P.out[(int64_t)(tok0 + j) * P.ld + t / kBlock] = sc;
             const uint32_t key = score_key(sc);
-            if (P.hist && key) atomicAdd(P.hist + (int64_t)(tok0 + j) * kHistBins + (key >> kHistShift), 1u);
+            if (P.hist && key) atomicAdd(hist_s + j * kHistBins + (key >> kHistShift), 1u);
           }
         }
       }
     }
+    tc::named_sync(7, kEpiThreads);  // the last group's counts are complete
+    if (P.hist && cur_g >= 0) flush_counts();
   }
   // after a failed wait some tile loads may still be in flight: give them
   // time to land before the CTA's shared memory is released (bounded)
