@@ -503,9 +503,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every other use (odd count: the parity of the slot's stages alternates)
       const uint32_t ph = (P.n_slots & 1) ? (u - 1) >> 1 : u - 1;
       if (lane == 0) {
-        bool ok = wait_or_abort(bar_full + 8 * s, n & 1, P, abort);      // codes landed
-        if (ok) ok = wait_or_abort(bar_sf + 8 * s, n & 1, P, abort);     // scale factors in TMEM
-        if (ok && u > 0) ok = wait_or_abort(bar_acce + 8 * (slot * 2 + mw), ph & 1, P, abort);  // slot read
+        // the three conditions probed together first (their latencies
+        // overlap); a bounded wait on each only when one is not yet met
+        const uint32_t b_acce = bar_acce + 8 * (slot * 2 + mw);
+        const bool r0 = mbar_try_wait(bar_full + 8 * s, n & 1);
+        const bool r1 = mbar_try_wait(bar_sf + 8 * s, n & 1);
+        const bool r2 = u == 0 || mbar_try_wait(b_acce, ph & 1);
+        bool ok = r0 && r1 && r2 && !*abort;
+        if (!ok) {
+          ok = wait_or_abort(bar_full + 8 * s, n & 1, P, abort);                    // codes landed
+          if (ok) ok = wait_or_abort(bar_sf + 8 * s, n & 1, P, abort);              // scale factors in TMEM
+          if (ok && u > 0) ok = wait_or_abort(b_acce, ph & 1, P, abort);            // slot read
+        }
         if (ok) {
           tc::fence_after_sync();
           if (kRescore) tc::fence_proxy_async_smem();  // codes written by cp.async (generic proxy)
@@ -551,22 +560,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int box_rows = kRescore ? kBlock : P.box_rows;
     const int bshift = __ffs(box_rows) - 1;  // box_rows is a power of two (256, 128, 64 or 8)
     const int slot_bytes = kRescore ? 128 : box_rows * spr;
+    const bool one_box4 = !kRescore && box_rows >= kRows && spr == 4;
     for (; ti.valid(); ti.next(P), (++s == kStages ? (s = 0, ++n) : 0u)) {
       if (!warp_wait_or_abort(bar_full + 8 * s, n & 1, P, abort)) break;
       const uint8_t* raw = smem + kOffRaw + s * kRawStage;
       // tile m of the stage: rows m*128 + m1*32 + lane, columns m*8 ..
       uint32_t r[kSub][8];
+      if (one_box4) {  // the stage's scales are one [rows][4] array: word rw is row rw's
+        const uint32_t* raw32 = reinterpret_cast<const uint32_t*>(raw) + lane;
 #pragma unroll
-      for (int m = 0; m < kSub; ++m)
+        for (int m = 0; m < kSub; ++m)
 #pragma unroll
-        for (int m1 = 0; m1 < 4; ++m1) {
-          const int rw = m * kTile + m1 * 32 + lane;
-          const uint8_t* src = raw + (rw >> bshift) * slot_bytes + (rw & (box_rows - 1)) * spr;
-          const uint32_t wv = (spr == 4) ? *reinterpret_cast<const uint32_t*>(src)
-                                         : (uint32_t)*reinterpret_cast<const uint16_t*>(src);
-          r[m][m1] = __byte_perm(wv, 0, 0x1100u);      // K step 0: scales 0, 1
-          r[m][4 + m1] = __byte_perm(wv, 0, 0x3322u);  // K step 1: scales 2, 3
-        }
+          for (int m1 = 0; m1 < 4; ++m1) {
+            const uint32_t wv = raw32[m * kTile + m1 * 32];
+            r[m][m1] = __byte_perm(wv, 0, 0x1100u);      // K step 0: scales 0, 1
+            r[m][4 + m1] = __byte_perm(wv, 0, 0x3322u);  // K step 1: scales 2, 3
+          }
+      } else {
+#pragma unroll
+        for (int m = 0; m < kSub; ++m)
+#pragma unroll
+          for (int m1 = 0; m1 < 4; ++m1) {
+            const int rw = m * kTile + m1 * 32 + lane;
+            const uint8_t* src = raw + (rw >> bshift) * slot_bytes + (rw & (box_rows - 1)) * spr;
+            const uint32_t wv = (spr == 4) ? *reinterpret_cast<const uint32_t*>(src)
+                                           : (uint32_t)*reinterpret_cast<const uint16_t*>(src);
+            r[m][m1] = __byte_perm(wv, 0, 0x1100u);      // K step 0: scales 0, 1
+            r[m][4 + m1] = __byte_perm(wv, 0, 0x3322u);  // K step 1: scales 2, 3
+          }
+      }
       const uint32_t ta = tmem + lane_base + kColSfa + (uint32_t)s * 8 * kSub;
       if (ksteps == 2) {
         if (kSub == 2) {
@@ -618,7 +640,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (++wgc == kEpiWG) wgc = 0;
     };
     int cur_g = -1, W = 0, tok0 = 0, sel0 = 0;
-    bool dead = false;  // warpgroup-uniform: a wait of this warpgroup gave up
+    bool dead = false;  // a wait of this warp (two-tile stages) or warpgroup gave up
     const int ng = P.Nh / 16;
     // The group's key counts gather in shared memory (per CTA) and go to the
     // global counts, one atomic per non-empty bin, when the CTA leaves the
@@ -668,9 +690,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         mj1 = nu;
       }
       if (mj0 >= mj1 || dead) continue;  // no unit of this stage (or nothing left to do)
-      // one prober per warpgroup; the other warps park on the named barrier
-      if (!mbar_wait_group(bar_done + 8 * s, n & 1, P.wait_ns, ept == 0, *abort != 0, 1 + wg, 128)) {
-        if (ept == 0 && !*abort) {
+      // two-tile stages: every warp probes for itself (measured faster);
+      // otherwise one prober per warpgroup, the other warps parked on the
+      // named barrier
+      const uint32_t b_done = bar_done + 8 * s;
+      const bool got = kSub == 2 ? (*abort == 0 && mbar_wait_warp(b_done, n & 1, P.wait_ns))
+                                 : mbar_wait_group(b_done, n & 1, P.wait_ns, ept == 0, *abort != 0, 1 + wg, 128);
+      if (!got) {
+        if ((kSub == 2 ? lane : ept) == 0 && !*abort) {
           set_status(P.status, CSA2_ERR_TIMEOUT);
           *abort = 1;
         }
