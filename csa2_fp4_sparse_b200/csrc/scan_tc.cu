@@ -157,13 +157,53 @@ __device__ __forceinline__ int group_tiles(const Params& P, int g) {
   return (int)((max(vis, (int64_t)0) + P.rows - 1) / P.rows);
 }
 
-// this CTA's contiguous range of (group, stage) work in group-major order
+// This CTA's contiguous range of (group, stage) work in group-major order,
+// found by all threads of the CTA together: each sums the stages of a run of
+// consecutive groups, a block scan places the runs, and the thread whose run
+// holds the CTA's first stage finds its group (a serial walk over every group
+// cost up to a dependent load chain per group).  Results in shared memory:
+// first group, first stage in it, number of stages (0: no work).
 template <bool kRescore>
-__device__ __forceinline__ void work_range(const Params& P, int64_t* begin, int64_t* end) {
-  int64_t total = 0;
-  for (int g = 0; g < n_groups<kRescore>(P); ++g) total += group_tiles<kRescore>(P, g);
-  *begin = total * blockIdx.x / gridDim.x;
-  *end = total * (blockIdx.x + 1) / gridDim.x;
+__device__ void work_start(const Params& P, long long* s_wsum, int* s_g0, int* s_t0, long long* s_n) {
+  const int ng = n_groups<kRescore>(P);
+  const int per = (ng + kThreads - 1) / kThreads;
+  const int g_lo = min(ng, (int)threadIdx.x * per), g_hi = min(ng, g_lo + per);
+  long long mine = 0;
+  for (int g = g_lo; g < g_hi; ++g) mine += group_tiles<kRescore>(P, g);
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  long long incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) s_wsum[wid] = incl;
+  if (threadIdx.x == 0) {
+    *s_g0 = 0;
+    *s_t0 = 0;
+  }
+  __syncthreads();
+  long long before = 0, total = 0;
+  for (int w = 0; w < kThreads / 32; ++w) {
+    const long long v = s_wsum[w];
+    if (w < wid) before += v;
+    total += v;
+  }
+  const long long excl = before + incl - mine;
+  const long long begin = total * blockIdx.x / gridDim.x, end = total * (blockIdx.x + 1) / gridDim.x;
+  if (mine > 0 && begin < end && excl <= begin && begin < excl + mine) {  // one thread
+    long long acc = excl;
+    int g = g_lo;
+    for (; g < g_hi - 1; ++g) {
+      const int t = group_tiles<kRescore>(P, g);
+      if (acc + t > begin) break;
+      acc += t;
+    }
+    *s_g0 = g;
+    *s_t0 = (int)(begin - acc);
+  }
+  if (threadIdx.x == 0) *s_n = end - begin;
+  __syncthreads();
 }
 
 // iterator over the stages of [begin, end)
@@ -171,18 +211,12 @@ template <bool kRescore>
 struct TileIter {
   int b, tile, ntile;  // b: group
   int64_t left;
-  __device__ void init(const Params& P, int64_t begin, int64_t end) {
-    b = 0;
-    int64_t acc = 0;
-    const int ng = n_groups<kRescore>(P);
-    ntile = group_tiles<kRescore>(P, 0);
-    while (b < ng - 1 && acc + ntile <= begin) {
-      acc += ntile;
-      ++b;
-      ntile = group_tiles<kRescore>(P, b);
-    }
-    tile = (int)(begin - acc);
-    left = end - begin;
+  // start at stage t0 of group g0 (from work_start), n stages in all
+  __device__ void init(const Params& P, int g0, int t0, int64_t n) {
+    b = g0;
+    tile = t0;
+    left = n;
+    ntile = n > 0 ? group_tiles<kRescore>(P, g0) : 0;
   }
   __device__ bool valid() const { return left > 0; }
   __device__ void next(const Params& P) {
@@ -289,8 +323,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_holder;
 
-  int64_t wb, we;
-  work_range<kRescore>(P, &wb, &we);
+  __shared__ long long s_wsum[kThreads / 32], s_nwork;
+  __shared__ int s_g0, s_t0;
+  work_start<kRescore>(P, s_wsum, &s_g0, &s_t0, &s_nwork);
+  const int w_g0 = s_g0, w_t0 = s_t0;
+  const int64_t w_n = s_nwork;
 
   if (warp < kMma0) {
     // ------------------------------------------------------------ producers
@@ -301,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nbox = kRescore ? 16 : kRows / box_rows;
     const uint32_t tx = (uint32_t)kRows * row_bytes + (uint32_t)kRows * spr;
     TileIter<kRescore> ti;
-    ti.init(P, wb, we);
+    ti.init(P, w_g0, w_t0, w_n);
     int it = 0, s = 0;  // this CTA's stage count, ring stage
     uint32_t n = 0;     // use of the ring stage
     auto adv = [&]() {
@@ -405,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const tc::SmemLayout sw = (P.DI == 128) ? tc::kSwizzle64B : tc::kSwizzle32B;
     const uint32_t sbo = 8u * row_bytes;  // 8 rows per swizzle atom
     TileIter<kRescore> ti;
-    ti.init(P, wb, we);
+    ti.init(P, w_g0, w_t0, w_n);
     int it = 0, s = 0, slot = 0;  // stage count, ring stage, accumulator slot
     uint32_t n = 0, u = 0;        // uses of the ring stage and of the slot
     auto adv = [&]() {
@@ -554,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     TileIter<kRescore> ti;
-    ti.init(P, wb, we);
+    ti.init(P, w_g0, w_t0, w_n);
     int s = 0;
     uint32_t n = 0;
     const int box_rows = kRescore ? kBlock : P.box_rows;
@@ -620,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* w_g = reinterpret_cast<float*>(smem + kOffW) + wg * kMaxWc * 64;
     int64_t* pos_g = reinterpret_cast<int64_t*>(smem + kOffPos) + wg * kMaxWc;
     TileIter<kRescore> ti;
-    ti.init(P, wb, we);
+    ti.init(P, w_g0, w_t0, w_n);
     // stage count, ring stage, slot, first warpgroup of the stage.  A scan
     // stage's units (its MMA tiles x query columns) are split between its
     // warpgroup wgc (the first half) and the next one (the rest), so that the
