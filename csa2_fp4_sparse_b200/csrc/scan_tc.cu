@@ -658,10 +658,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     int64_t* pos_g = reinterpret_cast<int64_t*>(smem + kOffPos) + wg * kMaxWc;
     TileIter<kRescore> ti;
     ti.init(P, w_g0, w_t0, w_n);
-    // stage count, ring stage, slot, first warpgroup of the stage.  A scan
-    // stage's units (its MMA tiles x query columns) are split between its
-    // warpgroup wgc (the first half) and the next one (the rest), so that the
-    // tiles of one stage are reduced in parallel.  Every warpgroup takes
+    // stage count, ring stage, slot, first warpgroup of the stage.  A stage's
+    // units (its MMA tiles x query columns) are split between its warpgroup
+    // wgc (the first half) and the next one (the rest), so that they are
+    // reduced in parallel.  Every warpgroup takes
     // part in every third stage, so before it waits for a stage's commit it
     // has seen the commit of a stage of the same MMA warp at most six stages
     // back: the barrier cannot be a phase behind the one waited for.
@@ -716,9 +716,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ept < W) pos_g[ept] = __ldg(P.qb.tok_pos + (kRescore ? tok0 : tok0 + ept));
         tc::named_sync(1 + wg, 128);
       }
-      // units of this stage; rescoring keeps a stage's units on one
-      // warpgroup (its units share the gathered block ids; measured faster)
-      const int nu = kSub * W, half = kRescore ? nu : (nu + 1) / 2;
+      // units of this stage, the first half to warpgroup wgc, the rest to the
+      // next (with one accumulator slot, as in rescoring four selectors at a
+      // time, the slot is free once both halves are read: half the wait)
+      const int nu = kSub * W, half = (nu + 1) / 2;
       int mj0 = 0, mj1 = 0;  // this warpgroup's units
       if (wgc == wg) {
         mj1 = half;
