@@ -422,7 +422,9 @@ __device__ __forceinline__ void sel_scan2(int a, int b, int* sh, int* ea, int* e
 }
 
 // grid (S, T, n_sel), clusters of (S, 1, 1); dynamic shared memory SelCLayout
-__global__ void __launch_bounds__(kSelThreads) k_select_cluster(const __grid_constant__ SelCParams P) {
+// (at most 64 registers: two CTAs of a launch with more groups than SMs
+// share an SM, one's serial phases hiding the other's)
+__global__ void __launch_bounds__(kSelThreads, 2) k_select_cluster(const __grid_constant__ SelCParams P) {
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ int hist_s[kHistBins];
   __shared__ int sh[2 * kSelWarps + 4];
