@@ -11,18 +11,21 @@
 // rescore only the pool).
 //
 // Work: one persistent CTA per SM walks a contiguous range of (group, stage)
-// items.  A stage is 128 positions of the FP4 indexer K cache; a group is up
-// to four "query columns" that share its stages: the scan's group is up to
-// four query tokens of one sequence (one pass over the sequence's keys per
-// group), the rescoring's group is one query token and up to four selector
-// layers (the token's pool is gathered once for all of them).
+// items (its first item found by all threads with a block scan over the
+// groups' stage counts).  A stage is 256 positions of the FP4 indexer K cache
+// (two 128-row MMA tiles) when every sequence has one query token, else 128
+// positions; a group is up to four "query columns" that share its stages: the
+// scan's group is query tokens of one sequence (one pass over the sequence's
+// keys per group), the rescoring's group is one query token and up to four
+// selector layers (the token's pool is gathered once for all of them).
 //
-// Warp roles (16 warps):
-//   0, 1    TMA producers, alternate stages: the stage's codes (a 128-row box,
-//           two 64-row boxes when pages hold 64 rows, or 16 gathered 8-row
-//           pool blocks) in the 64B/32B swizzle the MMA reads, and the rows'
-//           per-32 E4M3 scales (the scale array seen as rows of 16 bytes);
-//   2, 3    MMA issuers, alternate stages: per query column two
+// Warp roles (20 warps):
+//   0, 1    producers, alternate stages: scan, TMA boxes of up to 256 rows of
+//           codes (in the 64B/32B swizzle the MMA reads) and of the rows'
+//           per-32 E4M3 scales, loaded with an L2 evict-first policy (the key
+//           stream is read once); rescoring, 16 pool blocks of 8 rows
+//           gathered with per-lane 16-byte cp.async;
+//   2, 3    MMA issuers, alternate stages: per tile and query column two
 //           tcgen05.mma.kind::mxf4nvf4.block_scale.block16 (M = 128 positions,
 //           N = heads, K = 64 each) into the column's part of a TMEM
 //           accumulator slot, then one commit per stage, which frees the
@@ -31,14 +34,17 @@
 //           stage's scales in the block-scale layout with tcgen05.st (each
 //           per-32 scale twice: the MMA takes one UE4M3 scale per 16
 //           elements) and arrives on the stage's scale barrier;
-//   8 .. 19 epilogue, three warpgroups taking stages in turn: TMEM -> registers
-//           (one position per thread), ReLU, weighted head sum, block max
-//           over 8 lanes (scan) and the score stores; the slot is released as
-//           soon as its last load has landed.
+//   8 .. 19 epilogue, three warpgroups: a stage's units (tiles x columns) go
+//           half to one warpgroup and half to the next, the warpgroups taking
+//           stages in turn; TMEM -> registers (one position per thread),
+//           ReLU, weighted head sum, block max over 8 lanes (scan) and the
+//           score stores; the slot is released as soon as the last load of a
+//           unit has landed.  Every score's key is counted by its top 12 bits
+//           in shared memory; the counts go to the group's global histogram
+//           (one atomic per non-empty bin) when the CTA leaves the group.
 // A tcgen05 instruction costs its issuing thread 60-170 cycles and a TMA
 // instruction several hundred, while different warps issue concurrently; the
-// roles above keep every issuing thread's per-stage instruction count small
-// (producer: 2 TMA; MMA: 2 per column + 1 commit; SF warps: one tcgen05.st).
+// roles above keep every issuing thread's per-stage instruction count small.
 // All waits are bounded; on timeout the kernel records CSA2_ERR_TIMEOUT,
 // drains its own copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -53,7 +59,7 @@ namespace csa2 {
 namespace scan_tc {
 
 constexpr int kTile = 128;      // positions per MMA tile = MMA M
-constexpr int kMaxWc = 4;       // query columns per group
+constexpr int kMaxWc = 4;       // query columns per group at most
 constexpr int kEpiWG = 3;       // epilogue warpgroups
 constexpr int kThreads = 32 * (8 + 4 * kEpiWG);
 constexpr int kProd0 = 0;       // producer warps 0, 1
