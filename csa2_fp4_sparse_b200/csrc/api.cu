@@ -35,6 +35,14 @@ int cuda_check(cudaError_t e, const char* what) {
   return fail(CSA2_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
+bool overlap_launches(int kind) {
+  static const int mask = [] {
+    const char* e = std::getenv("CSA2_OVERLAP");
+    return e ? std::atoi(e) : kOverlapQuantize | kOverlapScan | kOverlapAttend;
+  }();
+  return (mask & kind) != 0;
+}
+
 int* status_ptr() {
   static int* cache[64] = {nullptr};
   int dev = 0;
@@ -190,8 +198,9 @@ static int launch_quantize_jobs(QuantJobs& J, cudaStream_t st) {
   int64_t grid = (total + 255) / 256;
   if (grid > 148 * 32) grid = 148 * 32;
   Launch L_("quantize_fp4", st);
-  k_quantize_fp4<<<(int)grid, 256, 0, st>>>(J, status_ptr());
-  return cuda_check(cudaGetLastError(), "k_quantize_fp4");
+  return cuda_check(
+      launch_overlapped(kOverlapQuantize, k_quantize_fp4, dim3((unsigned)grid), dim3(256), 0, st, J, status_ptr()),
+      "k_quantize_fp4");
 }
 
 // appends a job of `rows` rows to J (returns false when J is full)
@@ -305,13 +314,15 @@ static int launch_select_cluster(const csa2_query_batch* qb, const float* score,
     while (S * 2 <= want) S *= 2;
   }
   cudaLaunchConfig_t cfg{};
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   cfg.blockDim = dim3(kSelThreads);
   cfg.dynamicSmemBytes = lay.bytes;
   cfg.stream = st;
   cfg.attrs = at;
   cfg.numAttrs = 1;
   at[0].id = cudaLaunchAttributeClusterDimension;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   for (;; S /= 2) {
     cfg.gridDim = dim3(S, qb->n_tok, n_sel);
     at[0].val.clusterDim.x = S;
@@ -321,6 +332,7 @@ static int launch_select_cluster(const csa2_query_batch* qb, const float* score,
     if (S == 1 || (cudaOccupancyMaxActiveClusters(&nc, k_select_cluster, &cfg) == cudaSuccess && nc >= 1)) break;
     cudaGetLastError();  // a refused shape is not an error of the call
   }
+  cfg.numAttrs = overlap_launches(kOverlapSelect) ? 2 : 1;
   Launch L_(mode == 0 ? "select_blocks" : "select_positions", st);
   return cuda_check(cudaLaunchKernelEx(&cfg, k_select_cluster, sp), "k_select_cluster");
 }
@@ -344,8 +356,7 @@ static int launch_select_multi(const csa2_query_batch* qb, const float* score, i
   sp.status = status_ptr();
   const dim3 grid(1, qb->n_tok, n_sel);
   Launch L_(mode == 0 ? "select_blocks" : "select_positions", st);
-  k_select<<<grid, kSelThreads, 0, st>>>(sp);
-  return cuda_check(cudaGetLastError(), "k_select");
+  return cuda_check(launch_overlapped(kOverlapSelect, k_select, grid, dim3(kSelThreads), 0, st, sp), "k_select");
 }
 
 int launch_select(const csa2_query_batch* qb, const float* score, int64_t ld, int mode, const int32_t* pool,
@@ -644,6 +655,13 @@ int csa2_decode_stack(const csa2_stack_desc* d, void* workspace, size_t workspac
   }
   if (d->new_k_idx && !d->new_slot_k_idx) return fail(CSA2_ERR_INVALID_ARG, "new_k_idx needs new_slot_k_idx");
   if (d->new_kv && !d->new_slot_kv) return fail(CSA2_ERR_INVALID_ARG, "new_kv needs new_slot_kv");
+  Carve sc_c{sub, sub_bytes};
+  const int64_t ld = n_blocks_max(qb);
+  float* bs = static_cast<float*>(sc_c.take((size_t)T * ld * 4));
+  float* sc = static_cast<float*>(sc_c.take((size_t)std::min(n_sel, kMaxSel) * T * d->P * kBlock * 4));
+  const SelPlan sel = take_select_scratch(sc_c, qb, d->P, std::min(n_sel, kMaxSel));
+  // cleared first, so that the step's kernels follow one another directly
+  if (int rc = clear_select_counts(sel, st)) return rc;
   // this step's appended keys and Main KV rows and every selector's indexer
   // queries: one quantisation launch (more when there are many selectors)
   {
@@ -660,12 +678,6 @@ int csa2_decode_stack(const csa2_stack_desc* d, void* workspace, size_t workspac
     }
     if (int rc = launch_quantize_jobs(J, st)) return rc;
   }
-  Carve sc_c{sub, sub_bytes};
-  const int64_t ld = n_blocks_max(qb);
-  float* bs = static_cast<float*>(sc_c.take((size_t)T * ld * 4));
-  float* sc = static_cast<float*>(sc_c.take((size_t)std::min(n_sel, kMaxSel) * T * d->P * kBlock * 4));
-  const SelPlan sel = take_select_scratch(sc_c, qb, d->P, std::min(n_sel, kMaxSel));
-  if (int rc = clear_select_counts(sel, st)) return rc;
   // each FULL layer builds the pool that it and the REINDEX layers after it
   // rescore; the rescoring and position selection of consecutive selectors
   // run up to kMaxSel at a time

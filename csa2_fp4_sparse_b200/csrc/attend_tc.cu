@@ -179,8 +179,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
   const int tok = blockIdx.y, split = blockIdx.x, nsplit = gridDim.x, layer = blockIdx.z;
   const LayerIO& io = P.io[layer];  // read from parameter space where used
   const int64_t slot0 = ((int64_t)layer * P.qb.n_tok + tok) * nsplit;  // this token's partial slots
-  const int b = __ldg(P.qb.tok_seq + tok);
-  const int64_t p = __ldg(P.qb.tok_pos + tok);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -198,6 +196,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
     tc::tmem_relinquish();
     tc::fence_before_sync();
   }
+  grid_dep_wait();  // the previous kernel's index lists
+  grid_dep_launch();
+  const int b = __ldg(P.qb.tok_seq + tok);
+  const int64_t p = __ldg(P.qb.tok_pos + tok);
   // this CTA's chunks: c = split + nsplit * i (sparse chunks first, then window chunks)
   const int n_sel = min(__ldg(io.idx_n + tok), P.K);
   const int n_sp = (n_sel + kRows - 1) / kRows;
@@ -853,8 +855,9 @@ int launch_t(const Params& p, int nsplit, int n_layers, cudaStream_t st) {
     attr[dev] = true;
   }
   Launch L_("attend_tc", st);
-  k_attend_tc<D, HQ, QLO, PLO><<<dim3(nsplit, p.qb.n_tok, n_layers), kThreads, Ly::kBytes, st>>>(p);
-  return cuda_check(cudaGetLastError(), "k_attend_tc");
+  return cuda_check(launch_overlapped(kOverlapAttend, k_attend_tc<D, HQ, QLO, PLO>,
+                                      dim3(nsplit, p.qb.n_tok, n_layers), dim3(kThreads), Ly::kBytes, st, p),
+                    "k_attend_tc");
 }
 
 // fp32 queries (the fp16 residual copy) exist for D * Hq <= 16384 only

@@ -51,6 +51,20 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ---------------------------------------------------------------- overlapped launches
+// A kernel of the decode step is launched with programmatic stream
+// serialisation, so that its CTAs can be placed, and can set up their shared
+// memory, barriers and tensor memory, while the previous kernel on the stream
+// still runs. grid_dep_wait() returns once that kernel has completed and its
+// writes are visible (at once when the launch had no such predecessor); every
+// thread calls it before its first read or write of global memory.
+// grid_dep_launch() lets the next kernel's CTAs be placed; a kernel calls it
+// after its own wait, and so after its tensor-memory allocation: a placed
+// dependant can then never hold tensor memory that a CTA of an earlier
+// kernel still has to allocate.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

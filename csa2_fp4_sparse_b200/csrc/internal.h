@@ -47,4 +47,30 @@ struct Launch {
   int slot;
 };
 
+// Overlapped launches (programmatic stream serialisation) by kernel kind:
+// the quantiser, the scan and attention by default. The selections launch
+// plainly (overlapped, they made every decode workload slower), and so does
+// the rescoring (faster at four tokens of 1M context and at chunked
+// prefill, slower at the four other workloads). The environment variable
+// CSA2_OVERLAP, a mask of the kinds below, overrides the default (0: none).
+// Every kernel launched this way calls grid_dep_wait() before it touches
+// global memory.
+enum { kOverlapQuantize = 1, kOverlapScan = 2, kOverlapRescore = 4, kOverlapSelect = 8, kOverlapAttend = 16 };
+bool overlap_launches(int kind);
+template <typename... KArgs, typename... Args>
+cudaError_t launch_overlapped(int kind, void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute at[1];
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = overlap_launches(kind) ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k, args...);
+}
+
 }  // namespace csa2

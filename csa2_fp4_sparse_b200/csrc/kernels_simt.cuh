@@ -33,6 +33,8 @@ struct QuantJobs {
 };
 
 __global__ void __launch_bounds__(256) k_quantize_fp4(const __grid_constant__ QuantJobs J, int* status) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int64_t total = J.begin[J.n];
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t base = (int64_t)blockIdx.x * blockDim.x; base < total; base += stride) {

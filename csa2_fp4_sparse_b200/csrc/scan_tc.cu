@@ -328,6 +328,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_holder;
+  grid_dep_wait();  // the previous kernel's queries, pools and cleared counts
+  grid_dep_launch();
 
   __shared__ long long s_wsum[kThreads / 32], s_nwork;
   __shared__ int s_g0, s_t0;
@@ -991,8 +993,9 @@ static int launch_index_tc(const csa2_query_batch* qb, const uint8_t* qc, const 
     attr_done[dev] = true;
   }
   Launch L_(kRescore ? "rescore_tc" : "scan_tc", st);
-  k_index_tc<kRescore, kSub><<<num_sms(), kThreads, Lay::kSmemBytes, st>>>(tmc, tms, p);
-  return cuda_check(cudaGetLastError(), "k_index_tc");
+  return cuda_check(launch_overlapped(kRescore ? kOverlapRescore : kOverlapScan, k_index_tc<kRescore, kSub>,
+                                      dim3(num_sms()), dim3(kThreads), Lay::kSmemBytes, st, tmc, tms, p),
+                    "k_index_tc");
 }
 
 int launch_scan_tc(const csa2_query_batch* qb, const uint8_t* qc, const uint8_t* qs, const float* w, int H,

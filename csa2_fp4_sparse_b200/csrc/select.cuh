@@ -77,6 +77,8 @@ __global__ void __launch_bounds__(kSelThreads) k_select(const __grid_constant__ 
   const int T = P.qb.n_tok;
   const int64_t g = (int64_t)blockIdx.z * T + tok;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  grid_dep_wait();  // the scores of the previous kernel
+  grid_dep_launch();
   const int64_t p = __ldg(P.qb.tok_pos + tok);
   int n = P.mode == 0 ? (int)max((p + kBlock) / kBlock, (int64_t)0) : min(__ldg(P.pool_n + tok), P.P) * kBlock;
   n = (int)max((int64_t)0, min((int64_t)n, P.ld));  // never past the score row
@@ -435,6 +437,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select_cluster(const __grid_
   const int64_t g = (int64_t)blockIdx.z * T + tok;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const SelCLayout Lo(P.words, P.cap, P.mode == 1 ? P.P : 0);
+  grid_dep_wait();  // the scores and key counts of the previous kernel
+  grid_dep_launch();
   uint32_t* bsel = reinterpret_cast<uint32_t*>(sm + Lo.sel);
   uint32_t* btie = reinterpret_cast<uint32_t*>(sm + Lo.tie);
   uint2* cand = reinterpret_cast<uint2*>(sm + Lo.cand);

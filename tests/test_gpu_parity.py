@@ -297,3 +297,47 @@ def test_stack_attend_wait_event():
     assert _status() == 0
     torch.cuda.synchronize()
     assert torch.equal(dw.out_all, ref)
+
+
+_OVERLAP_CHILD = r"""
+import ctypes, hashlib, sys
+sys.path.insert(0, sys.argv[1])
+import torch
+import csa2_fp4_sparse_b200 as C
+from synth.gpu import DeviceWorkload
+from synth.workloads import CONFIGS
+cfg = CONFIGS[int(sys.argv[2])].with_(B=int(sys.argv[3]), lengths=("fixed", int(sys.argv[4])))
+from synth.workloads import make_workload
+w = make_workload(cfg)
+dw = DeviceWorkload(w)
+dw.fill_caches(include_new=False)
+desc = dw.stack_desc(append=True, copies=False)
+ws = dw.stack_workspace(desc)
+sp = torch.cuda.current_stream().cuda_stream
+for _ in range(4):  # back to back: each step's first kernel follows the last one's attention
+    C.check(C.csa2_decode_stack(ctypes.byref(desc), ws.data_ptr(), ws.numel(), sp))
+torch.cuda.synchronize()
+assert C.csa2_get_status(sp) == 0
+print(hashlib.sha256(dw.out_all.cpu().view(torch.uint8).numpy().tobytes()).hexdigest())
+"""
+
+
+@pytest.mark.parametrize("i,B,L", [(2, 3, 9000), (4, 2, 40000), (5, 6, 3000)])
+def test_stack_overlapped_launches_bit_identical(i, B, L):
+    """Decode steps with no overlapped launch (CSA2_OVERLAP=0), the default
+    set and every kernel kind overlapped (31) give bit-identical outputs"""
+    import os
+    import subprocess
+    import sys
+    root = os.path.abspath(os.path.join(os.path.dirname(__file__), ".."))
+    digests = {}
+    for mask in ("0", None, "31"):
+        env = dict(os.environ)
+        env.pop("CSA2_OVERLAP", None)
+        if mask is not None:
+            env["CSA2_OVERLAP"] = mask
+        r = subprocess.run([sys.executable, "-c", _OVERLAP_CHILD, root, str(i), str(B), str(L)], env=env,
+                           capture_output=True, text=True, timeout=600)
+        assert r.returncode == 0, r.stderr[-2000:]
+        digests[mask] = r.stdout.strip().splitlines()[-1]
+    assert len(set(digests.values())) == 1, digests
