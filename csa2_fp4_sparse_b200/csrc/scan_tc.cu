@@ -356,8 +356,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++n;
       }
     };
-    int cur_g = -1, tok0 = 0, b = 0;
+    int cur_g = -1, tok0 = 0, b = 0, np_g = 0;
     int64_t base = 0, len = 0;
+    // rescore: lane e < 16 holds the pool id of block e of stage (pf_g,
+    // pf_tile), loaded one stage of this warp ahead of its use
+    int pf_g = -1, pf_tile = -1;
+    int32_t pf_blk = -1;
     const uint64_t l2_ef = tc::l2_policy_evict_first();
     for (; ti.valid(); ti.next(P), adv()) {
       if ((it & 1) != pw || *abort) continue;
@@ -374,6 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         group_info<kRescore>(P, cur_g, &tok0, &W, &b, &sel0);
         len = __ldg(P.qb.seq_len + b);
         base = P.page_table ? 0 : __ldg(P.seq_base + b);
+        if (kRescore) np_g = min(__ldg(P.pool_n + tok0), P.pool_cap);  // the token's pool size in blocks
       }
       if (kRescore) {
         // gather: 16 pool blocks of 8 rows, 16-byte asynchronous copies from
@@ -381,16 +386,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         // warp hundreds of cycles each); codes land in the swizzle the MMA
         // reads, each block's scales at its 128-byte slot.  Rows outside the
         // cache are zero-filled.
-        int64_t my_row0 = -1;  // lane e < 16: first cache row of block e
+        int32_t blk = -1;
         if (lane < 16) {
           const int e = ti.tile * 16 + lane;
-          const int np = min(__ldg(P.pool_n + tok0), P.pool_cap);
-          const int32_t blk = e < np ? __ldg(P.pool + (int64_t)tok0 * P.pool_cap + e) : -1;
-          if (blk >= 0) {
-            const int64_t row0 = key_row(P, b, (int64_t)blk * kBlock, base);
-            if (row0 >= 0 && ((row0 * spr) & 15) == 0) my_row0 = row0;
-            else set_status(P.status, CSA2_ERR_RANGE);
-          }
+          blk = (pf_g == ti.b && pf_tile == ti.tile) ? pf_blk
+                                                     : (e < np_g ? __ldg(P.pool + (int64_t)tok0 * P.pool_cap + e) : -1);
+        }
+        // this warp's next stage (two on), when in the same group: its pool
+        // ids load while this stage's copies are issued
+        if (ti.left > 2 && ti.tile + 2 < ti.ntile) {
+          pf_g = ti.b;
+          pf_tile = ti.tile + 2;
+          const int e2 = pf_tile * 16 + lane;
+          pf_blk = (lane < 16 && e2 < np_g) ? __ldg(P.pool + (int64_t)tok0 * P.pool_cap + e2) : -1;
+        }
+        int64_t my_row0 = -1;  // lane e < 16: first cache row of block e
+        if (blk >= 0) {
+          const int64_t row0 = key_row(P, b, (int64_t)blk * kBlock, base);
+          if (row0 >= 0 && ((row0 * spr) & 15) == 0) my_row0 = row0;
+          else set_status(P.status, CSA2_ERR_RANGE);
         }
         const int cpr = row_bytes / 16;  // 16-byte chunks a code row
         const uint32_t a_base = sbase + kOffA + s * kCodeStage;
@@ -684,7 +698,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (++slot == P.n_slots) slot = 0;
       if (++wgc == kEpiWG) wgc = 0;
     };
-    int cur_g = -1, W = 0, tok0 = 0, sel0 = 0;
+    int cur_g = -1, W = 0, tok0 = 0, sel0 = 0, np_e = 0;
     bool dead = false;  // a wait of this warp (two-tile stages) or warpgroup gave up
     const int ng = P.Nh / 16;
     // The group's key counts gather in shared memory (per CTA) and go to the
@@ -722,6 +736,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           w_g[e] = h < P.H ? 0.5f * __ldg(wsrc + h) : 0.0f;
         }
         if (ept < W) pos_g[ept] = __ldg(P.qb.tok_pos + (kRescore ? tok0 : tok0 + ept));
+        if (kRescore) np_e = min(__ldg(P.pool_n + tok0), P.pool_cap);
         tc::named_sync(1 + wg, 128);
       }
       // units of this stage, the first half to warpgroup wgc, the rest to the
@@ -736,6 +751,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         mj1 = nu;
       }
       if (mj0 >= mj1 || dead) continue;  // no unit of this stage (or nothing left to do)
+      int32_t blk = -1;  // rescore: this thread's pool block, loaded while the stage's MMAs run
+      if (kRescore) {
+        const int i = ti.tile * kTile + row;
+        blk = (i / kBlock) < np_e ? __ldg(P.pool + (int64_t)tok0 * P.pool_cap + i / kBlock) : -1;
+      }
       // two-tile stages: every warp probes for itself (measured faster);
       // otherwise one prober per warpgroup, the other warps parked on the
       // named barrier
@@ -753,12 +773,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::fence_after_sync();
       const int64_t t0 = (int64_t)ti.tile * kRows;
       const uint32_t taddr0 = tmem + ((uint32_t)(quarter * 32) << 16) + kColAcc + (uint32_t)(slot * P.slot_cols);
-      int32_t blk = -1;  // rescore: this thread's pool block
-      if (kRescore) {
-        const int i = ti.tile * kTile + row;
-        const int np = min(__ldg(P.pool_n + tok0), P.pool_cap);
-        blk = (i / kBlock) < np ? __ldg(P.pool + (int64_t)tok0 * P.pool_cap + i / kBlock) : -1;
-      }
       for (int mj = mj0; mj < mj1; ++mj) {  // unit: tile m = mj / W of the stage, query column j = mj % W
         // two-tile stages only serve one query token per sequence (W = 1)
         const int m = kSub == 1 ? 0 : mj, j = kSub == 1 ? mj : 0;
