@@ -197,7 +197,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
     tc::fence_before_sync();
   }
   grid_dep_wait();  // the previous kernel's index lists
-  grid_dep_launch();
   const int b = __ldg(P.qb.tok_seq + tok);
   const int64_t p = __ldg(P.qb.tok_pos + tok);
   // this CTA's chunks: c = split + nsplit * i (sparse chunks first, then window chunks)
@@ -824,6 +823,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
     }
   }
   // no MMA of ours may be in flight when TMEM is released
+  grid_dep_launch();
   if (threadIdx.x == 0) {
     if (!mbar_wait_bounded(bar_drain, 0, P.wait_ns)) set_status(P.status, CSA2_ERR_TIMEOUT);
   }

@@ -61,7 +61,9 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // grid_dep_launch() lets the next kernel's CTAs be placed; a kernel calls it
 // after its own wait, and so after its tensor-memory allocation: a placed
 // dependant can then never hold tensor memory that a CTA of an earlier
-// kernel still has to allocate.
+// kernel still has to allocate. The persistent scoring kernels and attention
+// call it when their CTA's work is done (measured faster than at the start:
+// the dependants are placed on the SMs the tail frees).
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 

@@ -329,7 +329,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_holder;
   grid_dep_wait();  // the previous kernel's queries, pools and cleared counts
-  grid_dep_launch();
 
   __shared__ long long s_wsum[kThreads / 32], s_nwork;
   __shared__ int s_g0, s_t0;
@@ -845,6 +844,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::named_sync(7, kEpiThreads);  // the last group's counts are complete
     if (P.hist && cur_g >= 0) flush_counts();
   }
+  grid_dep_launch();
   // after a failed wait some tile loads may still be in flight: give them
   // time to land before the CTA's shared memory is released (bounded)
   if (threadIdx.x == 0 && *abort) {

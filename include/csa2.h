@@ -33,6 +33,13 @@
  *   - Index outputs are ascending, padded with -1, with a count array.
  *   - Functions are thread-safe as long as concurrent calls use different
  *     output and workspace buffers.  csa2_last_error() is per thread.
+ *   - The quantiser, scan and attention kernels are launched with
+ *     programmatic stream serialisation: their CTAs may be placed while the
+ *     previous kernel on the stream runs, but each waits for that kernel's
+ *     completion before touching global memory, so stream order is kept.
+ *     The environment variable CSA2_OVERLAP (read once per process: a mask of
+ *     1 quantiser, 2 scan, 4 rescoring, 8 selections, 16 attention; 0 = none)
+ *     replaces the default set (1 | 2 | 16).
  */
 #ifndef CSA2_H
 #define CSA2_H
