@@ -405,10 +405,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (row0 >= 0 && ((row0 * spr) & 15) == 0) my_row0 = row0;
           else set_status(P.status, CSA2_ERR_RANGE);
         }
-        const int cpr = row_bytes / 16;  // 16-byte chunks a code row
+        // 16-byte chunks a code row: 1 << cshift (d_I is 64 or 128); shifts,
+        // not divisions by a runtime value, keep this loop short
+        const int cshift = P.DI == 128 ? 2 : 1;
         const uint32_t a_base = sbase + kOffA + s * kCodeStage;
-        for (int c = lane; c < kTile * cpr; c += 32) {
-          const int r = c / cpr, ch = c % cpr;
+        for (int c = lane; c < (kTile << cshift); c += 32) {
+          const int r = c >> cshift, ch = c & ((1 << cshift) - 1);
           const int64_t row0 = __shfl_sync(0xffffffffu, my_row0, r / kBlock);
           const int64_t gr = row0 + r % kBlock;
           const bool in = row0 >= 0 && gr < P.n_rows;
@@ -501,16 +503,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           };
           // B operand: query codes, swizzled like the TMA-written A tiles,
           // in 16-byte asynchronous copies that are all in flight together
-          // (heads past H zero-filled)
-          const int chunks_per_row = row_bytes / 16;
-          for (int e = lane; e < W * 64 * chunks_per_row; e += 32) {
-            const int j = e / (64 * chunks_per_row);
-            const int n = (e / chunks_per_row) % 64;
-            const int ch = e % chunks_per_row;
-            const int sch = (P.DI == 128) ? (ch ^ ((n >> 1) & 3)) : (ch ^ ((n >> 2) & 1));
-            const bool in = n < P.H;
-            tc::cp_async_16(sbase + kOffB + j * 4096 + n * row_bytes + sch * 16,
-                            in ? P.q_codes + (qrow(j) * P.H + n) * row_bytes + ch * 16 : P.q_codes, in ? 16u : 0u);
+          // (heads past H zero-filled); a code row is 1 << cshift chunks
+          // (shifts, not divisions by a runtime value: this loop is one
+          // warp's serial work on the way to the first MMA)
+          const int cshift = P.DI == 128 ? 2 : 1;
+          for (int j = 0; j < W; ++j) {
+            const uint8_t* src = P.q_codes + qrow(j) * P.H * row_bytes;
+            const uint32_t dst = sbase + kOffB + j * 4096;
+            for (int e = lane; e < (64 << cshift); e += 32) {
+              const int n = e >> cshift, ch = e & ((1 << cshift) - 1);
+              const int sch = (P.DI == 128) ? (ch ^ ((n >> 1) & 3)) : (ch ^ ((n >> 2) & 1));
+              const bool in = n < P.H;
+              tc::cp_async_16(dst + n * row_bytes + sch * 16, in ? src + n * row_bytes + ch * 16 : P.q_codes,
+                              in ? 16u : 0u);
+            }
           }
           // B scale factors, [m0 (32)][m1 (4)][k (4)] per 64-element K step:
           // lane m0 first loads the scale words of its heads m1*32 + m0 of
