@@ -254,12 +254,15 @@ __device__ __forceinline__ bool warp_wait_or_abort(uint32_t bar, uint32_t parity
   return __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
 }
 
-// cache row of position `pos` of sequence b, or -1 when outside the cache
+// cache row of position `pos` (0 <= pos < max_seq_len, so 32-bit) of
+// sequence b, or -1 when outside the cache
 __device__ __forceinline__ int64_t key_row(const Params& P, int b, int64_t pos, int64_t base) {
   int64_t row;
   if (P.page_table) {
-    const int32_t pg = __ldg(P.page_table + (int64_t)b * P.max_pages + pos / P.page_size);
-    row = (int64_t)pg * P.page_size + pos % P.page_size;
+    const uint32_t p32 = (uint32_t)pos, ps = (uint32_t)P.page_size;  // unsigned 32-bit divide: the short one
+    const uint32_t q = p32 / ps;
+    const int32_t pg = __ldg(P.page_table + (int64_t)b * P.max_pages + q);
+    row = (int64_t)pg * P.page_size + (p32 - q * ps);
   } else {
     row = base + pos;
   }
@@ -400,7 +403,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           pf_blk = (lane < 16 && e2 < np_g) ? __ldg(P.pool + (int64_t)tok0 * P.pool_cap + e2) : -1;
         }
         int64_t my_row0 = -1;  // lane e < 16: first cache row of block e
-        if (blk >= 0) {
+        // (a block past the sequence holds no key: zero-filled, scored -inf)
+        if (blk >= 0 && (int64_t)blk * kBlock < len) {
           const int64_t row0 = key_row(P, b, (int64_t)blk * kBlock, base);
           if (row0 >= 0 && ((row0 * spr) & 15) == 0) my_row0 = row0;
           else set_status(P.status, CSA2_ERR_RANGE);
