@@ -234,7 +234,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
       const int32_t t = tv[u];
       pg[u] = 0;
       if (t >= 0 && t <= p)
-        pg[u] = P.kv.page_table ? (int64_t)__ldg(P.kv.page_table + (int64_t)b * P.kv.max_pages + t / P.kv.page_size)
+        pg[u] = P.kv.page_table ? (int64_t)__ldg(P.kv.page_table + (int64_t)b * P.kv.max_pages +
+                                                 (uint32_t)t / (uint32_t)P.kv.page_size)
                                 : __ldg(P.kv.seq_base + b);
     }
   };
@@ -319,7 +320,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
       }
       int64_t row = -1;
       if (t >= 0 && t <= p) {
-        row = P.kv.page_table ? pg[u] * P.kv.page_size + t % P.kv.page_size : pg[u] + t;
+        row = P.kv.page_table ? pg[u] * P.kv.page_size + (int64_t)((uint32_t)t % (uint32_t)P.kv.page_size)
+                              : pg[u] + t;
         if (row < 0 || row >= P.kv.n_rows) row = -1;
       }
       if (row < 0) set_status(P.status, CSA2_ERR_RANGE);
@@ -348,7 +350,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_tc(const __grid_constant
           row = rows_s[i * kRows + r];
         } else {
           const int64_t t = w_lo + (int64_t)(c - n_sp) * kRows + r;
-          if (t <= p) row = (int64_t)b * P.swa_cap + t % P.swa_cap;
+          // 0 <= t < max_seq_len: an unsigned 32-bit remainder (a 64-bit one
+          // costs the loader a long instruction sequence per unit)
+          if (t <= p) row = (int64_t)b * P.swa_cap + (int64_t)((uint32_t)t % (uint32_t)P.swa_cap);
         }
         pf.c[k] = make_uint4(0, 0, 0, 0);
         pf.s[k] = 0;
