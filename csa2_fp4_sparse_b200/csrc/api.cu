@@ -305,12 +305,13 @@ static int launch_select_cluster(const csa2_query_batch* qb, const float* score,
       return rc;
     attr_done[dev] = true;
   }
-  // CTAs per group: about 8192 candidates each, a power of two <= 16, the
-  // whole grid within the SMs, and a cluster shape the GPU can place
+  // CTAs per group: about 4096 candidates each (measured: 8192 and 2048
+  // slower where the groups are few), a power of two <= 16, the whole grid
+  // within the SMs, and a cluster shape the GPU can place
   int S = 1;
   const int sms = std::min(num_sms_dev(), kSelMaxGroups);
   if (groups < sms) {
-    int want = (int)std::min<int64_t>({(int64_t)(n_max + 8191) / 8192, 16, sms / groups});
+    int want = (int)std::min<int64_t>({(int64_t)(n_max + 4095) / 4096, 16, sms / groups});
     while (S * 2 <= want) S *= 2;
   }
   cudaLaunchConfig_t cfg{};
